@@ -1,0 +1,240 @@
+"""Plain fp64 CPU oracle for the Lookahead Sparse Attention (LSA) decode step.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, calls or links
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it.  It shares no code with the CUDA library and imports
+nothing from it.  Every input arrives as a numpy array (bf16 values already
+widened exactly to float32/float64 by the caller, or raw integers for the byte
+copies); every floating-point step runs in float64.
+
+What it computes, and the passages it follows
+---------------------------------------------
+Sources are the web pages about "FlashMemory-DeepSeek-V4: Lightning Index
+Ultra-Long Context via Lookahead Sparse Attention" (cited below as *FM-DS-V4
+summary*, with its section), the handbook page "DeepSeek-V4: Architecting for
+Ultra-Long Contexts" (*DS-V4 handbook*, with its section) and the Korean review
+of the same paper (*FM-DS-V4 review*, with its section).
+
+1. ``index_scores`` -- the Neural Memory Indexer.  Every tau decode steps the
+   indexer scores each historical chunk from the current query state against
+   the chunk's cached indexer key (FM-DS-V4 summary, 1 Introduction and
+   2.1 Architecture; DS-V4 handbook, "The Neural Memory Indexer", items 2-3),
+   through a sigmoid (FM-DS-V4 review, 1. Key Terms, "Neural Memory Indexer")
+   over a dot product (FM-DS-V4 summary, 3 Experiments "Limitations").  The
+   specified form is score_c = sum_h w_h * sigmoid(q_h . k_c / sqrt(d_I)) over
+   H_I = 16 indexer heads, d_I = 128.
+2. ``topk_chunks`` -- keep the K highest-scoring chunks among all but the latest
+   one, ordered by (score descending, chunk index ascending), and always keep
+   the latest chunk (the non-offloadable recent context of FM-DS-V4 summary,
+   2.1 Architecture).  The kept list is returned in ascending chunk order.
+3. ``gather_chunks`` -- copy the kept chunks, in kept order, into one compact
+   buffer, so that only the chunks the query needs stay resident on the GPU
+   (FM-DS-V4 summary, Abstract and 2.1 Architecture).
+4. ``sparse_decode_attn`` -- GQA decode attention over the kept tokens only:
+   softmax(Q K^T / sqrt(d_k)) V per query head (DS-V4 handbook, "Grouped Query
+   Attention (GQA) vs. Multi-Head Attention (MHA)", the attention equation), 64
+   query heads sharing 8 KV heads, head dimension 128, every 8 consecutive query
+   heads on one KV head (same section, the DeepSeek-V4 configuration list).
+   Plain two-pass softmax, no splitting.
+5. ``threshold_chunks`` -- the pages' own selection rule: sigmoid thresholding
+   at 0.5 in place of a fixed top-k (FM-DS-V4 summary, 2.1 Architecture and
+   2.4 Configuration), read as score_c / sum_h w_h > 0.5, latest chunk kept.
+
+Readings taken where the pages are silent are listed in the design notes of
+this repository and marked "Reading:" at the point of use.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, special cases reducing to library routines, brute force).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# Shapes fixed by the method (DS-V4 handbook, GQA section: 64 query heads,
+# 8 KV heads, head dim 128).  Indexer heads and dims: H_I = 16, d_I = 128.
+# Chunk length: 64 tokens.
+NUM_Q_HEADS = 64
+NUM_KV_HEADS = 8
+HEAD_DIM = 128
+GROUP = NUM_Q_HEADS // NUM_KV_HEADS
+CHUNK_TOKENS = 64
+INDEX_HEADS = 16
+INDEX_DIM = 128
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of raw bf16 bit patterns (uint16/int16) to float64."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _slot(chunk_table, b: int, c: int, max_chunks: int) -> int:
+    # Reading: a missing table means the identity layout, slot = b*max_chunks + c.
+    if chunk_table is None:
+        return b * max_chunks + c
+    return int(chunk_table[b, c])
+
+
+def index_scores(q_idx, w, chunk_keys, chunk_table, n_chunks, max_chunks=None):
+    """Indexer scores for every chunk of every sequence.
+
+    q_idx      [B, H_I, d_I]  indexer query of the window (one per sequence).
+    w          [H_I]          per-head indexer weights.
+    chunk_keys [n_slots, d_I] cached indexer key of each physical chunk slot.
+    chunk_table[B, max_chunks] logical chunk -> physical slot, or None.
+    n_chunks   [B]            number of chunks in each sequence.
+
+    Returns float64 [B, max_chunks]; entries c >= n_chunks[b] are NaN.
+    score[b, c] = sum_h w_h * sigmoid(q_idx[b, h] . k[slot(b, c)] / sqrt(d_I)).
+    """
+    q_idx = np.asarray(q_idx, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    keys = np.asarray(chunk_keys, dtype=np.float64)
+    n_chunks = np.asarray(n_chunks).astype(np.int64)
+    B = q_idx.shape[0]
+    if max_chunks is None:
+        max_chunks = int(chunk_table.shape[1]) if chunk_table is not None else int(n_chunks.max(initial=0))
+    out = np.full((B, max_chunks), np.nan, dtype=np.float64)
+    for b in range(B):
+        n = int(n_chunks[b])
+        if n == 0:
+            continue
+        slots = np.array([_slot(chunk_table, b, c, max_chunks) for c in range(n)], dtype=np.int64)
+        logits = q_idx[b] @ keys[slots].T / math.sqrt(INDEX_DIM)      # [H_I, n]
+        sig = 1.0 / (1.0 + np.exp(-logits))                             # sigmoid, fp64 libm exp
+        out[b, :n] = w @ sig                                            # weighted sum over heads
+    return out
+
+
+def topk_chunks(scores, n_chunks, k_per_seq):
+    """Per-sequence kept chunk lists.
+
+    Candidates are the chunks 0 .. n-2 (all but the latest).  They are ordered
+    by score descending, then chunk index ascending; the first K are kept, the
+    latest chunk n-1 is added, and the list is returned in ascending order.
+    Reading: the latest chunk is outside the K budget, so exactly min(K, n-1)+1
+    chunks are kept; K >= n-1 keeps every chunk; n == 0 keeps none.
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    out = []
+    for b in range(len(n_chunks)):
+        n = int(n_chunks[b])
+        k = int(k_per_seq[b])
+        if n == 0:
+            out.append(np.zeros(0, dtype=np.int64))
+            continue
+        cand = np.arange(n - 1, dtype=np.int64)
+        s = scores[b, : n - 1]
+        # np.lexsort sorts by the last key first: primary key -score, then index.
+        order = np.lexsort((cand, -s))
+        chosen = cand[order[: max(0, min(k, n - 1))]]
+        kept = np.sort(np.concatenate([chosen, np.array([n - 1], dtype=np.int64)]))
+        out.append(kept)
+    return out
+
+
+def threshold_chunks(scores, n_chunks, w, threshold=0.5):
+    """The pages' sigmoid-threshold selection (FM-DS-V4 summary, 2.1 and 2.4).
+
+    Reading: a chunk is recalled when its weighted mean sigmoid probability
+    score_c / sum_h w_h exceeds the threshold; the latest chunk is always kept.
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    wsum = float(np.sum(np.asarray(w, dtype=np.float64)))
+    out = []
+    for b in range(len(n_chunks)):
+        n = int(n_chunks[b])
+        if n == 0:
+            out.append(np.zeros(0, dtype=np.int64))
+            continue
+        cand = np.arange(n - 1, dtype=np.int64)
+        chosen = cand[scores[b, : n - 1] / wsum > threshold]
+        out.append(np.concatenate([chosen, np.array([n - 1], dtype=np.int64)]))
+    return out
+
+
+def cumulative_kept(kept_lists):
+    """cu_kept[B+1]: start of each sequence's kept chunks in the compact buffer."""
+    cu = np.zeros(len(kept_lists) + 1, dtype=np.int64)
+    for b, k in enumerate(kept_lists):
+        cu[b + 1] = cu[b] + len(k)
+    return cu
+
+
+def gather_chunks(k_pool, v_pool, chunk_table, kept_lists, max_chunks=None):
+    """Copy kept chunks into the compact buffers, sequence by sequence, in kept order.
+
+    Pools are [n_slots, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM] of any dtype; the
+    copy is element-exact.  Returns (k_buf, v_buf, cu_kept).
+    """
+    if max_chunks is None and chunk_table is not None:
+        max_chunks = chunk_table.shape[1]
+    cu = cumulative_kept(kept_lists)
+    total = int(cu[-1])
+    k_buf = np.empty((total,) + tuple(k_pool.shape[1:]), dtype=k_pool.dtype)
+    v_buf = np.empty((total,) + tuple(v_pool.shape[1:]), dtype=v_pool.dtype)
+    for b, kept in enumerate(kept_lists):
+        for j, c in enumerate(kept):
+            s = _slot(chunk_table, b, int(c), max_chunks)
+            k_buf[cu[b] + j] = k_pool[s]
+            v_buf[cu[b] + j] = v_pool[s]
+    return k_buf, v_buf, cu
+
+
+def attend_one(q_h, K, V, scale):
+    """softmax(q K^T * scale) V for one query vector over T tokens (two-pass)."""
+    s = (K @ q_h) * scale          # [T]
+    m = np.max(s)
+    p = np.exp(s - m)
+    return (p @ V) / np.sum(p)
+
+
+def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=None):
+    """GQA decode attention of each query head over its sequence's kept tokens.
+
+    q      [B, 64, 128]
+    k_buf  [total_kept, 8, 64, 128], v_buf the same
+    cu_kept[B+1]
+    Query head h reads KV head h // 8 (8 consecutive query heads per KV head).
+    Returns float64 [B, 64, 128]; a sequence with no kept chunk gives zeros
+    (Reading: the empty softmax is defined as a zero output).
+    ``seqs``/``heads`` restrict the work to a sample; other rows stay NaN.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    q = np.asarray(q, dtype=np.float64)
+    B = q.shape[0]
+    out = np.full((B, NUM_Q_HEADS, HEAD_DIM), np.nan, dtype=np.float64)
+    seqs = range(B) if seqs is None else seqs
+    heads = range(NUM_Q_HEADS) if heads is None else heads
+    for b in seqs:
+        lo, hi = int(cu_kept[b]), int(cu_kept[b + 1])
+        if hi == lo:
+            out[b, list(heads)] = 0.0
+            continue
+        for g in range(NUM_KV_HEADS):
+            group_heads = [h for h in heads if h // GROUP == g]
+            if not group_heads:
+                continue
+            K = np.asarray(k_buf[lo:hi, g], dtype=np.float64).reshape(-1, HEAD_DIM)
+            V = np.asarray(v_buf[lo:hi, g], dtype=np.float64).reshape(-1, HEAD_DIM)
+            for h in group_heads:
+                out[b, h] = attend_one(q[b, h], K, V, scale)
+    return out
+
+
+def decode_window(q_idx, w, chunk_keys, chunk_table, n_chunks, k_per_seq,
+                  k_pool, v_pool, q_steps, max_chunks=None, steps=None):
+    """One lookahead window: score, select, gather, then attention for each step.
+
+    q_steps [T, B, 64, 128]: the decode-step queries of the window.
+    Returns (scores, kept_lists, cu_kept, outputs[T, B, 64, 128]).
+    """
+    scores = index_scores(q_idx, w, chunk_keys, chunk_table, n_chunks, max_chunks)
+    kept = topk_chunks(scores, n_chunks, k_per_seq)
+    k_buf, v_buf, cu = gather_chunks(k_pool, v_pool, chunk_table, kept, max_chunks)
+    steps = range(q_steps.shape[0]) if steps is None else steps
+    outs = {t: sparse_decode_attn(q_steps[t], k_buf, v_buf, cu) for t in steps}
+    return scores, kept, cu, outs

@@ -1,0 +1,341 @@
+"""Pins of the fp64 oracle against facts fixed outside the oracle itself.
+
+Each test ties one oracle function to something other than its own formula:
+a closed form, a special case that reduces to a library routine (scipy's
+``expit``, torch's ``scaled_dot_product_attention``, Python's ``sorted``), an
+invariant, or brute force on tiny inputs.  They are chosen so that a plausible
+slip (a dropped scale, a sign, a head mapped to the wrong KV head, a transposed
+operand, a wrong tie order, a lost latest chunk) fails at least one of them.
+CPU only.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+import oracle
+
+RNG = np.random.default_rng(1234)
+
+
+def bf16_round(x):
+    """Round float values to bf16 (nearest even) and widen back to float64."""
+    return torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+# ----------------------------------------------------------------- scoring ---
+
+def test_score_zero_query_is_half_weight_sum():
+    """q_I = 0: every logit is 0, sigmoid(0) = 1/2, so score = sum(w)/2 for every chunk."""
+    B, N = 2, 7
+    q = np.zeros((B, 16, 128))
+    w = RNG.uniform(0, 1, 16)
+    keys = bf16_round(RNG.standard_normal((B * N, 128)))
+    s = oracle.index_scores(q, w, keys, None, [N, N], max_chunks=N)
+    np.testing.assert_allclose(s, np.full((B, N), w.sum() / 2), rtol=1e-15, atol=0)
+
+
+def test_score_closed_form_scale_and_head_weights():
+    """q_h = a_h * ones, k = ones/8: q_h.k / sqrt(128) = a_h * 16 / sqrt(128) = a_h*sqrt(2).
+
+    The score is then sum_h w_h * expit(a_h * sqrt(2)), computed here with scipy's
+    expit.  Pins the 1/sqrt(d_I) scale (not 1/d_I, not none), the sigmoid sign and
+    that head h uses weight w_h.
+    """
+    a = np.array([0, 1, -1, 2, -2, 3, 0.5, -0.5, 1, 0, -3, 2, 1, -1, 0.25, 4], dtype=np.float64)
+    q = np.ones((1, 16, 128)) * a[None, :, None]
+    keys = np.full((3, 128), 0.125)
+    w = RNG.uniform(0, 1, 16)
+    s = oracle.index_scores(q, w, keys, None, [3], max_chunks=3)
+    expect = float(np.dot(w, expit(a * math.sqrt(2.0))))
+    np.testing.assert_allclose(s[0], [expect] * 3, rtol=1e-14)
+    # one-hot weights isolate each head
+    for h in range(16):
+        e = np.zeros(16)
+        e[h] = 1.0
+        s = oracle.index_scores(q, e, keys, None, [3], max_chunks=3)
+        np.testing.assert_allclose(s[0, 0], expit(a[h] * math.sqrt(2.0)), rtol=1e-14)
+
+
+def test_score_sigmoid_root2_high_precision():
+    """sigmoid(sqrt 2) evaluated with 40-digit decimal arithmetic, independent of numpy."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 40
+    expect = float(1 / (1 + (-Decimal(2).sqrt()).exp()))
+    q = np.ones((1, 16, 128))
+    keys = np.full((1, 128), 0.125)
+    e = np.zeros(16)
+    e[0] = 1.0
+    s = oracle.index_scores(q, e, keys, None, [1], max_chunks=1)
+    assert abs(s[0, 0] - expect) < 2e-16
+
+
+def test_score_chunk_table_indirection():
+    """score[b, c] depends only on the key in slot table[b, c].
+
+    Slot s holds the key x_s * ones with x_s = s/64 (exact in bf16), so with q = ones
+    on head 0 and w = e_0 the score of a slot is expit(sqrt(128) * x_s) in closed form.
+    """
+    B, M, S = 3, 6, 18
+    keys = np.repeat((np.arange(S) / 64.0)[:, None], 128, axis=1)
+    table = RNG.permutation(S)[: B * M].reshape(B, M)
+    n = [6, 4, 0]
+    q = np.zeros((B, 16, 128))
+    q[:, 0, :] = 1.0
+    e = np.zeros(16)
+    e[0] = 1.0
+    s = oracle.index_scores(q, e, keys, table, n)
+    for b in range(B):
+        for c in range(M):
+            if c < n[b]:
+                np.testing.assert_allclose(s[b, c], expit(math.sqrt(128) * table[b, c] / 64.0), rtol=1e-14)
+            else:
+                assert np.isnan(s[b, c])
+
+
+def test_score_range_invariant():
+    """0 < score < sum(w) on random bf16 inputs."""
+    B, N = 2, 50
+    q = bf16_round(RNG.standard_normal((B, 16, 128)))
+    keys = bf16_round(RNG.standard_normal((B * N, 128)))
+    w = RNG.uniform(0, 1, 16)
+    s = oracle.index_scores(q, w, keys, None, [N, N], max_chunks=N)
+    assert np.all(s > 0) and np.all(s < w.sum())
+
+
+def test_score_brute_force_loops():
+    """Independent triple loop with math.exp on a tiny paged case."""
+    B, M = 2, 5
+    q = bf16_round(RNG.standard_normal((B, 16, 128)))
+    keys = bf16_round(RNG.standard_normal((12, 128)))
+    table = RNG.permutation(12)[:10].reshape(B, M)
+    w = RNG.uniform(0, 1, 16)
+    s = oracle.index_scores(q, w, keys, table, [5, 3])
+    for b in range(B):
+        for c in range([5, 3][b]):
+            tot = 0.0
+            for h in range(16):
+                dot = sum(q[b, h, i] * keys[table[b, c], i] for i in range(128))
+                tot += w[h] * (1.0 / (1.0 + math.exp(-dot / math.sqrt(128))))
+            assert abs(s[b, c] - tot) <= 1e-13 * abs(tot)
+
+
+# ------------------------------------------------------------------- top-K ---
+
+def _brute_topk(scores_row, n, k):
+    if n == 0:
+        return []
+    cand = sorted(range(n - 1), key=lambda c: (-scores_row[c], c))
+    return sorted(cand[: max(0, min(k, n - 1))] + [n - 1])
+
+
+@pytest.mark.parametrize("trial", range(30))
+def test_topk_matches_full_sort(trial):
+    rng = np.random.default_rng(trial)
+    B = int(rng.integers(1, 5))
+    M = int(rng.integers(1, 65))
+    n = rng.integers(0, M + 1, B)
+    k = rng.integers(0, M + 2, B)
+    if trial % 3 == 0:      # many exact ties
+        scores = rng.integers(0, 4, (B, M)).astype(np.float64)
+    else:
+        scores = rng.standard_normal((B, M))
+    got = oracle.topk_chunks(scores, n, k)
+    for b in range(B):
+        assert list(got[b]) == _brute_topk(list(scores[b]), int(n[b]), int(k[b]))
+
+
+def test_topk_all_ties_closed_form():
+    """All scores equal: the lowest indices win: kept = {0..K-1} + {N-1}."""
+    N, K = 40, 9
+    got = oracle.topk_chunks(np.full((1, N), 0.37), [N], [K])
+    assert list(got[0]) == list(range(K)) + [N - 1]
+
+
+def test_topk_boundaries():
+    s = RNG.standard_normal((1, 10))
+    assert list(oracle.topk_chunks(s, [10], [9])[0]) == list(range(10))      # K = N-1
+    assert list(oracle.topk_chunks(s, [10], [50])[0]) == list(range(10))     # K > N-1
+    assert list(oracle.topk_chunks(s, [1], [4])[0]) == [0]                   # only the latest
+    assert list(oracle.topk_chunks(s, [0], [4])[0]) == []                    # empty sequence
+    assert list(oracle.topk_chunks(s, [10], [0])[0]) == [9]                  # K = 0
+
+
+def test_topk_latest_not_double_counted():
+    """The latest chunk has the highest score: it is kept once, plus K others."""
+    s = np.arange(12, dtype=np.float64)[None, :]          # latest (11) scores highest
+    got = oracle.topk_chunks(s, [12], [3])[0]
+    assert list(got) == [8, 9, 10, 11]
+    s2 = -np.arange(12, dtype=np.float64)[None, :]        # latest scores lowest
+    assert list(oracle.topk_chunks(s2, [12], [3])[0]) == [0, 1, 2, 11]
+
+
+def test_threshold_rule():
+    w = np.array([0.5, 1.5] + [0.0] * 14)
+    s = np.array([[0.2, 1.2, 1.0, 1.01, 0.0]]) * 1.0     # score / sum(w) = s / 2
+    got = oracle.threshold_chunks(s, [5], w)[0]
+    assert list(got) == [1, 3, 4]                           # 0.6 and 0.505 pass; latest kept
+
+
+# ------------------------------------------------------------------ gather ---
+
+def test_gather_closed_form_positions():
+    """Pools filled with their own flat index: the gathered element at
+    (i = cu[b] + j, h, t, d) must equal the flat index of (table[b, kept_j], h, t, d)."""
+    S, B, M = 11, 2, 5
+    shape = (S, 8, 64, 128)
+    k_pool = np.arange(np.prod(shape), dtype=np.int64).reshape(shape)
+    v_pool = -k_pool
+    table = RNG.permutation(S)[: B * M].reshape(B, M)
+    kept = [np.array([0, 3, 4]), np.array([1, 4])]
+    k_buf, v_buf, cu = oracle.gather_chunks(k_pool, v_pool, table, kept)
+    assert list(cu) == [0, 3, 5]
+    h, t, d = np.meshgrid(np.arange(8), np.arange(64), np.arange(128), indexing="ij")
+    for b in range(B):
+        for j, c in enumerate(kept[b]):
+            flat = ((table[b, c] * 8 + h) * 64 + t) * 128 + d
+            assert np.array_equal(k_buf[cu[b] + j], flat)
+            assert np.array_equal(v_buf[cu[b] + j], -flat)
+
+
+# --------------------------------------------------------------- attention ---
+
+def _rand_bufs(n_chunks, rng):
+    k = bf16_round(rng.standard_normal((n_chunks, 8, 64, 128)))
+    v = bf16_round(rng.standard_normal((n_chunks, 8, 64, 128)))
+    return k, v
+
+
+def test_attention_all_chunks_equals_dense_sdpa():
+    """With every chunk kept, the result is dense GQA attention: torch's fp64
+    scaled_dot_product_attention with K/V repeated 8x per KV head."""
+    rng = np.random.default_rng(7)
+    B, n = 2, [3, 2]
+    cu = np.array([0, 3, 5])
+    k_buf, v_buf = _rand_bufs(5, rng)
+    q = bf16_round(rng.standard_normal((B, 64, 128)))
+    got = oracle.sparse_decode_attn(q, k_buf, v_buf, cu)
+    for b in range(B):
+        K = torch.from_numpy(k_buf[cu[b]:cu[b + 1]]).permute(1, 0, 2, 3).reshape(8, -1, 128)
+        V = torch.from_numpy(v_buf[cu[b]:cu[b + 1]]).permute(1, 0, 2, 3).reshape(8, -1, 128)
+        K = K.repeat_interleave(8, dim=0)
+        V = V.repeat_interleave(8, dim=0)
+        Q = torch.from_numpy(q[b]).reshape(64, 1, 128)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V).reshape(64, 128).numpy()
+        np.testing.assert_allclose(got[b], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_attention_identical_keys_give_mean_of_v():
+    rng = np.random.default_rng(8)
+    k_buf, v_buf = _rand_bufs(3, rng)
+    k_buf[:] = k_buf[0, 0, 0]               # every key equal
+    q = bf16_round(rng.standard_normal((1, 64, 128)))
+    got = oracle.sparse_decode_attn(q, k_buf, v_buf, [0, 3])
+    for h in range(64):
+        g = h // 8
+        np.testing.assert_allclose(got[0, h], v_buf[:, g].reshape(-1, 128).mean(axis=0), rtol=1e-12, atol=1e-14)
+
+
+def test_attention_single_chunk_closed_form():
+    """q = e_0, k_j = (s_j, 0, ...), v_j = e_j (j < 64): o_h[j] = softmax_j(s_j / sqrt(128))."""
+    s_int = (np.arange(64) % 7) - 3.0
+    k = np.zeros((1, 8, 64, 128))
+    k[0, :, :, 0] = s_int
+    v = np.zeros((1, 8, 64, 128))
+    for j in range(64):
+        v[0, :, j, j] = 1.0
+    q = np.zeros((1, 64, 128))
+    q[0, :, 0] = 1.0
+    got = oracle.sparse_decode_attn(q, k, v, [0, 1])
+    e = np.array([math.exp(x / math.sqrt(128)) for x in s_int])
+    expect = np.zeros(128)
+    expect[:64] = e / e.sum()
+    for h in range(64):
+        np.testing.assert_allclose(got[0, h], expect, rtol=1e-13, atol=1e-16)
+
+
+def test_attention_gqa_head_mapping():
+    """V of KV head g is the constant g+1: every query head h must return h // 8 + 1."""
+    rng = np.random.default_rng(9)
+    k_buf, v_buf = _rand_bufs(2, rng)
+    for g in range(8):
+        v_buf[:, g] = g + 1.0
+    q = bf16_round(rng.standard_normal((1, 64, 128)))
+    got = oracle.sparse_decode_attn(q, k_buf, v_buf, [0, 2])
+    for h in range(64):
+        np.testing.assert_allclose(got[0, h], np.full(128, h // 8 + 1.0), rtol=1e-13)
+
+
+def test_attention_scale_pin_two_tokens():
+    """Two tokens with logits 0 and 1 after scaling: weights 1/(1+e) and e/(1+e)."""
+    k = np.zeros((1, 8, 64, 128))
+    v = np.zeros((1, 8, 64, 128))
+    # token 0: k = 0, v = (1, 0, ..); token 1: k = sqrt(128) e_0, v = (0, 1, ..);
+    # tokens 2..63 get a very negative logit (k = -sqrt(128)*40 e_0) and v = 0.
+    k[0, :, 1, 0] = math.sqrt(128)
+    k[0, :, 2:, 0] = -math.sqrt(128) * 40
+    v[0, :, 0, 0] = 1.0
+    v[0, :, 1, 1] = 1.0
+    q = np.zeros((1, 64, 128))
+    q[0, :, 0] = 1.0
+    got = oracle.sparse_decode_attn(q, k, v, [0, 1])
+    np.testing.assert_allclose(got[0, 5, 0], 1 / (1 + math.e), rtol=1e-13)
+    np.testing.assert_allclose(got[0, 5, 1], math.e / (1 + math.e), rtol=1e-13)
+
+
+def test_attention_large_logits_stay_finite():
+    """Logits 1000 and 1001 (scaled): the softmax is shift-invariant, so the weights are
+    still 1/(1+e) and e/(1+e); an implementation without the max shift overflows."""
+    k = np.zeros((1, 8, 64, 128))
+    v = np.zeros((1, 8, 64, 128))
+    k[0, :, 0, 0] = 1000 * math.sqrt(128)
+    k[0, :, 1, 0] = 1001 * math.sqrt(128)
+    k[0, :, 2:, 0] = -1000 * math.sqrt(128)
+    v[0, :, 0, 0] = 1.0
+    v[0, :, 1, 1] = 1.0
+    q = np.zeros((1, 64, 128))
+    q[0, :, 0] = 1.0
+    got = oracle.sparse_decode_attn(q, k, v, [0, 1])
+    np.testing.assert_allclose(got[0, 63, :2], [1 / (1 + math.e), math.e / (1 + math.e)], rtol=1e-12)
+
+
+def test_attention_chunk_permutation_invariance():
+    rng = np.random.default_rng(10)
+    k_buf, v_buf = _rand_bufs(4, rng)
+    q = bf16_round(rng.standard_normal((1, 64, 128)))
+    a = oracle.sparse_decode_attn(q, k_buf, v_buf, [0, 4])
+    p = [2, 0, 3, 1]
+    b = oracle.sparse_decode_attn(q, k_buf[p], v_buf[p], [0, 4])
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-15)
+
+
+def test_attention_empty_sequence_is_zero():
+    rng = np.random.default_rng(11)
+    k_buf, v_buf = _rand_bufs(2, rng)
+    q = bf16_round(rng.standard_normal((3, 64, 128)))
+    got = oracle.sparse_decode_attn(q, k_buf, v_buf, [0, 2, 2, 2])
+    assert np.all(got[1] == 0) and np.all(got[2] == 0)
+    assert np.all(np.isfinite(got[0]))
+
+
+def test_bf16_bits_widening():
+    x = torch.tensor([1.0, -2.5, 3.140625, 0.0, -0.0, 65280.0]).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy()
+    np.testing.assert_array_equal(oracle.bf16_bits_to_f64(bits), x.to(torch.float64).numpy())
+
+
+def test_decode_window_composition():
+    """A whole window equals its stages run one after another (tiny sizes)."""
+    rng = np.random.default_rng(12)
+    N, K = 10, 3
+    keys = bf16_round(rng.standard_normal((N, 128)))
+    kp, vp = _rand_bufs(N, rng)
+    q_idx = bf16_round(rng.standard_normal((1, 16, 128)))
+    w = rng.uniform(0, 1, 16)
+    qs = bf16_round(rng.standard_normal((2, 1, 64, 128)))
+    scores, kept, cu, outs = oracle.decode_window(q_idx, w, keys, None, [N], [K], kp, vp, qs, max_chunks=N)
+    assert len(kept[0]) == K + 1 and kept[0][-1] == N - 1
+    ref = oracle.sparse_decode_attn(qs[1], kp[kept[0]], vp[kept[0]], [0, K + 1])
+    np.testing.assert_array_equal(outs[1], ref)
