@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Benchmark of the LSA decode hot path on B200: one JSON line on stdout.
+
+A *step* is one lookahead window of one layer (of every layer for the batched
+workload): indexer scoring of every chunk, top-K plus latest chunk, gather of
+the kept chunks into the compact buffer (a host-tier fetch for ``1m_host``),
+then 64 decode steps of split-K GQA attention over the kept chunks.  All
+inputs (KV pools, indexer keys, queries of every window) are resident on the
+device before timing starts; the window's selection and its 64 attention
+launches are replayed from two captured CUDA graphs per window index.
+
+Metric: decode tokens per second per layer (64 * B tokens per window and
+layer), with the achieved HBM bandwidth of the whole window and of the
+attention kernel against the measured copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 500k]
+    python bench.py --impl reference ...   # the fp64 oracle on the host cores
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload on its own GPU (the path shards by sequence and needs no
+collective); the timing is the max over ranks and ``value`` sums the tokens of
+all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "LSA decode tok/s/layer at 128K-1M ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "tok/s/layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "500k"
+ATTN_KERNEL = "sparse_decode_attn_kernel"
+
+
+# ----------------------------------------------------------------- helpers --
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    """Digest of the attention kernel's sources (ties ncu traffic to a build)."""
+    h = hashlib.sha256()
+    for name in ("lsa_attn.cu", "lsa_common.cuh"):
+        with open(os.path.join(ROOT, "kv_chunk_selection_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"sparse_decode_attn_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != source_digest():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def copy_probe_gbs(device, nbytes=1 << 31, reps=10):
+    """Streaming copy (read + write bytes) in the same run: torch copy_ of 1 Gi bf16."""
+    a = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=device)
+    b = torch.empty_like(a)
+    a.fill_(1.0)
+    best = float("inf")
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        b.copy_(a)
+        e.record()
+        e.synchronize()
+        best = min(best, s.elapsed_time(e) / 1e3)
+    del a, b
+    return 2 * (nbytes // 2) * 2 / best / 1e9
+
+
+def window_bytes(n_chunks, kept_total, layers):
+    """Algorithmic bytes of one window: indexer keys of every chunk once, and per
+    decode step the kept K/V, the query and the fp32 output (gather excluded).
+    ``kept_total`` is the number of kept chunks the selection produced."""
+    n = n_chunks.to(torch.int64).cpu()
+    B = int(n.numel())
+    keys = 256 * int(n.sum()) + B * 16 * 128 * 2 + 16 * 4
+    attn_launch = int(kept_total) * 2 * workloads.CHUNK_BYTES_ONE + B * (64 * 128 * 2 + 64 * 128 * 4)
+    per_layer = keys + workloads.TAU * attn_launch
+    return per_layer * layers, attn_launch, int(n.sum())
+
+
+# -------------------------------------------------------------- our arm ------
+
+def run_ours(args, rank, world, local_rank):
+    import kv_chunk_selection_b200 as lsa
+    from kv_chunk_selection_b200.window import LayerWindow
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lsa.lib()
+    wl = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(args.workload, dev, base_seed=workloads.BASE_SEED + rank)
+    B, layers, n_win = inp.batch, len(inp.layers), inp.workload.windows
+    host_tier = inp.workload.host_pool
+    lws = [LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev) for _ in range(layers)]
+    outs = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def select_phase(w):
+        for l, L in enumerate(inp.layers):
+            lws[l].select(L.q_idx[w], L.w, L.chunk_keys)
+            if host_tier:
+                lws[l].fetch(L.k_pool, L.v_pool, num_ctas=args.fetch_ctas)
+            else:
+                lws[l].gather(L.k_pool, L.v_pool)
+
+    def attn_phase(w):
+        for t in range(workloads.TAU):
+            for l, L in enumerate(inp.layers):
+                lws[l].attend(L.q[w, t], outs[l][t])
+
+    # warm every path once, then capture one pair of graphs per window index
+    with torch.cuda.stream(stream):
+        select_phase(0)
+        attn_phase(0)
+    torch.cuda.synchronize()
+    bits = lsa.read_device_status()
+    if bits:
+        raise RuntimeError(f"device status after warm-up: {lsa.decode_status(bits)}")
+    graphs = []
+    if args.graphs:
+        for w in range(n_win):
+            gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs, stream=stream):
+                select_phase(w)
+            with torch.cuda.graph(ga, stream=stream):
+                attn_phase(w)
+            graphs.append((gs, ga))
+    torch.cuda.synchronize()
+
+    def step(i, evs=None):
+        w = i % n_win
+        if evs is not None:
+            evs[0].record(stream)
+        if graphs:
+            graphs[w][0].replay()
+        else:
+            select_phase(w)
+        if evs is not None:
+            evs[1].record(stream)
+        if graphs:
+            graphs[w][1].replay()
+        else:
+            attn_phase(w)
+        if evs is not None:
+            evs[2].record(stream)
+
+    copy_gbs = copy_probe_gbs(dev)
+    peak, peak_kind = measured_peaks()
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    elapsed = t0.elapsed_time(t1) / 1e3
+    sel_s = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    att_s = sum(e[1].elapsed_time(e[2]) for e in evs) / 1e3
+    bits = lsa.read_device_status()
+    if bits:
+        raise RuntimeError(f"device status after timing: {lsa.decode_status(bits)}")
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    # tok/s/layer: every window decodes 64 tokens per sequence in each layer; a
+    # window of `layers` layers takes `elapsed / steps`, i.e. 1/layers of it per layer.
+    value = world * workloads.TAU * B * layers * args.steps / elapsed
+    kept_total = int(lws[0].cu_kept[0][-1].item())
+    wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers)
+    hbm_gbs = wbytes * args.steps / elapsed / 1e9
+    n_attn = workloads.TAU * layers * args.steps
+    attn_avg = att_s / n_attn
+    attn_gbs = attn_bytes / attn_avg / 1e9
+    traffic = profiled_traffic(args.workload)
+
+    # ---- end to end through the public API, inputs from pinned host memory ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, inp, lws, dev, stream)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": inp.workload.description, "name": args.workload, "batch": B, "layers": layers,
+            "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
+            "tau": workloads.TAU, "gqa": "64q/8kv/d128", "indexer": "16 heads x 128",
+            "kv_dtype": "bf16", "softmax_accumulate": "fp32",
+            "l2": ("inputs larger than L2: each attention launch streams "
+                   f"{attn_bytes / 2**20:.1f} MiB of kept KV (L2 is 126 MB)" if attn_bytes > 126e6 else
+                   f"compact buffer {attn_bytes / 2**20:.1f} MiB is smaller than L2 and re-read by the 64 steps"),
+            "cuda_graphs": bool(args.graphs), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "roofline": {
+            "kernel": ATTN_KERNEL, "bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+            "frac": attn_gbs / peak, "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
+            "algorithmic_bytes_per_launch": attn_bytes, "avg_launch_us": attn_avg * 1e6,
+        },
+        "hbm": {"window_gbs": hbm_gbs, "frac_of_measured": hbm_gbs / peak,
+                "frac_of_nominal_8tbs": hbm_gbs / NOMINAL_HBM_GBS, "copy_probe_gbs": copy_gbs,
+                "frac_of_copy_probe": hbm_gbs / copy_gbs, "algorithmic_bytes_per_step": wbytes},
+        "indexer_chunks_per_s": world * total_chunks * layers * args.steps / sel_s if sel_s > 0 else None,
+        "stage_us": {"select_and_gather_per_window": sel_s / args.steps * 1e6,
+                     "attention_per_decode_step": attn_avg * 1e6,
+                     "attention_64_steps": att_s / args.steps * 1e6},
+        "gpu_launches": args.steps * layers * (3 + workloads.TAU),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    return out
+
+
+def run_e2e(args, inp, lws, dev, stream):
+    """Same metric through the public API: every window copies its queries in from
+    pinned host memory and its 64 outputs back to pinned host memory."""
+    B, layers = inp.batch, len(inp.layers)
+    n_win = inp.workload.windows
+    host_q_idx = [[L.q_idx[w].cpu().pin_memory() for w in range(n_win)] for L in inp.layers]
+    host_q = [[L.q[w].cpu().pin_memory() for w in range(n_win)] for L in inp.layers]
+    dq_idx = [torch.empty_like(inp.layers[l].q_idx[0]) for l in range(layers)]
+    dq = [torch.empty_like(inp.layers[l].q[0]) for l in range(layers)]
+    douts = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
+    hout = [torch.empty((workloads.TAU, B, 64, 128)).pin_memory() for _ in range(layers)]
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def one(i):
+        w = i % n_win
+        for l, L in enumerate(inp.layers):
+            dq_idx[l].copy_(host_q_idx[l][w], non_blocking=True)
+            dq[l].copy_(host_q[l][w], non_blocking=True)
+        for l, L in enumerate(inp.layers):
+            lws[l].select(dq_idx[l], L.w, L.chunk_keys)
+            if inp.workload.host_pool:
+                lws[l].fetch(L.k_pool, L.v_pool, num_ctas=args.fetch_ctas)
+            else:
+                lws[l].gather(L.k_pool, L.v_pool)
+        for t in range(workloads.TAU):
+            for l in range(layers):
+                lws[l].attend(dq[l][t], douts[l][t])
+        for l in range(layers):
+            hout[l].copy_(douts[l], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            one(i)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record(stream)
+        for i in range(steps):
+            one(i)
+        e.record(stream)
+    torch.cuda.synchronize()
+    el = s.elapsed_time(e) / 1e3
+    h2d = layers * (B * 16 * 128 * 2 + workloads.TAU * B * 64 * 128 * 2)
+    d2h = layers * workloads.TAU * B * 64 * 128 * 4
+    return {"value": workloads.TAU * B * layers * steps / el, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "api": "kv_chunk_selection_b200.window.LayerWindow"}
+
+
+# ---------------------------------------------------------- oracle (CPU) arm --
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warmup=0):
+    """Times the fp64 oracle on a bounded sample of the workload.
+
+    The sample is one full selection of window 0 of layer 0 (scoring of every
+    chunk, top-K, gather of the kept chunks) plus decode-attention steps of that
+    window, each over one KV head group (8 query heads), rotating over groups
+    and steps until ``budget_s`` seconds (or ``group_steps`` steps) are spent.
+    Throughput is extrapolated to whole windows: 64 * B tokens per
+    (selection + 64 steps x 8 groups).
+    """
+    import numpy as np
+
+    import oracle
+    dev = "cuda" if (on_gpu_inputs and torch.cuda.is_available()) else "cpu"
+    inp = workloads.make_inputs(workload, dev, layers=1, windows=1)
+    L = inp.layers[0]
+    B = inp.batch
+    q_idx = L.q_idx[0].float().cpu().numpy()
+    w = L.w.cpu().double().numpy()
+    keys = L.chunk_keys.float().cpu().numpy()
+    table = inp.chunk_table.cpu().numpy()
+    n = inp.n_chunks.cpu().numpy()
+    k = inp.k_per_seq.cpu().numpy()
+    kpool = L.k_pool.view(torch.int16).cpu().numpy()
+    vpool = L.v_pool.view(torch.int16).cpu().numpy()
+    qs = L.q[0].float().cpu().numpy()
+    del inp, L
+    t0 = time.perf_counter()
+    scores = oracle.index_scores(q_idx, w, keys, table, n, int(table.shape[1]))
+    kept = oracle.topk_chunks(scores, n, k)
+    kb_bits, vb_bits, cu = oracle.gather_chunks(kpool, vpool, table, kept, int(table.shape[1]))
+    kb = oracle.bf16_bits_to_f64(kb_bits)
+    vb = oracle.bf16_bits_to_f64(vb_bits)
+    t_sel = time.perf_counter() - t0
+    del kpool, vpool
+    times = []
+    i = 0
+    start = time.perf_counter()
+    while True:
+        g = i % 8
+        t = (i * 7) % workloads.TAU
+        heads = list(range(8 * g, 8 * g + 8))
+        a = time.perf_counter()
+        oracle.sparse_decode_attn(qs[t], kb, vb, cu, heads=heads)
+        if i >= warmup:
+            times.append(time.perf_counter() - a)
+        i += 1
+        if group_steps is not None and len(times) >= group_steps:
+            break
+        if group_steps is None and time.perf_counter() - start > budget_s and len(times) >= 1:
+            break
+    t_group = float(np.mean(times))
+    window_s = t_sel + workloads.TAU * 8 * t_group
+    value = workloads.TAU * B / window_s
+    sample = (f"{workload}: one selection of window 0 (score {int(n.sum())} chunks, top-K, gather "
+              f"{int(cu[-1])} chunks) timed once ({t_sel:.2f} s) + {len(times)} decode-attention steps over one "
+              f"KV-head group (8 query heads) each ({t_group * 1e3:.1f} ms mean); extrapolated to a window of "
+              f"64 steps x 8 groups")
+    return {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", "sample": sample,
+            "window_s_extrapolated": window_s, "host_cpus": os.cpu_count()}, times, t_sel
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    t_start = time.perf_counter()
+    base, times, t_sel = oracle_sample(args.workload, budget_s=1e9, group_steps=args.steps + args.warmup,
+                                       warmup=0)
+    times = times[args.warmup:]
+    import numpy as np
+    t_group = float(np.mean(times))
+    inp_b = workloads.WORKLOADS[args.workload].batch
+    window_s = t_sel + workloads.TAU * 8 * t_group
+    value = workloads.TAU * inp_b / window_s
+    base["value"] = value
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_group * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workloads.WORKLOADS[args.workload].description, "name": args.workload,
+                   "step": "one decode-attention step over one KV-head group, selection timed once and "
+                           "amortised over the 64-step window"},
+        "cpu_baseline": base, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t_start,
+    }
+
+
+# --------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-graphs", dest="graphs", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--fetch-ctas", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    # The oracle sample runs before any CUDA work of this process (rank 0, N = 1 only).
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu, _, _ = oracle_sample(args.workload, args.cpu_budget_s, on_gpu_inputs=True)
+        torch.cuda.empty_cache()
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+    out["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

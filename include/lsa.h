@@ -1,0 +1,212 @@
+/*
+ * lsa.h -- C ABI of liblsa, the B200 (sm_100a) decode hot path of Lookahead
+ * Sparse Attention (LSA).
+ *
+ * The method (pages on "FlashMemory-DeepSeek-V4: Lightning Index Ultra-Long
+ * Context via Lookahead Sparse Attention"): every tau = 64 decode steps a neural
+ * memory indexer scores each 64-token chunk of the context (summary page,
+ * sections 1 Introduction and 2.1 Architecture); only the chunks the coming
+ * window needs are kept on the GPU (summary page, Abstract and 2.1), fetched
+ * from a CPU tier when the cache lives there (summary page, 3 Experiments,
+ * "Experimental Setup"; handbook page "DeepSeek-V4: Architecting for Ultra-Long
+ * Contexts", "The Neural Memory Indexer", item 3); decode attention then runs
+ * over the kept chunks only, as GQA with 64 query heads, 8 KV heads and head
+ * dimension 128 (handbook page, "Grouped Query Attention (GQA) vs. Multi-Head
+ * Attention (MHA)").
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Pointers marked "device" are CUDA device (or managed) memory of the
+ *    current device; "host" pointers are CPU memory.  The caller owns every
+ *    buffer, stream and event.  The library allocates no device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every compute call only enqueues work on `stream` and returns.
+ *  - Return value: LSA_OK (0) or a negative lsa_status.  Argument checks are
+ *    done on the host, before anything is launched; a failed check launches
+ *    nothing.  LSA_ERR_CUDA reports a launch error (cudaGetLastError).
+ *  - Conditions only the device can see (a count or slot index out of range, a
+ *    compact buffer too small, a bounded wait that ran out) set bits of a
+ *    device status word (LSA_DEV_ERR_*) instead of trapping; the offending
+ *    work item is skipped.  lsa_read_device_status() returns and clears it.
+ *  - Shapes are fixed: 64 query heads, 8 KV heads, head dim 128, 64-token
+ *    chunks, 16 indexer heads of dim 128.  bf16 is IEEE-style bfloat16 stored
+ *    as 2 bytes; all bf16 arrays must be 16-byte aligned.
+ *  - Layouts (row-major, last index fastest):
+ *      KV pool / compact buffer : bf16 [slot][8 kv heads][64 tokens][128]
+ *                                 (LSA_CHUNK_BYTES bytes per slot, per K or V)
+ *      indexer keys             : bf16 [slot][128]
+ *      indexer query            : bf16 [B][16][128]
+ *      decode query             : bf16 [B][64][128]
+ *      attention output         : fp32 [B][64][128]
+ *      chunk table              : int32 [B][max_chunks], logical chunk -> slot;
+ *                                 NULL means slot = b * max_chunks + c.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LSA_NUM_Q_HEADS 64
+#define LSA_NUM_KV_HEADS 8
+#define LSA_HEAD_DIM 128
+#define LSA_CHUNK_TOKENS 64
+#define LSA_INDEX_HEADS 16
+#define LSA_INDEX_DIM 128
+/* Bytes of one chunk of K (or of V): 8 heads x 64 tokens x 128 dims x 2 B. */
+#define LSA_CHUNK_BYTES 131072
+/* Largest batch the attention and top-K calls accept. */
+#define LSA_MAX_BATCH 4096
+
+typedef enum {
+  LSA_OK = 0,
+  LSA_ERR_INVALID_ARG = -1,       /* null pointer, negative size, bad value   */
+  LSA_ERR_UNSUPPORTED_SHAPE = -2, /* size beyond what a kernel supports       */
+  LSA_ERR_WORKSPACE = -3,         /* workspace missing or too small           */
+  LSA_ERR_CUDA = -4,              /* CUDA runtime/launch error                */
+  LSA_ERR_NOT_PINNED = -5,        /* host pool is not page-locked memory      */
+  LSA_ERR_MISALIGNED = -6,        /* pointer not 16-byte aligned              */
+  LSA_ERR_NO_DEVICE = -7          /* no usable sm_100 device                  */
+} lsa_status;
+
+/* Bits of the device status word. */
+#define LSA_DEV_ERR_BAD_COUNT 1u   /* n_chunks / k_per_seq / cu_kept out of range */
+#define LSA_DEV_ERR_BAD_SLOT 2u    /* chunk table entry outside [0, n_slots)     */
+#define LSA_DEV_ERR_BAD_CHUNK 4u   /* kept chunk index outside [0, max_chunks)   */
+#define LSA_DEV_ERR_CAPACITY 8u    /* compact buffer or kept row too small        */
+#define LSA_DEV_ERR_TIMEOUT 16u    /* a bounded in-kernel wait ran out            */
+#define LSA_DEV_ERR_WORKSPACE 32u  /* attention workspace not zero-initialised    */
+
+/* Human-readable name of an lsa_status value. */
+const char* lsa_status_string(int status);
+
+/* ABI version of this library (major * 100 + minor). */
+int lsa_version(void);
+
+/*
+ * Synchronises `stream`, stores the device status word of the current device
+ * in *bits (0 = no device-side error since the last read) and clears it.
+ */
+int lsa_read_device_status(void* stream, unsigned int* bits);
+
+/*
+ * lsa_index_score -- indexer scores of every chunk (the Neural Memory Indexer
+ * of the summary page, 2.1 Architecture; sigmoid scoring per the review page,
+ * "1. Key Terms & Definitions"):
+ *
+ *   scores[b*max_chunks + c] = sum_h w[h] * sigmoid(q_idx[b,h,:] . keys[slot(b,c),:] / sqrt(128))
+ *
+ * for c < n_chunks[b]; entries c >= n_chunks[b] are left untouched.
+ *   q_idx      device bf16 [B][16][128]
+ *   w          device fp32 [16]
+ *   chunk_keys device bf16 [n_slots][128]
+ *   chunk_table device int32 [B][max_chunks] or NULL (identity layout)
+ *   n_chunks   device int32 [B], each in [0, max_chunks]
+ *   scores     device fp32 [B][max_chunks]
+ * Device errors: BAD_COUNT (n_chunks out of range: the sequence is skipped),
+ * BAD_SLOT (that chunk's score is not written).
+ */
+int lsa_index_score(const void* q_idx, const float* w, const void* chunk_keys, int64_t n_slots,
+                    const int32_t* chunk_table, const int32_t* n_chunks, int B, int max_chunks,
+                    float* scores, void* stream);
+
+/*
+ * lsa_topk_chunks -- per-sequence selection: among chunks 0 .. n-2 keep the
+ * K = k_per_seq[b] best by (score descending, chunk index ascending), then add
+ * the latest chunk n-1.  kept[b*max_kept + j], j < n_kept[b], lists the kept
+ * chunk indices in ascending order (the latest is last);
+ * n_kept[b] = min(K, n-1) + 1 (0 when n == 0); cu_kept[0] = 0 and
+ * cu_kept[b+1] = cu_kept[b] + n_kept[b] (offsets into the compact buffer, in
+ * chunks).  Fixed-budget form of the recall step of the summary page, 2.1
+ * Architecture.
+ *   scores    device fp32 [B][max_chunks] (from lsa_index_score)
+ *   n_chunks, k_per_seq  device int32 [B]
+ *   kept      device int32 [B][max_kept]; n_kept device int32 [B];
+ *   cu_kept   device int32 [B+1]
+ * B <= LSA_MAX_BATCH.  Device errors: BAD_COUNT (negative K, n out of range:
+ * the sequence keeps nothing), CAPACITY (n_kept would exceed max_kept: the
+ * sequence keeps nothing).
+ */
+int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq,
+                    int B, int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept,
+                    int32_t* cu_kept, void* stream);
+
+/*
+ * lsa_gather_chunks -- copy every kept chunk from the device KV pools into the
+ * compact buffers, bit for bit: for i = cu_kept[b] + j,
+ *   k_buf[i] = k_pool[slot(b, kept[b*max_kept + j])], same for V.
+ *   k_pool, v_pool device bf16 [n_slots][8][64][128]
+ *   k_buf,  v_buf  device bf16 [buf_chunks][8][64][128]
+ * Device errors: CAPACITY (cu_kept[B] > buf_chunks: nothing is copied),
+ * BAD_CHUNK / BAD_SLOT (that chunk is not copied).
+ */
+int lsa_gather_chunks(const void* k_pool, const void* v_pool, int64_t n_slots,
+                      const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept,
+                      int B, int max_chunks, int max_kept, void* k_buf, void* v_buf,
+                      int64_t buf_chunks, void* stream);
+
+/*
+ * lsa_fetch_from_host -- the same copy as lsa_gather_chunks, but the pools
+ * live in page-locked host memory (the CPU cold tier of the summary page,
+ * 3 Experiments; prefetch over the host link, handbook page, "The Neural
+ * Memory Indexer").  SM threads read the mapped host pages directly (no
+ * host-side loop, no copy of `kept` to the host), so the call is fully
+ * asynchronous and can run on a side stream while attention runs on another.
+ *   host_k_pool, host_v_pool  page-locked host bf16 [n_slots][8][64][128]
+ *                             (cudaHostAlloc / cudaHostRegister); anything
+ *                             else returns LSA_ERR_NOT_PINNED.
+ *   num_ctas   thread blocks used for the copy (<= 0: library default), kept
+ *              small so the fetch leaves SMs to concurrent kernels.
+ *   done_event optional cudaEvent_t (void*) recorded on `stream` after the copy.
+ * Other arguments and device errors as lsa_gather_chunks.
+ */
+int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                        const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept,
+                        int B, int max_chunks, int max_kept, void* k_buf, void* v_buf,
+                        int64_t buf_chunks, int num_ctas, void* stream, void* done_event);
+
+/*
+ * Bytes of workspace lsa_sparse_decode_attn needs for a batch of B sequences.
+ * The workspace must be zero-filled once before its first use; every call
+ * leaves it ready for the next one.
+ */
+size_t lsa_attn_workspace_size(int B);
+
+/*
+ * lsa_sparse_decode_attn -- one decode step of GQA attention over the kept
+ * chunks (handbook page, "Grouped Query Attention (GQA) vs. Multi-Head
+ * Attention (MHA)": softmax(q K^T / sqrt(d_k)) V, every 8 consecutive query
+ * heads sharing one KV head).  For sequence b, query head h and KV head
+ * g = h / 8, the keys and values are the 64 * (cu_kept[b+1] - cu_kept[b])
+ * tokens of head g in k_buf / v_buf chunks cu_kept[b] .. cu_kept[b+1]-1:
+ *
+ *   out[b,h,:] = sum_j softmax_j(scale * q[b,h,:] . k_j) v_j    (fp32)
+ *
+ * A sequence with no kept chunk gets zeros.  The work is split over all SMs
+ * along the kept tokens (split-K flash decoding) and the partial results are
+ * merged with their log-sum-exp weights in a fixed order, so repeated calls
+ * are bit-identical.
+ *   q            device bf16 [B][64][128]
+ *   k_buf, v_buf device bf16 [buf_chunks][8][64][128]
+ *   cu_kept      device int32 [B+1]
+ *   softmax_scale  usually 1/sqrt(128)
+ *   out          device fp32 [B][64][128]
+ *   workspace    device, >= lsa_attn_workspace_size(B) bytes, zero-filled
+ *                before first use.
+ * B <= LSA_MAX_BATCH.  Device errors: CAPACITY (cu_kept[B] > buf_chunks or
+ * cu_kept decreasing: nothing is computed), TIMEOUT, WORKSPACE.
+ */
+int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
+                           int64_t buf_chunks, const int32_t* cu_kept, int B,
+                           float softmax_scale, float* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

@@ -1,0 +1,225 @@
+"""Python binding of liblsa, the B200 decode hot path of Lookahead Sparse Attention.
+
+Argument marshalling only: every function below checks dtypes, devices and
+contiguity of torch tensors, passes raw pointers and sizes to the C ABI of the
+same name (``include/lsa.h``) on the current torch CUDA stream, and raises
+:class:`LsaError` on a non-zero status.  All computation happens in the CUDA
+kernels of ``liblsa.so``; there is no fallback.  If the library has not been
+built, importing works but the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "liblsa.so")
+
+NUM_Q_HEADS = 64
+NUM_KV_HEADS = 8
+HEAD_DIM = 128
+CHUNK_TOKENS = 64
+INDEX_HEADS = 16
+INDEX_DIM = 128
+CHUNK_BYTES = NUM_KV_HEADS * CHUNK_TOKENS * HEAD_DIM * 2
+
+DEV_ERR_BITS = {1: "BAD_COUNT", 2: "BAD_SLOT", 4: "BAD_CHUNK", 8: "CAPACITY", 16: "TIMEOUT", 32: "WORKSPACE"}
+
+_lib = None
+
+
+class LsaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = _load().lsa_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{fn} failed: {name} ({status})")
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"liblsa.so not found at {LIB_PATH}; build it with `python -m kv_chunk_selection_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "lsa_status_string": ([I], ctypes.c_char_p),
+        "lsa_version": ([], I),
+        "lsa_read_device_status": ([P, ctypes.POINTER(ctypes.c_uint)], I),
+        "lsa_index_score": ([P, P, P, I64, P, P, I, I, P, P], I),
+        "lsa_topk_chunks": ([P, P, P, I, I, I, P, P, P, P], I),
+        "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
+        "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
+        "lsa_attn_workspace_size": ([I], S),
+        "lsa_sparse_decode_attn": ([P, P, P, I64, P, I, F, P, P, S, P], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def lib():
+    """The loaded ctypes library (raw C ABI)."""
+    return _load()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype, cuda=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise LsaError(fn, st)
+
+
+def read_device_status(stream=None) -> int:
+    """Synchronises the stream, returns and clears the device status bits."""
+    bits = ctypes.c_uint(0)
+    _check("lsa_read_device_status", _load().lsa_read_device_status(_stream(stream), ctypes.byref(bits)))
+    return bits.value
+
+
+def decode_status(bits: int) -> list:
+    return [n for b, n in DEV_ERR_BITS.items() if bits & b]
+
+
+def lsa_index_score(q_idx, w, chunk_keys, chunk_table, n_chunks, scores, stream=None):
+    """scores[b, c] = sum_h w[h] sigmoid(q_idx[b,h].k[slot(b,c)] / sqrt(128)) for c < n_chunks[b]."""
+    _need(q_idx, "q_idx", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(chunk_keys, "chunk_keys", torch.bfloat16)
+    _need(n_chunks, "n_chunks", torch.int32)
+    _need(scores, "scores", torch.float32)
+    if chunk_table is not None:
+        _need(chunk_table, "chunk_table", torch.int32)
+    B = q_idx.shape[0]
+    if tuple(q_idx.shape) != (B, INDEX_HEADS, INDEX_DIM) or scores.dim() != 2 or scores.shape[0] != B:
+        raise ValueError("bad shapes")
+    max_chunks = scores.shape[1]
+    if chunk_table is not None and tuple(chunk_table.shape) != (B, max_chunks):
+        raise ValueError("chunk_table must be [B, max_chunks]")
+    n_slots = chunk_keys.shape[0]
+    _check("lsa_index_score", _load().lsa_index_score(
+        _ptr(q_idx), _ptr(w), _ptr(chunk_keys), n_slots, _ptr(chunk_table), _ptr(n_chunks), B, max_chunks,
+        _ptr(scores), _stream(stream)))
+
+
+def lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu_kept, stream=None):
+    """Top-K chunks per sequence (score desc, index asc) plus the latest, ascending."""
+    for t, n in ((scores, "scores"),):
+        _need(t, n, torch.float32)
+    for t, n in ((n_chunks, "n_chunks"), (k_per_seq, "k_per_seq"), (kept, "kept"), (n_kept, "n_kept"),
+                 (cu_kept, "cu_kept")):
+        _need(t, n, torch.int32)
+    B, max_chunks = scores.shape
+    max_kept = kept.shape[1]
+    if kept.shape[0] != B or cu_kept.numel() != B + 1 or n_kept.numel() != B:
+        raise ValueError("bad shapes")
+    _check("lsa_topk_chunks", _load().lsa_topk_chunks(
+        _ptr(scores), _ptr(n_chunks), _ptr(k_per_seq), B, max_chunks, max_kept, _ptr(kept), _ptr(n_kept),
+        _ptr(cu_kept), _stream(stream)))
+
+
+def lsa_gather_chunks(k_pool, v_pool, chunk_table, kept, cu_kept, max_chunks, k_buf, v_buf, stream=None):
+    """Copy the kept chunks of the device pools into the compact buffers."""
+    for t, n in ((k_pool, "k_pool"), (v_pool, "v_pool"), (k_buf, "k_buf"), (v_buf, "v_buf")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((kept, "kept"), (cu_kept, "cu_kept")):
+        _need(t, n, torch.int32)
+    if chunk_table is not None:
+        _need(chunk_table, "chunk_table", torch.int32)
+    B, max_kept = kept.shape
+    _check("lsa_gather_chunks", _load().lsa_gather_chunks(
+        _ptr(k_pool), _ptr(v_pool), k_pool.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(cu_kept), B,
+        int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _stream(stream)))
+
+
+def lsa_fetch_from_host(host_k_pool, host_v_pool, chunk_table, kept, cu_kept, max_chunks, k_buf, v_buf,
+                        num_ctas=0, stream=None, done_event: Optional[torch.cuda.Event] = None):
+    """Same copy as lsa_gather_chunks from page-locked host pools (SM zero-copy reads)."""
+    for t, n in ((host_k_pool, "host_k_pool"), (host_v_pool, "host_v_pool")):
+        _need(t, n, torch.bfloat16, cuda=False)
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((kept, "kept"), (cu_kept, "cu_kept")):
+        _need(t, n, torch.int32)
+    if chunk_table is not None:
+        _need(chunk_table, "chunk_table", torch.int32)
+    B, max_kept = kept.shape
+    ev = None
+    if done_event is not None:
+        if not done_event.cuda_event:
+            # torch creates the CUDA event lazily on its first record
+            done_event.record(stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream())
+        ev = ctypes.c_void_p(done_event.cuda_event)
+    _check("lsa_fetch_from_host", _load().lsa_fetch_from_host(
+        _ptr(host_k_pool), _ptr(host_v_pool), host_k_pool.shape[0], _ptr(chunk_table), _ptr(kept),
+        _ptr(cu_kept), B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], int(num_ctas),
+        _stream(stream), ev))
+
+
+def lsa_attn_workspace_size(B: int) -> int:
+    return int(_load().lsa_attn_workspace_size(int(B)))
+
+
+def new_attn_workspace(B: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace for lsa_sparse_decode_attn (zeroing is required once)."""
+    n = lsa_attn_workspace_size(B)
+    if n == 0:
+        raise ValueError("unsupported batch")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_scale=None, stream=None):
+    """out[b,h] = softmax(scale q[b,h] K^T) V over the kept tokens of KV head h // 8."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_buf, "k_buf", torch.bfloat16)
+    _need(v_buf, "v_buf", torch.bfloat16)
+    _need(cu_kept, "cu_kept", torch.int32)
+    _need(out, "out", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    B = q.shape[0]
+    if tuple(q.shape) != (B, NUM_Q_HEADS, HEAD_DIM) or tuple(out.shape) != (B, NUM_Q_HEADS, HEAD_DIM):
+        raise ValueError("q and out must be [B, 64, 128]")
+    if k_buf.shape != v_buf.shape or cu_kept.numel() != B + 1:
+        raise ValueError("bad shapes")
+    scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
+    _check("lsa_sparse_decode_attn", _load().lsa_sparse_decode_attn(
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+__all__ = [
+    "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
+    "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_attn_workspace_size", "new_attn_workspace",
+    "lsa_sparse_decode_attn", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
+    "INDEX_DIM", "CHUNK_BYTES",
+]

@@ -1,0 +1,468 @@
+// lsa_sparse_decode_attn: one GQA decode step over the kept chunks.
+//
+// Method: softmax(q K^T / sqrt(d)) V per query head, 8 consecutive query heads
+// per KV head (handbook page "DeepSeek-V4: Architecting for Ultra-Long
+// Contexts", section "Grouped Query Attention (GQA) vs. Multi-Head Attention
+// (MHA)"), over only the chunks kept for the window (summary page
+// "FlashMemory-DeepSeek-V4 ...", Abstract and 2.1 Architecture).
+//
+// B200 design
+// -----------
+// * Work unit = one (sequence b, KV head g, kept chunk j) tile: 64 tokens of K
+//   and of V, 16 KiB each, contiguous in the compact buffer.  The units of all
+//   (b, g) pairs are laid end to end, and the grid (one CTA per SM) cuts that
+//   list into equal contiguous ranges (split-K over the kept tokens, balanced
+//   to within one unit per CTA for any batch mix).
+// * A producer warp streams units into a 6-stage shared-memory ring with TMA
+//   (cp.async.bulk.tensor, 128-byte swizzle, evict-first L2 hint) completing
+//   on mbarriers; 4 consumer warps each take 16 of the 64 tokens of a unit.
+// * Per warp, scores are computed transposed, S^T = K Q^T, on the tensor
+//   cores (mma.sync m16n8k16: M = 16 tokens, N = the 8 query heads of the
+//   group, K = 128), so no MMA row is padding.  The online softmax runs in
+//   fp32 (exp2 domain); probabilities are rounded to bf16, transposed in
+//   registers with movmatrix and used as the B operand of O^T += V^T P^T
+//   (M = 128 dims, N = 8 heads, K = 16 tokens, V^T read with ldmatrix.trans).
+// * At the end of each (b, g) segment the 4 warps combine their (max, sum,
+//   acc) in shared memory.  A segment that covers the whole pair writes the
+//   output; otherwise it writes a normalised partial and its log-sum-exp, and
+//   the last CTA to finish the pair (atomic ticket) merges all partials of the
+//   pair in CTA order, so the result does not depend on timing.
+#include <math.h>
+
+#include <mutex>
+
+#include "lsa_common.cuh"
+#include "lsa_runtime.cuh"
+
+namespace lsa {
+namespace attn {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kStages = 6;
+constexpr int kBoxBytes = 8192;              // 64 tokens x 64 dims of bf16
+constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo, V hi
+constexpr int kAccStride = 132;              // padded row of the combine buffer
+constexpr int kRecFloats = kGroup * kHeadDim + kGroup;  // partial o[8][128] + lse[8]
+constexpr int kMaxCtas = 1024;
+constexpr int kSmemBytes = 1024 /*align*/ + kStages * kStageBytes +
+                           kConsumerWarps * kGroup * kAccStride * 4 + 2 * kConsumerWarps * kGroup * 4 +
+                           2 * kStages * 8 + 16;
+
+// CTA that owns unit u when T units are cut into G equal contiguous ranges
+// [floor(T c / G), floor(T (c+1) / G)).
+__device__ __forceinline__ int cta_of(int64_t u, int64_t T, int G) {
+  return static_cast<int>(((u + 1) * G - 1) / T);
+}
+__device__ __forceinline__ int64_t range_lo(int c, int64_t T, int G) { return T * c / G; }
+
+// Largest b in [0, B) with 8 * cu[b] <= u (the sequence that holds unit u).
+__device__ __forceinline__ int seq_of_unit(const int32_t* cu, int B, int64_t u) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (8 * static_cast<int64_t>(__ldg(cu + mid)) <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+struct UnitCursor {
+  int b, g, j;
+  __device__ void start(const int32_t* cu, int B, int64_t u) {
+    b = seq_of_unit(cu, B, u);
+    const int64_t r = u - 8 * static_cast<int64_t>(__ldg(cu + b));
+    const int n = __ldg(cu + b + 1) - __ldg(cu + b);
+    g = static_cast<int>(r / n);
+    j = static_cast<int>(r - static_cast<int64_t>(g) * n);
+  }
+  __device__ void advance(const int32_t* cu, int B, int n_b) {
+    if (++j == n_b) {
+      j = 0;
+      if (++g == kNumKVHeads) {
+        g = 0;
+        ++b;
+        while (b < B && __ldg(cu + b + 1) == __ldg(cu + b)) ++b;
+      }
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu, int B,
+                          int64_t buf_chunks, float scale_log2, float* __restrict__ out,
+                          int* __restrict__ counters, float* __restrict__ records, unsigned* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* accbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  float* mbuf = accbuf + kConsumerWarps * kGroup * kAccStride;
+  float* lbuf = mbuf + kConsumerWarps * kGroup;
+  uint64_t* full = reinterpret_cast<uint64_t*>(lbuf + kConsumerWarps * kGroup);
+  uint64_t* empty = full + kStages;
+  int* flags = reinterpret_cast<int*>(empty + kStages);  // [0] abort, [1] last-CTA
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ---- validate cu_kept (every thread reaches the same verdict) -------------
+  const int total = __ldg(cu + B);
+  int bad = (__ldg(cu) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) ? 1 : 0;
+  for (int b = tid; b < B; b += kThreads) bad |= (__ldg(cu + b + 1) < __ldg(cu + b));
+  bad = __syncthreads_or(bad);
+  if (bad) {
+    if (blockIdx.x == 0 && tid == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
+    return;
+  }
+  const int64_t T = 8 * static_cast<int64_t>(total);
+  const int G = gridDim.x;
+  const int64_t u0 = range_lo(blockIdx.x, T, G), u1 = range_lo(blockIdx.x + 1, T, G);
+
+  // Sequences without kept chunks get zeros.
+  for (int b = blockIdx.x; b < B; b += G) {
+    if (__ldg(cu + b + 1) == __ldg(cu + b)) {
+      float4* o = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * kNumQHeads * kHeadDim);
+      for (int i = tid; i < kNumQHeads * kHeadDim / 4; i += kThreads) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  if (u0 >= u1) return;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = flags;
+
+  if (warp == kConsumerWarps) {
+    // ====================== producer warp: TMA stream ========================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint64_t policy = l2_policy_evict_first();
+      UnitCursor cur;
+      cur.start(cu, B, u0);
+      const int64_t n_units = u1 - u0;
+      int64_t issued = 0;
+      for (int64_t i = 0; i < n_units; ++i) {
+        const int s = static_cast<int>(i % kStages);
+        if (i >= kStages) {
+          const unsigned par = static_cast<unsigned>(((i / kStages) - 1) & 1);
+          if (!mbar_wait_bounded(&empty[s], par, abort_flag)) {
+            if (!*abort_flag) set_status(status, LSA_DEV_ERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        const int cb = __ldg(cu + cur.b);
+        const int n_b = __ldg(cu + cur.b + 1) - cb;
+        const int row = ((cb + cur.j) * kNumKVHeads + cur.g) * kChunkTokens;
+        uint8_t* st = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        tma_load_2d(st, &tm_k, 0, row, &full[s], policy);
+        tma_load_2d(st + kBoxBytes, &tm_k, 64, row, &full[s], policy);
+        tma_load_2d(st + 2 * kBoxBytes, &tm_v, 0, row, &full[s], policy);
+        tma_load_2d(st + 3 * kBoxBytes, &tm_v, 64, row, &full[s], policy);
+        issued = i + 1;
+        cur.advance(cu, B, n_b);
+      }
+      if (*abort_flag) {
+        // Let every copy already issued land before the CTA exits.
+        int never = 0;
+        for (int64_t i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+          mbar_wait_bounded(&full[i % kStages], static_cast<unsigned>((i / kStages) & 1), &never);
+      }
+    }
+    return;
+  }
+
+  // ========================= consumer warps ==================================
+  const int gl = lane >> 2;   // row group of the mma fragments
+  const int c4 = lane & 3;    // column pair of the mma fragments
+  const int mi = lane >> 3, r8 = lane & 7;
+  // ldmatrix row addresses of this lane (see the fragment maps in the header comment)
+  const int krow = warp * 16 + r8 + ((mi & 1) << 3);
+  const int kx = mi >> 1;
+  const int vrow = warp * 16 + r8 + ((mi >> 1) << 3);
+  const int vx = mi & 1;
+  const uint32_t smem_base = smem_u32(smem);
+
+  UnitCursor cur;
+  cur.start(cu, B, u0);
+  int64_t u = u0;
+  int64_t unit_i = 0;
+  while (u < u1) {
+    const int b = cur.b, g = cur.g;
+    const int cb = __ldg(cu + b);
+    const int n_b = __ldg(cu + b + 1) - cb;
+    const int j0 = cur.j;
+    const int64_t seg_cap = static_cast<int64_t>(j0) + (u1 - u);
+    const int jend = seg_cap < n_b ? static_cast<int>(seg_cap) : n_b;
+    const bool whole_pair = (j0 == 0 && jend == n_b);
+
+    // Q^T fragments (B operand of S^T = K Q^T): head 8g+gl, dims 16t + 2c4 (+8).
+    uint32_t bq[8][2];
+    {
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          q + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + gl) * kHeadDim);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        bq[t][0] = __ldg(qrow + 8 * t + c4);
+        bq[t][1] = __ldg(qrow + 8 * t + 4 + c4);
+      }
+    }
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+    for (int jj = j0; jj < jend; ++jj, ++unit_i) {
+      const int s = static_cast<int>(unit_i % kStages);
+      bool ok = !*abort_flag;
+      if (ok) {
+        ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((unit_i / kStages) & 1), abort_flag);
+        if (!ok) {
+          if (!*abort_flag) set_status(status, LSA_DEV_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+      }
+      if (ok) {
+        const uint32_t kbase = smem_base + s * kStageBytes;
+        const uint32_t vbase = kbase + 2 * kBoxBytes;
+        // ---- S^T[16 tokens x 8 heads] = K[16 x 128] Q^T[128 x 8] ----------
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const uint32_t addr = kbase + (t >> 2) * kBoxBytes + krow * 128 +
+                                ((((t & 3) * 2 + kx) ^ (krow & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(addr, a0, a1, a2, a3);
+          mma_bf16_16816((t & 1) ? sb : sa, a0, a1, a2, a3, bq[t][0], bq[t][1]);
+        }
+        // s[0]: (token gl, head 2c4)  s[1]: (gl, 2c4+1)  s[2]: (gl+8, 2c4)  s[3]: (gl+8, 2c4+1)
+        const float s0 = (sa[0] + sb[0]) * scale_log2, s1 = (sa[1] + sb[1]) * scale_log2;
+        const float s2 = (sa[2] + sb[2]) * scale_log2, s3 = (sa[3] + sb[3]) * scale_log2;
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        const uint32_t ptop = pack_bf16(fast_exp2(s0 - mn0), fast_exp2(s1 - mn1));
+        const uint32_t pbot = pack_bf16(fast_exp2(s2 - mn0), fast_exp2(s3 - mn1));
+        l0 = l0 * al0 + bf16_lo(ptop) + bf16_lo(pbot);
+        l1 = l1 * al1 + bf16_hi(ptop) + bf16_hi(pbot);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          acc[i][0] *= al0;
+          acc[i][1] *= al1;
+          acc[i][2] *= al0;
+          acc[i][3] *= al1;
+        }
+        // P^T as the B operand (k = token, n = head): transpose the 8x8 blocks.
+        const uint32_t pb0 = movmatrix_trans(ptop);
+        const uint32_t pb1 = movmatrix_trans(pbot);
+        // ---- O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] P^T[16 x 8] ---
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t addr = vbase + (i >> 2) * kBoxBytes + vrow * 128 +
+                                ((((i & 3) * 2 + vx) ^ (vrow & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+          mma_bf16_16816(acc[i], a0, a1, a2, a3, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---- end of segment: combine the 4 warps --------------------------------
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    if (gl == 0) {
+      mbuf[warp * kGroup + 2 * c4] = m0;
+      mbuf[warp * kGroup + 2 * c4 + 1] = m1;
+      lbuf[warp * kGroup + 2 * c4] = l0;
+      lbuf[warp * kGroup + 2 * c4 + 1] = l1;
+    }
+    {
+      float* ab = accbuf + warp * kGroup * kAccStride;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ab[(2 * c4) * kAccStride + 16 * i + gl] = acc[i][0];
+        ab[(2 * c4 + 1) * kAccStride + 16 * i + gl] = acc[i][1];
+        ab[(2 * c4) * kAccStride + 16 * i + gl + 8] = acc[i][2];
+        ab[(2 * c4 + 1) * kAccStride + 16 * i + gl + 8] = acc[i][3];
+      }
+    }
+    named_barrier(1, kConsumerThreads);
+
+    const int hh = tid >> 4;          // head within the group
+    const int d0 = (tid & 15) * 8;    // 8 consecutive dims
+    float mw[kConsumerWarps], M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      mw[w] = mbuf[w * kGroup + hh];
+      M = fmaxf(M, mw[w]);
+    }
+    float L = 0.f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float sc = fast_exp2(mw[w] - M);
+      L += sc * lbuf[w * kGroup + hh];
+      const float* ab = accbuf + (w * kGroup + hh) * kAccStride + d0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] += sc * ab[k];
+    }
+    const float inv = 1.f / L;
+    const int p = b * kNumKVHeads + g;
+    float* dst = out + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + hh) * kHeadDim + d0;
+    if (whole_pair) {
+      reinterpret_cast<float4*>(dst)[0] = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv);
+    } else {
+      float* rec = records + static_cast<int64_t>(p + blockIdx.x) * kRecFloats;
+      reinterpret_cast<float4*>(rec + hh * kHeadDim + d0)[0] =
+          make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+      reinterpret_cast<float4*>(rec + hh * kHeadDim + d0)[1] =
+          make_float4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv);
+      if ((tid & 15) == 0) rec[kGroup * kHeadDim + hh] = M + __log2f(L);
+      __threadfence();
+      named_barrier(1, kConsumerThreads);
+      // Contributing CTAs of pair p: those whose unit range meets [a_p, a_p + n_b).
+      const int64_t a_p = 8 * static_cast<int64_t>(cb) + static_cast<int64_t>(g) * n_b;
+      const int c_lo = cta_of(a_p, T, G), c_hi = cta_of(a_p + n_b - 1, T, G);
+      if (tid == 0) {
+        int n_contrib = 0;
+        for (int c = c_lo; c <= c_hi; ++c) n_contrib += (range_lo(c + 1, T, G) > range_lo(c, T, G));
+        const int old = atomicAdd(&counters[p], 1);
+        if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
+        flags[1] = (old == n_contrib - 1);
+      }
+      named_barrier(1, kConsumerThreads);
+      if (flags[1]) {
+        __threadfence();
+        float lse_max = -INFINITY;
+        for (int c = c_lo; c <= c_hi; ++c) {
+          if (range_lo(c + 1, T, G) == range_lo(c, T, G)) continue;
+          const float* rc = records + static_cast<int64_t>(p + c) * kRecFloats;
+          lse_max = fmaxf(lse_max, __ldcg(rc + kGroup * kHeadDim + hh));
+        }
+        float den = 0.f, r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c = c_lo; c <= c_hi; ++c) {
+          if (range_lo(c + 1, T, G) == range_lo(c, T, G)) continue;
+          const float* rc = records + static_cast<int64_t>(p + c) * kRecFloats;
+          const float wgt = fast_exp2(__ldcg(rc + kGroup * kHeadDim + hh) - lse_max);
+          den += wgt;
+          const float4 x0 = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
+          const float4 x1 = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0) + 1);
+          r[0] += wgt * x0.x; r[1] += wgt * x0.y; r[2] += wgt * x0.z; r[3] += wgt * x0.w;
+          r[4] += wgt * x1.x; r[5] += wgt * x1.y; r[6] += wgt * x1.z; r[7] += wgt * x1.w;
+        }
+        const float id = 1.f / den;
+        reinterpret_cast<float4*>(dst)[0] = make_float4(r[0] * id, r[1] * id, r[2] * id, r[3] * id);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(r[4] * id, r[5] * id, r[6] * id, r[7] * id);
+        if (tid == 0) counters[p] = 0;   // ready for the next call
+      }
+    }
+    named_barrier(1, kConsumerThreads);   // combine buffer free for the next segment
+
+    // Move the cursor to the unit after this segment.
+    u += jend - j0;
+    cur.j = jend - 1;
+    cur.advance(cu, B, n_b);
+  }
+}
+
+// Workspace: int counters[B*8] (padded to 256 B), then fp32 records[(B*8 + kMaxCtas)][kRecFloats].
+size_t workspace_bytes(int B) {
+  const size_t cnt = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
+  return cnt + (static_cast<size_t>(B) * kNumKVHeads + kMaxCtas) * kRecFloats * sizeof(float);
+}
+
+}  // namespace attn
+}  // namespace lsa
+
+namespace {
+std::mutex g_attn_mu;
+bool g_attn_attr_set[64] = {};
+
+int encode_kv_map(CUtensorMap* map, const void* base, int64_t buf_chunks) {
+  lsa::EncodeTiledFn enc = lsa::tensor_map_encoder();
+  if (!enc) return LSA_ERR_NO_DEVICE;
+  // 2-D view of the compact buffer: rows = (chunk, KV head, token), 128 bf16 per row.
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(lsa::kHeadDim),
+                              static_cast<cuuint64_t>(buf_chunks) * lsa::kNumKVHeads * lsa::kChunkTokens};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(lsa::kHeadDim) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(lsa::kChunkTokens)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LSA_OK : LSA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+size_t lsa_attn_workspace_size(int B) {
+  if (B <= 0 || B > LSA_MAX_BATCH) return 0;
+  return lsa::attn::workspace_bytes(B);
+}
+
+int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
+                           const int32_t* cu_kept, int B, float softmax_scale, float* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  using namespace lsa;
+  if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  // TMA row coordinates are 32-bit: (buf_chunks * 512) rows must fit.
+  if (buf_chunks > (int64_t{1} << 22)) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out) || !aligned16(workspace))
+    return LSA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < attn::workspace_bytes(B)) return LSA_ERR_WORKSPACE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return LSA_ERR_NO_DEVICE;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(g_attn_mu);
+    if (dev < 64 && !g_attn_attr_set[dev]) {
+      if (cudaFuncSetAttribute(attn::sparse_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn::kSmemBytes) != cudaSuccess) {
+        cudaGetLastError();
+        return LSA_ERR_CUDA;
+      }
+      g_attn_attr_set[dev] = true;
+    }
+  }
+  CUtensorMap tm_k, tm_v;
+  int st = encode_kv_map(&tm_k, k_buf, buf_chunks);
+  if (st != LSA_OK) return st;
+  st = encode_kv_map(&tm_v, v_buf, buf_chunks);
+  if (st != LSA_OK) return st;
+  const size_t cnt_bytes = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
+  int* counters = static_cast<int*>(workspace);
+  float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cnt_bytes);
+  const int grid = sms < attn::kMaxCtas ? sms : attn::kMaxCtas;
+  const float scale_log2 = softmax_scale * 1.4426950408889634f;
+  attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks, scale_log2, out, counters, records,
+      lsa_device_status_ptr());
+  return launch_status();
+}
+
+}  // extern "C"

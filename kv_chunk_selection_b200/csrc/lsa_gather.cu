@@ -1,0 +1,154 @@
+// lsa_gather_chunks / lsa_fetch_from_host: build the compact resident buffer.
+//
+// Method: only the chunks recalled for the coming window are kept in GPU
+// memory (summary page "FlashMemory-DeepSeek-V4 ...", Abstract and 2.1
+// Architecture); when the full cache lives in CPU memory they are fetched from
+// there every tau steps (summary page, 3 Experiments "Experimental Setup";
+// handbook page "DeepSeek-V4: Architecting for Ultra-Long Contexts", "The
+// Neural Memory Indexer", item 3).
+//
+// B200 design: a pure bandwidth copy.  The work item is one 16 KiB
+// (chunk, KV head, K-or-V) tile, contiguous at both ends; a 256-thread CTA
+// moves it with 16-byte loads issued four per thread before any store, and the
+// grid strides over all items of the batch (the total is read on the device
+// from cu_kept, so nothing is copied back to the host and the call can be
+// captured in a CUDA graph).  The host-tier variant runs the same kernel on a
+// small grid over the device alias of page-locked host memory: SMs pull the
+// scattered chunks over the host link directly, on the caller's side stream,
+// without a host loop or a device-to-host copy of the kept list.
+#include "lsa_common.cuh"
+#include "lsa_runtime.cuh"
+
+namespace lsa {
+namespace gather {
+
+constexpr int kThreads = 256;
+constexpr int kVecPerTile = kTileBytes / 16;        // 1024 x 16 B
+constexpr int kVecPerThread = kVecPerTile / kThreads;  // 4
+
+__device__ __forceinline__ int seq_of(const int32_t* cu, int B, int i) {
+  int lo = 0, hi = B - 1;  // largest b with cu[b] <= i
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kThreads)
+gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool, int64_t n_slots,
+              const int32_t* __restrict__ table, const int32_t* __restrict__ kept, const int32_t* __restrict__ cu,
+              int B, int max_chunks, int max_kept, uint4* __restrict__ k_buf, uint4* __restrict__ v_buf,
+              int64_t buf_chunks, unsigned* status) {
+  const int total = __ldg(cu + B);
+  if (__ldg(cu) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
+    return;
+  }
+  const int64_t items = static_cast<int64_t>(total) * 2 * kNumKVHeads;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int i = static_cast<int>(it >> 4);        // compact chunk index
+    const int kv = static_cast<int>((it >> 3) & 1);  // 0 = K, 1 = V
+    const int h = static_cast<int>(it & 7);
+    const int b = seq_of(cu, B, i);
+    const int j = i - __ldg(cu + b);
+    if (j < 0 || j >= max_kept) {
+      if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
+      continue;
+    }
+    const int c = __ldg(kept + static_cast<int64_t>(b) * max_kept + j);
+    if (c < 0 || c >= max_chunks) {
+      if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
+      continue;
+    }
+    const int64_t slot = table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c)
+                               : static_cast<int64_t>(b) * max_chunks + c;
+    if (slot < 0 || slot >= n_slots) {
+      if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_BAD_SLOT);
+      continue;
+    }
+    const int64_t tile = static_cast<int64_t>(kNumKVHeads) * kVecPerTile;  // uint4 per chunk
+    const uint4* src = (kv ? v_pool : k_pool) + slot * tile + h * kVecPerTile;
+    uint4* dst = (kv ? v_buf : k_buf) + static_cast<int64_t>(i) * tile + h * kVecPerTile;
+    uint4 r[kVecPerThread];
+#pragma unroll
+    for (int v = 0; v < kVecPerThread; ++v) r[v] = __ldcs(src + v * kThreads + threadIdx.x);
+#pragma unroll
+    for (int v = 0; v < kVecPerThread; ++v) dst[v * kThreads + threadIdx.x] = r[v];
+  }
+}
+
+int check_common(const void* k_pool, const void* v_pool, int64_t n_slots, const int32_t* kept,
+                 const int32_t* cu_kept, int B, int max_chunks, int max_kept, const void* k_buf, const void* v_buf,
+                 int64_t buf_chunks) {
+  if (!k_pool || !v_pool || !kept || !cu_kept || !k_buf || !v_buf || B <= 0 || max_chunks <= 0 ||
+      max_kept <= 0 || n_slots <= 0 || buf_chunks <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(k_buf) || !aligned16(v_buf)) return LSA_ERR_MISALIGNED;
+  return LSA_OK;
+}
+
+}  // namespace gather
+}  // namespace lsa
+
+extern "C" {
+
+int lsa_gather_chunks(const void* k_pool, const void* v_pool, int64_t n_slots, const int32_t* chunk_table,
+                      const int32_t* kept, const int32_t* cu_kept, int B, int max_chunks, int max_kept, void* k_buf,
+                      void* v_buf, int64_t buf_chunks, void* stream) {
+  using namespace lsa;
+  const int st =
+      gather::check_common(k_pool, v_pool, n_slots, kept, cu_kept, B, max_chunks, max_kept, k_buf, v_buf, buf_chunks);
+  if (st != LSA_OK) return st;
+  const int sms = device_sm_count();
+  if (sms <= 0) return LSA_ERR_NO_DEVICE;
+  gather::gather_kernel<<<sms * 8, gather::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_pool), static_cast<const uint4*>(v_pool), n_slots, chunk_table, kept, cu_kept, B,
+      max_chunks, max_kept, static_cast<uint4*>(k_buf), static_cast<uint4*>(v_buf), buf_chunks,
+      lsa_device_status_ptr());
+  return launch_status();
+}
+
+int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                        const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept, int B,
+                        int max_chunks, int max_kept, void* k_buf, void* v_buf, int64_t buf_chunks, int num_ctas,
+                        void* stream, void* done_event) {
+  using namespace lsa;
+  const int st = gather::check_common(host_k_pool, host_v_pool, n_slots, kept, cu_kept, B, max_chunks, max_kept,
+                                      k_buf, v_buf, buf_chunks);
+  if (st != LSA_OK) return st;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  // The pools must be page-locked host memory; use their device aliases.
+  void* dk = nullptr;
+  void* dv = nullptr;
+  cudaPointerAttributes ak, av;
+  if (cudaPointerGetAttributes(&ak, host_k_pool) != cudaSuccess ||
+      cudaPointerGetAttributes(&av, host_v_pool) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_NOT_PINNED;
+  }
+  if (ak.type != cudaMemoryTypeHost || av.type != cudaMemoryTypeHost) return LSA_ERR_NOT_PINNED;
+  if (cudaHostGetDevicePointer(&dk, const_cast<void*>(host_k_pool), 0) != cudaSuccess ||
+      cudaHostGetDevicePointer(&dv, const_cast<void*>(host_v_pool), 0) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_NOT_PINNED;
+  }
+  const int grid = num_ctas > 0 ? num_ctas : 64;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gather::gather_kernel<<<grid, gather::kThreads, 0, s>>>(
+      static_cast<const uint4*>(dk), static_cast<const uint4*>(dv), n_slots, chunk_table, kept, cu_kept, B,
+      max_chunks, max_kept, static_cast<uint4*>(k_buf), static_cast<uint4*>(v_buf), buf_chunks,
+      lsa_device_status_ptr());
+  int rc = launch_status();
+  if (rc == LSA_OK && done_event) {
+    if (cudaEventRecord(static_cast<cudaEvent_t>(done_event), s) != cudaSuccess) {
+      cudaGetLastError();
+      rc = LSA_ERR_CUDA;
+    }
+  }
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,202 @@
+// lsa_topk_chunks: per-sequence top-K of the indexer scores plus the latest chunk.
+//
+// Method: the recalled set is the fixed-budget form of the indexer's selection
+// (summary page "FlashMemory-DeepSeek-V4 ...", 2.1 Architecture): the K best
+// chunks among all but the latest, ordered by score descending then chunk
+// index ascending, plus the latest chunk, listed in ascending order.
+//
+// B200 design: one 1024-thread CTA per sequence runs an exact radix select on
+// a 32-bit key that orders scores descending (the float bits mapped to an
+// order-preserving unsigned and complemented).  Four 8-bit digit passes find
+// the boundary key; chunk index breaks ties among equal keys.  Histograms use
+// shared-memory atomics aggregated per warp with __match_any_sync, since the
+// high digits of scores in a narrow range are nearly all equal.  The kept set
+// is then written in index order with two block-wide prefix scans, so the
+// output is ascending without a sort.  Scores are read from L2 on each pass
+// (at most 64 KiB per sequence).
+#include "lsa_common.cuh"
+#include "lsa_runtime.cuh"
+
+namespace lsa {
+namespace topk {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+
+// Smaller key <=> larger score (IEEE order-preserving map, then complement).
+// -0.0 and +0.0 get the same key (they are equal scores, so the chunk index
+// decides), and NaN sorts after every number.
+__device__ __forceinline__ uint32_t desc_key(float s) {
+  if (s != s) return 0xffffffffu;
+  uint32_t u = __float_as_uint(s);
+  if ((u << 1) == 0) u = 0;
+  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ~ord;
+}
+
+// Kept count of one sequence, or 0 with *err set when its counts are invalid.
+__device__ __forceinline__ int kept_count(int n, int k, int max_chunks, int max_kept, unsigned* err) {
+  if (n < 0 || n > max_chunks || k < 0) {
+    *err |= LSA_DEV_ERR_BAD_COUNT;
+    return 0;
+  }
+  if (n == 0) return 0;
+  const int nk = min(k, n - 1) + 1;
+  if (nk > max_kept) {
+    *err |= LSA_DEV_ERR_CAPACITY;
+    return 0;
+  }
+  return nk;
+}
+
+// Exclusive block-wide prefix sum of one int per thread; *total gets the sum.
+__device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ws, off);
+      if (lane >= off) ws += y;
+    }
+    warp_sums[lane] = ws;  // inclusive
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (total) *total = warp_sums[kWarps - 1];
+  __syncthreads();
+  return excl;
+}
+
+__global__ void __launch_bounds__(kThreads)
+topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
+            const int32_t* __restrict__ k_per_seq, int B, int max_chunks, int max_kept,
+            int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, int32_t* __restrict__ cu_kept,
+            unsigned* status) {
+  __shared__ int hist[256];
+  __shared__ int warp_sums[32];
+  __shared__ int sel[2];
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+
+  // cu_kept[b+1] = sum of the kept counts of sequences 0..b.
+  int part = 0;
+  unsigned dummy = 0;
+  for (int bb = tid; bb <= b; bb += kThreads)
+    part += kept_count(__ldg(n_chunks + bb), __ldg(k_per_seq + bb), max_chunks, max_kept, &dummy);
+  int tot = 0;
+  block_exclusive_scan(part, warp_sums, &tot);
+  unsigned err = 0;
+  const int n = __ldg(n_chunks + b);
+  const int nk = kept_count(n, __ldg(k_per_seq + b), max_chunks, max_kept, &err);
+  if (tid == 0) {
+    cu_kept[b + 1] = tot;
+    if (b == 0) cu_kept[0] = 0;
+    n_kept[b] = nk;
+    if (err) set_status(status, err);
+  }
+  if (nk == 0) return;
+  int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
+  const int cand = n - 1;
+  const int kc = nk - 1;
+  if (kc == cand) {  // keep every chunk
+    for (int c = tid; c < n; c += kThreads) out[c] = c;
+    return;
+  }
+  if (tid == 0) out[kc] = n - 1;  // the latest chunk, always last
+  if (kc == 0) return;
+  const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
+
+  // ---- radix select of the kc-th smallest key (1-based) -----------------------
+  uint32_t prefix = 0, mask = 0;
+  int krem = kc;
+  const int cand_pad = (cand + kThreads - 1) / kThreads * kThreads;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < cand_pad; i += kThreads) {
+      const bool valid = i < cand;
+      const uint32_t key = valid ? desc_key(__ldg(sc + i)) : 0u;
+      const bool match = valid && ((key & mask) == prefix);
+      const int digit = match ? static_cast<int>((key >> shift) & 255u) : 256;
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+    }
+    __syncthreads();
+    // Inclusive prefix over the 256 bins (warps 0..7), then locate the bin
+    // that holds the krem-th smallest remaining key.
+    int count = 0, incl = 0;
+    if (tid < 256) {
+      count = hist[tid];
+      incl = count;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) warp_sums[tid >> 5] = incl;
+    }
+    __syncthreads();
+    if (tid < 256) {
+      for (int w = 0; w < (tid >> 5); ++w) incl += warp_sums[w];
+      const int excl = incl - count;
+      if (excl < krem && incl >= krem) {
+        sel[0] = tid;
+        sel[1] = krem - excl;
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel[0]) << shift;
+    mask |= 255u << shift;
+    krem = sel[1];
+    __syncthreads();
+  }
+  const uint32_t boundary = prefix;  // the kc-th smallest key; take krem of its ties
+
+  // ---- write the kept candidates in ascending index order ---------------------
+  const int per = (cand + kThreads - 1) / kThreads;
+  const int lo = min(cand, tid * per), hi = min(cand, lo + per);
+  int n_eq = 0;
+  for (int i = lo; i < hi; ++i) n_eq += (desc_key(__ldg(sc + i)) == boundary);
+  const int eq_before = block_exclusive_scan(n_eq, warp_sums, nullptr);
+  int n_sel = 0, eq_seen = eq_before;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t key = desc_key(__ldg(sc + i));
+    if (key < boundary) ++n_sel;
+    else if (key == boundary) n_sel += (eq_seen++ < krem);
+  }
+  int pos = block_exclusive_scan(n_sel, warp_sums, nullptr);
+  eq_seen = eq_before;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t key = desc_key(__ldg(sc + i));
+    bool take = key < boundary;
+    if (key == boundary) take = (eq_seen++ < krem);
+    if (take) out[pos++] = i;
+  }
+}
+
+}  // namespace topk
+}  // namespace lsa
+
+extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq, int B,
+                               int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
+                               void* stream) {
+  using namespace lsa;
+  if (!scores || !n_chunks || !k_per_seq || !kept || !n_kept || !cu_kept || B <= 0 || max_chunks <= 0 ||
+      max_kept <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  topk::topk_kernel<<<B, topk::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      scores, n_chunks, k_per_seq, B, max_chunks, max_kept, kept, n_kept, cu_kept, lsa_device_status_ptr());
+  return launch_status();
+}

@@ -1,0 +1,88 @@
+"""The lookahead window schedule of one layer, on top of the C ABI.
+
+Every tau = 64 decode steps the indexer scores all chunks, the selection keeps
+the top-K plus the latest chunk, and the kept chunks are gathered into the
+compact buffer (or fetched from a page-locked host pool); the next 64 decode
+steps attend over that buffer only (summary page "FlashMemory-DeepSeek-V4 ...",
+1 Introduction and 2.1 Architecture; handbook page "DeepSeek-V4: Architecting
+for Ultra-Long Contexts", "The Neural Memory Indexer").
+
+This module only owns buffers and issues the library calls in order; it does
+no arithmetic of the method itself.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_attn_workspace_size,
+               lsa_fetch_from_host, lsa_gather_chunks, lsa_index_score, lsa_sparse_decode_attn,
+               lsa_topk_chunks)
+
+TAU = 64
+
+
+class LayerWindow:
+    """Buffers and calls of one layer's decode window.
+
+    Sizes: ``max_kept`` = max_b K_b + 1 kept chunks per sequence row, and the
+    compact buffer holds ``sum_b (K_b + 1)`` chunks (an upper bound of the kept
+    total).  With ``double_buffer`` two compact buffers alternate, so the
+    selection of the next window can be fetched while the current one is read.
+    """
+
+    def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
+                 max_chunks: int, device="cuda", double_buffer: bool = False):
+        self.device = torch.device(device)
+        self.n_chunks = n_chunks
+        self.k_per_seq = k_per_seq
+        self.chunk_table = chunk_table
+        self.max_chunks = int(max_chunks)
+        self.B = int(n_chunks.shape[0])
+        k_host = k_per_seq.to("cpu", torch.int64)
+        self.max_kept = int(k_host.max()) + 1
+        self.buf_chunks = int((k_host + 1).sum())
+        nbuf = 2 if double_buffer else 1
+        shape = (self.buf_chunks, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM)
+        self.k_bufs = [torch.empty(shape, dtype=torch.bfloat16, device=self.device) for _ in range(nbuf)]
+        self.v_bufs = [torch.empty(shape, dtype=torch.bfloat16, device=self.device) for _ in range(nbuf)]
+        self.scores = torch.empty((self.B, self.max_chunks), dtype=torch.float32, device=self.device)
+        self.kept = [torch.zeros((self.B, self.max_kept), dtype=torch.int32, device=self.device) for _ in range(nbuf)]
+        self.n_kept = [torch.zeros((self.B,), dtype=torch.int32, device=self.device) for _ in range(nbuf)]
+        self.cu_kept = [torch.zeros((self.B + 1,), dtype=torch.int32, device=self.device) for _ in range(nbuf)]
+        self.workspace = torch.zeros(lsa_attn_workspace_size(self.B), dtype=torch.uint8, device=self.device)
+        self.active = 0
+
+    def select(self, q_idx, w, chunk_keys, buf: int = 0, stream=None):
+        """Indexer scores, then top-K plus latest, into selection slot ``buf``."""
+        lsa_index_score(q_idx, w, chunk_keys, self.chunk_table, self.n_chunks, self.scores, stream=stream)
+        lsa_topk_chunks(self.scores, self.n_chunks, self.k_per_seq, self.kept[buf], self.n_kept[buf],
+                        self.cu_kept[buf], stream=stream)
+
+    def gather(self, k_pool, v_pool, buf: int = 0, stream=None):
+        lsa_gather_chunks(k_pool, v_pool, self.chunk_table, self.kept[buf], self.cu_kept[buf], self.max_chunks,
+                          self.k_bufs[buf], self.v_bufs[buf], stream=stream)
+
+    def fetch(self, host_k_pool, host_v_pool, buf: int = 0, num_ctas: int = 0, stream=None, done_event=None):
+        lsa_fetch_from_host(host_k_pool, host_v_pool, self.chunk_table, self.kept[buf], self.cu_kept[buf],
+                            self.max_chunks, self.k_bufs[buf], self.v_bufs[buf], num_ctas=num_ctas,
+                            stream=stream, done_event=done_event)
+
+    def attend(self, q, out, buf: int = 0, stream=None):
+        """One decode step: out[B, 64, 128] fp32 from q[B, 64, 128] bf16."""
+        lsa_sparse_decode_attn(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], out, self.workspace,
+                               stream=stream)
+
+    def run_window(self, q_idx, w, chunk_keys, k_pool, v_pool, q_steps, outs, stream=None):
+        """Select, gather, then one attention call per step of ``q_steps`` [T, B, 64, 128]."""
+        self.select(q_idx, w, chunk_keys, 0, stream)
+        self.gather(k_pool, v_pool, 0, stream)
+        for t in range(q_steps.shape[0]):
+            self.attend(q_steps[t], outs[t], 0, stream)
+
+    def kept_lists(self, buf: int = 0):
+        """Host copy of the kept chunk lists (for inspection and tests)."""
+        kept = self.kept[buf].cpu()
+        n = self.n_kept[buf].cpu()
+        return [kept[b, : int(n[b])].tolist() for b in range(self.B)]

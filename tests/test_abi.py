@@ -1,0 +1,116 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+its header declares, and rejects bad arguments on the host before launching.
+
+Only argument errors that the host checks catch before any launch are used
+here (null pointers, bad sizes, misaligned addresses), so these tests are safe
+on any machine; the "no device" answers are only asserted without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import kv_chunk_selection_b200 as lsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA, NOT_PINNED, MISALIGNED, NO_DEVICE = 0, -1, -2, -3, -4, -5, -6, -7
+NO_GPU = not torch.cuda.is_available()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from kv_chunk_selection_b200 import build
+    build.build()
+    return lsa.lib()
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ("lsa_index_score", "lsa_topk_chunks", "lsa_gather_chunks", "lsa_sparse_decode_attn",
+                 "lsa_fetch_from_host", "lsa_attn_workspace_size", "lsa_read_device_status",
+                 "lsa_status_string", "lsa_version"):
+        assert name in fns
+
+
+def test_library_exports_every_header_symbol(L):
+    raw = ctypes.CDLL(lsa.LIB_PATH)
+    missing = [f for f in header_functions() if not hasattr(raw, f)]
+    assert missing == []
+
+
+def test_status_strings_and_version(L):
+    assert L.lsa_status_string(OK) == b"LSA_OK"
+    assert L.lsa_status_string(NOT_PINNED) == b"LSA_ERR_NOT_PINNED"
+    assert L.lsa_status_string(12345) == b"LSA_ERR_UNKNOWN"
+    assert L.lsa_version() == 100
+
+
+def test_workspace_size(L):
+    assert L.lsa_attn_workspace_size(0) == 0
+    assert L.lsa_attn_workspace_size(4097) == 0
+    s1, s32 = L.lsa_attn_workspace_size(1), L.lsa_attn_workspace_size(32)
+    assert 0 < s1 < s32
+    # 8 counters (padded to 256 B) + (8 + 1024) partial records of 1032 floats
+    assert s1 == 256 + (8 + 1024) * 1032 * 4
+
+
+def test_host_checks_null_pointers(L):
+    n = None
+    assert L.lsa_index_score(n, n, n, 1, n, n, 1, 1, n, n) == INVALID
+    assert L.lsa_topk_chunks(n, n, n, 1, 1, 1, n, n, n, n) == INVALID
+    assert L.lsa_gather_chunks(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, n) == INVALID
+    assert L.lsa_fetch_from_host(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, 0, n, n) == INVALID
+    assert L.lsa_sparse_decode_attn(n, n, n, 1, n, 1, 0.1, n, n, 0, n) == INVALID
+    assert L.lsa_read_device_status(n, None) == INVALID
+
+
+def test_host_checks_sizes_and_alignment(L):
+    odd = ctypes.c_void_p(0x1001)         # misaligned, never dereferenced
+    ok = ctypes.c_void_p(0x100000)        # aligned, never dereferenced (checks fail first)
+    # non-positive sizes
+    assert L.lsa_index_score(ok, ok, ok, 0, None, ok, 1, 4, ok, None) == INVALID
+    assert L.lsa_index_score(ok, ok, ok, 4, None, ok, 0, 4, ok, None) == INVALID
+    assert L.lsa_topk_chunks(ok, ok, ok, 1, 4, 0, ok, ok, ok, None) == INVALID
+    assert L.lsa_topk_chunks(ok, ok, ok, LSA_MAX_BATCH + 1, 4, 2, ok, ok, ok, None) == UNSUPPORTED
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, -1.0, ok, ok, 1 << 30, None) == INVALID
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, LSA_MAX_BATCH + 1, 0.1, ok, ok, 1 << 30, None) == UNSUPPORTED
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, (1 << 22) + 1, ok, 1, 0.1, ok, ok, 1 << 30, None) == UNSUPPORTED
+    # misaligned bf16 arrays
+    assert L.lsa_index_score(odd, ok, ok, 4, None, ok, 1, 4, ok, None) == MISALIGNED
+    assert L.lsa_gather_chunks(ok, odd, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, None) == MISALIGNED
+    assert L.lsa_sparse_decode_attn(ok, ok, odd, 4, ok, 1, 0.1, ok, ok, 1 << 30, None) == MISALIGNED
+    assert L.lsa_fetch_from_host(odd, ok, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, 0, None, None) == MISALIGNED
+    # workspace too small
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, 16, None) == WORKSPACE
+
+
+LSA_MAX_BATCH = 4096
+
+
+@pytest.mark.skipif(not NO_GPU, reason="asserts the answer on a machine without a GPU")
+def test_no_device_answer(L):
+    ok = ctypes.c_void_p(0x100000)
+    ws = L.lsa_attn_workspace_size(1)
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, ws, None) == NO_DEVICE
+    assert L.lsa_gather_chunks(ok, ok, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, None) == NO_DEVICE
+    bits = ctypes.c_uint(0)
+    assert L.lsa_read_device_status(None, ctypes.byref(bits)) == NO_DEVICE
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    monkeypatch.setattr(lsa, "_lib", None)
+    monkeypatch.setattr(lsa, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="liblsa.so not found"):
+        lsa.lib()
+    importlib.reload(lsa)

@@ -1,0 +1,405 @@
+"""GPU parity: every kernel of liblsa against the fp64 oracle, through the C ABI.
+
+Sizes: full windows at the tiny workload; the 128K workload in full for
+scoring, selection and gather and at sampled decode steps for attention;
+hand-made ragged batches that split (sequence, KV head) pairs across CTAs and
+leave ragged tails; and the 500K / batched / 1M host-tier workloads at full
+size on sampled outputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kv_chunk_selection_b200 as lsa
+import oracle
+import workloads
+from kv_chunk_selection_b200.window import LayerWindow
+from lsa_testlib import (assert_attention_close, assert_kept_matches, assert_scores_close, f64, i64,
+                         kept_from_gpu)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from kv_chunk_selection_b200 import build
+    build.build()
+    lsa.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def status_clean():
+    bits = lsa.read_device_status()
+    assert bits == 0, f"device status {lsa.decode_status(bits)}"
+
+
+def score_on_gpu(inp, layer=0, window=0):
+    L = inp.layers[layer]
+    scores = torch.full((inp.batch, inp.max_chunks), float("nan"), device=DEV)
+    lsa.lsa_index_score(L.q_idx[window], L.w, L.chunk_keys, inp.chunk_table, inp.n_chunks, scores)
+    return scores
+
+
+def oracle_scores(inp, layer=0, window=0):
+    L = inp.layers[layer]
+    return oracle.index_scores(f64(L.q_idx[window]), f64(L.w), f64(L.chunk_keys), i64(inp.chunk_table),
+                               i64(inp.n_chunks), inp.max_chunks)
+
+
+# ------------------------------------------------------------------ scoring --
+
+@pytest.mark.parametrize("name", ["tiny", "128k", "500k", "1m_host", "batched"])
+def test_index_score_matches_oracle(name):
+    inp = workloads.make_inputs(name, DEV, pools=False, layers=1)
+    for w in range(min(2, inp.workload.windows)):
+        g = score_on_gpu(inp, 0, w)
+        o = oracle_scores(inp, 0, w)
+        assert_scores_close(g, o, i64(inp.n_chunks))
+        # entries past each sequence's end are left untouched
+        gh = f64(g)
+        for b, n in enumerate(i64(inp.n_chunks)):
+            assert np.all(np.isnan(gh[b, n:]))
+    status_clean()
+
+
+# ---------------------------------------------------------------- selection --
+
+def run_topk(scores, n_chunks, k_per_seq, max_kept):
+    B = scores.shape[0]
+    kept = torch.full((B, max_kept), -7, dtype=torch.int32, device=DEV)
+    n_kept = torch.zeros(B, dtype=torch.int32, device=DEV)
+    cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu)
+    return kept, n_kept, cu
+
+
+@pytest.mark.parametrize("name", ["tiny", "128k", "500k", "1m_host", "batched"])
+def test_topk_matches_oracle(name):
+    inp = workloads.make_inputs(name, DEV, pools=False, layers=1)
+    n, k = i64(inp.n_chunks), i64(inp.k_per_seq)
+    g = score_on_gpu(inp)
+    kept, n_kept, cu = run_topk(g, inp.n_chunks, inp.k_per_seq, int(k.max()) + 1)
+    got = kept_from_gpu(kept, n_kept)
+    # same decision in the same precision: the oracle's selection run on the GPU's fp32 scores
+    ref_same = oracle.topk_chunks(f64(g), n, k)
+    for b in range(len(n)):
+        assert got[b] == list(ref_same[b]), f"seq {b}"
+    # against the oracle's own fp64 scores, with the tie window
+    assert_kept_matches(got, oracle_scores(inp), n, k)
+    assert i64(cu).tolist() == oracle.cumulative_kept(ref_same).tolist()
+    if inp.layers[0].planted is not None:
+        planted = set(inp.layers[0].planted.tolist())
+        recall = len(planted & set(got[0])) / len(planted)
+        print(f"planted-chunk recall {recall:.2f}")  # diagnostic only
+    status_clean()
+
+
+def test_topk_edge_cases():
+    cases = [(0, 3), (1, 0), (1, 5), (2, 0), (2, 1), (5, 4), (5, 10), (64, 8), (3000, 300), (16384, 1638),
+             (4097, 4095), (100, 0), (777, 776), (1025, 513)]
+    B = len(cases)
+    M = max(c[0] for c in cases)
+    rng = np.random.default_rng(5)
+    scores = np.zeros((B, M), dtype=np.float32)
+    for b, (n, _) in enumerate(cases):
+        kind = b % 4
+        if kind == 0:
+            scores[b, :n] = 0.25                                     # all ties
+        elif kind == 1:
+            scores[b, :n] = rng.integers(-3, 4, n) * 0.5             # heavy ties, negatives
+        elif kind == 2:
+            scores[b, :n] = rng.standard_normal(n)
+        else:
+            v = rng.standard_normal(n).astype(np.float32)
+            v[::7] = 0.0
+            v[3::7] = -0.0                                           # signed zeros tie
+            scores[b, :n] = v
+    n_chunks = torch.tensor([c[0] for c in cases], dtype=torch.int32, device=DEV)
+    k_per_seq = torch.tensor([c[1] for c in cases], dtype=torch.int32, device=DEV)
+    kept, n_kept, cu = run_topk(torch.from_numpy(scores).to(DEV), n_chunks, k_per_seq, M)
+    got = kept_from_gpu(kept, n_kept)
+    ref = oracle.topk_chunks(scores.astype(np.float64), i64(n_chunks), i64(k_per_seq))
+    for b in range(B):
+        assert got[b] == list(ref[b]), f"case {cases[b]}"
+    assert i64(cu).tolist() == oracle.cumulative_kept(ref).tolist()
+    status_clean()
+
+
+def test_topk_nan_and_inf_order():
+    s = np.array([[1.0, np.nan, np.inf, -np.inf, 2.0, np.nan, 0.5, 0.0]], dtype=np.float32)
+    n = torch.tensor([8], dtype=torch.int32, device=DEV)
+    for K in range(0, 8):
+        k = torch.tensor([K], dtype=torch.int32, device=DEV)
+        kept, n_kept, _ = run_topk(torch.from_numpy(s).to(DEV), n, k, 8)
+        ref = oracle.topk_chunks(s.astype(np.float64), [8], [K])
+        assert kept_from_gpu(kept, n_kept)[0] == list(ref[0]), K
+    status_clean()
+
+
+# ------------------------------------------------------------------ gather --
+
+def paged_case(B=6, seed=3, max_chunks=40):
+    rng = np.random.default_rng(seed)
+    n = rng.integers(1, max_chunks + 1, B)
+    n[1] = 1
+    n_slots = int(n.sum()) + 5
+    perm = rng.permutation(n_slots)
+    table = np.zeros((B, max_chunks), dtype=np.int32)
+    off = 0
+    for b in range(B):
+        table[b, : n[b]] = perm[off: off + n[b]]
+        off += n[b]
+    k = np.array([max(0, int(x) // 3) for x in n])
+    return n.astype(np.int32), k.astype(np.int32), table, n_slots
+
+
+def test_gather_paged_bit_exact():
+    n, k, table, n_slots = paged_case()
+    B, M = table.shape
+    g = torch.Generator(device=DEV).manual_seed(11)
+    shape = (n_slots, 8, 64, 128)
+    k_pool = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    v_pool = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    scores = torch.rand((B, M), generator=g, device=DEV)
+    n_t = torch.from_numpy(n).to(DEV)
+    k_t = torch.from_numpy(k).to(DEV)
+    tab = torch.from_numpy(table).to(DEV)
+    kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
+    buf_chunks = int((k + 1).sum())
+    kb = torch.zeros((buf_chunks,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    vb = torch.zeros_like(kb)
+    lsa.lsa_gather_chunks(k_pool, v_pool, tab, kept, cu, M, kb, vb)
+    kept_l = kept_from_gpu(kept, n_kept)
+    rk, rv, rcu = oracle.gather_chunks(k_pool.view(torch.int16).cpu().numpy(), v_pool.view(torch.int16).cpu().numpy(),
+                                       table, kept_l, M)
+    total = int(rcu[-1])
+    assert np.array_equal(kb[:total].view(torch.int16).cpu().numpy(), rk)
+    assert np.array_equal(vb[:total].view(torch.int16).cpu().numpy(), rv)
+    status_clean()
+
+
+# --------------------------------------------------------------- attention --
+
+def ragged_buffers(n_kept, seed=21):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    total = int(sum(n_kept))
+    shape = (max(total, 1), 8, 64, 128)
+    kb = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    vb = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(n_kept)]), dtype=torch.int32, device=DEV)
+    q = torch.randn((len(n_kept), 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    return q, kb, vb, cu
+
+
+def run_attn(q, kb, vb, cu):
+    B = q.shape[0]
+    out = torch.full((B, 64, 128), float("nan"), device=DEV)
+    ws = lsa.new_attn_workspace(B)
+    lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out, ws)
+    return out, ws
+
+
+@pytest.mark.parametrize("n_kept", [[1], [9], [257], [1, 0, 37, 3, 150, 9], [0, 0, 5, 0], [2] * 40,
+                                    [300, 1, 1, 1, 1, 1, 1, 1, 299]])
+def test_attention_ragged_matches_oracle(n_kept):
+    q, kb, vb, cu = ragged_buffers(n_kept)
+    out, _ = run_attn(q, kb, vb, cu)
+    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu))
+    assert_attention_close(out, ref)
+    status_clean()
+
+
+def test_attention_closed_forms():
+    n_kept = [3, 70]
+    q, kb, vb, cu = ragged_buffers(n_kept, seed=4)
+    kb[:] = kb[0, 0, 0]                       # identical keys: output = mean of V
+    out, _ = run_attn(q, kb, vb, cu)
+    o = f64(out)
+    c = i64(cu)
+    for b in range(2):
+        for h in (0, 13, 63):
+            mean = f64(vb[c[b]: c[b + 1], h // 8]).reshape(-1, 128).mean(axis=0)
+            np.testing.assert_allclose(o[b, h], mean, atol=2e-3, rtol=1e-3)
+    # GQA mapping: V of KV head g is the constant g + 1
+    q, kb, vb, cu = ragged_buffers(n_kept, seed=5)
+    for g in range(8):
+        vb[:, g] = g + 1.0
+    out, _ = run_attn(q, kb, vb, cu)
+    o = f64(out)
+    for h in range(64):
+        np.testing.assert_allclose(o[:, h], h // 8 + 1.0, rtol=1e-5)
+    status_clean()
+
+
+def test_attention_deterministic_and_workspace_reusable():
+    q, kb, vb, cu = ragged_buffers([400, 3, 77])
+    out1, ws = run_attn(q, kb, vb, cu)
+    out2 = torch.empty_like(out1)
+    for _ in range(3):
+        lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out2, ws)
+    assert torch.equal(out1, out2)
+    # every call leaves the ticket counters at zero
+    assert int(ws[: 3 * 8 * 4].view(torch.int32).abs().sum()) == 0
+    status_clean()
+
+
+def test_attention_scale_argument():
+    q, kb, vb, cu = ragged_buffers([5])
+    out = torch.empty((1, 64, 128), device=DEV)
+    ws = lsa.new_attn_workspace(1)
+    lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out, ws, softmax_scale=0.3)
+    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), scale=0.3)
+    assert_attention_close(out, ref)
+
+
+# ------------------------------------------------------------ whole window --
+
+def f32(t: torch.Tensor) -> np.ndarray:
+    """Exact float32 host copy of a bf16 tensor (half the memory of float64)."""
+    return t.detach().float().cpu().numpy()
+
+
+def window_parity(name, steps, layer=0, window=0, heads=None, seqs=None, **kw):
+    inp = workloads.make_inputs(name, DEV, layers=1, **kw)
+    L = inp.layers[layer]
+    lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, DEV)
+    lw.select(L.q_idx[window], L.w, L.chunk_keys)
+    if inp.workload.host_pool:
+        lw.fetch(L.k_pool, L.v_pool)
+    else:
+        lw.gather(L.k_pool, L.v_pool)
+    outs = {}
+    for t in steps:
+        out = torch.empty((inp.batch, 64, 128), device=DEV)
+        lw.attend(L.q[window, t], out)
+        outs[t] = out
+    torch.cuda.synchronize()
+    status_clean()
+    # scores and selection
+    n, k = i64(inp.n_chunks), i64(inp.k_per_seq)
+    o_scores = oracle_scores(inp, layer, window)
+    assert_scores_close(lw.scores, o_scores, n)
+    got = lw.kept_lists()
+    assert_kept_matches(got, o_scores, n, k)
+    cu = i64(lw.cu_kept[0])
+    total = int(cu[-1])
+    # gather: every kept chunk equals its pool slot, bit for bit
+    table = i64(inp.chunk_table)
+    idx = torch.tensor([int(table[b, c]) for b in range(inp.batch) for c in got[b]], device=L.k_pool.device)
+    assert torch.equal(lw.k_bufs[0][:total], L.k_pool[idx].to(DEV))
+    assert torch.equal(lw.v_bufs[0][:total], L.v_pool[idx].to(DEV))
+    # attention at the sampled steps: the oracle on the kept set the GPU chose
+    kb, vb = f32(lw.k_bufs[0][:total]), f32(lw.v_bufs[0][:total])
+    errs = []
+    for t in steps:
+        ref = oracle.sparse_decode_attn(f64(L.q[window, t]), kb, vb, cu, heads=heads, seqs=seqs)
+        errs.append(assert_attention_close(outs[t], ref, heads=heads, seqs=seqs))
+    return inp, lw, outs, errs
+
+
+def test_window_tiny_full():
+    """Whole window of the tiny workload, all 64 steps, against the oracle's own window."""
+    inp = workloads.make_inputs("tiny", DEV)
+    L = inp.layers[0]
+    lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, DEV)
+    outs = torch.empty((64, 1, 64, 128), device=DEV)
+    lw.run_window(L.q_idx[0], L.w, L.chunk_keys, L.k_pool, L.v_pool, L.q[0], outs)
+    torch.cuda.synchronize()
+    status_clean()
+    scores, kept, cu, o_outs = oracle.decode_window(
+        f64(L.q_idx[0]), f64(L.w), f64(L.chunk_keys), i64(inp.chunk_table), i64(inp.n_chunks),
+        i64(inp.k_per_seq), f64(L.k_pool), f64(L.v_pool), f64(L.q[0]), inp.max_chunks)
+    assert_scores_close(lw.scores, scores, i64(inp.n_chunks))
+    assert lw.kept_lists()[0] == list(kept[0])
+    for t in range(64):
+        assert_attention_close(outs[t], o_outs[t])
+
+
+def test_window_128k_sampled_steps():
+    window_parity("128k", steps=[0, 31, 63], window=1)
+
+
+@pytest.mark.slow
+def test_window_500k_sampled_steps():
+    window_parity("500k", steps=[0, 63], heads=[0, 9, 18, 27, 36, 45, 54, 63])
+
+
+@pytest.mark.slow
+def test_window_batched_one_layer_sampled():
+    window_parity("batched", steps=[0, 63], heads=[0, 15, 22, 31, 36, 47, 53, 63])
+
+
+@pytest.mark.slow
+def test_window_1m_host_tier_sampled():
+    inp, lw, outs, errs = window_parity("1m_host", steps=[0], heads=[0, 27, 63])
+
+
+# ------------------------------------------------------------ host fetch ----
+
+def test_fetch_from_host_equals_gather():
+    n, k, table, n_slots = paged_case(B=4, seed=9, max_chunks=30)
+    B, M = table.shape
+    g = torch.Generator(device=DEV).manual_seed(12)
+    shape = (n_slots, 8, 64, 128)
+    k_dev = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    v_dev = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    k_host = k_dev.cpu().pin_memory()
+    v_host = v_dev.cpu().pin_memory()
+    scores = torch.rand((B, M), generator=g, device=DEV)
+    n_t, k_t, tab = (torch.from_numpy(x).to(DEV) for x in (n, k, table))
+    kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
+    buf = int((k + 1).sum())
+    a_k = torch.zeros((buf,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    a_v, b_k, b_v = torch.zeros_like(a_k), torch.zeros_like(a_k), torch.zeros_like(a_k)
+    lsa.lsa_gather_chunks(k_dev, v_dev, tab, kept, cu, M, a_k, a_v)
+    side = torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    side.wait_stream(torch.cuda.current_stream())
+    lsa.lsa_fetch_from_host(k_host, v_host, tab, kept, cu, M, b_k, b_v, num_ctas=16, stream=side, done_event=ev)
+    torch.cuda.current_stream().wait_event(ev)
+    assert torch.equal(a_k, b_k) and torch.equal(a_v, b_v)
+    status_clean()
+
+
+def test_fetch_rejects_unpinned_pool():
+    k_host = torch.zeros((4, 8, 64, 128), dtype=torch.bfloat16)     # pageable
+    kept = torch.zeros((1, 2), dtype=torch.int32, device=DEV)
+    cu = torch.tensor([0, 1], dtype=torch.int32, device=DEV)
+    buf = torch.zeros((2, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(lsa.LsaError, match="NOT_PINNED"):
+        lsa.lsa_fetch_from_host(k_host, k_host, None, kept, cu, 4, buf, buf)
+
+
+# ------------------------------------------------------- device-side errors --
+
+def test_device_errors_are_reported_not_trapped():
+    shape = (4, 8, 64, 128)
+    pool = torch.zeros(shape, dtype=torch.bfloat16, device=DEV)
+    buf = torch.zeros((2,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    kept = torch.tensor([[0, 9]], dtype=torch.int32, device=DEV)      # 9 >= max_chunks (4)
+    cu = torch.tensor([0, 2], dtype=torch.int32, device=DEV)
+    lsa.lsa_gather_chunks(pool, pool, None, kept, cu, 4, buf, buf)
+    assert lsa.read_device_status() & 4                                 # BAD_CHUNK
+    table = torch.tensor([[0, 1, 2, 77]], dtype=torch.int32, device=DEV)  # slot 77 >= n_slots
+    kept = torch.tensor([[0, 3]], dtype=torch.int32, device=DEV)
+    lsa.lsa_gather_chunks(pool, pool, table, kept, cu, 4, buf, buf)
+    assert lsa.read_device_status() & 2                                 # BAD_SLOT
+    cu_big = torch.tensor([0, 3], dtype=torch.int32, device=DEV)        # 3 chunks > buffer of 2
+    lsa.lsa_gather_chunks(pool, pool, None, kept, cu_big, 4, buf, buf)
+    assert lsa.read_device_status() & 8                                 # CAPACITY
+    q = torch.zeros((1, 64, 128), dtype=torch.bfloat16, device=DEV)
+    out = torch.zeros((1, 64, 128), device=DEV)
+    ws = lsa.new_attn_workspace(1)
+    lsa.lsa_sparse_decode_attn(q, buf, buf, cu_big, out, ws)
+    assert lsa.read_device_status() & 8
+    keys = torch.zeros((4, 128), dtype=torch.bfloat16, device=DEV)
+    scores = torch.zeros((1, 4), device=DEV)
+    lsa.lsa_index_score(torch.zeros((1, 16, 128), dtype=torch.bfloat16, device=DEV),
+                        torch.ones(16, device=DEV), keys, None,
+                        torch.tensor([5], dtype=torch.int32, device=DEV), scores)
+    assert lsa.read_device_status() & 1                                 # BAD_COUNT
+    assert lsa.read_device_status() == 0

@@ -164,9 +164,10 @@ def lengths_for(wl: Workload, base_seed: int = BASE_SEED):
 
 def make_inputs(name_or_wl, device="cuda", base_seed: int = BASE_SEED, layers: Optional[int] = None,
                 windows: Optional[int] = None, steps: int = TAU, chunks: Optional[int] = None,
-                k: Optional[int] = None, batch: Optional[int] = None) -> Inputs:
+                k: Optional[int] = None, batch: Optional[int] = None, pools: bool = True) -> Inputs:
     """Draw every input of a workload.  ``chunks``/``k``/``batch`` override the
-    sizes (used for reduced parity cases with the same distributions)."""
+    sizes (used for reduced parity cases with the same distributions); with
+    ``pools=False`` the KV pools are left out (scoring and selection only)."""
     wl = WORKLOADS[name_or_wl] if isinstance(name_or_wl, str) else name_or_wl
     if chunks is not None or k is not None or batch is not None:
         wl = dataclasses.replace(
@@ -216,7 +217,9 @@ def make_inputs(name_or_wl, device="cuda", base_seed: int = BASE_SEED, layers: O
         else:
             chunk_keys = randn_bf16((n_slots, INDEX_DIM), _seed(base_seed, "keys", l), device)
         shape = (n_slots, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM)
-        if wl.host_pool:
+        if not pools:
+            k_pool = v_pool = None
+        elif wl.host_pool:
             k_pool = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
             v_pool = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
             randn_bf16(shape, _seed(base_seed, "kpool", l), device, out=k_pool)
