@@ -205,6 +205,37 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
                            float softmax_scale, float* out, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/*
+ * lsa_sparse_decode_attn_noalloc -- lsa_sparse_decode_attn without a
+ * caller-provided workspace, for callers that cannot allocate device memory:
+ * programs with no device allocator of their own, plug-ins inside a framework
+ * that owns all device memory and forbids cudaMalloc after start-up, and
+ * latency-critical loops that must not call cudaMalloc (it can synchronise the
+ * device).  The pages have no counterpart of this call; it is a convenience of
+ * this library.
+ *
+ * The split-K scratch lives in a fixed array inside the library
+ * (LSA_NOALLOC_SCRATCH_BYTES of device memory, held by every GPU that loads
+ * the library until the process exits).  The caller still owns and passes q,
+ * the compact buffers, cu_kept and out; arguments, results and device errors
+ * are those of lsa_sparse_decode_attn.  Limits: B <= LSA_NOALLOC_MAX_BATCH
+ * and a device of at most LSA_NOALLOC_MAX_CTAS SMs, otherwise
+ * LSA_ERR_UNSUPPORTED_SHAPE.  The call allocates nothing (no cudaMalloc, no
+ * cudaFree).  Its first call on a device looks up the array's device address
+ * and sets the kernel's shared-memory limit; make that first call before any
+ * stream capture.  Every call on a device uses the same array: calls whose
+ * work may overlap on the GPU (other streams, other host threads) race and
+ * must be serialised by the caller.  Each call clears the array's counters on
+ * `stream` before its kernel runs.
+ */
+#define LSA_NOALLOC_MAX_BATCH 32
+#define LSA_NOALLOC_MAX_CTAS 256
+/* 1 KiB of counters + (32*8 + 256) partial records of 1032 floats. */
+#define LSA_NOALLOC_SCRATCH_BYTES 2114560
+int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, const void* v_buf,
+                                   int64_t buf_chunks, const int32_t* cu_kept, int B,
+                                   float softmax_scale, float* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -58,6 +58,7 @@ def _load():
         "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
         "lsa_attn_workspace_size": ([I], S),
         "lsa_sparse_decode_attn": ([P, P, P, I64, P, I, F, P, P, S, P], I),
+        "lsa_sparse_decode_attn_noalloc": ([P, P, P, I64, P, I, F, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -217,9 +218,29 @@ def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_sca
         _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
+def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=None, stream=None):
+    """lsa_sparse_decode_attn without a workspace argument, for callers that cannot
+    allocate device memory; its scratch is a fixed array inside the library, shared
+    by every call on the device (calls that may overlap on the GPU must be
+    serialised by the caller).  At most 32 sequences."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_buf, "k_buf", torch.bfloat16)
+    _need(v_buf, "v_buf", torch.bfloat16)
+    _need(cu_kept, "cu_kept", torch.int32)
+    _need(out, "out", torch.float32)
+    B = q.shape[0]
+    if tuple(q.shape) != (B, NUM_Q_HEADS, HEAD_DIM) or tuple(out.shape) != (B, NUM_Q_HEADS, HEAD_DIM):
+        raise ValueError("q and out must be [B, 64, 128]")
+    if k_buf.shape != v_buf.shape or cu_kept.numel() != B + 1:
+        raise ValueError("bad shapes")
+    scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
+    _check("lsa_sparse_decode_attn_noalloc", _load().lsa_sparse_decode_attn_noalloc(
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(out), _stream(stream)))
+
+
 __all__ = [
     "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_attn_workspace_size", "new_attn_workspace",
-    "lsa_sparse_decode_attn", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
+    "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

@@ -466,3 +466,103 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// lsa_sparse_decode_attn_noalloc: the same decode step for callers that cannot
+// allocate device memory.  Some callers have no device allocator of their own
+// (a plain C host program, or a plug-in living inside a framework that owns
+// all device memory and forbids cudaMalloc once it has started), and some
+// cannot allocate at the moment they call (cudaMalloc may synchronise the
+// device, which a latency-critical decode loop must not do).  For them the
+// split-K scratch (ticket counters and partial results) lives in a fixed
+// array inside this library instead of a caller-provided workspace.
+//
+// The array is a file-scope __device__ variable of LSA_NOALLOC_SCRATCH_BYTES
+// bytes: every GPU that loads the library holds it until the process exits.
+// Its size fixes the limits: at most LSA_NOALLOC_MAX_BATCH sequences and a
+// grid of at most LSA_NOALLOC_MAX_CTAS CTAs (one per SM); larger requests are
+// rejected with LSA_ERR_UNSUPPORTED_SHAPE.  All calls on a device share the
+// one array, so calls whose kernels may overlap on the GPU (different
+// streams, or different host threads) race with each other and must be
+// serialised by the caller.  The ticket counters are cleared on the stream
+// before every launch, so leftovers of an earlier call do not matter.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocCounterBytes =
+    ((static_cast<size_t>(LSA_NOALLOC_MAX_BATCH) * lsa::kNumKVHeads * 4 + 255) / 256) * 256;
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocCounterBytes + (static_cast<size_t>(LSA_NOALLOC_MAX_BATCH) * lsa::kNumKVHeads + LSA_NOALLOC_MAX_CTAS) *
+                               lsa::attn::kRecFloats * sizeof(float);
+static_assert(kNoAllocScratchBytes == LSA_NOALLOC_SCRATCH_BYTES, "header constant out of date");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+bool g_noalloc_attr_set[64] = {};
+
+// Device address of the scratch array for the current device.  The host-side
+// symbol is only a stand-in, so the address is looked up once per device
+// (with that device current) through cudaGetSymbolAddress.
+int noalloc_setup(int dev, void** scratch) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return LSA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  if (!g_noalloc_attr_set[dev]) {
+    if (cudaFuncSetAttribute(lsa::attn::sparse_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lsa::attn::kSmemBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return LSA_ERR_CUDA;
+    }
+    g_noalloc_attr_set[dev] = true;
+  }
+  *scratch = g_noalloc_ptr[dev];
+  return LSA_OK;
+}
+}  // namespace
+
+extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, const void* v_buf,
+                                              int64_t buf_chunks, const int32_t* cu_kept, int B,
+                                              float softmax_scale, float* out, void* stream) {
+  using namespace lsa;
+  if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
+  if (B > LSA_NOALLOC_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (buf_chunks > (int64_t{1} << 22)) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out)) return LSA_ERR_MISALIGNED;
+  const int sms = device_sm_count();
+  if (sms <= 0) return LSA_ERR_NO_DEVICE;
+  const int grid = sms < attn::kMaxCtas ? sms : attn::kMaxCtas;
+  if (grid > LSA_NOALLOC_MAX_CTAS) return LSA_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return LSA_ERR_NO_DEVICE;
+  }
+  void* scratch = nullptr;
+  int st = noalloc_setup(dev, &scratch);
+  if (st != LSA_OK) return st;
+  CUtensorMap tm_k, tm_v;
+  st = encode_kv_map(&tm_k, k_buf, buf_chunks);
+  if (st != LSA_OK) return st;
+  st = encode_kv_map(&tm_v, v_buf, buf_chunks);
+  if (st != LSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* counters = static_cast<int*>(scratch);
+  float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocCounterBytes);
+  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(B) * kNumKVHeads * sizeof(int), s) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  const float scale_log2 = softmax_scale * 1.4426950408889634f;
+  attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
+      tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks, scale_log2, out, counters, records,
+      lsa_device_status_ptr());
+  return launch_status();
+}
