@@ -358,6 +358,58 @@ def run_e2e(args, inp, lws, dev, stream):
             "d2h_bytes_per_step": d2h, "steps": steps, "api": "kv_chunk_selection_b200.window.LayerWindow"}
 
 
+def run_attn_only(args):
+    """Attention launches alone over a random compact buffer of the workload's
+    kept size (no pools, no selection): the small case for kernel profiling."""
+    import kv_chunk_selection_b200 as lsa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = workloads.WORKLOADS[args.workload]
+    n, k = workloads.lengths_for(wl)
+    kept = [min(int(kb), int(nb) - 1) + 1 if int(nb) > 0 else 0 for nb, kb in zip(n, k)]
+    B = len(kept)
+    cu = torch.tensor([0] + list(torch.tensor(kept).cumsum(0).tolist()), dtype=torch.int32, device=dev)
+    total = int(sum(kept))
+    shape = (total, 8, 64, 128)
+    kbuf = workloads.randn_bf16(shape, 1, dev)
+    vbuf = workloads.randn_bf16(shape, 2, dev)
+    qs = workloads.randn_bf16((workloads.TAU, B, 64, 128), 3, dev)
+    out = torch.empty((B, 64, 128), device=dev)
+    ws = lsa.new_attn_workspace(B, dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        lsa.lsa_sparse_decode_attn(qs[0], kbuf, vbuf, cu, out, ws)     # first call sets kernel attributes
+    torch.cuda.synchronize()
+    # One graph of `steps` back-to-back launches (as in a decode window), replayed:
+    # events bracket whole replays, so host launch cost is not timed.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            lsa.lsa_sparse_decode_attn(qs[i % workloads.TAU], kbuf, vbuf, cu, out, ws)
+    for _ in range(max(1, args.warmup // max(1, args.steps))):
+        graph.replay()
+    torch.cuda.synchronize()
+    per_launch = []
+    for _ in range(args.repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        with torch.cuda.stream(stream):
+            graph.replay()
+        b.record(stream)
+        b.synchronize()
+        per_launch.append(a.elapsed_time(b) / 1e3 / args.steps)
+    torch.cuda.synchronize()
+    bits = lsa.read_device_status()
+    times = sorted(per_launch)
+    nbytes = total * 2 * workloads.CHUNK_BYTES_ONE + B * (64 * 128 * 2 + 64 * 128 * 4)
+    peak, kind = measured_peaks()
+    med = times[len(times) // 2]
+    return {"mode": "attn-only", "workload": args.workload, "kept_chunks": total, "launches_per_replay": args.steps,
+            "replays": args.repeats, "median_us": med * 1e6, "min_us": times[0] * 1e6, "bytes_per_launch": nbytes,
+            "median_gbs": nbytes / med / 1e9, "frac_of_measured": nbytes / med / 1e9 / peak,
+            "peak_source": kind, "device_status": bits, "source_digest": source_digest()}
+
+
 # ---------------------------------------------------------- oracle (CPU) arm --
 
 def _blas_threads():
@@ -472,6 +524,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--fetch-ctas", type=int, default=64)
+    ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
+    ap.add_argument("--attn-only", action="store_true",
+                    help="time attention launches alone on a random compact buffer (profiling case)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -479,6 +534,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.attn_only:
+        print(json.dumps(run_attn_only(args)), flush=True)
+        return
 
     if args.impl == "reference":
         line = run_reference(args, rank, world)

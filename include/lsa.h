@@ -80,6 +80,7 @@ typedef enum {
 #define LSA_DEV_ERR_CAPACITY 8u    /* compact buffer or kept row too small        */
 #define LSA_DEV_ERR_TIMEOUT 16u    /* a bounded in-kernel wait ran out            */
 #define LSA_DEV_ERR_WORKSPACE 32u  /* attention workspace not zero-initialised    */
+#define LSA_DEV_ERR_INTERNAL 64u   /* launch-layout assumption violated (a bug)    */
 
 /* Human-readable name of an lsa_status value. */
 const char* lsa_status_string(int status);
@@ -219,7 +220,7 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
  * the library until the process exits).  The caller still owns and passes q,
  * the compact buffers, cu_kept and out; arguments, results and device errors
  * are those of lsa_sparse_decode_attn.  Limits: B <= LSA_NOALLOC_MAX_BATCH
- * and a device of at most LSA_NOALLOC_MAX_CTAS SMs, otherwise
+ * and a device of at most 256 SMs (two CTAs per SM), otherwise
  * LSA_ERR_UNSUPPORTED_SHAPE.  The call allocates nothing (no cudaMalloc, no
  * cudaFree).  Its first call on a device looks up the array's device address
  * and sets the kernel's shared-memory limit; make that first call before any
@@ -229,9 +230,9 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
  * `stream` before its kernel runs.
  */
 #define LSA_NOALLOC_MAX_BATCH 32
-#define LSA_NOALLOC_MAX_CTAS 256
-/* 1 KiB of counters + (32*8 + 256) partial records of 1032 floats. */
-#define LSA_NOALLOC_SCRATCH_BYTES 2114560
+#define LSA_NOALLOC_MAX_CTAS 512
+/* 1 KiB of counters + (32*8 + 512) partial records of 1032 floats. */
+#define LSA_NOALLOC_SCRATCH_BYTES 3171328
 int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, const void* v_buf,
                                    int64_t buf_chunks, const int32_t* cu_kept, int B,
                                    float softmax_scale, float* out, void* stream);

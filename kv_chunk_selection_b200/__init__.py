@@ -27,7 +27,8 @@ INDEX_HEADS = 16
 INDEX_DIM = 128
 CHUNK_BYTES = NUM_KV_HEADS * CHUNK_TOKENS * HEAD_DIM * 2
 
-DEV_ERR_BITS = {1: "BAD_COUNT", 2: "BAD_SLOT", 4: "BAD_CHUNK", 8: "CAPACITY", 16: "TIMEOUT", 32: "WORKSPACE"}
+DEV_ERR_BITS = {1: "BAD_COUNT", 2: "BAD_SLOT", 4: "BAD_CHUNK", 8: "CAPACITY", 16: "TIMEOUT", 32: "WORKSPACE",
+                64: "INTERNAL"}
 
 _lib = None
 

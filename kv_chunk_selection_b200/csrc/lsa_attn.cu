@@ -40,22 +40,31 @@ namespace attn {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kStages = 6;
+constexpr int kStages = 3;
+constexpr int kCtasPerSm = 2;                // two CTAs share each SM (8 consumer warps)
 constexpr int kBoxBytes = 8192;              // 64 tokens x 64 dims of bf16
 constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo, V hi
 constexpr int kAccStride = 132;              // padded row of the combine buffer
 constexpr int kRecFloats = kGroup * kHeadDim + kGroup;  // partial o[8][128] + lse[8]
 constexpr int kMaxCtas = 1024;
-constexpr int kSmemBytes = 1024 /*align*/ + kStages * kStageBytes +
+constexpr int kSmemBytes = kStages * kStageBytes +
                            kConsumerWarps * kGroup * kAccStride * 4 + 2 * kConsumerWarps * kGroup * 4 +
                            2 * kStages * 8 + 16;
 
-// CTA that owns unit u when T units are cut into G equal contiguous ranges
-// [floor(T c / G), floor(T (c+1) / G)).
-__device__ __forceinline__ int cta_of(int64_t u, int64_t T, int G) {
-  return static_cast<int>(((u + 1) * G - 1) / T);
-}
-__device__ __forceinline__ int64_t range_lo(int c, int64_t T, int G) { return T * c / G; }
+// T units cut into G contiguous ranges: the first `rem` CTAs take base + 1
+// units, the others base (base = T / G, rem = T % G).  Everything is 32-bit
+// (T <= 8 * 2^22).  When T < G the CTAs c >= T are empty and sit after every
+// non-empty one, so the CTAs between the first and last owner of any unit
+// range all own part of it.
+struct Partition {
+  int base, rem;
+  __device__ Partition(int T, int G) : base(T / G), rem(T % G) {}
+  __device__ int start(int c) const { return c * base + min(c, rem); }
+  __device__ int cta_of(int u) const {
+    const int big = rem * (base + 1);
+    return u < big ? u / (base + 1) : rem + (u - big) / base;
+  }
+};
 
 // Largest b in [0, B) with 8 * cu[b] <= u (the sequence that holds unit u).
 __device__ __forceinline__ int seq_of_unit(const int32_t* cu, int B, int64_t u) {
@@ -88,13 +97,22 @@ struct UnitCursor {
   }
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Grid: kCtasPerSm CTAs per SM, capped at kMaxCtas.
+inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasPerSm : kMaxCtas; }
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu, int B,
                           int64_t buf_chunks, float scale_log2, float* __restrict__ out,
                           int* __restrict__ counters, float* __restrict__ records, unsigned* status) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte TMA swizzle pattern repeats every 1024 bytes and the fragment
+  // addressing below assumes each box starts on such a boundary.
+  if (smem_u32(smem_raw) & 1023u) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   float* accbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);
   float* mbuf = accbuf + kConsumerWarps * kGroup * kAccStride;
   float* lbuf = mbuf + kConsumerWarps * kGroup;
@@ -114,9 +132,10 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     if (blockIdx.x == 0 && tid == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
     return;
   }
-  const int64_t T = 8 * static_cast<int64_t>(total);
+  const int T = 8 * total;
   const int G = gridDim.x;
-  const int64_t u0 = range_lo(blockIdx.x, T, G), u1 = range_lo(blockIdx.x + 1, T, G);
+  const Partition part(T, G);
+  const int64_t u0 = part.start(blockIdx.x), u1 = part.start(blockIdx.x + 1);
 
   // Sequences without kept chunks get zeros.
   for (int b = blockIdx.x; b < B; b += G) {
@@ -191,6 +210,14 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   const int vrow = warp * 16 + r8 + ((mi >> 1) << 3);
   const int vx = mi & 1;
   const uint32_t smem_base = smem_u32(smem);
+  // Swizzled byte offsets of this lane's ldmatrix rows within a stage, for the
+  // 8 k-steps of S^T (K boxes) and the 8 dim tiles of O^T (V boxes).
+  uint32_t kofs[8], vofs[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    kofs[t] = (t >> 2) * kBoxBytes + krow * 128 + ((((t & 3) * 2 + kx) ^ (krow & 7)) << 4);
+    vofs[t] = 2 * kBoxBytes + (t >> 2) * kBoxBytes + vrow * 128 + ((((t & 3) * 2 + vx) ^ (vrow & 7)) << 4);
+  }
 
   UnitCursor cur;
   cur.start(cu, B, u0);
@@ -232,16 +259,13 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
       }
       if (ok) {
-        const uint32_t kbase = smem_base + s * kStageBytes;
-        const uint32_t vbase = kbase + 2 * kBoxBytes;
+        const uint32_t sbase = smem_base + s * kStageBytes;
         // ---- S^T[16 tokens x 8 heads] = K[16 x 128] Q^T[128 x 8] ----------
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          const uint32_t addr = kbase + (t >> 2) * kBoxBytes + krow * 128 +
-                                ((((t & 3) * 2 + kx) ^ (krow & 7)) << 4);
           uint32_t a0, a1, a2, a3;
-          ldmatrix_x4(addr, a0, a1, a2, a3);
+          ldmatrix_x4(sbase + kofs[t], a0, a1, a2, a3);
           mma_bf16_16816((t & 1) ? sb : sa, a0, a1, a2, a3, bq[t][0], bq[t][1]);
         }
         // s[0]: (token gl, head 2c4)  s[1]: (gl, 2c4+1)  s[2]: (gl+8, 2c4)  s[3]: (gl+8, 2c4+1)
@@ -261,12 +285,16 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         const uint32_t pbot = pack_bf16(fast_exp2(s2 - mn0), fast_exp2(s3 - mn1));
         l0 = l0 * al0 + bf16_lo(ptop) + bf16_lo(pbot);
         l1 = l1 * al1 + bf16_hi(ptop) + bf16_hi(pbot);
+        // Rescale only when some running max moved (warp-uniform branch); once
+        // the maxima settle, alpha is exactly 1 and the 32 multiplies are skipped.
+        if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          acc[i][0] *= al0;
-          acc[i][1] *= al1;
-          acc[i][2] *= al0;
-          acc[i][3] *= al1;
+          for (int i = 0; i < 8; ++i) {
+            acc[i][0] *= al0;
+            acc[i][1] *= al1;
+            acc[i][2] *= al0;
+            acc[i][3] *= al1;
+          }
         }
         // P^T as the B operand (k = token, n = head): transpose the 8x8 blocks.
         const uint32_t pb0 = movmatrix_trans(ptop);
@@ -274,10 +302,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         // ---- O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] P^T[16 x 8] ---
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint32_t addr = vbase + (i >> 2) * kBoxBytes + vrow * 128 +
-                                ((((i & 3) * 2 + vx) ^ (vrow & 7)) << 4);
           uint32_t a0, a1, a2, a3;
-          ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+          ldmatrix_x4_trans(sbase + vofs[i], a0, a1, a2, a3);
           mma_bf16_16816(acc[i], a0, a1, a2, a3, pb0, pb1);
         }
       }
@@ -343,10 +369,9 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       named_barrier(1, kConsumerThreads);
       // Contributing CTAs of pair p: those whose unit range meets [a_p, a_p + n_b).
       const int64_t a_p = 8 * static_cast<int64_t>(cb) + static_cast<int64_t>(g) * n_b;
-      const int c_lo = cta_of(a_p, T, G), c_hi = cta_of(a_p + n_b - 1, T, G);
+      const int c_lo = part.cta_of(static_cast<int>(a_p)), c_hi = part.cta_of(static_cast<int>(a_p + n_b - 1));
       if (tid == 0) {
-        int n_contrib = 0;
-        for (int c = c_lo; c <= c_hi; ++c) n_contrib += (range_lo(c + 1, T, G) > range_lo(c, T, G));
+        const int n_contrib = c_hi - c_lo + 1;   // every CTA in [c_lo, c_hi] owns part of the pair
         const int old = atomicAdd(&counters[p], 1);
         if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
         flags[1] = (old == n_contrib - 1);
@@ -354,22 +379,39 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       named_barrier(1, kConsumerThreads);
       if (flags[1]) {
         __threadfence();
-        float lse_max = -INFINITY;
-        for (int c = c_lo; c <= c_hi; ++c) {
-          if (range_lo(c + 1, T, G) == range_lo(c, T, G)) continue;
-          const float* rc = records + static_cast<int64_t>(p + c) * kRecFloats;
-          lse_max = fmaxf(lse_max, __ldcg(rc + kGroup * kHeadDim + hh));
-        }
-        float den = 0.f, r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int c = c_lo; c <= c_hi; ++c) {
-          if (range_lo(c + 1, T, G) == range_lo(c, T, G)) continue;
-          const float* rc = records + static_cast<int64_t>(p + c) * kRecFloats;
-          const float wgt = fast_exp2(__ldcg(rc + kGroup * kHeadDim + hh) - lse_max);
-          den += wgt;
-          const float4 x0 = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
-          const float4 x1 = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0) + 1);
-          r[0] += wgt * x0.x; r[1] += wgt * x0.y; r[2] += wgt * x0.z; r[3] += wgt * x0.w;
-          r[4] += wgt * x1.x; r[5] += wgt * x1.y; r[6] += wgt * x1.z; r[7] += wgt * x1.w;
+        // Merge the partials of pair p in CTA order.  Records of the
+        // contributing CTAs are contiguous (index p + c).  The log-sum-exps of
+        // all of them are staged in shared memory (the combine buffer is free
+        // now), then every thread folds its 8 dims of one head, with the
+        // record loads unrolled so several are in flight.
+        const int n_rec = c_hi - c_lo + 1;
+        const float* rbase = records + static_cast<int64_t>(p + c_lo) * kRecFloats;
+        float* lse_s = accbuf;                 // [n_rec chunk of 512][8]
+        float lse_max = -INFINITY, den = 0.f;
+        float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c0 = 0; c0 < n_rec; c0 += 512) {
+          const int nc = min(512, n_rec - c0);
+          for (int i = tid; i < nc * kGroup; i += kConsumerThreads)
+            lse_s[i] = __ldcg(rbase + static_cast<int64_t>(c0 + (i >> 3)) * kRecFloats + kGroup * kHeadDim + (i & 7));
+          named_barrier(1, kConsumerThreads);
+          float m_new = lse_max;
+          for (int c = 0; c < nc; ++c) m_new = fmaxf(m_new, lse_s[c * kGroup + hh]);
+          const float resc = fast_exp2(lse_max - m_new);   // 0 on the first chunk
+          den *= resc;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) r[k] *= resc;
+          lse_max = m_new;
+#pragma unroll 8
+          for (int c = 0; c < nc; ++c) {
+            const float* rc = rbase + static_cast<int64_t>(c0 + c) * kRecFloats + hh * kHeadDim + d0;
+            const float4 x0 = __ldcg(reinterpret_cast<const float4*>(rc));
+            const float4 x1 = __ldcg(reinterpret_cast<const float4*>(rc) + 1);
+            const float wgt = fast_exp2(lse_s[c * kGroup + hh] - lse_max);
+            den += wgt;
+            r[0] += wgt * x0.x; r[1] += wgt * x0.y; r[2] += wgt * x0.z; r[3] += wgt * x0.w;
+            r[4] += wgt * x1.x; r[5] += wgt * x1.y; r[6] += wgt * x1.z; r[7] += wgt * x1.w;
+          }
+          named_barrier(1, kConsumerThreads);
         }
         const float id = 1.f / den;
         reinterpret_cast<float4*>(dst)[0] = make_float4(r[0] * id, r[1] * id, r[2] * id, r[3] * id);
@@ -457,7 +499,7 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
   const size_t cnt_bytes = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
   int* counters = static_cast<int*>(workspace);
   float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cnt_bytes);
-  const int grid = sms < attn::kMaxCtas ? sms : attn::kMaxCtas;
+  const int grid = attn::grid_for(sms);
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks, scale_log2, out, counters, records,
@@ -480,7 +522,7 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
 // The array is a file-scope __device__ variable of LSA_NOALLOC_SCRATCH_BYTES
 // bytes: every GPU that loads the library holds it until the process exits.
 // Its size fixes the limits: at most LSA_NOALLOC_MAX_BATCH sequences and a
-// grid of at most LSA_NOALLOC_MAX_CTAS CTAs (one per SM); larger requests are
+// grid of at most LSA_NOALLOC_MAX_CTAS CTAs (two per SM); larger requests are
 // rejected with LSA_ERR_UNSUPPORTED_SHAPE.  All calls on a device share the
 // one array, so calls whose kernels may overlap on the GPU (different
 // streams, or different host threads) race with each other and must be
@@ -538,7 +580,7 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out)) return LSA_ERR_MISALIGNED;
   const int sms = device_sm_count();
   if (sms <= 0) return LSA_ERR_NO_DEVICE;
-  const int grid = sms < attn::kMaxCtas ? sms : attn::kMaxCtas;
+  const int grid = attn::grid_for(sms);
   if (grid > LSA_NOALLOC_MAX_CTAS) return LSA_ERR_UNSUPPORTED_SHAPE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
