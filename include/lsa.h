@@ -170,6 +170,12 @@ int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_
                         int B, int max_chunks, int max_kept, void* k_buf, void* v_buf,
                         int64_t buf_chunks, int num_ctas, void* stream, void* done_event);
 
+/* Flags of lsa_sparse_decode_attn. */
+/* The kernel that ran just before this call on `stream` did not write k_buf,
+ * v_buf or cu_kept (true for every decode step of a window after the first):
+ * the call may then stream K/V while that kernel is still finishing. */
+#define LSA_ATTN_KV_UNCHANGED 1u
+
 /*
  * Bytes of workspace lsa_sparse_decode_attn needs for a batch of B sequences.
  * The workspace must be zero-filled once before its first use; every call
@@ -198,13 +204,18 @@ size_t lsa_attn_workspace_size(int B);
  *   out          device fp32 [B][64][128]
  *   workspace    device, >= lsa_attn_workspace_size(B) bytes, zero-filled
  *                before first use.
+ *   flags        0 or LSA_ATTN_KV_UNCHANGED.  The kernel is launched as a
+ *                programmatic dependent of the preceding kernel on `stream`
+ *                (its start overlaps that kernel's tail); it waits for that
+ *                kernel before reading q or cu_kept (without the flag) and
+ *                before writing out or the workspace.
  * B <= LSA_MAX_BATCH.  Device errors: CAPACITY (cu_kept[B] > buf_chunks or
  * cu_kept decreasing: nothing is computed), TIMEOUT, WORKSPACE.
  */
 int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
                            int64_t buf_chunks, const int32_t* cu_kept, int B,
                            float softmax_scale, float* out, void* workspace,
-                           size_t workspace_bytes, void* stream);
+                           size_t workspace_bytes, unsigned int flags, void* stream);
 
 /*
  * lsa_sparse_decode_attn_noalloc -- lsa_sparse_decode_attn without a

@@ -58,7 +58,7 @@ def _load():
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
         "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
         "lsa_attn_workspace_size": ([I], S),
-        "lsa_sparse_decode_attn": ([P, P, P, I64, P, I, F, P, P, S, P], I),
+        "lsa_sparse_decode_attn": ([P, P, P, I64, P, I, F, P, P, S, ctypes.c_uint, P], I),
         "lsa_sparse_decode_attn_noalloc": ([P, P, P, I64, P, I, F, P, P], I),
     }
     for name, (args, res) in sig.items():
@@ -200,8 +200,16 @@ def new_attn_workspace(B: int, device=None) -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_scale=None, stream=None):
-    """out[b,h] = softmax(scale q[b,h] K^T) V over the kept tokens of KV head h // 8."""
+ATTN_KV_UNCHANGED = 1
+
+
+def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_scale=None, stream=None,
+                           kv_unchanged=False):
+    """out[b,h] = softmax(scale q[b,h] K^T) V over the kept tokens of KV head h // 8.
+
+    ``kv_unchanged=True`` tells the library that the kernel just before this
+    call on the stream did not write k_buf, v_buf or cu_kept (every decode step
+    of a window after the first), so K/V streaming may overlap its tail."""
     _need(q, "q", torch.bfloat16)
     _need(k_buf, "k_buf", torch.bfloat16)
     _need(v_buf, "v_buf", torch.bfloat16)
@@ -216,7 +224,7 @@ def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_sca
     scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
     _check("lsa_sparse_decode_attn", _load().lsa_sparse_decode_attn(
         _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(out),
-        _ptr(workspace), workspace.numel(), _stream(stream)))
+        _ptr(workspace), workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
 
 
 def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=None, stream=None):

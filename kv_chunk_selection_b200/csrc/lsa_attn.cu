@@ -104,7 +104,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu, int B,
                           int64_t buf_chunks, float scale_log2, float* __restrict__ out,
-                          int* __restrict__ counters, float* __restrict__ records, unsigned* status) {
+                          int* __restrict__ counters, float* __restrict__ records, unsigned* status,
+                          int kv_unchanged) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte TMA swizzle pattern repeats every 1024 bytes and the fragment
   // addressing below assumes each box starts on such a boundary.
@@ -123,6 +124,11 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
+  // With kv_unchanged the caller guarantees that the preceding kernel on the
+  // stream did not write k_buf, v_buf or cu_kept, so those may be read before
+  // it has finished; everything else (q, out, the workspace) waits for it.
+  if (!kv_unchanged) griddep_wait();
+
   // ---- validate cu_kept (every thread reaches the same verdict) -------------
   const int total = __ldg(cu + B);
   int bad = (__ldg(cu) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) ? 1 : 0;
@@ -137,14 +143,21 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   const Partition part(T, G);
   const int64_t u0 = part.start(blockIdx.x), u1 = part.start(blockIdx.x + 1);
 
-  // Sequences without kept chunks get zeros.
-  for (int b = blockIdx.x; b < B; b += G) {
-    if (__ldg(cu + b + 1) == __ldg(cu + b)) {
-      float4* o = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * kNumQHeads * kHeadDim);
-      for (int i = tid; i < kNumQHeads * kHeadDim / 4; i += kThreads) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // Sequences without kept chunks get zeros (written after the wait).
+  auto zero_empty = [&](int first, int stride) {
+    for (int b = blockIdx.x; b < B; b += G) {
+      if (__ldg(cu + b + 1) == __ldg(cu + b)) {
+        float4* o = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * kNumQHeads * kHeadDim);
+        for (int i = first; i < kNumQHeads * kHeadDim / 4; i += stride) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
+  };
+  if (u0 >= u1) {
+    if (kv_unchanged) griddep_wait();
+    zero_empty(tid, kThreads);
+    griddep_launch_dependents();
+    return;
   }
-  if (u0 >= u1) return;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -156,6 +169,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     mbar_fence_init();
   }
   __syncthreads();
+  griddep_launch_dependents();
   volatile int* abort_flag = flags;
 
   if (warp == kConsumerWarps) {
@@ -201,6 +215,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   }
 
   // ========================= consumer warps ==================================
+  if (kv_unchanged) griddep_wait();
+  zero_empty(tid, kConsumerThreads);
   const int gl = lane >> 2;   // row group of the mma fragments
   const int c4 = lane & 3;    // column pair of the mma fragments
   const int mi = lane >> 3, r8 = lane & 7;
@@ -380,38 +396,41 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       if (flags[1]) {
         __threadfence();
         // Merge the partials of pair p in CTA order.  Records of the
-        // contributing CTAs are contiguous (index p + c).  The log-sum-exps of
-        // all of them are staged in shared memory (the combine buffer is free
-        // now), then every thread folds its 8 dims of one head, with the
-        // record loads unrolled so several are in flight.
+        // contributing CTAs are contiguous (index p + c).  They are folded in
+        // batches of 8 with a running log-sum-exp: each batch issues all of
+        // its loads (8 lse + 16 float4 per thread) before using any, so a
+        // batch costs one L2 round trip.
         const int n_rec = c_hi - c_lo + 1;
         const float* rbase = records + static_cast<int64_t>(p + c_lo) * kRecFloats;
-        float* lse_s = accbuf;                 // [n_rec chunk of 512][8]
         float lse_max = -INFINITY, den = 0.f;
         float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int c0 = 0; c0 < n_rec; c0 += 512) {
-          const int nc = min(512, n_rec - c0);
-          for (int i = tid; i < nc * kGroup; i += kConsumerThreads)
-            lse_s[i] = __ldcg(rbase + static_cast<int64_t>(c0 + (i >> 3)) * kRecFloats + kGroup * kHeadDim + (i & 7));
-          named_barrier(1, kConsumerThreads);
+        for (int c0 = 0; c0 < n_rec; c0 += 8) {
+          float lse[8];
+          float4 x[8][2];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int c = min(c0 + k, n_rec - 1);   // tail lanes re-read the last record (weight 0)
+            const float* rc = rbase + static_cast<int64_t>(c) * kRecFloats;
+            lse[k] = __ldcg(rc + kGroup * kHeadDim + hh);
+            x[k][0] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
+            x[k][1] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0) + 1);
+          }
           float m_new = lse_max;
-          for (int c = 0; c < nc; ++c) m_new = fmaxf(m_new, lse_s[c * kGroup + hh]);
-          const float resc = fast_exp2(lse_max - m_new);   // 0 on the first chunk
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (c0 + k < n_rec) m_new = fmaxf(m_new, lse[k]);
+          const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
           den *= resc;
 #pragma unroll
           for (int k = 0; k < 8; ++k) r[k] *= resc;
           lse_max = m_new;
-#pragma unroll 8
-          for (int c = 0; c < nc; ++c) {
-            const float* rc = rbase + static_cast<int64_t>(c0 + c) * kRecFloats + hh * kHeadDim + d0;
-            const float4 x0 = __ldcg(reinterpret_cast<const float4*>(rc));
-            const float4 x1 = __ldcg(reinterpret_cast<const float4*>(rc) + 1);
-            const float wgt = fast_exp2(lse_s[c * kGroup + hh] - lse_max);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float wgt = (c0 + k < n_rec) ? fast_exp2(lse[k] - lse_max) : 0.f;
             den += wgt;
-            r[0] += wgt * x0.x; r[1] += wgt * x0.y; r[2] += wgt * x0.z; r[3] += wgt * x0.w;
-            r[4] += wgt * x1.x; r[5] += wgt * x1.y; r[6] += wgt * x1.z; r[7] += wgt * x1.w;
+            r[0] += wgt * x[k][0].x; r[1] += wgt * x[k][0].y; r[2] += wgt * x[k][0].z; r[3] += wgt * x[k][0].w;
+            r[4] += wgt * x[k][1].x; r[5] += wgt * x[k][1].y; r[6] += wgt * x[k][1].z; r[7] += wgt * x[k][1].w;
           }
-          named_barrier(1, kConsumerThreads);
         }
         const float id = 1.f / den;
         reinterpret_cast<float4*>(dst)[0] = make_float4(r[0] * id, r[1] * id, r[2] * id, r[3] * id);
@@ -466,10 +485,11 @@ size_t lsa_attn_workspace_size(int B) {
 
 int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
                            const int32_t* cu_kept, int B, float softmax_scale, float* out, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+                           size_t workspace_bytes, unsigned int flags, void* stream) {
   using namespace lsa;
   if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
+  if (flags & ~static_cast<unsigned>(LSA_ATTN_KV_UNCHANGED)) return LSA_ERR_INVALID_ARG;
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   // TMA row coordinates are 32-bit: (buf_chunks * 512) rows must fit.
   if (buf_chunks > (int64_t{1} << 22)) return LSA_ERR_UNSUPPORTED_SHAPE;
@@ -499,11 +519,27 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
   const size_t cnt_bytes = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
   int* counters = static_cast<int*>(workspace);
   float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cnt_bytes);
-  const int grid = attn::grid_for(sms);
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
-  attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks, scale_log2, out, counters, records,
-      lsa_device_status_ptr());
+  // Launched as a programmatic dependent of the preceding kernel: its
+  // prologue (and, with LSA_ATTN_KV_UNCHANGED, its K/V stream) overlaps the
+  // tail of that kernel; the kernel waits for it before touching its outputs.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(attn::grid_for(sms));
+  cfg.blockDim = dim3(attn::kThreads);
+  cfg.dynamicSmemBytes = attn::kSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int kv_unchanged = (flags & LSA_ATTN_KV_UNCHANGED) ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, attn::sparse_decode_attn_kernel, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
+                         cu_kept, B, buf_chunks, scale_log2, out, counters, records, lsa_device_status_ptr(),
+                         kv_unchanged) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -605,6 +641,6 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
       tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks, scale_log2, out, counters, records,
-      lsa_device_status_ptr());
+      lsa_device_status_ptr(), 0);
   return launch_status();
 }

@@ -69,17 +69,20 @@ class LayerWindow:
                             self.max_chunks, self.k_bufs[buf], self.v_bufs[buf], num_ctas=num_ctas,
                             stream=stream, done_event=done_event)
 
-    def attend(self, q, out, buf: int = 0, stream=None):
-        """One decode step: out[B, 64, 128] fp32 from q[B, 64, 128] bf16."""
+    def attend(self, q, out, buf: int = 0, stream=None, kv_unchanged: bool = False):
+        """One decode step: out[B, 64, 128] fp32 from q[B, 64, 128] bf16.
+
+        ``kv_unchanged``: the previous kernel on the stream did not write this
+        window's compact buffer or offsets (true for every step but the first)."""
         lsa_sparse_decode_attn(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], out, self.workspace,
-                               stream=stream)
+                               stream=stream, kv_unchanged=kv_unchanged)
 
     def run_window(self, q_idx, w, chunk_keys, k_pool, v_pool, q_steps, outs, stream=None):
         """Select, gather, then one attention call per step of ``q_steps`` [T, B, 64, 128]."""
         self.select(q_idx, w, chunk_keys, 0, stream)
         self.gather(k_pool, v_pool, 0, stream)
         for t in range(q_steps.shape[0]):
-            self.attend(q_steps[t], outs[t], 0, stream)
+            self.attend(q_steps[t], outs[t], 0, stream, kv_unchanged=t > 0)
 
     def kept_lists(self, buf: int = 0):
         """Host copy of the kept chunk lists (for inspection and tests)."""

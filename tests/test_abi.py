@@ -70,7 +70,7 @@ def test_host_checks_null_pointers(L):
     assert L.lsa_topk_chunks(n, n, n, 1, 1, 1, n, n, n, n) == INVALID
     assert L.lsa_gather_chunks(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, n) == INVALID
     assert L.lsa_fetch_from_host(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, 0, n, n) == INVALID
-    assert L.lsa_sparse_decode_attn(n, n, n, 1, n, 1, 0.1, n, n, 0, n) == INVALID
+    assert L.lsa_sparse_decode_attn(n, n, n, 1, n, 1, 0.1, n, n, 0, 0, n) == INVALID
     assert L.lsa_read_device_status(n, None) == INVALID
 
 
@@ -82,16 +82,17 @@ def test_host_checks_sizes_and_alignment(L):
     assert L.lsa_index_score(ok, ok, ok, 4, None, ok, 0, 4, ok, None) == INVALID
     assert L.lsa_topk_chunks(ok, ok, ok, 1, 4, 0, ok, ok, ok, None) == INVALID
     assert L.lsa_topk_chunks(ok, ok, ok, LSA_MAX_BATCH + 1, 4, 2, ok, ok, ok, None) == UNSUPPORTED
-    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, -1.0, ok, ok, 1 << 30, None) == INVALID
-    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, LSA_MAX_BATCH + 1, 0.1, ok, ok, 1 << 30, None) == UNSUPPORTED
-    assert L.lsa_sparse_decode_attn(ok, ok, ok, (1 << 22) + 1, ok, 1, 0.1, ok, ok, 1 << 30, None) == UNSUPPORTED
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, -1.0, ok, ok, 1 << 30, 0, None) == INVALID
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, 1 << 30, 2, None) == INVALID   # unknown flag
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, LSA_MAX_BATCH + 1, 0.1, ok, ok, 1 << 30, 0, None) == UNSUPPORTED
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, (1 << 22) + 1, ok, 1, 0.1, ok, ok, 1 << 30, 0, None) == UNSUPPORTED
     # misaligned bf16 arrays
     assert L.lsa_index_score(odd, ok, ok, 4, None, ok, 1, 4, ok, None) == MISALIGNED
     assert L.lsa_gather_chunks(ok, odd, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, None) == MISALIGNED
-    assert L.lsa_sparse_decode_attn(ok, ok, odd, 4, ok, 1, 0.1, ok, ok, 1 << 30, None) == MISALIGNED
+    assert L.lsa_sparse_decode_attn(ok, ok, odd, 4, ok, 1, 0.1, ok, ok, 1 << 30, 0, None) == MISALIGNED
     assert L.lsa_fetch_from_host(odd, ok, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, 0, None, None) == MISALIGNED
     # workspace too small
-    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, 16, None) == WORKSPACE
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, 16, 0, None) == WORKSPACE
 
 
 LSA_MAX_BATCH = 4096
@@ -101,7 +102,7 @@ LSA_MAX_BATCH = 4096
 def test_no_device_answer(L):
     ok = ctypes.c_void_p(0x100000)
     ws = L.lsa_attn_workspace_size(1)
-    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, ws, None) == NO_DEVICE
+    assert L.lsa_sparse_decode_attn(ok, ok, ok, 4, ok, 1, 0.1, ok, ok, ws, 0, None) == NO_DEVICE
     assert L.lsa_gather_chunks(ok, ok, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, None) == NO_DEVICE
     bits = ctypes.c_uint(0)
     assert L.lsa_read_device_status(None, ctypes.byref(bits)) == NO_DEVICE

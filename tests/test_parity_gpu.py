@@ -247,6 +247,41 @@ def test_attention_deterministic_and_workspace_reusable():
     status_clean()
 
 
+def test_attention_overlapped_steps_match():
+    """Steps launched with kv_unchanged (K/V streamed while the previous step's
+    merge finishes) give bit-identical results, also right after a gather."""
+    n, k, table, n_slots = paged_case(B=5, seed=15, max_chunks=60)
+    B, M = table.shape
+    g = torch.Generator(device=DEV).manual_seed(16)
+    shape = (n_slots, 8, 64, 128)
+    k_pool = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    v_pool = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    n_t, k_t, tab = (torch.from_numpy(x).to(DEV) for x in (n, k, table))
+    scores = torch.rand((B, M), generator=g, device=DEV)
+    kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
+    buf = int((k + 1).sum())
+    kb = torch.empty((buf,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    vb = torch.empty_like(kb)
+    qs = torch.randn((6, B, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    ws = lsa.new_attn_workspace(B)
+    ref = torch.empty((6, B, 64, 128), device=DEV)
+    got = torch.empty_like(ref)
+    lsa.lsa_gather_chunks(k_pool, v_pool, tab, kept, cu, M, kb, vb)
+    for t in range(6):
+        lsa.lsa_sparse_decode_attn(qs[t], kb, vb, cu, ref[t], ws)
+    torch.cuda.synchronize()
+    kb.zero_()
+    vb.zero_()
+    lsa.lsa_gather_chunks(k_pool, v_pool, tab, kept, cu, M, kb, vb)   # rewrite, then overlap the steps
+    for t in range(6):
+        lsa.lsa_sparse_decode_attn(qs[t], kb, vb, cu, got[t], ws, kv_unchanged=t > 0)
+    torch.cuda.synchronize()
+    assert torch.equal(ref, got)
+    o = oracle.sparse_decode_attn(f64(qs[3]), f64(kb), f64(vb), i64(cu))
+    assert_attention_close(got[3], o)
+    status_clean()
+
+
 def test_attention_scale_argument():
     q, kb, vb, cu = ragged_buffers([5])
     out = torch.empty((1, 64, 128), device=DEV)

@@ -61,7 +61,7 @@ def test_noalloc_matches_workspace_entry_point_twice(L):
     ref = torch.empty((B, 64, 128), device=DEV)
     ws = torch.zeros(L.lsa_attn_workspace_size(B), dtype=torch.uint8, device=DEV)
     assert L.lsa_sparse_decode_attn(_p(q), _p(kb), _p(vb), kb.shape[0], _p(cu), B, scale, _p(ref), _p(ws),
-                                    ws.numel(), stream) == 0
+                                    ws.numel(), 0, stream) == 0
 
     for call in range(2):
         out = torch.full((B, 64, 128), float("nan"), device=DEV)
