@@ -161,6 +161,16 @@ def window_bytes(n_chunks, kept_total, layers):
     return per_layer * layers, attn_launch, int(n.sum())
 
 
+def combine_ranks(elapsed_s: float, tokens_per_rank: float, world: int, device="cpu"):
+    """Whole-job result of `world` replicas: the slowest rank's time (max over
+    ranks) and the tokens of all ranks divided by it."""
+    if world > 1:
+        t = torch.tensor([elapsed_s], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_s = float(t.item())
+    return elapsed_s, world * tokens_per_rank / elapsed_s
+
+
 # -------------------------------------------------------------- our arm ------
 
 def run_ours(args, rank, world, local_rank):
@@ -256,14 +266,9 @@ def run_ours(args, rank, world, local_rank):
     bits = lsa.read_device_status()
     if bits:
         raise RuntimeError(f"device status after timing: {lsa.decode_status(bits)}")
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed = float(t.item())
-
     # tok/s/layer: every window decodes 64 tokens per sequence in each layer; a
     # window of `layers` layers takes `elapsed / steps`, i.e. 1/layers of it per layer.
-    value = world * workloads.TAU * B * layers * args.steps / elapsed
+    elapsed, value = combine_ranks(elapsed, workloads.TAU * B * layers * args.steps, world, dev)
     kept_total = int(lws[0].cu_kept[0][-1].item())
     wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers)
     hbm_gbs = wbytes * args.steps / elapsed / 1e9
