@@ -171,6 +171,122 @@ def combine_ranks(elapsed_s: float, tokens_per_rank: float, world: int, device="
     return elapsed_s, world * tokens_per_rank / elapsed_s
 
 
+def h2d_probe_gbs(device, nbytes=1 << 30, reps=5):
+    """Pinned host to device copy bandwidth in the same run (the host link)."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    best = float("inf")
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        d.copy_(h, non_blocking=True)
+        e.record()
+        e.synchronize()
+        best = min(best, s.elapsed_time(e) / 1e3)
+    del h, d
+    return nbytes / best / 1e9
+
+
+def run_host_tier(args, rank, world, local_rank):
+    """Host-tier window pipeline: while the main stream runs the 64 attention
+    steps of window w over compact buffer w % 2, a side stream scores and selects
+    window w + 1 and fetches its kept chunks from the page-locked host pool into
+    the other buffer.  The indexer query of window w + 1 is taken as known when
+    window w starts (the selection looks one window ahead), which is what lets the
+    fetch hide behind attention."""
+    import kv_chunk_selection_b200 as lsa
+    from kv_chunk_selection_b200.window import LayerWindow
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lsa.lib()
+    inp = workloads.make_inputs(args.workload, dev, base_seed=workloads.BASE_SEED + rank)
+    assert len(inp.layers) == 1
+    L = inp.layers[0]
+    B, n_win = inp.batch, inp.workload.windows
+    lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev, double_buffer=True)
+    out = torch.empty((workloads.TAU, B, 64, 128), device=dev)
+    main, side = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    n_total = args.steps + args.warmup
+    ev_fetched = [torch.cuda.Event() for _ in range(n_total + 1)]
+    ev_attn_done = [torch.cuda.Event() for _ in range(n_total)]
+    f0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_total + 1)]
+    f1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_total + 1)]
+
+    def prepare(w):            # on the side stream: select + fetch window w into buffer w % 2
+        buf = w % 2
+        if w >= 2:
+            side.wait_event(ev_attn_done[w - 2])     # buffer w % 2 was read by window w - 2
+        with torch.cuda.stream(side):
+            lw.select(L.q_idx[w % n_win], L.w, L.chunk_keys, buf=buf)
+            f0[w].record(side)
+            lw.fetch(L.k_pool, L.v_pool, buf=buf, num_ctas=args.fetch_ctas)
+            f1[w].record(side)
+            ev_fetched[w].record(side)
+
+    def attend(w):             # on the main stream: 64 steps over buffer w % 2
+        main.wait_event(ev_fetched[w])
+        with torch.cuda.stream(main):
+            for t in range(workloads.TAU):
+                lw.attend(L.q[w % n_win, t], out[t], buf=w % 2, kv_unchanged=t > 0)
+            ev_attn_done[w].record(main)
+
+    probe = h2d_probe_gbs(dev)
+    copy_gbs = copy_probe_gbs(dev)
+    peak, peak_kind = measured_peaks()
+    prepare(0)
+    for w in range(args.warmup):
+        prepare(w + 1)
+        attend(w)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0.record(main)
+    for w in range(args.warmup, n_total):
+        prepare(w + 1)
+        attend(w)
+    t1.record(main)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    bits = lsa.read_device_status()
+    if bits:
+        raise RuntimeError(f"device status after timing: {lsa.decode_status(bits)}")
+    elapsed = t0.elapsed_time(t1) / 1e3
+    fetch_s = [f0[w].elapsed_time(f1[w]) / 1e3 for w in range(args.warmup + 1, n_total + 1)]
+    kept_total = int(lw.cu_kept[0][-1].item())
+    fetch_bytes = kept_total * 2 * workloads.CHUNK_BYTES_ONE
+    elapsed, value = combine_ranks(elapsed, workloads.TAU * B * args.steps, world, dev)
+    wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, 1)
+    fetch_gbs = fetch_bytes / statistics.median(fetch_s) / 1e9
+    window_s = elapsed / args.steps
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": window_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": inp.workload.description, "name": args.workload, "batch": B, "layers": 1,
+                   "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
+                   "tau": workloads.TAU, "schedule": "double-buffered: select + fetch of window w+1 on a side "
+                   "stream overlaps the 64 attention steps of window w", "fetch_ctas": args.fetch_ctas,
+                   "l2": "inputs larger than L2 (host pool 8 GiB, 410 MiB per attention launch)"},
+        "roofline": {"kernel": "gather_kernel (host-tier fetch)", "bound": "pcie", "achieved": fetch_gbs,
+                     "peak": probe, "unit": "GB/s", "frac": fetch_gbs / probe,
+                     "peak_source": "same-run pinned H2D copy probe (cudaMemcpyAsync, 1 GiB)", "traffic": None,
+                     "algorithmic_bytes_per_launch": fetch_bytes, "avg_launch_us": statistics.median(fetch_s) * 1e6},
+        "hbm": {"window_gbs": wbytes * args.steps / elapsed / 1e9, "copy_probe_gbs": copy_gbs,
+                "frac_of_measured": wbytes * args.steps / elapsed / 1e9 / peak},
+        "pcie": {"fetch_bytes_per_window": fetch_bytes, "fetch_gbs_median": fetch_gbs, "h2d_probe_gbs": probe,
+                 "window_bound_by_fetch_ms": fetch_bytes / probe / 1e6},
+        "gpu_launches": args.steps * (3 + workloads.TAU),
+        "clocks": clocks, "e2e": None,
+    }
+
+
 # -------------------------------------------------------------- our arm ------
 
 def run_ours(args, rank, world, local_rank):
@@ -561,7 +677,10 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        if workloads.WORKLOADS[args.workload].host_pool:
+            out = run_host_tier(args, rank, world, local_rank)
+        else:
+            out = run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.barrier()
