@@ -47,6 +47,9 @@ constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo
 constexpr int kAccStride = 132;              // padded row of the combine buffer
 constexpr int kRecFloats = kGroup * kHeadDim + kGroup;  // partial o[8][128] + lse[8]
 constexpr int kMaxCtas = 1024;
+constexpr int kRecBytes = kRecFloats * 4;    // 4128, a multiple of 16
+// Partial records that fit in the stage ring plus the combine buffer.
+constexpr int kStagedRecs = (kStages * kStageBytes + kConsumerWarps * kGroup * kAccStride * 4) / kRecBytes;
 constexpr int kSmemBytes = kStages * kStageBytes +
                            kConsumerWarps * kGroup * kAccStride * 4 + 2 * kConsumerWarps * kGroup * 4 +
                            2 * kStages * 8 + 16;
@@ -396,40 +399,74 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       if (flags[1]) {
         __threadfence();
         // Merge the partials of pair p in CTA order.  Records of the
-        // contributing CTAs are contiguous (index p + c).  They are folded in
-        // batches of 8 with a running log-sum-exp: each batch issues all of
-        // its loads (8 lse + 16 float4 per thread) before using any, so a
-        // batch costs one L2 round trip.
+        // contributing CTAs are contiguous (index p + c).
         const int n_rec = c_hi - c_lo + 1;
         const float* rbase = records + static_cast<int64_t>(p + c_lo) * kRecFloats;
         float lse_max = -INFINITY, den = 0.f;
         float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int c0 = 0; c0 < n_rec; c0 += 8) {
-          float lse[8];
-          float4 x[8][2];
+        if (u + (jend - j0) == u1) {
+          // Last segment of this CTA: the stage ring and the combine buffer
+          // are free, so whole batches of records are pulled into shared
+          // memory with asynchronous 16-byte copies (one L2 round trip per
+          // batch) and folded from there with a running log-sum-exp.
+          const float* srec = reinterpret_cast<const float*>(smem);
+          const char* gsrc = reinterpret_cast<const char*>(rbase);
+          for (int c0 = 0; c0 < n_rec; c0 += kStagedRecs) {
+            const int nc = min(kStagedRecs, n_rec - c0);
+            const char* g = gsrc + static_cast<int64_t>(c0) * kRecBytes;
+            for (int i = tid; i < nc * (kRecBytes / 16); i += kConsumerThreads)
+              cp_async_16_cg(smem_base + i * 16, g + static_cast<int64_t>(i) * 16);
+            cp_async_wait_all();
+            named_barrier(1, kConsumerThreads);
+            float m_new = lse_max;
+            for (int c = 0; c < nc; ++c) m_new = fmaxf(m_new, srec[c * kRecFloats + kGroup * kHeadDim + hh]);
+            const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
+            den *= resc;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int c = min(c0 + k, n_rec - 1);   // tail lanes re-read the last record (weight 0)
-            const float* rc = rbase + static_cast<int64_t>(c) * kRecFloats;
-            lse[k] = __ldcg(rc + kGroup * kHeadDim + hh);
-            x[k][0] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
-            x[k][1] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0) + 1);
+            for (int k = 0; k < 8; ++k) r[k] *= resc;
+            lse_max = m_new;
+#pragma unroll 4
+            for (int c = 0; c < nc; ++c) {
+              const float* rc = srec + c * kRecFloats;
+              const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - lse_max);
+              const float4 x0 = reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0)[0];
+              const float4 x1 = reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0)[1];
+              den += wgt;
+              r[0] += wgt * x0.x; r[1] += wgt * x0.y; r[2] += wgt * x0.z; r[3] += wgt * x0.w;
+              r[4] += wgt * x1.x; r[5] += wgt * x1.y; r[6] += wgt * x1.z; r[7] += wgt * x1.w;
+            }
+            named_barrier(1, kConsumerThreads);
           }
-          float m_new = lse_max;
+        } else {
+          // Mid-CTA (the producer may still be filling the ring): fold the
+          // records in batches of 8 from L2, all loads of a batch in flight.
+          for (int c0 = 0; c0 < n_rec; c0 += 8) {
+            float lse[8];
+            float4 x[8][2];
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (c0 + k < n_rec) m_new = fmaxf(m_new, lse[k]);
-          const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
-          den *= resc;
+            for (int k = 0; k < 8; ++k) {
+              const int c = min(c0 + k, n_rec - 1);   // tail lanes re-read the last record (weight 0)
+              const float* rc = rbase + static_cast<int64_t>(c) * kRecFloats;
+              lse[k] = __ldcg(rc + kGroup * kHeadDim + hh);
+              x[k][0] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
+              x[k][1] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0) + 1);
+            }
+            float m_new = lse_max;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) r[k] *= resc;
-          lse_max = m_new;
+            for (int k = 0; k < 8; ++k)
+              if (c0 + k < n_rec) m_new = fmaxf(m_new, lse[k]);
+            const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
+            den *= resc;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float wgt = (c0 + k < n_rec) ? fast_exp2(lse[k] - lse_max) : 0.f;
-            den += wgt;
-            r[0] += wgt * x[k][0].x; r[1] += wgt * x[k][0].y; r[2] += wgt * x[k][0].z; r[3] += wgt * x[k][0].w;
-            r[4] += wgt * x[k][1].x; r[5] += wgt * x[k][1].y; r[6] += wgt * x[k][1].z; r[7] += wgt * x[k][1].w;
+            for (int k = 0; k < 8; ++k) r[k] *= resc;
+            lse_max = m_new;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float wgt = (c0 + k < n_rec) ? fast_exp2(lse[k] - lse_max) : 0.f;
+              den += wgt;
+              r[0] += wgt * x[k][0].x; r[1] += wgt * x[k][0].y; r[2] += wgt * x[k][0].z; r[3] += wgt * x[k][0].w;
+              r[4] += wgt * x[k][1].x; r[5] += wgt * x[k][1].y; r[6] += wgt * x[k][1].z; r[7] += wgt * x[k][1].w;
+            }
           }
         }
         const float id = 1.f / den;

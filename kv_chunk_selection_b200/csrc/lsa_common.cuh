@@ -141,6 +141,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// Ampere-style asynchronous 16-byte copy global -> shared through L2 only
+// (.cg), and waits on the thread's outstanding copies (hardware waits).
+__device__ __forceinline__ void cp_async_16_cg(uint32_t smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Programmatic dependent launch: wait until the preceding grid on the stream
 // has completed and its writes are visible (a no-op without such a launch),
 // and allow the next grid to be scheduled before this one finishes.
