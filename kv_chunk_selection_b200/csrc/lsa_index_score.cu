@@ -7,27 +7,37 @@
 // (summary page, 3 Experiments, "Limitations"):
 //     score_c = sum_h w_h * sigmoid(q_h . k_c / sqrt(128)),  16 heads.
 //
-// B200 design: the [chunks x 128] x [128 x 16 heads] product is a dense
-// contraction, computed on the tensor cores with mma.sync m16n8k16 (M = 16
-// chunks, N = 8 heads, two N tiles).  Key rows are fetched straight from HBM
-// into the A fragments with 16-byte loads: the contraction index is permuted
-// consistently in A and B so that each lane's 16 bytes (8 consecutive dims of
-// one key row) feed two k-steps, and a warp instruction covers 8 rows x 64
-// contiguous bytes.  The sigmoid and the weighted head sum run in fp32 on the
-// accumulator fragments; a 2-step shuffle finishes each chunk's sum.
+// B200 design: per sequence the scores are one dense contraction
+// [chunks x 128] x [128 x 16 heads].  A CTA takes a tile of 128 chunks and
+// computes D[128 x 16] = K_tile Q^T on the 5th-generation tensor cores:
+// tcgen05.mma kind::f16 (M = 128 chunks, N = 16 heads, K = 16 per
+// instruction, 8 instructions), bf16 operands in shared memory in the
+// 128-byte swizzled K-major layout, the fp32 accumulator in tensor memory
+// (16 of the 32 allocated columns).  Key rows are gathered through the chunk
+// table with 16-byte loads (one row per thread) and written swizzled; one
+// thread issues the MMAs and commits them to an mbarrier; each warp then reads
+// its 32 TMEM lanes (one chunk per thread, 16 head logits) with tcgen05.ld and
+// applies the sigmoid and the weighted head sum in fp32.
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
 namespace lsa {
 namespace score {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kChunksPerCta = kWarps * 16;
+constexpr int kThreads = 128;       // one thread per chunk row = one TMEM lane
+constexpr int kTile = 128;          // chunks per CTA (MMA M)
+constexpr int kKBlockBytes = 128;   // 64 bf16 per row per swizzle atom
+constexpr int kABytes = kTile * 2 * kKBlockBytes;          // 32 KiB: 2 K-blocks of [128 x 128 B]
+constexpr int kBBytes = kIndexHeads * 2 * kKBlockBytes;    // 4 KiB: 2 K-blocks of [16 x 128 B]
+constexpr int kSmemBytes = kABytes + kBBytes + 64;
+constexpr uint32_t kTmemCols = 32;  // allocation unit (>= 16 accumulator columns)
+constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kTile, kIndexHeads);
 
-__device__ __forceinline__ float sigmoid_from_logit2(float neg_logit_log2) {
-  // sigmoid(x) = 1 / (1 + 2^(-x log2 e)); the argument is already -x log2 e.
-  return 1.f / (1.f + fast_exp2(neg_logit_log2));
+// Byte offset of the 16-byte piece j (0..15, 8 bf16 each) of row r in a
+// K-major SW128 operand with `rows` rows per K-block.
+__device__ __forceinline__ uint32_t sw128_offset(int r, int j, int rows) {
+  const int kb = j >> 3, jj = j & 7;
+  return kb * rows * kKBlockBytes + r * kKBlockBytes + ((jj ^ (r & 7)) << 4);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -35,73 +45,95 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
                    const __nv_bfloat16* __restrict__ keys, int64_t n_slots, const int32_t* __restrict__ table,
                    const int32_t* __restrict__ n_chunks, int max_chunks, float* __restrict__ scores,
                    float neg_scale_log2, unsigned* status) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   const int b = blockIdx.y;
   const int n = __ldg(n_chunks + b);
   if (n < 0 || n > max_chunks) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_BAD_COUNT);
     return;
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int base = blockIdx.x * kChunksPerCta + warp * 16;
+  const int base = blockIdx.x * kTile;
   if (base >= n) return;
-  const int gl = lane >> 2, c4 = lane & 3;
-
-  // B operand: Q^T for heads gl (tile 0) and 8+gl (tile 1); lane c4 holds dims
-  // [32 s + 8 c4, 32 s + 8 c4 + 8) of k-step pair s.
-  const uint4* q0 = reinterpret_cast<const uint4*>(q_idx + (static_cast<int64_t>(b) * kIndexHeads + gl) * kIndexDim);
-  const uint4* q1 = q0 + 8 * kIndexDim / 8;
-  uint4 qa[4], qb[4];
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    qa[s] = __ldg(q0 + 4 * s + c4);
-    qb[s] = __ldg(q1 + 4 * s + c4);
+  if (smem_u32(smem) & 1023u) {   // the swizzle atoms assume 1024-byte alignment
+    if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
+    return;
   }
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + kABytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kABytes + kBBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  const int tid = threadIdx.x, warp = tid >> 5;
 
-  // A operand rows: chunks base+gl and base+gl+8.
-  const int r0 = base + gl, r1 = base + gl + 8;
-  int64_t slot0 = -1, slot1 = -1;
-  if (r0 < n) slot0 = table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + r0)
-                            : static_cast<int64_t>(b) * max_chunks + r0;
-  if (r1 < n) slot1 = table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + r1)
-                            : static_cast<int64_t>(b) * max_chunks + r1;
-  bool bad0 = (r0 < n) && (slot0 < 0 || slot0 >= n_slots);
-  bool bad1 = (r1 < n) && (slot1 < 0 || slot1 >= n_slots);
-  if (bad0 || bad1) set_status(status, LSA_DEV_ERR_BAD_SLOT);
-  const bool ok0 = (r0 < n) && !bad0, ok1 = (r1 < n) && !bad1;
-  uint4 ka[4], kb[4];
-  const uint4 z = make_uint4(0, 0, 0, 0);
-  const uint4* k0 = reinterpret_cast<const uint4*>(keys + (ok0 ? slot0 : 0) * kIndexDim);
-  const uint4* k1 = reinterpret_cast<const uint4*>(keys + (ok1 ? slot1 : 0) * kIndexDim);
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    ka[s] = ok0 ? __ldg(k0 + 4 * s + c4) : z;
-    kb[s] = ok1 ? __ldg(k1 + 4 * s + c4) : z;
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
   }
 
-  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+  // A: key row of chunk base + tid, gathered through the chunk table.
+  const int c = base + tid;
+  bool ok = c < n;
+  int64_t slot = 0;
+  if (ok) {
+    slot = table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
+    if (slot < 0 || slot >= n_slots) {
+      set_status(status, LSA_DEV_ERR_BAD_SLOT);
+      ok = false;
+    }
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(keys + (ok ? slot : 0) * kIndexDim);
+    uint4 v[16];
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    mma_bf16_16816(d0, ka[s].x, kb[s].x, ka[s].y, kb[s].y, qa[s].x, qa[s].y);
-    mma_bf16_16816(d1, ka[s].x, kb[s].x, ka[s].y, kb[s].y, qb[s].x, qb[s].y);
-    mma_bf16_16816(d0, ka[s].z, kb[s].z, ka[s].w, kb[s].w, qa[s].z, qa[s].w);
-    mma_bf16_16816(d1, ka[s].z, kb[s].z, ka[s].w, kb[s].w, qb[s].z, qb[s].w);
+    for (int j = 0; j < 16; ++j) v[j] = ok ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) *reinterpret_cast<uint4*>(sa + sw128_offset(tid, j, kTile)) = v[j];
   }
-  // d0: heads 2c4, 2c4+1; d1: heads 8+2c4, 9+2c4.  [0],[1] chunk r0; [2],[3] chunk r1.
-  const float w0 = __ldg(w + 2 * c4), w1 = __ldg(w + 2 * c4 + 1);
-  const float w2 = __ldg(w + 8 + 2 * c4), w3 = __ldg(w + 9 + 2 * c4);
-  float p0 = w0 * sigmoid_from_logit2(d0[0] * neg_scale_log2) + w1 * sigmoid_from_logit2(d0[1] * neg_scale_log2) +
-             w2 * sigmoid_from_logit2(d1[0] * neg_scale_log2) + w3 * sigmoid_from_logit2(d1[1] * neg_scale_log2);
-  float p1 = w0 * sigmoid_from_logit2(d0[2] * neg_scale_log2) + w1 * sigmoid_from_logit2(d0[3] * neg_scale_log2) +
-             w2 * sigmoid_from_logit2(d1[2] * neg_scale_log2) + w3 * sigmoid_from_logit2(d1[3] * neg_scale_log2);
-  p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
-  p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
-  p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
-  p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
-  if (c4 == 0) {
-    float* row = scores + static_cast<int64_t>(b) * max_chunks;
-    if (ok0) row[r0] = p0;
-    if (ok1) row[r1] = p1;
+  // B: the 16 indexer query rows of sequence b (K-major, one row per head).
+  {
+    const uint4* qb = reinterpret_cast<const uint4*>(q_idx + static_cast<int64_t>(b) * kIndexHeads * kIndexDim);
+#pragma unroll
+    for (int i = tid; i < kIndexHeads * 16; i += kThreads) {
+      const int h = i >> 4, j = i & 15;
+      *reinterpret_cast<uint4*>(sb + sw128_offset(h, j, kIndexHeads)) = __ldg(qb + i);
+    }
   }
+  fence_proxy_async_smem();   // generic-proxy smem writes -> visible to the tensor core
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ad = umma_desc_kmajor_sw128(a0 + kb * kTile * kKBlockBytes + k * 32);
+        const uint64_t bd = umma_desc_kmajor_sw128(b0 + kb * kIndexHeads * kKBlockBytes + k * 32);
+        umma_bf16(tmem, ad, bd, kIdesc, (kb | k) != 0);
+      }
+    }
+    umma_commit(bar);
+  }
+  int never = 0;
+  // warp-uniform, so the .sync.aligned TMEM load below never diverges
+  const bool done = __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0, &never));
+  tcgen05_fence_after();
+  if (!done) {
+    if (tid == 0) set_status(status, LSA_DEV_ERR_TIMEOUT);
+  } else {
+    float logit[16];
+    tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16), logit);
+    float s = 0.f;
+#pragma unroll
+    for (int h = 0; h < kIndexHeads; ++h) s += __ldg(w + h) * (1.f / (1.f + fast_exp2(logit[h] * neg_scale_log2)));
+    if (ok) scores[static_cast<int64_t>(b) * max_chunks + c] = s;
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace score
@@ -116,9 +148,9 @@ extern "C" int lsa_index_score(const void* q_idx, const float* w, const void* ch
   if (B > 65535) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q_idx) || !aligned16(chunk_keys)) return LSA_ERR_MISALIGNED;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
-  const dim3 grid((max_chunks + score::kChunksPerCta - 1) / score::kChunksPerCta, B);
+  const dim3 grid((max_chunks + score::kTile - 1) / score::kTile, B);
   const float neg_scale_log2 = -1.4426950408889634f / sqrtf(static_cast<float>(kIndexDim));
-  score::index_score_kernel<<<grid, score::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+  score::index_score_kernel<<<grid, score::kThreads, score::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(chunk_keys), n_slots,
       chunk_table, n_chunks, max_chunks, scores, neg_scale_log2, lsa_device_status_ptr());
   return launch_status();
