@@ -7,13 +7,14 @@
 //
 // B200 design: one 1024-thread CTA per sequence runs an exact radix select on
 // a 32-bit key that orders scores descending (the float bits mapped to an
-// order-preserving unsigned and complemented).  Four 8-bit digit passes find
-// the boundary key; chunk index breaks ties among equal keys.  Histograms use
-// shared-memory atomics aggregated per warp with __match_any_sync, since the
-// high digits of scores in a narrow range are nearly all equal.  The kept set
-// is then written in index order with two block-wide prefix scans, so the
-// output is ascending without a sort.  Scores are read from L2 on each pass
-// (at most 64 KiB per sequence).
+// order-preserving unsigned and complemented); the chunk index breaks ties
+// among equal keys.  Each thread owns a contiguous run of candidates and keeps
+// their keys in registers (up to 16 per thread, N <= 16384; larger N re-reads
+// the scores).  The bits that every key shares (found from a block-wide min
+// and max) need no pass, so scores in a narrow range take 3 or fewer 8-bit
+// digit passes, each a shared-memory histogram and a 256-bin scan.  The kept
+// set is then written in index order with two block-wide prefix scans, so the
+// output is ascending without a sort.
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
@@ -76,6 +77,155 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return excl;
 }
 
+constexpr int kMaxPerThread = 16;   // candidates kept in registers per thread (N <= 16384)
+
+// Selects the kc smallest keys among candidates 0..cand-1 (kc < cand) and
+// writes their indices in ascending order to out[0..kc).  Thread t owns the
+// contiguous candidates [t*per, (t+1)*per); with kCached their keys live in
+// registers for all passes, otherwise they are re-read from the scores.
+template <bool kCached>
+__device__ void select_and_write(const float* __restrict__ sc, int cand, int kc, int per, int32_t* __restrict__ out,
+                                 int* hist, int* warp_sums, int* sel) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int lo = min(cand, tid * per), hi = min(cand, lo + per);
+  uint32_t kr[kCached ? kMaxPerThread : 1];
+  if (kCached) {
+#pragma unroll
+    for (int e = 0; e < kMaxPerThread; ++e) kr[e] = (lo + e < hi) ? desc_key(__ldg(sc + lo + e)) : 0u;
+  }
+  auto key_of = [&](int e) -> uint32_t { return kCached ? kr[e] : desc_key(__ldg(sc + lo + e)); };
+  const int n_own = hi - lo;
+
+  // Bits shared by every candidate key need no pass: start below the highest
+  // bit where the smallest and largest key differ.
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  if (kCached) {
+#pragma unroll
+    for (int e = 0; e < kMaxPerThread; ++e)
+      if (e < n_own) { kmin = min(kmin, kr[e]); kmax = max(kmax, kr[e]); }
+  } else {
+    for (int e = 0; e < n_own; ++e) { const uint32_t k = key_of(e); kmin = min(kmin, k); kmax = max(kmax, k); }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+  }
+  if (lane == 0) { warp_sums[tid >> 5] = static_cast<int>(kmin); hist[tid >> 5] = static_cast<int>(kmax); }
+  __syncthreads();
+  if (tid < 32) {
+    uint32_t a = static_cast<uint32_t>(warp_sums[tid]), z = static_cast<uint32_t>(hist[tid]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, off));
+      z = max(z, __shfl_xor_sync(0xffffffffu, z, off));
+    }
+    if (tid == 0) { sel[0] = static_cast<int>(a); sel[1] = static_cast<int>(z); }
+  }
+  __syncthreads();
+  kmin = static_cast<uint32_t>(sel[0]);
+  kmax = static_cast<uint32_t>(sel[1]);
+  __syncthreads();
+  const uint32_t diff = kmin ^ kmax;
+  int hi_bit = diff ? 31 - __clz(diff) : -1;
+  uint32_t mask = hi_bit >= 31 ? 0u : (0xffffffffu << (hi_bit + 1));
+  uint32_t prefix = kmin & mask;
+  int krem = kc;
+
+  // ---- radix select of the kc-th smallest key over the remaining bits ---------
+  while (hi_bit >= 0) {
+    const int width = min(8, hi_bit + 1);
+    const int shift = hi_bit - width + 1;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    if (kCached) {
+#pragma unroll
+      for (int e = 0; e < kMaxPerThread; ++e)
+        if (e < n_own && (kr[e] & mask) == prefix) atomicAdd(&hist[(kr[e] >> shift) & dmask], 1);
+    } else {
+      for (int e = 0; e < n_own; ++e) {
+        const uint32_t k = key_of(e);
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1);
+      }
+    }
+    __syncthreads();
+    // Inclusive prefix over the bins (warps 0..7), then locate the bin that
+    // holds the krem-th smallest remaining key.
+    int count = 0, incl = 0;
+    if (tid < 256) {
+      count = hist[tid];
+      incl = count;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) warp_sums[tid >> 5] = incl;
+    }
+    __syncthreads();
+    if (tid < 256) {
+      for (int w = 0; w < (tid >> 5); ++w) incl += warp_sums[w];
+      const int excl = incl - count;
+      if (excl < krem && incl >= krem) {
+        sel[0] = tid;
+        sel[1] = krem - excl;
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel[0]) << shift;
+    mask |= dmask << shift;
+    krem = sel[1];
+    hi_bit -= width;
+    __syncthreads();
+  }
+  const uint32_t boundary = prefix;  // the kc-th smallest key; take krem of its ties
+
+  // ---- write the kept candidates in ascending index order ---------------------
+  int n_eq = 0;
+  if (kCached) {
+#pragma unroll
+    for (int e = 0; e < kMaxPerThread; ++e) n_eq += (e < n_own && kr[e] == boundary);
+  } else {
+    for (int e = 0; e < n_own; ++e) n_eq += (key_of(e) == boundary);
+  }
+  const int eq_before = block_exclusive_scan(n_eq, warp_sums, nullptr);
+  int n_sel = 0, eq_seen = eq_before;
+  bool take[kCached ? kMaxPerThread : 1];
+  if (kCached) {
+#pragma unroll
+    for (int e = 0; e < kMaxPerThread; ++e) {
+      bool t = false;
+      if (e < n_own) {
+        if (kr[e] < boundary) t = true;
+        else if (kr[e] == boundary) t = (eq_seen++ < krem);
+      }
+      take[e] = t;
+      n_sel += t;
+    }
+  } else {
+    for (int e = 0; e < n_own; ++e) {
+      const uint32_t k = key_of(e);
+      if (k < boundary) ++n_sel;
+      else if (k == boundary) n_sel += (eq_seen++ < krem);
+    }
+  }
+  int pos = block_exclusive_scan(n_sel, warp_sums, nullptr);
+  if (kCached) {
+#pragma unroll
+    for (int e = 0; e < kMaxPerThread; ++e)
+      if (take[e]) out[pos++] = lo + e;
+  } else {
+    eq_seen = eq_before;
+    for (int e = 0; e < n_own; ++e) {
+      const uint32_t k = key_of(e);
+      bool t = k < boundary;
+      if (k == boundary) t = (eq_seen++ < krem);
+      if (t) out[pos++] = lo + e;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
             const int32_t* __restrict__ k_per_seq, int B, int max_chunks, int max_kept,
@@ -85,7 +235,7 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   __shared__ int warp_sums[32];
   __shared__ int sel[2];
   const int b = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
 
   // cu_kept[b+1] = sum of the kept counts of sequences 0..b.
   int part = 0;
@@ -114,73 +264,11 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   if (tid == 0) out[kc] = n - 1;  // the latest chunk, always last
   if (kc == 0) return;
   const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
-
-  // ---- radix select of the kc-th smallest key (1-based) -----------------------
-  uint32_t prefix = 0, mask = 0;
-  int krem = kc;
-  const int cand_pad = (cand + kThreads - 1) / kThreads * kThreads;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < cand_pad; i += kThreads) {
-      const bool valid = i < cand;
-      const uint32_t key = valid ? desc_key(__ldg(sc + i)) : 0u;
-      const bool match = valid && ((key & mask) == prefix);
-      const int digit = match ? static_cast<int>((key >> shift) & 255u) : 256;
-      const unsigned peers = __match_any_sync(0xffffffffu, digit);
-      if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
-    }
-    __syncthreads();
-    // Inclusive prefix over the 256 bins (warps 0..7), then locate the bin
-    // that holds the krem-th smallest remaining key.
-    int count = 0, incl = 0;
-    if (tid < 256) {
-      count = hist[tid];
-      incl = count;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      if (lane == 31) warp_sums[tid >> 5] = incl;
-    }
-    __syncthreads();
-    if (tid < 256) {
-      for (int w = 0; w < (tid >> 5); ++w) incl += warp_sums[w];
-      const int excl = incl - count;
-      if (excl < krem && incl >= krem) {
-        sel[0] = tid;
-        sel[1] = krem - excl;
-      }
-    }
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(sel[0]) << shift;
-    mask |= 255u << shift;
-    krem = sel[1];
-    __syncthreads();
-  }
-  const uint32_t boundary = prefix;  // the kc-th smallest key; take krem of its ties
-
-  // ---- write the kept candidates in ascending index order ---------------------
   const int per = (cand + kThreads - 1) / kThreads;
-  const int lo = min(cand, tid * per), hi = min(cand, lo + per);
-  int n_eq = 0;
-  for (int i = lo; i < hi; ++i) n_eq += (desc_key(__ldg(sc + i)) == boundary);
-  const int eq_before = block_exclusive_scan(n_eq, warp_sums, nullptr);
-  int n_sel = 0, eq_seen = eq_before;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t key = desc_key(__ldg(sc + i));
-    if (key < boundary) ++n_sel;
-    else if (key == boundary) n_sel += (eq_seen++ < krem);
-  }
-  int pos = block_exclusive_scan(n_sel, warp_sums, nullptr);
-  eq_seen = eq_before;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t key = desc_key(__ldg(sc + i));
-    bool take = key < boundary;
-    if (key == boundary) take = (eq_seen++ < krem);
-    if (take) out[pos++] = i;
-  }
+  if (per <= kMaxPerThread)
+    select_and_write<true>(sc, cand, kc, per, out, hist, warp_sums, sel);
+  else
+    select_and_write<false>(sc, cand, kc, per, out, hist, warp_sums, sel);
 }
 
 }  // namespace topk

@@ -100,7 +100,7 @@ def test_topk_matches_oracle(name):
 
 def test_topk_edge_cases():
     cases = [(0, 3), (1, 0), (1, 5), (2, 0), (2, 1), (5, 4), (5, 10), (64, 8), (3000, 300), (16384, 1638),
-             (4097, 4095), (100, 0), (777, 776), (1025, 513)]
+             (4097, 4095), (100, 0), (777, 776), (1025, 513), (20000, 2000), (16386, 9000), (30001, 7)]
     B = len(cases)
     M = max(c[0] for c in cases)
     rng = np.random.default_rng(5)
