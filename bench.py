@@ -156,7 +156,7 @@ def window_bytes(n_chunks, kept_total, layers):
     n = n_chunks.to(torch.int64).cpu()
     B = int(n.numel())
     keys = 256 * int(n.sum()) + B * 16 * 128 * 2 + 16 * 4
-    attn_launch = int(kept_total) * 2 * workloads.CHUNK_BYTES_ONE + B * (64 * 128 * 2 + 64 * 128 * 4)
+    attn_launch = int(round(kept_total * 2 * workloads.CHUNK_BYTES_ONE)) + B * (64 * 128 * 2 + 64 * 128 * 4)
     per_layer = keys + workloads.TAU * attn_launch
     return per_layer * layers, attn_launch, int(n.sum())
 
@@ -300,7 +300,8 @@ def run_ours(args, rank, world, local_rank):
     inp = workloads.make_inputs(args.workload, dev, base_seed=workloads.BASE_SEED + rank)
     B, layers, n_win = inp.batch, len(inp.layers), inp.workload.windows
     host_tier = inp.workload.host_pool
-    lws = [LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev) for _ in range(layers)]
+    lws = [LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev,
+                       selection=args.selection, threshold=args.threshold) for _ in range(layers)]
     outs = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
     stream = torch.cuda.Stream(device=dev)
 
@@ -317,10 +318,16 @@ def run_ours(args, rank, world, local_rank):
             for l, L in enumerate(inp.layers):
                 lws[l].attend(L.q[w, t], outs[l][t], kv_unchanged=t > 0)
 
-    # warm every path once, then capture one pair of graphs per window index
+    # warm every path once (and record the kept total of every window index,
+    # which the threshold selection makes data-dependent), then capture one pair
+    # of graphs per window index
+    kept_totals = []
     with torch.cuda.stream(stream):
-        select_phase(0)
-        attn_phase(0)
+        for w in range(n_win):
+            select_phase(w)
+            torch.cuda.synchronize()
+            kept_totals.append(sum(int(lw.cu_kept[0][-1].item()) for lw in lws) / layers)
+        attn_phase(n_win - 1)
     torch.cuda.synchronize()
     bits = lsa.read_device_status()
     if bits:
@@ -385,7 +392,8 @@ def run_ours(args, rank, world, local_rank):
     # tok/s/layer: every window decodes 64 tokens per sequence in each layer; a
     # window of `layers` layers takes `elapsed / steps`, i.e. 1/layers of it per layer.
     elapsed, value = combine_ranks(elapsed, workloads.TAU * B * layers * args.steps, world, dev)
-    kept_total = int(lws[0].cu_kept[0][-1].item())
+    # mean kept total over the timed windows (identical for every window with top-K)
+    kept_total = sum(kept_totals[i % n_win] for i in range(args.steps)) / args.steps
     wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers)
     hbm_gbs = wbytes * args.steps / elapsed / 1e9
     n_attn = workloads.TAU * layers * args.steps
@@ -405,6 +413,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": inp.workload.description, "name": args.workload, "batch": B, "layers": layers,
             "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
+            "selection": args.selection if args.selection == "topk" else f"threshold {args.threshold}",
             "tau": workloads.TAU, "gqa": "64q/8kv/d128", "indexer": "16 heads x 128",
             "kv_dtype": "bf16", "softmax_accumulate": "fp32",
             "l2": ("inputs larger than L2: each attention launch streams "
@@ -645,6 +654,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--fetch-ctas", type=int, default=64)
+    ap.add_argument("--selection", choices=["topk", "threshold"], default="topk",
+                    help="chunk selection: fixed top-K budget (default) or the sigmoid threshold")
+    ap.add_argument("--threshold", type=float, default=0.5)
     ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
     ap.add_argument("--attn-only", action="store_true",
                     help="time attention launches alone on a random compact buffer (profiling case)")

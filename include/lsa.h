@@ -137,6 +137,26 @@ int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t*
                     int32_t* cu_kept, void* stream);
 
 /*
+ * lsa_threshold_chunks -- the pages' own selection rule: sigmoid thresholding
+ * in place of a fixed top-k (summary page, 2.1 Architecture; the 0.5
+ * classification threshold of 2.4 Configuration).  Chunk c < n-1 is kept when
+ * score_c / sum_h w[h] > threshold, i.e. when the weighted mean of the heads'
+ * sigmoid probabilities exceeds it (fp32: the sum of w in head order, then
+ * one division per chunk); the latest chunk n-1 is always kept.  Outputs as
+ * lsa_topk_chunks: kept[b*max_kept + j] ascending with the latest last,
+ * n_kept[b], cu_kept[B+1].  The kept count depends on the data, so size
+ * max_kept for the worst case (max n) or accept CAPACITY.
+ *   scores   device fp32 [B][max_chunks]; w device fp32 [16] (as for scoring)
+ *   threshold  finite; 0.5 in the pages
+ * Two kernels are launched (per-sequence compaction, then offsets); B <=
+ * LSA_MAX_BATCH.  Device errors: BAD_COUNT (n out of range) and CAPACITY (the
+ * kept set would exceed max_kept): that sequence keeps nothing.
+ */
+int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks, const float* w, float threshold,
+                         int B, int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept,
+                         int32_t* cu_kept, void* stream);
+
+/*
  * lsa_gather_chunks -- copy every kept chunk from the device KV pools into the
  * compact buffers, bit for bit: for i = cu_kept[b] + j,
  *   k_buf[i] = k_pool[slot(b, kept[b*max_kept + j])], same for V.

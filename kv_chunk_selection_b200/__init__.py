@@ -55,6 +55,7 @@ def _load():
         "lsa_read_device_status": ([P, ctypes.POINTER(ctypes.c_uint)], I),
         "lsa_index_score": ([P, P, P, I64, P, P, I, I, P, P], I),
         "lsa_topk_chunks": ([P, P, P, I, I, I, P, P, P, P], I),
+        "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
         "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
         "lsa_attn_workspace_size": ([I], S),
@@ -148,6 +149,21 @@ def lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu_kept, stream=N
     _check("lsa_topk_chunks", _load().lsa_topk_chunks(
         _ptr(scores), _ptr(n_chunks), _ptr(k_per_seq), B, max_chunks, max_kept, _ptr(kept), _ptr(n_kept),
         _ptr(cu_kept), _stream(stream)))
+
+
+def lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu_kept, threshold=0.5, stream=None):
+    """Sigmoid-threshold selection: chunks with score / sum(w) > threshold, plus the latest, ascending."""
+    _need(scores, "scores", torch.float32)
+    _need(w, "w", torch.float32)
+    for t, n in ((n_chunks, "n_chunks"), (kept, "kept"), (n_kept, "n_kept"), (cu_kept, "cu_kept")):
+        _need(t, n, torch.int32)
+    B, max_chunks = scores.shape
+    max_kept = kept.shape[1]
+    if kept.shape[0] != B or cu_kept.numel() != B + 1 or n_kept.numel() != B:
+        raise ValueError("bad shapes")
+    _check("lsa_threshold_chunks", _load().lsa_threshold_chunks(
+        _ptr(scores), _ptr(n_chunks), _ptr(w), float(threshold), B, max_chunks, max_kept, _ptr(kept),
+        _ptr(n_kept), _ptr(cu_kept), _stream(stream)))
 
 
 def lsa_gather_chunks(k_pool, v_pool, chunk_table, kept, cu_kept, max_chunks, k_buf, v_buf, stream=None):
@@ -249,6 +265,7 @@ def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=
 
 __all__ = [
     "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
+    "lsa_threshold_chunks",
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_attn_workspace_size", "new_attn_workspace",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",

@@ -288,3 +288,100 @@ extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, con
       scores, n_chunks, k_per_seq, B, max_chunks, max_kept, kept, n_kept, cu_kept, lsa_device_status_ptr());
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// lsa_threshold_chunks: the pages' own selection rule, sigmoid thresholding in
+// place of a fixed top-k (summary page, 2.1 Architecture and 2.4
+// Configuration): chunk c < n-1 is kept when score_c / sum_h w_h (the weighted
+// mean of the heads' sigmoid probabilities) exceeds the threshold; the latest
+// chunk is always kept.  The kept count is data-dependent, so a first kernel
+// compacts each sequence (one CTA per sequence, contiguous candidate runs per
+// thread, one block scan, index order preserved) and a second one-CTA kernel
+// turns the counts into cu_kept.
+// ---------------------------------------------------------------------------
+namespace lsa {
+namespace topk {
+
+__global__ void __launch_bounds__(kThreads)
+threshold_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
+                 const float* __restrict__ w, float threshold, int max_chunks, int max_kept,
+                 int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, unsigned* status) {
+  __shared__ int warp_sums[32];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int n = __ldg(n_chunks + b);
+  if (n < 0 || n > max_chunks) {
+    if (tid == 0) { n_kept[b] = 0; set_status(status, LSA_DEV_ERR_BAD_COUNT); }
+    return;
+  }
+  if (n == 0) {
+    if (tid == 0) n_kept[b] = 0;
+    return;
+  }
+  float wsum = 0.f;   // fixed order: every thread gets the same fp32 sum
+#pragma unroll
+  for (int h = 0; h < kIndexHeads; ++h) wsum += __ldg(w + h);
+  const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
+  const int cand = n - 1;
+  const int per = (cand + kThreads - 1) / kThreads;
+  const int lo = min(cand, tid * per), hi = min(cand, lo + per);
+  int cnt = 0;
+  for (int i = lo; i < hi; ++i) cnt += (__ldg(sc + i) / wsum > threshold);
+  int total = 0;
+  int pos = block_exclusive_scan(cnt, warp_sums, &total);
+  if (total + 1 > max_kept) {
+    if (tid == 0) { n_kept[b] = 0; set_status(status, LSA_DEV_ERR_CAPACITY); }
+    return;
+  }
+  int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
+  for (int i = lo; i < hi; ++i)
+    if (__ldg(sc + i) / wsum > threshold) out[pos++] = i;
+  if (tid == 0) {
+    out[total] = n - 1;
+    n_kept[b] = total + 1;
+  }
+}
+
+// cu_kept[0] = 0, cu_kept[b+1] = cu_kept[b] + n_kept[b]  (one CTA, B <= 4096).
+__global__ void __launch_bounds__(kThreads)
+offsets_kernel(const int32_t* __restrict__ n_kept, int B, int32_t* __restrict__ cu_kept) {
+  __shared__ int warp_sums[32];
+  const int tid = threadIdx.x;
+  constexpr int kPer = (LSA_MAX_BATCH + kThreads - 1) / kThreads;   // 4
+  int v[kPer], s = 0;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int b = tid * kPer + e;
+    v[e] = b < B ? n_kept[b] : 0;
+    s += v[e];
+  }
+  int run = block_exclusive_scan(s, warp_sums, nullptr);
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int b = tid * kPer + e;
+    run += v[e];
+    if (b < B) cu_kept[b + 1] = run;
+  }
+  if (tid == 0) cu_kept[0] = 0;
+}
+
+}  // namespace topk
+}  // namespace lsa
+
+extern "C" int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks, const float* w, float threshold,
+                                    int B, int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept,
+                                    int32_t* cu_kept, void* stream) {
+  using namespace lsa;
+  if (!scores || !n_chunks || !w || !kept || !n_kept || !cu_kept || B <= 0 || max_chunks <= 0 || max_kept <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (!isfinite(threshold)) return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  topk::threshold_kernel<<<B, topk::kThreads, 0, s>>>(scores, n_chunks, w, threshold, max_chunks, max_kept, kept,
+                                                       n_kept, lsa_device_status_ptr());
+  int st = launch_status();
+  if (st != LSA_OK) return st;
+  topk::offsets_kernel<<<1, topk::kThreads, 0, s>>>(n_kept, B, cu_kept);
+  return launch_status();
+}

@@ -18,7 +18,7 @@ import torch
 
 from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_attn_workspace_size,
                lsa_fetch_from_host, lsa_gather_chunks, lsa_index_score, lsa_sparse_decode_attn,
-               lsa_topk_chunks)
+               lsa_threshold_chunks, lsa_topk_chunks)
 
 TAU = 64
 
@@ -26,23 +26,37 @@ TAU = 64
 class LayerWindow:
     """Buffers and calls of one layer's decode window.
 
-    Sizes: ``max_kept`` = max_b K_b + 1 kept chunks per sequence row, and the
-    compact buffer holds ``sum_b (K_b + 1)`` chunks (an upper bound of the kept
-    total).  With ``double_buffer`` two compact buffers alternate, so the
+    Selection is the fixed top-K budget (``selection="topk"``) or the pages'
+    sigmoid threshold (``selection="threshold"``, keep a chunk when its weighted
+    mean probability exceeds ``threshold``).  Sizes: with top-K, ``max_kept`` =
+    max_b K_b + 1 kept chunks per sequence row and the compact buffer holds
+    ``sum_b (K_b + 1)`` chunks (an upper bound of the kept total); with the
+    threshold the kept count depends on the data, so both are sized for every
+    chunk.  With ``double_buffer`` two compact buffers alternate, so the
     selection of the next window can be fetched while the current one is read.
     """
 
     def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
-                 max_chunks: int, device="cuda", double_buffer: bool = False):
+                 max_chunks: int, device="cuda", double_buffer: bool = False, selection: str = "topk",
+                 threshold: float = 0.5):
         self.device = torch.device(device)
         self.n_chunks = n_chunks
         self.k_per_seq = k_per_seq
         self.chunk_table = chunk_table
         self.max_chunks = int(max_chunks)
         self.B = int(n_chunks.shape[0])
-        k_host = k_per_seq.to("cpu", torch.int64)
-        self.max_kept = int(k_host.max()) + 1
-        self.buf_chunks = int((k_host + 1).sum())
+        if selection not in ("topk", "threshold"):
+            raise ValueError("selection must be 'topk' or 'threshold'")
+        self.selection = selection
+        self.threshold = float(threshold)
+        if selection == "topk":
+            k_host = k_per_seq.to("cpu", torch.int64)
+            self.max_kept = int(k_host.max()) + 1
+            self.buf_chunks = int((k_host + 1).sum())
+        else:
+            n_host = n_chunks.to("cpu", torch.int64)
+            self.max_kept = int(max_chunks)
+            self.buf_chunks = int(n_host.sum())
         nbuf = 2 if double_buffer else 1
         shape = (self.buf_chunks, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM)
         self.k_bufs = [torch.empty(shape, dtype=torch.bfloat16, device=self.device) for _ in range(nbuf)]
@@ -55,10 +69,14 @@ class LayerWindow:
         self.active = 0
 
     def select(self, q_idx, w, chunk_keys, buf: int = 0, stream=None):
-        """Indexer scores, then top-K plus latest, into selection slot ``buf``."""
+        """Indexer scores, then the selection (top-K or threshold) plus latest, into slot ``buf``."""
         lsa_index_score(q_idx, w, chunk_keys, self.chunk_table, self.n_chunks, self.scores, stream=stream)
-        lsa_topk_chunks(self.scores, self.n_chunks, self.k_per_seq, self.kept[buf], self.n_kept[buf],
-                        self.cu_kept[buf], stream=stream)
+        if self.selection == "topk":
+            lsa_topk_chunks(self.scores, self.n_chunks, self.k_per_seq, self.kept[buf], self.n_kept[buf],
+                            self.cu_kept[buf], stream=stream)
+        else:
+            lsa_threshold_chunks(self.scores, self.n_chunks, w, self.kept[buf], self.n_kept[buf], self.cu_kept[buf],
+                                 threshold=self.threshold, stream=stream)
 
     def gather(self, k_pool, v_pool, buf: int = 0, stream=None):
         lsa_gather_chunks(k_pool, v_pool, self.chunk_table, self.kept[buf], self.cu_kept[buf], self.max_chunks,

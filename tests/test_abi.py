@@ -36,7 +36,8 @@ def L():
 
 def test_header_declares_the_boundary():
     fns = header_functions()
-    for name in ("lsa_index_score", "lsa_topk_chunks", "lsa_gather_chunks", "lsa_sparse_decode_attn",
+    for name in ("lsa_index_score", "lsa_topk_chunks", "lsa_threshold_chunks", "lsa_gather_chunks",
+                 "lsa_sparse_decode_attn",
                  "lsa_fetch_from_host", "lsa_attn_workspace_size", "lsa_read_device_status",
                  "lsa_status_string", "lsa_version"):
         assert name in fns
@@ -68,6 +69,7 @@ def test_host_checks_null_pointers(L):
     n = None
     assert L.lsa_index_score(n, n, n, 1, n, n, 1, 1, n, n) == INVALID
     assert L.lsa_topk_chunks(n, n, n, 1, 1, 1, n, n, n, n) == INVALID
+    assert L.lsa_threshold_chunks(n, n, n, ctypes.c_float(0.5), 1, 1, 1, n, n, n, n) == INVALID
     assert L.lsa_gather_chunks(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, n) == INVALID
     assert L.lsa_fetch_from_host(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, 0, n, n) == INVALID
     assert L.lsa_sparse_decode_attn(n, n, n, 1, n, 1, 0.1, n, n, 0, 0, n) == INVALID

@@ -140,6 +140,82 @@ def test_topk_nan_and_inf_order():
     status_clean()
 
 
+def run_threshold(scores, n_chunks, w, threshold, max_kept):
+    B = scores.shape[0]
+    kept = torch.full((B, max_kept), -7, dtype=torch.int32, device=DEV)
+    n_kept = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu, threshold=threshold)
+    return kept, n_kept, cu
+
+
+def assert_threshold_matches(got, scores64, n, w64, t):
+    """Exact match with the oracle's rule on the same scores, except chunks whose
+    weighted mean probability is within 1e-6 (relative) of the threshold."""
+    ref = oracle.threshold_chunks(scores64, n, w64, t)
+    wsum = float(np.sum(w64))
+    for b in range(len(n)):
+        g, r = set(got[b]), set(ref[b].tolist())
+        for c in g ^ r:
+            assert abs(scores64[b, c] / wsum - t) <= 1e-6 * abs(t), f"seq {b}: chunk {c} differs away from the threshold"
+        assert sorted(got[b]) == got[b]
+
+
+@pytest.mark.parametrize("name,t", [("tiny", 0.5), ("128k", 0.5), ("128k", 0.6), ("batched", 0.55)])
+def test_threshold_matches_oracle(name, t):
+    inp = workloads.make_inputs(name, DEV, pools=False, layers=1)
+    n = i64(inp.n_chunks)
+    g = score_on_gpu(inp)
+    kept, n_kept, cu = run_threshold(g, inp.n_chunks, inp.layers[0].w, t, inp.max_chunks)
+    got = kept_from_gpu(kept, n_kept)
+    assert_threshold_matches(got, f64(g), n, f64(inp.layers[0].w), t)
+    assert i64(cu).tolist() == oracle.cumulative_kept(got).tolist()
+    # the oracle's own fp64 scores give the same set outside the threshold window
+    assert_threshold_matches(got, oracle_scores(inp), n, f64(inp.layers[0].w), t)
+    status_clean()
+
+
+def test_threshold_edge_cases():
+    w = torch.full((16,), 0.5, device=DEV)                     # sum(w) = 8
+    n = torch.tensor([0, 1, 5, 5, 40], dtype=torch.int32, device=DEV)
+    s = torch.zeros((5, 40), device=DEV)
+    s[2, :5] = 8.0                                               # every mean probability 1.0: all kept
+    s[3, :5] = 1.0                                               # 0.125: only the latest kept
+    s[4, :40] = torch.linspace(0, 8, 40, device=DEV)
+    kept, n_kept, cu = run_threshold(s, n, w, 0.5, 40)
+    got = kept_from_gpu(kept, n_kept)
+    assert got[0] == [] and got[1] == [0] and got[2] == [0, 1, 2, 3, 4] and got[3] == [4]
+    ref = oracle.threshold_chunks(f64(s), i64(n), f64(w), 0.5)
+    assert got[4] == list(ref[4])
+    assert i64(cu).tolist() == oracle.cumulative_kept(got).tolist()
+    status_clean()
+    # a kept set larger than max_kept: that sequence keeps nothing, CAPACITY is reported
+    kept, n_kept, cu = run_threshold(s, n, w, 0.5, 4)
+    assert lsa.read_device_status() & 8
+    assert i64(n_kept).tolist()[2] == 0 and i64(n_kept).tolist()[1] == 1
+
+
+def test_threshold_window_attention():
+    """Threshold selection feeds the same gather and attention: whole step vs the oracle."""
+    inp = workloads.make_inputs("128k", DEV, layers=1, windows=1, steps=2)
+    L = inp.layers[0]
+    g = score_on_gpu(inp)
+    kept, n_kept, cu = run_threshold(g, inp.n_chunks, L.w, 0.6, inp.max_chunks)
+    total = int(cu[-1])
+    kb = torch.empty((total, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    vb = torch.empty_like(kb)
+    lsa.lsa_gather_chunks(L.k_pool, L.v_pool, inp.chunk_table, kept, cu, inp.max_chunks, kb, vb)
+    out = torch.empty((1, 64, 128), device=DEV)
+    ws = lsa.new_attn_workspace(1)
+    lsa.lsa_sparse_decode_attn(L.q[0, 1], kb, vb, cu, out, ws)
+    got = kept_from_gpu(kept, n_kept)
+    assert_threshold_matches(got, f64(g), i64(inp.n_chunks), f64(L.w), 0.6)
+    assert torch.equal(kb, L.k_pool[torch.tensor(got[0], device=DEV)])
+    ref = oracle.sparse_decode_attn(f64(L.q[0, 1]), f64(kb), f64(vb), i64(cu))
+    assert_attention_close(out, ref)
+    status_clean()
+
+
 # ------------------------------------------------------------------ gather --
 
 def paged_case(B=6, seed=3, max_chunks=40):
