@@ -95,6 +95,18 @@ int lsa_version(void);
 int lsa_read_device_status(void* stream, unsigned int* bits);
 
 /*
+ * lsa_selftest_bounded_wait -- diagnostic of the failure detection every
+ * kernel relies on (a device-side wait that cannot complete must not hang the
+ * GPU).  Launches one warp that waits, through the same bounded-wait helpers
+ * the kernels use, on an mbarrier nothing completes (mode 0) or until the
+ * device int *flag is non-zero (mode 1; flag device memory).  After limit_us
+ * microseconds (1 .. 2,000,000) a wait that has not completed sets
+ * LSA_DEV_ERR_TIMEOUT in the device status word and the kernel returns; the
+ * context stays usable.  Not part of the decode path.
+ */
+int lsa_selftest_bounded_wait(int mode, const int* flag, unsigned int limit_us, void* stream);
+
+/*
  * lsa_index_score -- indexer scores of every chunk (the Neural Memory Indexer
  * of the summary page, 2.1 Architecture; sigmoid scoring per the review page,
  * "1. Key Terms & Definitions"):

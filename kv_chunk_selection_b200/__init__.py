@@ -53,6 +53,7 @@ def _load():
         "lsa_status_string": ([I], ctypes.c_char_p),
         "lsa_version": ([], I),
         "lsa_read_device_status": ([P, ctypes.POINTER(ctypes.c_uint)], I),
+        "lsa_selftest_bounded_wait": ([I, P, ctypes.c_uint, P], I),
         "lsa_index_score": ([P, P, P, I64, P, P, I, I, P, P], I),
         "lsa_topk_chunks": ([P, P, P, I, I, I, P, P, P, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
@@ -108,6 +109,14 @@ def read_device_status(stream=None) -> int:
     bits = ctypes.c_uint(0)
     _check("lsa_read_device_status", _load().lsa_read_device_status(_stream(stream), ctypes.byref(bits)))
     return bits.value
+
+
+def lsa_selftest_bounded_wait(mode: int, flag: Optional[torch.Tensor], limit_us: int, stream=None):
+    """Runs the bounded-wait self-test (mode 0: mbarrier nothing completes; mode 1: device flag)."""
+    if flag is not None:
+        _need(flag, "flag", torch.int32)
+    _check("lsa_selftest_bounded_wait",
+           _load().lsa_selftest_bounded_wait(int(mode), _ptr(flag), int(limit_us), _stream(stream)))
 
 
 def decode_status(bits: int) -> list:

@@ -81,7 +81,38 @@ EncodeTiledFn tensor_map_encoder() {
 
 }  // namespace lsa
 
+namespace {
+// Self-test of the bounded waits every kernel relies on: mode 0 waits on an
+// mbarrier that nothing will complete, mode 1 on a device flag (complete when
+// the caller has set it).  A wait that runs out sets LSA_DEV_ERR_TIMEOUT and
+// the kernel returns normally, leaving the context usable.
+__global__ void selftest_wait_kernel(int mode, const int* flag, unsigned long long limit_ns, unsigned* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    lsa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    lsa::mbar_fence_init();
+  }
+  __syncthreads();
+  bool ok;
+  if (mode == 0) ok = lsa::mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns);
+  else ok = lsa::flag_wait_bounded(flag, limit_ns);
+  if (!ok && threadIdx.x == 0) lsa::set_status(status, LSA_DEV_ERR_TIMEOUT);
+}
+}  // namespace
+
 extern "C" {
+
+int lsa_selftest_bounded_wait(int mode, const int* flag, unsigned int limit_us, void* stream) {
+  if (mode != 0 && mode != 1) return LSA_ERR_INVALID_ARG;
+  if (mode == 1 && !flag) return LSA_ERR_INVALID_ARG;
+  if (limit_us == 0 || limit_us > 2000000u) return LSA_ERR_INVALID_ARG;
+  if (lsa::device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      mode, flag, static_cast<unsigned long long>(limit_us) * 1000ull, lsa_device_status_ptr());
+  return lsa::launch_status();
+}
 
 const char* lsa_status_string(int status) {
   switch (status) {

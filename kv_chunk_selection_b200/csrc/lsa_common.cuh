@@ -69,16 +69,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete.  Gives up (returns
-// false) after kWaitLimitNs, or as soon as *abort_flag becomes non-zero.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, volatile int* abort_flag) {
+// false) after `limit_ns` (default kWaitLimitNs), or as soon as *abort_flag
+// becomes non-zero.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, volatile int* abort_flag,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (unsigned it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+  }
+}
+// Waits until *flag (device memory) becomes non-zero, at most `limit_ns`.
+__device__ __forceinline__ bool flag_wait_bounded(const volatile int* flag, unsigned long long limit_ns) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (unsigned it = 0;; ++it) {
+    if (*flag) return true;
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(256);
   }
 }
 
