@@ -37,11 +37,13 @@
 namespace lsa {
 namespace attn {
 
-constexpr int kConsumerWarps = 4;
+constexpr int kGroups = 2;                   // consumer warp groups, taking alternate units
+constexpr int kWarpsPerGroup = 4;            // each warp of a group takes 16 of a unit's 64 tokens
+constexpr int kConsumerWarps = kGroups * kWarpsPerGroup;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kStages = 3;
-constexpr int kCtasPerSm = 2;                // two CTAs share each SM (8 consumer warps)
+constexpr int kStages = 6;
+constexpr int kCtasPerSm = 1;                // one CTA per SM: 8 consumer warps, 6 stages in flight
 constexpr int kBoxBytes = 8192;              // 64 tokens x 64 dims of bf16
 constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo, V hi
 constexpr int kAccStride = 132;              // padded row of the combine buffer
@@ -165,7 +167,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], kWarpsPerGroup);   // a stage is consumed by one warp group
     }
     flags[0] = 0;
     flags[1] = 0;
@@ -220,13 +222,15 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   // ========================= consumer warps ==================================
   if (kv_unchanged) griddep_wait();
   zero_empty(tid, kConsumerThreads);
+  const int grp = warp / kWarpsPerGroup;   // takes the units with unit_i % 2 == grp
+  const int wig = warp % kWarpsPerGroup;   // 16-token slice of a unit
   const int gl = lane >> 2;   // row group of the mma fragments
   const int c4 = lane & 3;    // column pair of the mma fragments
   const int mi = lane >> 3, r8 = lane & 7;
   // ldmatrix row addresses of this lane (see the fragment maps in the header comment)
-  const int krow = warp * 16 + r8 + ((mi & 1) << 3);
+  const int krow = wig * 16 + r8 + ((mi & 1) << 3);
   const int kx = mi >> 1;
-  const int vrow = warp * 16 + r8 + ((mi >> 1) << 3);
+  const int vrow = wig * 16 + r8 + ((mi >> 1) << 3);
   const int vx = mi & 1;
   const uint32_t smem_base = smem_u32(smem);
   // Swizzled byte offsets of this lane's ldmatrix rows within a stage, for the
@@ -268,6 +272,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
     for (int jj = j0; jj < jend; ++jj, ++unit_i) {
+      if (static_cast<int>(unit_i & 1) != grp) continue;   // the other group's unit
       const int s = static_cast<int>(unit_i % kStages);
       bool ok = !*abort_flag;
       if (ok) {
@@ -330,7 +335,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       if (lane == 0) mbar_arrive(&empty[s]);
     }
 
-    // ---- end of segment: combine the 4 warps --------------------------------
+    // ---- end of segment: combine the 8 warps --------------------------------
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, off);
@@ -354,36 +359,32 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     }
     named_barrier(1, kConsumerThreads);
 
-    const int hh = tid >> 4;          // head within the group
-    const int d0 = (tid & 15) * 8;    // 8 consecutive dims
+    const int hh = tid >> 5;          // head within the group (warp-uniform)
+    const int d0 = (tid & 31) * 4;    // 4 consecutive dims
     float mw[kConsumerWarps], M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
       mw[w] = mbuf[w * kGroup + hh];
       M = fmaxf(M, mw[w]);
     }
-    float L = 0.f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float L = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      const float sc = fast_exp2(mw[w] - M);
+      const float sc = fast_exp2(mw[w] - M);   // 0 for a warp that saw no unit of this segment
       L += sc * lbuf[w * kGroup + hh];
-      const float* ab = accbuf + (w * kGroup + hh) * kAccStride + d0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] += sc * ab[k];
+      const float4 x = *reinterpret_cast<const float4*>(accbuf + (w * kGroup + hh) * kAccStride + d0);
+      o.x += sc * x.x; o.y += sc * x.y; o.z += sc * x.z; o.w += sc * x.w;
     }
     const float inv = 1.f / L;
     const int p = b * kNumKVHeads + g;
     float* dst = out + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + hh) * kHeadDim + d0;
     if (whole_pair) {
-      reinterpret_cast<float4*>(dst)[0] = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
-      reinterpret_cast<float4*>(dst)[1] = make_float4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv);
+      *reinterpret_cast<float4*>(dst) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     } else {
       float* rec = records + static_cast<int64_t>(p + blockIdx.x) * kRecFloats;
-      reinterpret_cast<float4*>(rec + hh * kHeadDim + d0)[0] =
-          make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
-      reinterpret_cast<float4*>(rec + hh * kHeadDim + d0)[1] =
-          make_float4(o[4] * inv, o[5] * inv, o[6] * inv, o[7] * inv);
-      if ((tid & 15) == 0) rec[kGroup * kHeadDim + hh] = M + __log2f(L);
+      *reinterpret_cast<float4*>(rec + hh * kHeadDim + d0) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      if ((tid & 31) == 0) rec[kGroup * kHeadDim + hh] = M + __log2f(L);
       __threadfence();
       named_barrier(1, kConsumerThreads);
       // Contributing CTAs of pair p: those whose unit range meets [a_p, a_p + n_b).
@@ -403,37 +404,41 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         const int n_rec = c_hi - c_lo + 1;
         const float* rbase = records + static_cast<int64_t>(p + c_lo) * kRecFloats;
         float lse_max = -INFINITY, den = 0.f;
-        float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
         if (u + (jend - j0) == u1) {
           // Last segment of this CTA: the stage ring and the combine buffer
           // are free, so whole batches of records are pulled into shared
           // memory with asynchronous 16-byte copies (one L2 round trip per
-          // batch) and folded from there with a running log-sum-exp.
+          // batch) and folded from there with a running log-sum-exp.  The
+          // log-sum-exp a thread reads is warp-uniform (one head per warp).
           const float* srec = reinterpret_cast<const float*>(smem);
           const char* gsrc = reinterpret_cast<const char*>(rbase);
           for (int c0 = 0; c0 < n_rec; c0 += kStagedRecs) {
             const int nc = min(kStagedRecs, n_rec - c0);
-            const char* g = gsrc + static_cast<int64_t>(c0) * kRecBytes;
+            const char* gb = gsrc + static_cast<int64_t>(c0) * kRecBytes;
             for (int i = tid; i < nc * (kRecBytes / 16); i += kConsumerThreads)
-              cp_async_16_cg(smem_base + i * 16, g + static_cast<int64_t>(i) * 16);
+              cp_async_16_cg(smem_base + i * 16, gb + static_cast<int64_t>(i) * 16);
             cp_async_wait_all();
             named_barrier(1, kConsumerThreads);
-            float m_new = lse_max;
-            for (int c = 0; c < nc; ++c) m_new = fmaxf(m_new, srec[c * kRecFloats + kGroup * kHeadDim + hh]);
+            float m4[4] = {lse_max, lse_max, lse_max, lse_max};
+            int c = 0;
+            for (; c + 4 <= nc; c += 4) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], srec[(c + k) * kRecFloats + kGroup * kHeadDim + hh]);
+            }
+            for (; c < nc; ++c) m4[0] = fmaxf(m4[0], srec[c * kRecFloats + kGroup * kHeadDim + hh]);
+            const float m_new = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
             den *= resc;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) r[k] *= resc;
+            r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
             lse_max = m_new;
 #pragma unroll 4
-            for (int c = 0; c < nc; ++c) {
-              const float* rc = srec + c * kRecFloats;
+            for (int cc = 0; cc < nc; ++cc) {
+              const float* rc = srec + cc * kRecFloats;
               const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - lse_max);
-              const float4 x0 = reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0)[0];
-              const float4 x1 = reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0)[1];
+              const float4 x = *reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0);
               den += wgt;
-              r[0] += wgt * x0.x; r[1] += wgt * x0.y; r[2] += wgt * x0.z; r[3] += wgt * x0.w;
-              r[4] += wgt * x1.x; r[5] += wgt * x1.y; r[6] += wgt * x1.z; r[7] += wgt * x1.w;
+              r.x += wgt * x.x; r.y += wgt * x.y; r.z += wgt * x.z; r.w += wgt * x.w;
             }
             named_barrier(1, kConsumerThreads);
           }
@@ -442,14 +447,13 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           // records in batches of 8 from L2, all loads of a batch in flight.
           for (int c0 = 0; c0 < n_rec; c0 += 8) {
             float lse[8];
-            float4 x[8][2];
+            float4 x[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const int c = min(c0 + k, n_rec - 1);   // tail lanes re-read the last record (weight 0)
               const float* rc = rbase + static_cast<int64_t>(c) * kRecFloats;
               lse[k] = __ldcg(rc + kGroup * kHeadDim + hh);
-              x[k][0] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
-              x[k][1] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0) + 1);
+              x[k] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
             }
             float m_new = lse_max;
 #pragma unroll
@@ -457,21 +461,18 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
               if (c0 + k < n_rec) m_new = fmaxf(m_new, lse[k]);
             const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
             den *= resc;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) r[k] *= resc;
+            r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
             lse_max = m_new;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const float wgt = (c0 + k < n_rec) ? fast_exp2(lse[k] - lse_max) : 0.f;
               den += wgt;
-              r[0] += wgt * x[k][0].x; r[1] += wgt * x[k][0].y; r[2] += wgt * x[k][0].z; r[3] += wgt * x[k][0].w;
-              r[4] += wgt * x[k][1].x; r[5] += wgt * x[k][1].y; r[6] += wgt * x[k][1].z; r[7] += wgt * x[k][1].w;
+              r.x += wgt * x[k].x; r.y += wgt * x[k].y; r.z += wgt * x[k].z; r.w += wgt * x[k].w;
             }
           }
         }
         const float id = 1.f / den;
-        reinterpret_cast<float4*>(dst)[0] = make_float4(r[0] * id, r[1] * id, r[2] * id, r[3] * id);
-        reinterpret_cast<float4*>(dst)[1] = make_float4(r[4] * id, r[5] * id, r[6] * id, r[7] * id);
+        *reinterpret_cast<float4*>(dst) = make_float4(r.x * id, r.y * id, r.z * id, r.w * id);
         if (tid == 0) counters[p] = 0;   // ready for the next call
       }
     }
