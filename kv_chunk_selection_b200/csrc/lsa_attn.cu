@@ -242,6 +242,85 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     vofs[t] = 2 * kBoxBytes + (t >> 2) * kBoxBytes + vrow * 128 + ((((t & 3) * 2 + vx) ^ (vrow & 7)) << 4);
   }
 
+  const int hh = tid >> 5;          // combine / merge: head within the group (warp-uniform)
+  const int d0 = (tid & 31) * 4;    // 4 consecutive dims
+
+  // Merge of the partials of pair p in CTA order, run at the end of this CTA's
+  // work (the stage ring and the combine buffer are free).  Records of the
+  // contributing CTAs are contiguous (index p + c); whole batches of them are
+  // pulled into shared memory with asynchronous 16-byte copies (one L2 round
+  // trip per batch) and folded with a running log-sum-exp.  The log-sum-exp a
+  // thread reads is warp-uniform (one head per warp).
+  auto merge_pair = [&](int pp, int c_lo, int c_hi) {
+    const int n_rec = c_hi - c_lo + 1;
+    const char* gsrc = reinterpret_cast<const char*>(records + static_cast<int64_t>(pp + c_lo) * kRecFloats);
+    const float* srec = reinterpret_cast<const float*>(smem);
+    float lse_max = -INFINITY, den = 0.f;
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < n_rec; c0 += kStagedRecs) {
+      const int nc = min(kStagedRecs, n_rec - c0);
+      const char* gb = gsrc + static_cast<int64_t>(c0) * kRecBytes;
+      for (int i = tid; i < nc * (kRecBytes / 16); i += kConsumerThreads)
+        cp_async_16_cg(smem_base + i * 16, gb + static_cast<int64_t>(i) * 16);
+      cp_async_wait_all();
+      named_barrier(1, kConsumerThreads);
+      float m4[4] = {lse_max, lse_max, lse_max, lse_max};
+      int c = 0;
+      for (; c + 4 <= nc; c += 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], srec[(c + k) * kRecFloats + kGroup * kHeadDim + hh]);
+      }
+      for (; c < nc; ++c) m4[0] = fmaxf(m4[0], srec[c * kRecFloats + kGroup * kHeadDim + hh]);
+      const float m_new = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
+      den *= resc;
+      r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
+      lse_max = m_new;
+#pragma unroll 4
+      for (int cc = 0; cc < nc; ++cc) {
+        const float* rc = srec + cc * kRecFloats;
+        const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - lse_max);
+        const float4 x = *reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0);
+        den += wgt;
+        r.x += wgt * x.x; r.y += wgt * x.y; r.z += wgt * x.z; r.w += wgt * x.w;
+      }
+      named_barrier(1, kConsumerThreads);
+    }
+    const float id = 1.f / den;
+    const int bb = pp / kNumKVHeads, gg = pp % kNumKVHeads;
+    float* dst = out + (static_cast<int64_t>(bb) * kNumQHeads + gg * kGroup + hh) * kHeadDim + d0;
+    *reinterpret_cast<float4*>(dst) = make_float4(r.x * id, r.y * id, r.z * id, r.w * id);
+    if (tid == 0) counters[pp] = 0;   // ready for the next call
+  };
+
+  // Tickets of the deferred first segment (if any) and of the last segment
+  // (cur_p >= 0), taken by two threads in parallel after one fence over the
+  // records; the last contributor of a pair merges it.
+  int pend_p = -1, pend_lo = 0, pend_hi = 0;
+  auto settle = [&](int cur_p, int cur_lo, int cur_hi) {
+    __threadfence();
+    named_barrier(1, kConsumerThreads);
+    if (tid == 0 && pend_p >= 0) {
+      const int n_contrib = pend_hi - pend_lo + 1;   // every CTA in [lo, hi] owns part of the pair
+      const int old = atomicAdd(&counters[pend_p], 1);
+      if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
+      flags[2] = (old == n_contrib - 1);
+    }
+    if (tid == 32 && cur_p >= 0) {
+      const int n_contrib = cur_hi - cur_lo + 1;
+      const int old = atomicAdd(&counters[cur_p], 1);
+      if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
+      flags[1] = (old == n_contrib - 1);
+    }
+    named_barrier(1, kConsumerThreads);
+    const bool m_pend = pend_p >= 0 && flags[2] != 0;
+    const bool m_cur = cur_p >= 0 && flags[1] != 0;
+    if (m_pend || m_cur) __threadfence();
+    if (m_pend) merge_pair(pend_p, pend_lo, pend_hi);
+    if (m_cur) merge_pair(cur_p, cur_lo, cur_hi);
+    pend_p = -1;
+  };
+
   UnitCursor cur;
   cur.start(cu, B, u0);
   int64_t u = u0;
@@ -359,8 +438,6 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     }
     named_barrier(1, kConsumerThreads);
 
-    const int hh = tid >> 5;          // head within the group (warp-uniform)
-    const int d0 = (tid & 31) * 4;    // 4 consecutive dims
     float mw[kConsumerWarps], M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
@@ -378,102 +455,24 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     }
     const float inv = 1.f / L;
     const int p = b * kNumKVHeads + g;
-    float* dst = out + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + hh) * kHeadDim + d0;
     if (whole_pair) {
+      float* dst = out + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + hh) * kHeadDim + d0;
       *reinterpret_cast<float4*>(dst) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     } else {
       float* rec = records + static_cast<int64_t>(p + blockIdx.x) * kRecFloats;
       *reinterpret_cast<float4*>(rec + hh * kHeadDim + d0) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
       if ((tid & 31) == 0) rec[kGroup * kHeadDim + hh] = M + __log2f(L);
-      __threadfence();
-      named_barrier(1, kConsumerThreads);
       // Contributing CTAs of pair p: those whose unit range meets [a_p, a_p + n_b).
-      const int64_t a_p = 8 * static_cast<int64_t>(cb) + static_cast<int64_t>(g) * n_b;
-      const int c_lo = part.cta_of(static_cast<int>(a_p)), c_hi = part.cta_of(static_cast<int>(a_p + n_b - 1));
-      if (tid == 0) {
-        const int n_contrib = c_hi - c_lo + 1;   // every CTA in [c_lo, c_hi] owns part of the pair
-        const int old = atomicAdd(&counters[p], 1);
-        if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
-        flags[1] = (old == n_contrib - 1);
-      }
-      named_barrier(1, kConsumerThreads);
-      if (flags[1]) {
-        __threadfence();
-        // Merge the partials of pair p in CTA order.  Records of the
-        // contributing CTAs are contiguous (index p + c).
-        const int n_rec = c_hi - c_lo + 1;
-        const float* rbase = records + static_cast<int64_t>(p + c_lo) * kRecFloats;
-        float lse_max = -INFINITY, den = 0.f;
-        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (u + (jend - j0) == u1) {
-          // Last segment of this CTA: the stage ring and the combine buffer
-          // are free, so whole batches of records are pulled into shared
-          // memory with asynchronous 16-byte copies (one L2 round trip per
-          // batch) and folded from there with a running log-sum-exp.  The
-          // log-sum-exp a thread reads is warp-uniform (one head per warp).
-          const float* srec = reinterpret_cast<const float*>(smem);
-          const char* gsrc = reinterpret_cast<const char*>(rbase);
-          for (int c0 = 0; c0 < n_rec; c0 += kStagedRecs) {
-            const int nc = min(kStagedRecs, n_rec - c0);
-            const char* gb = gsrc + static_cast<int64_t>(c0) * kRecBytes;
-            for (int i = tid; i < nc * (kRecBytes / 16); i += kConsumerThreads)
-              cp_async_16_cg(smem_base + i * 16, gb + static_cast<int64_t>(i) * 16);
-            cp_async_wait_all();
-            named_barrier(1, kConsumerThreads);
-            float m4[4] = {lse_max, lse_max, lse_max, lse_max};
-            int c = 0;
-            for (; c + 4 <= nc; c += 4) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], srec[(c + k) * kRecFloats + kGroup * kHeadDim + hh]);
-            }
-            for (; c < nc; ++c) m4[0] = fmaxf(m4[0], srec[c * kRecFloats + kGroup * kHeadDim + hh]);
-            const float m_new = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
-            den *= resc;
-            r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
-            lse_max = m_new;
-#pragma unroll 4
-            for (int cc = 0; cc < nc; ++cc) {
-              const float* rc = srec + cc * kRecFloats;
-              const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - lse_max);
-              const float4 x = *reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0);
-              den += wgt;
-              r.x += wgt * x.x; r.y += wgt * x.y; r.z += wgt * x.z; r.w += wgt * x.w;
-            }
-            named_barrier(1, kConsumerThreads);
-          }
-        } else {
-          // Mid-CTA (the producer may still be filling the ring): fold the
-          // records in batches of 8 from L2, all loads of a batch in flight.
-          for (int c0 = 0; c0 < n_rec; c0 += 8) {
-            float lse[8];
-            float4 x[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int c = min(c0 + k, n_rec - 1);   // tail lanes re-read the last record (weight 0)
-              const float* rc = rbase + static_cast<int64_t>(c) * kRecFloats;
-              lse[k] = __ldcg(rc + kGroup * kHeadDim + hh);
-              x[k] = __ldcg(reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0));
-            }
-            float m_new = lse_max;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              if (c0 + k < n_rec) m_new = fmaxf(m_new, lse[k]);
-            const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
-            den *= resc;
-            r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
-            lse_max = m_new;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float wgt = (c0 + k < n_rec) ? fast_exp2(lse[k] - lse_max) : 0.f;
-              den += wgt;
-              r.x += wgt * x[k].x; r.y += wgt * x[k].y; r.z += wgt * x[k].z; r.w += wgt * x[k].w;
-            }
-          }
-        }
-        const float id = 1.f / den;
-        *reinterpret_cast<float4*>(dst) = make_float4(r.x * id, r.y * id, r.z * id, r.w * id);
-        if (tid == 0) counters[p] = 0;   // ready for the next call
+      const int a_p = 8 * cb + g * n_b;
+      const int c_lo = part.cta_of(a_p), c_hi = part.cta_of(a_p + n_b - 1);
+      if (u + (jend - j0) != u1) {
+        // Only a CTA's first segment can be partial without being its last:
+        // keep streaming and take this pair's ticket at the CTA's end.
+        pend_p = p;
+        pend_lo = c_lo;
+        pend_hi = c_hi;
+      } else {
+        settle(p, c_lo, c_hi);
       }
     }
     named_barrier(1, kConsumerThreads);   // combine buffer free for the next segment
@@ -483,6 +482,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     cur.j = jend - 1;
     cur.advance(cu, B, n_b);
   }
+  if (pend_p >= 0) settle(-1, 0, 0);
 }
 
 // Workspace: int counters[B*8] (padded to 256 B), then fp32 records[(B*8 + kMaxCtas)][kRecFloats].
