@@ -42,7 +42,15 @@ constexpr int kWarpsPerGroup = 4;            // each warp of a group takes 16 of
 constexpr int kConsumerWarps = kGroups * kWarpsPerGroup;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kStages = 6;
+#ifndef LSA_ATTN_STAGES
+#define LSA_ATTN_STAGES 4
+#endif
+constexpr int kStages = LSA_ATTN_STAGES;     // TMA ring depth (32 KiB per stage)
+// Unit i goes to stage i % kStages and to group i % kGroups.  With kStages a
+// multiple of kGroups every stage belongs to one group, which waits on its
+// phases strictly in order; otherwise a group could wait on a phase two ahead
+// of the barrier's and the parity test would succeed early.
+static_assert(kStages % kGroups == 0, "each stage must belong to a single consumer group");
 constexpr int kCtasPerSm = 1;                // one CTA per SM: 8 consumer warps, 6 stages in flight
 constexpr int kBoxBytes = 8192;              // 64 tokens x 64 dims of bf16
 constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo, V hi
