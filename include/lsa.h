@@ -263,7 +263,7 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
  * the library until the process exits).  The caller still owns and passes q,
  * the compact buffers, cu_kept and out; arguments, results and device errors
  * are those of lsa_sparse_decode_attn.  Limits: B <= LSA_NOALLOC_MAX_BATCH
- * and a device of at most 256 SMs (two CTAs per SM), otherwise
+ * and a device of at most 512 SMs (one CTA per SM), otherwise
  * LSA_ERR_UNSUPPORTED_SHAPE.  The call allocates nothing (no cudaMalloc, no
  * cudaFree).  Its first call on a device looks up the array's device address
  * and sets the kernel's shared-memory limit; make that first call before any

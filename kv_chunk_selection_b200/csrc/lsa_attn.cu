@@ -604,7 +604,7 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
 // The array is a file-scope __device__ variable of LSA_NOALLOC_SCRATCH_BYTES
 // bytes: every GPU that loads the library holds it until the process exits.
 // Its size fixes the limits: at most LSA_NOALLOC_MAX_BATCH sequences and a
-// grid of at most LSA_NOALLOC_MAX_CTAS CTAs (two per SM); larger requests are
+// grid of at most LSA_NOALLOC_MAX_CTAS CTAs (one per SM); larger requests are
 // rejected with LSA_ERR_UNSUPPORTED_SHAPE.  All calls on a device share the
 // one array, so calls whose kernels may overlap on the GPU (different
 // streams, or different host threads) race with each other and must be
