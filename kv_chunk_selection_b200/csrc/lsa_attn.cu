@@ -13,20 +13,25 @@
 //   (b, g) pairs are laid end to end, and the grid (one CTA per SM) cuts that
 //   list into equal contiguous ranges (split-K over the kept tokens, balanced
 //   to within one unit per CTA for any batch mix).
-// * A producer warp streams units into a 6-stage shared-memory ring with TMA
+// * A producer warp streams units into a 4-stage shared-memory ring with TMA
 //   (cp.async.bulk.tensor, 128-byte swizzle, evict-first L2 hint) completing
-//   on mbarriers; 4 consumer warps each take 16 of the 64 tokens of a unit.
+//   on mbarriers.  Two groups of 4 consumer warps take alternate units; each
+//   warp of a group takes 16 of the unit's 64 tokens.
 // * Per warp, scores are computed transposed, S^T = K Q^T, on the tensor
 //   cores (mma.sync m16n8k16: M = 16 tokens, N = the 8 query heads of the
 //   group, K = 128), so no MMA row is padding.  The online softmax runs in
 //   fp32 (exp2 domain); probabilities are rounded to bf16, transposed in
 //   registers with movmatrix and used as the B operand of O^T += V^T P^T
 //   (M = 128 dims, N = 8 heads, K = 16 tokens, V^T read with ldmatrix.trans).
-// * At the end of each (b, g) segment the 4 warps combine their (max, sum,
+// * At the end of each (b, g) segment the 8 warps combine their (max, sum,
 //   acc) in shared memory.  A segment that covers the whole pair writes the
-//   output; otherwise it writes a normalised partial and its log-sum-exp, and
-//   the last CTA to finish the pair (atomic ticket) merges all partials of the
-//   pair in CTA order, so the result does not depend on timing.
+//   output; otherwise it writes a normalised partial and its log-sum-exp.  At
+//   the CTA's end it takes the tickets of its (at most two) partial pairs; the
+//   last CTA to finish a pair merges all partials of the pair in CTA order
+//   from shared memory, so the result does not depend on timing.
+// * Launched as a programmatic dependent of the previous kernel: when the
+//   caller states that K/V did not change, the producer starts streaming
+//   before the previous kernel has finished.
 #include <math.h>
 
 #include <mutex>
@@ -51,7 +56,7 @@ constexpr int kStages = LSA_ATTN_STAGES;     // TMA ring depth (32 KiB per stage
 // phases strictly in order; otherwise a group could wait on a phase two ahead
 // of the barrier's and the parity test would succeed early.
 static_assert(kStages % kGroups == 0, "each stage must belong to a single consumer group");
-constexpr int kCtasPerSm = 1;                // one CTA per SM: 8 consumer warps, 6 stages in flight
+constexpr int kCtasPerSm = 1;                // one CTA per SM: 8 consumer warps
 constexpr int kBoxBytes = 8192;              // 64 tokens x 64 dims of bf16
 constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo, V hi
 constexpr int kAccStride = 132;              // padded row of the combine buffer
