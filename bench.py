@@ -213,6 +213,8 @@ def run_host_tier(args, rank, world, local_rank):
     f0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_total + 1)]
     f1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_total + 1)]
 
+    reused = torch.zeros(n_total + 1, dtype=torch.int32, device=dev)
+
     def prepare(w):            # on the side stream: select + fetch window w into buffer w % 2
         buf = w % 2
         if w >= 2:
@@ -220,7 +222,16 @@ def run_host_tier(args, rank, world, local_rank):
         with torch.cuda.stream(side):
             lw.select(L.q_idx[w % n_win], L.w, L.chunk_keys, buf=buf)
             f0[w].record(side)
-            lw.fetch(L.k_pool, L.v_pool, buf=buf, num_ctas=args.fetch_ctas)
+            if args.delta and w >= 1:
+                # chunks window w - 1 also kept come from its buffer (still being read by
+                # its attention: read-only sharing), the rest over the host link
+                pb = (w - 1) % 2
+                lsa.lsa_fetch_from_host_delta(L.k_pool, L.v_pool, inp.chunk_table, lw.kept[buf], lw.cu_kept[buf],
+                                              inp.max_chunks, lw.k_bufs[buf], lw.v_bufs[buf], lw.kept[pb],
+                                              lw.cu_kept[pb], lw.k_bufs[pb], lw.v_bufs[pb], reused[w:w + 1],
+                                              num_ctas=args.fetch_ctas, stream=side)
+            else:
+                lw.fetch(L.k_pool, L.v_pool, buf=buf, num_ctas=args.fetch_ctas)
             f1[w].record(side)
             ev_fetched[w].record(side)
 
@@ -261,6 +272,8 @@ def run_host_tier(args, rank, world, local_rank):
     fetch_s = [f0[w].elapsed_time(f1[w]) / 1e3 for w in range(args.warmup + 1, n_total + 1)]
     kept_total = int(lw.cu_kept[0][-1].item())
     fetch_bytes = kept_total * 2 * workloads.CHUNK_BYTES_ONE
+    reuse = reused[args.warmup + 1:n_total + 1].float().mean().item() if args.delta else 0.0
+    link_bytes = (kept_total - reuse) * 2 * workloads.CHUNK_BYTES_ONE
     elapsed, value = combine_ranks(elapsed, workloads.TAU * B * args.steps, world, dev)
     wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, 1)
     fetch_gbs = fetch_bytes / statistics.median(fetch_s) / 1e9
@@ -273,6 +286,8 @@ def run_host_tier(args, rank, world, local_rank):
                    "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
                    "tau": workloads.TAU, "schedule": "double-buffered: select + fetch of window w+1 on a side "
                    "stream overlaps the 64 attention steps of window w", "fetch_ctas": args.fetch_ctas,
+                   "residency": "chunks kept by the previous window are copied from its device buffer"
+                   if args.delta else "every kept chunk is fetched from the host pool",
                    "l2": "inputs larger than L2 (host pool 8 GiB, 410 MiB per attention launch)"},
         "roofline": {"kernel": "gather_kernel (host-tier fetch)", "bound": "pcie", "achieved": fetch_gbs,
                      "peak": probe, "unit": "GB/s", "frac": fetch_gbs / probe,
@@ -281,7 +296,9 @@ def run_host_tier(args, rank, world, local_rank):
         "hbm": {"window_gbs": wbytes * args.steps / elapsed / 1e9, "copy_probe_gbs": copy_gbs,
                 "frac_of_measured": wbytes * args.steps / elapsed / 1e9 / peak},
         "pcie": {"fetch_bytes_per_window": fetch_bytes, "fetch_gbs_median": fetch_gbs, "h2d_probe_gbs": probe,
-                 "window_bound_by_fetch_ms": fetch_bytes / probe / 1e6},
+                 "window_bound_by_fetch_ms": fetch_bytes / probe / 1e6, "delta": bool(args.delta),
+                 "reused_chunks_per_window": reuse, "host_link_bytes_per_window": link_bytes,
+                 "host_link_gbs": link_bytes / statistics.median(fetch_s) / 1e9},
         "gpu_launches": args.steps * (3 + workloads.TAU),
         "clocks": clocks, "e2e": None,
     }
@@ -654,6 +671,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--fetch-ctas", type=int, default=64)
+    ap.add_argument("--delta", action="store_true",
+                    help="host tier: reuse chunks the previous window kept from its device buffer")
     ap.add_argument("--selection", choices=["topk", "threshold"], default="topk",
                     help="chunk selection: fixed top-K budget (default) or the sigmoid threshold")
     ap.add_argument("--threshold", type=float, default=0.5)

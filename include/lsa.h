@@ -209,6 +209,30 @@ int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_
 #define LSA_ATTN_KV_UNCHANGED 1u
 
 /*
+ * lsa_fetch_from_host_delta -- lsa_fetch_from_host with residency across
+ * windows (the eviction of non-recalled entries and the retention of recalled
+ * ones, summary page, 2.1 Architecture): a kept chunk that was also kept in
+ * the previous window of the same sequence is copied from that window's
+ * compact buffer in device memory instead of over the host link.  The result
+ * is identical to lsa_fetch_from_host.
+ *   prev_kept, prev_cu_kept  device int32 [B][prev_max_kept], [B+1]: the
+ *                            previous window's selection (ascending lists)
+ *   prev_k_buf, prev_v_buf   device bf16 [prev_buf_chunks][8][64][128]: its
+ *                            compact buffers (must not be k_buf / v_buf)
+ *   reused_chunks            optional device int32 counter, incremented once
+ *                            per chunk copied from the previous buffers
+ * Other arguments and device errors as lsa_fetch_from_host.
+ */
+int lsa_fetch_from_host_delta(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                              const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept,
+                              int B, int max_chunks, int max_kept, void* k_buf, void* v_buf,
+                              int64_t buf_chunks, const int32_t* prev_kept,
+                              const int32_t* prev_cu_kept, int prev_max_kept,
+                              const void* prev_k_buf, const void* prev_v_buf,
+                              int64_t prev_buf_chunks, int32_t* reused_chunks, int num_ctas,
+                              void* stream, void* done_event);
+
+/*
  * Bytes of workspace lsa_sparse_decode_attn needs for a batch of B sequences.
  * The workspace must be zero-filled once before its first use; every call
  * leaves it ready for the next one.

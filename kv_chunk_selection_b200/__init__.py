@@ -59,6 +59,7 @@ def _load():
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
         "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
+        "lsa_fetch_from_host_delta": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P, P, I, P, P, I64, P, I, P, P], I),
         "lsa_attn_workspace_size": ([I], S),
         "lsa_sparse_decode_attn": ([P, P, P, I64, P, I, F, P, P, S, ctypes.c_uint, P], I),
         "lsa_sparse_decode_attn_noalloc": ([P, P, P, I64, P, I, F, P, P], I),
@@ -213,6 +214,33 @@ def lsa_fetch_from_host(host_k_pool, host_v_pool, chunk_table, kept, cu_kept, ma
         _stream(stream), ev))
 
 
+def lsa_fetch_from_host_delta(host_k_pool, host_v_pool, chunk_table, kept, cu_kept, max_chunks, k_buf, v_buf,
+                              prev_kept, prev_cu_kept, prev_k_buf, prev_v_buf, reused_chunks=None, num_ctas=0,
+                              stream=None, done_event: Optional[torch.cuda.Event] = None):
+    """lsa_fetch_from_host, copying chunks the previous window also kept from its device buffers."""
+    for t, n in ((host_k_pool, "host_k_pool"), (host_v_pool, "host_v_pool")):
+        _need(t, n, torch.bfloat16, cuda=False)
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf"), (prev_k_buf, "prev_k_buf"), (prev_v_buf, "prev_v_buf")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((kept, "kept"), (cu_kept, "cu_kept"), (prev_kept, "prev_kept"), (prev_cu_kept, "prev_cu_kept")):
+        _need(t, n, torch.int32)
+    if chunk_table is not None:
+        _need(chunk_table, "chunk_table", torch.int32)
+    if reused_chunks is not None:
+        _need(reused_chunks, "reused_chunks", torch.int32)
+    B, max_kept = kept.shape
+    ev = None
+    if done_event is not None:
+        if not done_event.cuda_event:
+            done_event.record(stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream())
+        ev = ctypes.c_void_p(done_event.cuda_event)
+    _check("lsa_fetch_from_host_delta", _load().lsa_fetch_from_host_delta(
+        _ptr(host_k_pool), _ptr(host_v_pool), host_k_pool.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(cu_kept),
+        B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(prev_kept),
+        _ptr(prev_cu_kept), prev_kept.shape[1], _ptr(prev_k_buf), _ptr(prev_v_buf), prev_k_buf.shape[0],
+        _ptr(reused_chunks), int(num_ctas), _stream(stream), ev))
+
+
 def lsa_attn_workspace_size(B: int) -> int:
     return int(_load().lsa_attn_workspace_size(int(B)))
 
@@ -275,7 +303,7 @@ def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=
 __all__ = [
     "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
     "lsa_threshold_chunks",
-    "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_attn_workspace_size", "new_attn_workspace",
+    "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

@@ -35,11 +35,37 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int B, int i) {
   return lo;
 }
 
+// Chunks kept in the previous window and still resident in its compact
+// buffer (residency across windows): a kept chunk found in the previous
+// window's kept list of the same sequence is copied from device memory
+// instead of the host pool.
+struct PrevWindow {
+  const int32_t* kept;     // [B][max_kept] ascending, or nullptr (no reuse)
+  const int32_t* cu;       // [B+1]
+  int max_kept;
+  int64_t buf_chunks;
+  const uint4* k_buf;
+  const uint4* v_buf;
+  int32_t* reused;         // optional counter of reused chunks
+};
+
+// Index of chunk c in the ascending list a[0..n), or -1.
+__device__ __forceinline__ int find_sorted(const int32_t* a, int n, int c) {
+  int lo = 0, hi = n - 1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = __ldg(a + mid);
+    if (v == c) return mid;
+    if (v < c) lo = mid + 1; else hi = mid - 1;
+  }
+  return -1;
+}
+
 __global__ void __launch_bounds__(kThreads)
 gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool, int64_t n_slots,
               const int32_t* __restrict__ table, const int32_t* __restrict__ kept, const int32_t* __restrict__ cu,
               int B, int max_chunks, int max_kept, uint4* __restrict__ k_buf, uint4* __restrict__ v_buf,
-              int64_t buf_chunks, unsigned* status) {
+              int64_t buf_chunks, unsigned* status, PrevWindow prev) {
   const int total = __ldg(cu + B);
   if (__ldg(cu) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
@@ -69,6 +95,16 @@ gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool
     }
     const int64_t tile = static_cast<int64_t>(kNumKVHeads) * kVecPerTile;  // uint4 per chunk
     const uint4* src = (kv ? v_pool : k_pool) + slot * tile + h * kVecPerTile;
+    if (prev.kept) {
+      const int pb = __ldg(prev.cu + b), pn = __ldg(prev.cu + b + 1) - pb;
+      if (pb >= 0 && pn > 0 && pn <= prev.max_kept && static_cast<int64_t>(pb) + pn <= prev.buf_chunks) {
+        const int jp = find_sorted(prev.kept + static_cast<int64_t>(b) * prev.max_kept, pn, c);
+        if (jp >= 0) {
+          src = (kv ? prev.v_buf : prev.k_buf) + (static_cast<int64_t>(pb) + jp) * tile + h * kVecPerTile;
+          if (prev.reused && kv == 0 && h == 0 && threadIdx.x == 0) atomicAdd(prev.reused, 1);
+        }
+      }
+    }
     uint4* dst = (kv ? v_buf : k_buf) + static_cast<int64_t>(i) * tile + h * kVecPerTile;
     uint4 r[kVecPerThread];
 #pragma unroll
@@ -107,14 +143,17 @@ int lsa_gather_chunks(const void* k_pool, const void* v_pool, int64_t n_slots, c
   gather::gather_kernel<<<sms * 8, gather::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(k_pool), static_cast<const uint4*>(v_pool), n_slots, chunk_table, kept, cu_kept, B,
       max_chunks, max_kept, static_cast<uint4*>(k_buf), static_cast<uint4*>(v_buf), buf_chunks,
-      lsa_device_status_ptr());
+      lsa_device_status_ptr(), gather::PrevWindow{});
   return launch_status();
 }
 
-int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
-                        const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept, int B,
-                        int max_chunks, int max_kept, void* k_buf, void* v_buf, int64_t buf_chunks, int num_ctas,
-                        void* stream, void* done_event) {
+}  // extern "C"
+
+namespace {
+int fetch_impl(const void* host_k_pool, const void* host_v_pool, int64_t n_slots, const int32_t* chunk_table,
+               const int32_t* kept, const int32_t* cu_kept, int B, int max_chunks, int max_kept, void* k_buf,
+               void* v_buf, int64_t buf_chunks, int num_ctas, void* stream, void* done_event,
+               const lsa::gather::PrevWindow& prev) {
   using namespace lsa;
   const int st = gather::check_common(host_k_pool, host_v_pool, n_slots, kept, cu_kept, B, max_chunks, max_kept,
                                       k_buf, v_buf, buf_chunks);
@@ -140,7 +179,7 @@ int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_
   gather::gather_kernel<<<grid, gather::kThreads, 0, s>>>(
       static_cast<const uint4*>(dk), static_cast<const uint4*>(dv), n_slots, chunk_table, kept, cu_kept, B,
       max_chunks, max_kept, static_cast<uint4*>(k_buf), static_cast<uint4*>(v_buf), buf_chunks,
-      lsa_device_status_ptr());
+      lsa_device_status_ptr(), prev);
   int rc = launch_status();
   if (rc == LSA_OK && done_event) {
     if (cudaEventRecord(static_cast<cudaEvent_t>(done_event), s) != cudaSuccess) {
@@ -149,6 +188,35 @@ int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_
     }
   }
   return rc;
+}
+}  // namespace
+
+extern "C" {
+
+int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                        const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept, int B,
+                        int max_chunks, int max_kept, void* k_buf, void* v_buf, int64_t buf_chunks, int num_ctas,
+                        void* stream, void* done_event) {
+  return fetch_impl(host_k_pool, host_v_pool, n_slots, chunk_table, kept, cu_kept, B, max_chunks, max_kept, k_buf,
+                    v_buf, buf_chunks, num_ctas, stream, done_event, lsa::gather::PrevWindow{});
+}
+
+int lsa_fetch_from_host_delta(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                              const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept, int B,
+                              int max_chunks, int max_kept, void* k_buf, void* v_buf, int64_t buf_chunks,
+                              const int32_t* prev_kept, const int32_t* prev_cu_kept, int prev_max_kept,
+                              const void* prev_k_buf, const void* prev_v_buf, int64_t prev_buf_chunks,
+                              int32_t* reused_chunks, int num_ctas, void* stream, void* done_event) {
+  using namespace lsa;
+  if (!prev_kept || !prev_cu_kept || !prev_k_buf || !prev_v_buf || prev_max_kept <= 0 || prev_buf_chunks <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (!aligned16(prev_k_buf) || !aligned16(prev_v_buf)) return LSA_ERR_MISALIGNED;
+  if (prev_k_buf == k_buf || prev_v_buf == v_buf) return LSA_ERR_INVALID_ARG;   // must not overlap the target
+  gather::PrevWindow prev{prev_kept, prev_cu_kept, prev_max_kept, prev_buf_chunks,
+                          static_cast<const uint4*>(prev_k_buf), static_cast<const uint4*>(prev_v_buf),
+                          reused_chunks};
+  return fetch_impl(host_k_pool, host_v_pool, n_slots, chunk_table, kept, cu_kept, B, max_chunks, max_kept, k_buf,
+                    v_buf, buf_chunks, num_ctas, stream, done_event, prev);
 }
 
 }  // extern "C"

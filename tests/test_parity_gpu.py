@@ -476,6 +476,38 @@ def test_fetch_from_host_equals_gather():
     status_clean()
 
 
+def test_fetch_delta_reuses_previous_window():
+    """Residency across windows: chunks kept in both windows come from the previous
+    compact buffer; the result equals a plain host fetch bit for bit, and the reuse
+    count equals the size of the intersection of the two kept sets."""
+    n, k, table, n_slots = paged_case(B=4, seed=21, max_chunks=48)
+    B, M = table.shape
+    g = torch.Generator(device=DEV).manual_seed(22)
+    shape = (n_slots, 8, 64, 128)
+    k_host = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16).cpu().pin_memory()
+    v_host = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16).cpu().pin_memory()
+    n_t, k_t, tab = (torch.from_numpy(x).to(DEV) for x in (n, k, table))
+    s_a = torch.rand((B, M), generator=g, device=DEV)
+    s_b = s_a.clone()
+    s_b[:, ::3] = torch.rand((B, (M + 2) // 3), generator=g, device=DEV)   # partly different selection
+    ka, na, cua = run_topk(s_a, n_t, k_t, int(k.max()) + 1)
+    kb_, nb, cub = run_topk(s_b, n_t, k_t, int(k.max()) + 1)
+    buf = int((k + 1).sum())
+    ak = torch.zeros((buf,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    av = torch.zeros_like(ak)
+    lsa.lsa_fetch_from_host(k_host, v_host, tab, ka, cua, M, ak, av)                 # window A
+    bk, bv, rk, rv = (torch.zeros_like(ak) for _ in range(4))
+    reused = torch.zeros(1, dtype=torch.int32, device=DEV)
+    lsa.lsa_fetch_from_host_delta(k_host, v_host, tab, kb_, cub, M, bk, bv, ka, cua, ak, av, reused)
+    lsa.lsa_fetch_from_host(k_host, v_host, tab, kb_, cub, M, rk, rv)                # plain window B
+    torch.cuda.synchronize()
+    assert torch.equal(bk, rk) and torch.equal(bv, rv)
+    la, lb = kept_from_gpu(ka, na), kept_from_gpu(kb_, nb)
+    inter = sum(len(set(x) & set(y)) for x, y in zip(la, lb))
+    assert int(reused.item()) == inter and inter > 0
+    status_clean()
+
+
 def test_fetch_rejects_unpinned_pool():
     k_host = torch.zeros((4, 8, 64, 128), dtype=torch.bfloat16)     # pageable
     kept = torch.zeros((1, 2), dtype=torch.int32, device=DEV)
