@@ -39,6 +39,14 @@ of the same paper (*FM-DS-V4 review*, with its section).
 5. ``threshold_chunks`` -- the pages' own selection rule: sigmoid thresholding
    at 0.5 in place of a fixed top-k (FM-DS-V4 summary, 2.1 Architecture and
    2.4 Configuration), read as score_c / sum_h w_h > 0.5, latest chunk kept.
+6. ``topk_chunks(..., n_local=L)`` -- the non-offloadable recent context kept
+   beside the recalled chunks (FM-DS-V4 summary, 2.1 Architecture; the local
+   window of 3 Experiments) generalised from the latest chunk to the latest L.
+7. ``sparse_decode_attn(..., k_local, v_local, local_len)`` -- the tokens
+   decoded inside the current window (the decoded window of FM-DS-V4 summary,
+   3 Experiments) are appended before each step attends: attention then runs
+   over the kept chunks plus the first local_len[b] tokens of the sequence's
+   local chunk.
 
 Readings taken where the pages are silent are listed in the design notes of
 this repository and marked "Reading:" at the point of use.
@@ -108,14 +116,16 @@ def index_scores(q_idx, w, chunk_keys, chunk_table, n_chunks, max_chunks=None):
     return out
 
 
-def topk_chunks(scores, n_chunks, k_per_seq):
+def topk_chunks(scores, n_chunks, k_per_seq, n_local=1):
     """Per-sequence kept chunk lists.
 
-    Candidates are the chunks 0 .. n-2 (all but the latest).  They are ordered
-    by score descending, then chunk index ascending; the first K are kept, the
-    latest chunk n-1 is added, and the list is returned in ascending order.
-    Reading: the latest chunk is outside the K budget, so exactly min(K, n-1)+1
-    chunks are kept; K >= n-1 keeps every chunk; n == 0 keeps none.
+    The latest ``n_local`` chunks are always kept (the recent context; one
+    chunk, the latest, by default).  Candidates are the chunks before them,
+    0 .. n-1-n_local.  They are ordered by score descending, then chunk index
+    ascending; the first K are kept, the recent chunks are added, and the list
+    is returned in ascending order.  Reading: the recent chunks are outside the
+    K budget, so exactly min(K, n-L) + L chunks are kept with L = min(n_local, n);
+    K >= n-L keeps every chunk; n == 0 keeps none.
     """
     scores = np.asarray(scores, dtype=np.float64)
     out = []
@@ -125,12 +135,14 @@ def topk_chunks(scores, n_chunks, k_per_seq):
         if n == 0:
             out.append(np.zeros(0, dtype=np.int64))
             continue
-        cand = np.arange(n - 1, dtype=np.int64)
-        s = scores[b, : n - 1]
+        n_rec = min(int(n_local), n)
+        cand = np.arange(n - n_rec, dtype=np.int64)
+        s = scores[b, : n - n_rec]
         # np.lexsort sorts by the last key first: primary key -score, then index.
         order = np.lexsort((cand, -s))
-        chosen = cand[order[: max(0, min(k, n - 1))]]
-        kept = np.sort(np.concatenate([chosen, np.array([n - 1], dtype=np.int64)]))
+        chosen = cand[order[: max(0, min(k, n - n_rec))]]
+        recent = np.arange(n - n_rec, n, dtype=np.int64)
+        kept = np.sort(np.concatenate([chosen, recent]))
         out.append(kept)
     return out
 
@@ -191,15 +203,19 @@ def attend_one(q_h, K, V, scale):
     return (p @ V) / np.sum(p)
 
 
-def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=None):
+def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=None,
+                       k_local=None, v_local=None, local_len=None):
     """GQA decode attention of each query head over its sequence's kept tokens.
 
     q      [B, 64, 128]
     k_buf  [total_kept, 8, 64, 128], v_buf the same
     cu_kept[B+1]
+    k_local, v_local [B, 8, 64, 128] and local_len [B] (optional): the tokens
+    decoded in the current window; the first local_len[b] of them are attended
+    after the kept chunks.
     Query head h reads KV head h // 8 (8 consecutive query heads per KV head).
-    Returns float64 [B, 64, 128]; a sequence with no kept chunk gives zeros
-    (Reading: the empty softmax is defined as a zero output).
+    Returns float64 [B, 64, 128]; a sequence with no token to attend gives
+    zeros (Reading: the empty softmax is defined as a zero output).
     ``seqs``/``heads`` restrict the work to a sample; other rows stay NaN.
     """
     if scale is None:
@@ -211,7 +227,8 @@ def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=No
     heads = range(NUM_Q_HEADS) if heads is None else heads
     for b in seqs:
         lo, hi = int(cu_kept[b]), int(cu_kept[b + 1])
-        if hi == lo:
+        n_loc = 0 if local_len is None else int(local_len[b])
+        if hi == lo and n_loc == 0:
             out[b, list(heads)] = 0.0
             continue
         for g in range(NUM_KV_HEADS):
@@ -220,6 +237,9 @@ def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=No
                 continue
             K = np.asarray(k_buf[lo:hi, g], dtype=np.float64).reshape(-1, HEAD_DIM)
             V = np.asarray(v_buf[lo:hi, g], dtype=np.float64).reshape(-1, HEAD_DIM)
+            if n_loc:
+                K = np.concatenate([K, np.asarray(k_local[b, g, :n_loc], dtype=np.float64)])
+                V = np.concatenate([V, np.asarray(v_local[b, g, :n_loc], dtype=np.float64)])
             for h in group_heads:
                 out[b, h] = attend_one(q[b, h], K, V, scale)
     return out

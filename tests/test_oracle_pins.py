@@ -172,6 +172,66 @@ def test_topk_latest_not_double_counted():
     assert list(oracle.topk_chunks(s2, [12], [3])[0]) == [0, 1, 2, 11]
 
 
+@pytest.mark.parametrize("trial", range(12))
+def test_topk_local_window_matches_full_sort(trial):
+    """Recent context of L chunks: brute force with Python's sorted()."""
+    rng = np.random.default_rng(100 + trial)
+    M = int(rng.integers(1, 50))
+    n = int(rng.integers(0, M + 1))
+    k = int(rng.integers(0, M + 2))
+    L = int(rng.integers(1, 6))
+    scores = rng.integers(0, 3, (1, M)).astype(np.float64) if trial % 2 else rng.standard_normal((1, M))
+    got = list(oracle.topk_chunks(scores, [n], [k], n_local=L)[0])
+    if n == 0:
+        assert got == []
+        return
+    r = min(L, n)
+    cand = sorted(range(n - r), key=lambda c: (-scores[0, c], c))
+    assert got == sorted(cand[: max(0, min(k, n - r))] + list(range(n - r, n)))
+
+
+def test_topk_local_window_default_is_latest_chunk():
+    s = RNG.standard_normal((2, 30))
+    a = oracle.topk_chunks(s, [30, 7], [5, 2])
+    b = oracle.topk_chunks(s, [30, 7], [5, 2], n_local=1)
+    assert all(list(x) == list(y) for x, y in zip(a, b))
+
+
+def test_attention_local_tokens_equal_an_appended_chunk():
+    """A full local chunk (64 decoded tokens) attends exactly like one more kept
+    chunk at the end of the compact buffer; local_len = 0 changes nothing."""
+    rng = np.random.default_rng(31)
+    k_buf, v_buf = _rand_bufs(3, rng)
+    kl, vl = _rand_bufs(2, rng)           # [B=2][8][64][128]
+    q = bf16_round(rng.standard_normal((2, 64, 128)))
+    cu = [0, 2, 3]
+    full = oracle.sparse_decode_attn(q, k_buf, v_buf, cu, k_local=kl, v_local=vl, local_len=[64, 64])
+    k_cat = np.concatenate([k_buf[0:2], kl[0:1], k_buf[2:3], kl[1:2]])
+    v_cat = np.concatenate([v_buf[0:2], vl[0:1], v_buf[2:3], vl[1:2]])
+    ref = oracle.sparse_decode_attn(q, k_cat, v_cat, [0, 3, 5])
+    np.testing.assert_allclose(full, ref, rtol=1e-12, atol=1e-15)
+    none = oracle.sparse_decode_attn(q, k_buf, v_buf, cu, k_local=kl, v_local=vl, local_len=[0, 0])
+    np.testing.assert_array_equal(none, oracle.sparse_decode_attn(q, k_buf, v_buf, cu))
+
+
+def test_attention_local_tokens_only_closed_form():
+    """No kept chunk, local_len = 3 tokens with keys (0, s, 2s) along e_0 and values e_j:
+    the output is the softmax of (0, s, 2s)/sqrt(128) over the first 3 dims."""
+    kl = np.zeros((1, 8, 64, 128))
+    vl = np.zeros((1, 8, 64, 128))
+    for j in range(3):
+        kl[0, :, j, 0] = 4.0 * j
+        vl[0, :, j, j] = 1.0
+    kl[0, :, 3:, 0] = 1e3                 # beyond local_len: must be ignored
+    q = np.zeros((1, 64, 128))
+    q[0, :, 0] = 1.0
+    got = oracle.sparse_decode_attn(q, np.zeros((0, 8, 64, 128)), np.zeros((0, 8, 64, 128)), [0, 0],
+                                    k_local=kl, v_local=vl, local_len=[3])
+    e = np.array([math.exp(4.0 * j / math.sqrt(128)) for j in range(3)])
+    np.testing.assert_allclose(got[0, 17, :3], e / e.sum(), rtol=1e-13)
+    assert np.all(got[0, :, 3:] == 0)
+
+
 def test_threshold_rule():
     w = np.array([0.5, 1.5] + [0.0] * 14)
     s = np.array([[0.2, 1.2, 1.0, 1.01, 0.0]]) * 1.0     # score / sum(w) = s / 2
