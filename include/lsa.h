@@ -149,6 +149,18 @@ int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t*
                     int32_t* cu_kept, void* stream);
 
 /*
+ * lsa_topk_chunks_local -- lsa_topk_chunks with a recent-context window of
+ * n_local >= 1 chunks (the non-offloadable recent context kept beside the
+ * recalled chunks, summary page, 2.1 Architecture and 3 Experiments): the
+ * latest min(n_local, n) chunks are always kept, and K are chosen among the
+ * chunks before them.  n_kept[b] = min(K, n - L) + L with L = min(n_local, n).
+ * lsa_topk_chunks is the n_local = 1 case.
+ */
+int lsa_topk_chunks_local(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq,
+                          int n_local, int B, int max_chunks, int max_kept, int32_t* kept,
+                          int32_t* n_kept, int32_t* cu_kept, void* stream);
+
+/*
  * lsa_threshold_chunks -- the pages' own selection rule: sigmoid thresholding
  * in place of a fixed top-k (summary page, 2.1 Architecture; the 0.5
  * classification threshold of 2.4 Configuration).  Chunk c < n-1 is kept when
@@ -303,6 +315,38 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
 int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, const void* v_buf,
                                    int64_t buf_chunks, const int32_t* cu_kept, int B,
                                    float softmax_scale, float* out, void* stream);
+
+/*
+ * Tokens decoded inside the current window (the local / decoded window the
+ * summary page keeps beside the recalled chunks, 3 Experiments "Experimental
+ * Setup"; it makes each decode step causal).  Each sequence has one local
+ * chunk, k_local / v_local device bf16 [B][8][64][128], holding the tokens
+ * decoded since the window started, and a count local_len device int32 [B]
+ * (0 at the start of a window; the caller resets it).
+ *
+ * lsa_append_token -- writes the new token of every sequence (k_new, v_new
+ * device bf16 [B][8][128]) at position local_len[b] of its local chunk and
+ * increments local_len[b].  Device error CAPACITY (the local chunk already
+ * holds 64 tokens: nothing is written for that sequence).
+ */
+int lsa_append_token(const void* k_new, const void* v_new, void* k_local, void* v_local,
+                     int32_t* local_len, int B, void* stream);
+
+/*
+ * lsa_sparse_decode_attn_local -- lsa_sparse_decode_attn over the kept chunks
+ * and, after them, the first local_len[b] tokens of each sequence's local
+ * chunk (every 8 query heads on their KV head, as for the kept tokens).  A
+ * sequence with no kept chunk and local_len 0 gets zeros.  The local chunk is
+ * read after the preceding kernel has finished (it is normally written by
+ * lsa_append_token just before), also with LSA_ATTN_KV_UNCHANGED, which then
+ * applies to k_buf, v_buf and cu_kept only.  local_len outside [0, 64] sets
+ * BAD_COUNT and is clamped.  Other arguments as lsa_sparse_decode_attn.
+ */
+int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v_buf,
+                                 int64_t buf_chunks, const int32_t* cu_kept, int B,
+                                 float softmax_scale, const void* k_local, const void* v_local,
+                                 const int32_t* local_len, float* out, void* workspace,
+                                 size_t workspace_bytes, unsigned int flags, void* stream);
 
 #ifdef __cplusplus
 }

@@ -56,6 +56,9 @@ def _load():
         "lsa_selftest_bounded_wait": ([I, P, ctypes.c_uint, P], I),
         "lsa_index_score": ([P, P, P, I64, P, P, I, I, P, P], I),
         "lsa_topk_chunks": ([P, P, P, I, I, I, P, P, P, P], I),
+        "lsa_topk_chunks_local": ([P, P, P, I, I, I, I, P, P, P, P], I),
+        "lsa_append_token": ([P, P, P, P, P, I, P], I),
+        "lsa_sparse_decode_attn_local": ([P, P, P, I64, P, I, F, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
         "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
@@ -145,8 +148,8 @@ def lsa_index_score(q_idx, w, chunk_keys, chunk_table, n_chunks, scores, stream=
         _ptr(scores), _stream(stream)))
 
 
-def lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu_kept, stream=None):
-    """Top-K chunks per sequence (score desc, index asc) plus the latest, ascending."""
+def lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu_kept, stream=None, n_local=1):
+    """Top-K chunks per sequence (score desc, index asc) plus the latest ``n_local``, ascending."""
     for t, n in ((scores, "scores"),):
         _need(t, n, torch.float32)
     for t, n in ((n_chunks, "n_chunks"), (k_per_seq, "k_per_seq"), (kept, "kept"), (n_kept, "n_kept"),
@@ -156,9 +159,9 @@ def lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu_kept, stream=N
     max_kept = kept.shape[1]
     if kept.shape[0] != B or cu_kept.numel() != B + 1 or n_kept.numel() != B:
         raise ValueError("bad shapes")
-    _check("lsa_topk_chunks", _load().lsa_topk_chunks(
-        _ptr(scores), _ptr(n_chunks), _ptr(k_per_seq), B, max_chunks, max_kept, _ptr(kept), _ptr(n_kept),
-        _ptr(cu_kept), _stream(stream)))
+    _check("lsa_topk_chunks_local", _load().lsa_topk_chunks_local(
+        _ptr(scores), _ptr(n_chunks), _ptr(k_per_seq), int(n_local), B, max_chunks, max_kept, _ptr(kept),
+        _ptr(n_kept), _ptr(cu_kept), _stream(stream)))
 
 
 def lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu_kept, threshold=0.5, stream=None):
@@ -280,6 +283,41 @@ def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_sca
         _ptr(workspace), workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
 
 
+def lsa_append_token(k_new, v_new, k_local, v_local, local_len, stream=None):
+    """Appends each sequence's new token ([B, 8, 128]) at local_len[b] of its local chunk; increments it."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_local, "k_local"), (v_local, "v_local")):
+        _need(t, n, torch.bfloat16)
+    _need(local_len, "local_len", torch.int32)
+    B = k_new.shape[0]
+    if tuple(k_new.shape) != (B, NUM_KV_HEADS, HEAD_DIM) or tuple(k_local.shape) != (B, NUM_KV_HEADS,
+                                                                                     CHUNK_TOKENS, HEAD_DIM):
+        raise ValueError("k_new must be [B, 8, 128] and k_local [B, 8, 64, 128]")
+    _check("lsa_append_token", _load().lsa_append_token(
+        _ptr(k_new), _ptr(v_new), _ptr(k_local), _ptr(v_local), _ptr(local_len), B, _stream(stream)))
+
+
+def lsa_sparse_decode_attn_local(q, k_buf, v_buf, cu_kept, k_local, v_local, local_len, out, workspace,
+                                 softmax_scale=None, stream=None, kv_unchanged=False):
+    """Attention over the kept chunks plus the first local_len[b] tokens of each local chunk."""
+    _need(q, "q", torch.bfloat16)
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf"), (k_local, "k_local"), (v_local, "v_local")):
+        _need(t, n, torch.bfloat16)
+    _need(cu_kept, "cu_kept", torch.int32)
+    _need(local_len, "local_len", torch.int32)
+    _need(out, "out", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    B = q.shape[0]
+    if tuple(q.shape) != (B, NUM_Q_HEADS, HEAD_DIM) or tuple(out.shape) != (B, NUM_Q_HEADS, HEAD_DIM):
+        raise ValueError("q and out must be [B, 64, 128]")
+    if tuple(k_local.shape) != (B, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM) or k_local.shape != v_local.shape:
+        raise ValueError("k_local and v_local must be [B, 8, 64, 128]")
+    scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
+    _check("lsa_sparse_decode_attn_local", _load().lsa_sparse_decode_attn_local(
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(k_local),
+        _ptr(v_local), _ptr(local_len), _ptr(out), _ptr(workspace), workspace.numel(),
+        ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
+
+
 def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=None, stream=None):
     """lsa_sparse_decode_attn without a workspace argument, for callers that cannot
     allocate device memory; its scratch is a fixed array inside the library, shared
@@ -304,6 +342,7 @@ __all__ = [
     "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
     "lsa_threshold_chunks",
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
-    "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
+    "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token",
+    "lsa_sparse_decode_attn_local", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

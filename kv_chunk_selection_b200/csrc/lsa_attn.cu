@@ -20,9 +20,10 @@
 // * Per warp, scores are computed transposed, S^T = K Q^T, on the tensor
 //   cores (mma.sync m16n8k16: M = 16 tokens, N = the 8 query heads of the
 //   group, K = 128), so no MMA row is padding.  The online softmax runs in
-//   fp32 (exp2 domain); probabilities are rounded to bf16, transposed in
-//   registers with movmatrix and used as the B operand of O^T += V^T P^T
-//   (M = 128 dims, N = 8 heads, K = 16 tokens, V^T read with ldmatrix.trans).
+//   fp32 (exp2 domain); probabilities are split into two bf16 parts
+//   (P = P_hi + P_lo, about 16 mantissa bits), transposed in registers with
+//   movmatrix and used as the B operands of O^T += V^T P^T (M = 128 dims,
+//   N = 8 heads, K = 16 tokens, V^T read once with ldmatrix.trans).
 // * At the end of each (b, g) segment the 8 warps combine their (max, sum,
 //   acc) in shared memory.  A segment that covers the whole pair writes the
 //   output; otherwise it writes a normalised partial and its log-sum-exp.  At
@@ -84,32 +85,41 @@ struct Partition {
   }
 };
 
-// Largest b in [0, B) with 8 * cu[b] <= u (the sequence that holds unit u).
-__device__ __forceinline__ int seq_of_unit(const int32_t* cu, int B, int64_t u) {
+// Units of sequence b: its kept chunks plus E local chunks (E = 1 when the
+// window's decoded tokens are attended), for each of the 8 KV heads.  The
+// units of sequence b start at 8 * (cu[b] + E * b).
+__device__ __forceinline__ int64_t seq_unit_base(const int32_t* cu, int E, int b) {
+  return 8 * (static_cast<int64_t>(__ldg(cu + b)) + static_cast<int64_t>(E) * b);
+}
+__device__ __forceinline__ int units_of(const int32_t* cu, int E, int b) {
+  return __ldg(cu + b + 1) - __ldg(cu + b) + E;
+}
+// Largest b in [0, B) whose units start at or before u (the sequence of unit u).
+__device__ __forceinline__ int seq_of_unit(const int32_t* cu, int E, int B, int64_t u) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (8 * static_cast<int64_t>(__ldg(cu + mid)) <= u) lo = mid; else hi = mid - 1;
+    if (seq_unit_base(cu, E, mid) <= u) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
 struct UnitCursor {
   int b, g, j;
-  __device__ void start(const int32_t* cu, int B, int64_t u) {
-    b = seq_of_unit(cu, B, u);
-    const int64_t r = u - 8 * static_cast<int64_t>(__ldg(cu + b));
-    const int n = __ldg(cu + b + 1) - __ldg(cu + b);
+  __device__ void start(const int32_t* cu, int E, int B, int64_t u) {
+    b = seq_of_unit(cu, E, B, u);
+    const int64_t r = u - seq_unit_base(cu, E, b);
+    const int n = units_of(cu, E, b);
     g = static_cast<int>(r / n);
     j = static_cast<int>(r - static_cast<int64_t>(g) * n);
   }
-  __device__ void advance(const int32_t* cu, int B, int n_b) {
+  __device__ void advance(const int32_t* cu, int E, int B, int n_b) {
     if (++j == n_b) {
       j = 0;
       if (++g == kNumKVHeads) {
         g = 0;
         ++b;
-        while (b < B && __ldg(cu + b + 1) == __ldg(cu + b)) ++b;
+        while (b < B && units_of(cu, E, b) == 0) ++b;
       }
     }
   }
@@ -120,10 +130,11 @@ inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasP
 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vl,
                           const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu, int B,
-                          int64_t buf_chunks, float scale_log2, float* __restrict__ out,
-                          int* __restrict__ counters, float* __restrict__ records, unsigned* status,
-                          int kv_unchanged) {
+                          int64_t buf_chunks, const int32_t* __restrict__ local_len, float scale_log2,
+                          float* __restrict__ out, int* __restrict__ counters, float* __restrict__ records,
+                          unsigned* status, int kv_unchanged) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte TMA swizzle pattern repeats every 1024 bytes and the fragment
   // addressing below assumes each box starts on such a boundary.
@@ -156,7 +167,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     if (blockIdx.x == 0 && tid == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
     return;
   }
-  const int T = 8 * total;
+  const int E = local_len ? 1 : 0;   // one local unit per (b, g) when decoded tokens are attended
+  const int T = 8 * (total + E * B);
   const int G = gridDim.x;
   const Partition part(T, G);
   const int64_t u0 = part.start(blockIdx.x), u1 = part.start(blockIdx.x + 1);
@@ -164,7 +176,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   // Sequences without kept chunks get zeros (written after the wait).
   auto zero_empty = [&](int first, int stride) {
     for (int b = blockIdx.x; b < B; b += G) {
-      if (__ldg(cu + b + 1) == __ldg(cu + b)) {
+      if (units_of(cu, E, b) == 0) {
         float4* o = reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * kNumQHeads * kHeadDim);
         for (int i = first; i < kNumQHeads * kHeadDim / 4; i += stride) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -197,9 +209,10 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       tma_prefetch_desc(&tm_v);
       const uint64_t policy = l2_policy_evict_first();
       UnitCursor cur;
-      cur.start(cu, B, u0);
+      cur.start(cu, E, B, u0);
       const int64_t n_units = u1 - u0;
       int64_t issued = 0;
+      bool waited = !kv_unchanged;   // the local chunks are written by the preceding kernel
       for (int64_t i = 0; i < n_units; ++i) {
         const int s = static_cast<int>(i % kStages);
         if (i >= kStages) {
@@ -211,16 +224,24 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           }
         }
         const int cb = __ldg(cu + cur.b);
-        const int n_b = __ldg(cu + cur.b + 1) - cb;
-        const int row = ((cb + cur.j) * kNumKVHeads + cur.g) * kChunkTokens;
+        const int n_kept_b = __ldg(cu + cur.b + 1) - cb;
+        const bool local = E && cur.j == n_kept_b;
         uint8_t* st = smem + s * kStageBytes;
+        if (local && !waited) {
+          griddep_wait();
+          waited = true;
+        }
+        const int row = local ? (cur.b * kNumKVHeads + cur.g) * kChunkTokens
+                              : ((cb + cur.j) * kNumKVHeads + cur.g) * kChunkTokens;
+        const CUtensorMap* mk = local ? &tm_kl : &tm_k;
+        const CUtensorMap* mv = local ? &tm_vl : &tm_v;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(st, &tm_k, 0, row, &full[s], policy);
-        tma_load_2d(st + kBoxBytes, &tm_k, 64, row, &full[s], policy);
-        tma_load_2d(st + 2 * kBoxBytes, &tm_v, 0, row, &full[s], policy);
-        tma_load_2d(st + 3 * kBoxBytes, &tm_v, 64, row, &full[s], policy);
+        tma_load_2d(st, mk, 0, row, &full[s], policy);
+        tma_load_2d(st + kBoxBytes, mk, 64, row, &full[s], policy);
+        tma_load_2d(st + 2 * kBoxBytes, mv, 0, row, &full[s], policy);
+        tma_load_2d(st + 3 * kBoxBytes, mv, 64, row, &full[s], policy);
         issued = i + 1;
-        cur.advance(cu, B, n_b);
+        cur.advance(cu, E, B, n_kept_b + E);
       }
       if (*abort_flag) {
         // Let every copy already issued land before the CTA exits.
@@ -285,21 +306,22 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       }
       for (; c < nc; ++c) m4[0] = fmaxf(m4[0], srec[c * kRecFloats + kGroup * kHeadDim + hh]);
       const float m_new = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      const float resc = fast_exp2(lse_max - m_new);   // 0 on the first batch
+      const float mref = m_new == -INFINITY ? 0.f : m_new;   // all partials empty so far
+      const float resc = fast_exp2(lse_max - mref);           // 0 on the first batch
       den *= resc;
       r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
       lse_max = m_new;
 #pragma unroll 4
       for (int cc = 0; cc < nc; ++cc) {
         const float* rc = srec + cc * kRecFloats;
-        const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - lse_max);
+        const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - mref);
         const float4 x = *reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0);
         den += wgt;
         r.x += wgt * x.x; r.y += wgt * x.y; r.z += wgt * x.z; r.w += wgt * x.w;
       }
       named_barrier(1, kConsumerThreads);
     }
-    const float id = 1.f / den;
+    const float id = den > 0.f ? 1.f / den : 0.f;
     const int bb = pp / kNumKVHeads, gg = pp % kNumKVHeads;
     float* dst = out + (static_cast<int64_t>(bb) * kNumQHeads + gg * kGroup + hh) * kHeadDim + d0;
     *reinterpret_cast<float4*>(dst) = make_float4(r.x * id, r.y * id, r.z * id, r.w * id);
@@ -335,13 +357,23 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   };
 
   UnitCursor cur;
-  cur.start(cu, B, u0);
+  cur.start(cu, E, B, u0);
   int64_t u = u0;
   int64_t unit_i = 0;
   while (u < u1) {
     const int b = cur.b, g = cur.g;
     const int cb = __ldg(cu + b);
-    const int n_b = __ldg(cu + b + 1) - cb;
+    const int n_kept_b = __ldg(cu + b + 1) - cb;
+    const int n_b = n_kept_b + E;   // units of the pair
+    // Valid tokens of the pair's local unit (its last unit, when E = 1).
+    int valid_local = 64;
+    if (E) {
+      valid_local = __ldg(local_len + b);
+      if (valid_local < 0 || valid_local > kChunkTokens) {
+        if (tid == 0 && g == 0) set_status(status, LSA_DEV_ERR_BAD_COUNT);
+        valid_local = min(max(valid_local, 0), kChunkTokens);
+      }
+    }
     const int j0 = cur.j;
     const int64_t seg_cap = static_cast<int64_t>(j0) + (u1 - u);
     const int jend = seg_cap < n_b ? static_cast<int>(seg_cap) : n_b;
@@ -385,8 +417,13 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           mma_bf16_16816((t & 1) ? sb : sa, a0, a1, a2, a3, bq[t][0], bq[t][1]);
         }
         // s[0]: (token gl, head 2c4)  s[1]: (gl, 2c4+1)  s[2]: (gl+8, 2c4)  s[3]: (gl+8, 2c4+1)
-        const float s0 = (sa[0] + sb[0]) * scale_log2, s1 = (sa[1] + sb[1]) * scale_log2;
-        const float s2 = (sa[2] + sb[2]) * scale_log2, s3 = (sa[3] + sb[3]) * scale_log2;
+        float s0 = (sa[0] + sb[0]) * scale_log2, s1 = (sa[1] + sb[1]) * scale_log2;
+        float s2 = (sa[2] + sb[2]) * scale_log2, s3 = (sa[3] + sb[3]) * scale_log2;
+        if (E && jj == n_kept_b) {   // local unit: tokens not yet decoded are masked
+          const int tok = wig * 16 + gl;
+          if (tok >= valid_local) s0 = s1 = -INFINITY;
+          if (tok + 8 >= valid_local) s2 = s3 = -INFINITY;
+        }
         float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -394,13 +431,22 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
         }
         const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+        // Reference for the exponentials: the new max, or 0 while every score
+        // seen is masked (keeps alpha and p at 0 instead of NaN).
+        const float rf0 = mn0 == -INFINITY ? 0.f : mn0, rf1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = fast_exp2(m0 - rf0), al1 = fast_exp2(m1 - rf1);
         m0 = mn0;
         m1 = mn1;
-        const uint32_t ptop = pack_bf16(fast_exp2(s0 - mn0), fast_exp2(s1 - mn1));
-        const uint32_t pbot = pack_bf16(fast_exp2(s2 - mn0), fast_exp2(s3 - mn1));
-        l0 = l0 * al0 + bf16_lo(ptop) + bf16_lo(pbot);
-        l1 = l1 * al1 + bf16_hi(ptop) + bf16_hi(pbot);
+        const float p0 = fast_exp2(s0 - rf0), p1 = fast_exp2(s1 - rf1);
+        const float p2 = fast_exp2(s2 - rf0), p3 = fast_exp2(s3 - rf1);
+        // P as a sum of two bf16 parts (P_hi + P_lo carries about 16 bits of
+        // mantissa): a single bf16 rounding of P is too coarse when a softmax
+        // spans only a few tokens.
+        const uint32_t ptop = pack_bf16(p0, p1), pbot = pack_bf16(p2, p3);
+        const uint32_t ptop_lo = pack_bf16(p0 - bf16_lo(ptop), p1 - bf16_hi(ptop));
+        const uint32_t pbot_lo = pack_bf16(p2 - bf16_lo(pbot), p3 - bf16_hi(pbot));
+        l0 = l0 * al0 + p0 + p2;
+        l1 = l1 * al1 + p1 + p3;
         // Rescale only when some running max moved (warp-uniform branch); once
         // the maxima settle, alpha is exactly 1 and the 32 multiplies are skipped.
         if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
@@ -413,14 +459,15 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           }
         }
         // P^T as the B operand (k = token, n = head): transpose the 8x8 blocks.
-        const uint32_t pb0 = movmatrix_trans(ptop);
-        const uint32_t pb1 = movmatrix_trans(pbot);
-        // ---- O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] P^T[16 x 8] ---
+        const uint32_t pb0 = movmatrix_trans(ptop), pb1 = movmatrix_trans(pbot);
+        const uint32_t pl0 = movmatrix_trans(ptop_lo), pl1 = movmatrix_trans(pbot_lo);
+        // ---- O^T[128 dims x 8 heads] += V^T[128 x 16 tokens] (P_hi + P_lo)^T ---
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           uint32_t a0, a1, a2, a3;
           ldmatrix_x4_trans(sbase + vofs[i], a0, a1, a2, a3);
           mma_bf16_16816(acc[i], a0, a1, a2, a3, pb0, pb1);
+          mma_bf16_16816(acc[i], a0, a1, a2, a3, pl0, pl1);
         }
       }
       __syncwarp();
@@ -459,14 +506,15 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     }
     float L = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float Mref = M == -INFINITY ? 0.f : M;   // every score of the segment masked: o = 0
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      const float sc = fast_exp2(mw[w] - M);   // 0 for a warp that saw no unit of this segment
+      const float sc = fast_exp2(mw[w] - Mref);   // 0 for a warp that saw no unit of this segment
       L += sc * lbuf[w * kGroup + hh];
       const float4 x = *reinterpret_cast<const float4*>(accbuf + (w * kGroup + hh) * kAccStride + d0);
       o.x += sc * x.x; o.y += sc * x.y; o.z += sc * x.z; o.w += sc * x.w;
     }
-    const float inv = 1.f / L;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
     const int p = b * kNumKVHeads + g;
     if (whole_pair) {
       float* dst = out + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + hh) * kHeadDim + d0;
@@ -476,7 +524,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       *reinterpret_cast<float4*>(rec + hh * kHeadDim + d0) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
       if ((tid & 31) == 0) rec[kGroup * kHeadDim + hh] = M + __log2f(L);
       // Contributing CTAs of pair p: those whose unit range meets [a_p, a_p + n_b).
-      const int a_p = 8 * cb + g * n_b;
+      const int a_p = static_cast<int>(seq_unit_base(cu, E, b)) + g * n_b;
       const int c_lo = part.cta_of(a_p), c_hi = part.cta_of(a_p + n_b - 1);
       if (u + (jend - j0) != u1) {
         // Only a CTA's first segment can be partial without being its last:
@@ -493,7 +541,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     // Move the cursor to the unit after this segment.
     u += jend - j0;
     cur.j = jend - 1;
-    cur.advance(cu, B, n_b);
+    cur.advance(cu, E, B, n_b);
   }
   if (pend_p >= 0) settle(-1, 0, 0);
 }
@@ -534,18 +582,26 @@ size_t lsa_attn_workspace_size(int B) {
   return lsa::attn::workspace_bytes(B);
 }
 
-int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
-                           const int32_t* cu_kept, int B, float softmax_scale, float* out, void* workspace,
-                           size_t workspace_bytes, unsigned int flags, void* stream) {
+}  // extern "C"
+
+namespace {
+// Shared launcher of lsa_sparse_decode_attn and lsa_sparse_decode_attn_local
+// (k_local == nullptr: no local units).
+int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
+                int B, float softmax_scale, const void* k_local, const void* v_local, const int32_t* local_len,
+                float* out, void* workspace, size_t workspace_bytes, unsigned int flags, void* stream) {
   using namespace lsa;
   if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
   if (flags & ~static_cast<unsigned>(LSA_ATTN_KV_UNCHANGED)) return LSA_ERR_INVALID_ARG;
+  const bool local = k_local != nullptr;
+  if (local && (!v_local || !local_len)) return LSA_ERR_INVALID_ARG;
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   // TMA row coordinates are 32-bit: (buf_chunks * 512) rows must fit.
   if (buf_chunks > (int64_t{1} << 22)) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out) || !aligned16(workspace))
     return LSA_ERR_MISALIGNED;
+  if (local && (!aligned16(k_local) || !aligned16(v_local))) return LSA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < attn::workspace_bytes(B)) return LSA_ERR_WORKSPACE;
   const int sms = device_sm_count();
   if (sms <= 0) return LSA_ERR_NO_DEVICE;
@@ -562,11 +618,20 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
       g_attn_attr_set[dev] = true;
     }
   }
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_k, tm_v, tm_kl, tm_vl;
   int st = encode_kv_map(&tm_k, k_buf, buf_chunks);
   if (st != LSA_OK) return st;
   st = encode_kv_map(&tm_v, v_buf, buf_chunks);
   if (st != LSA_OK) return st;
+  if (local) {   // the local chunks: [B][8][64][128], one chunk per sequence
+    st = encode_kv_map(&tm_kl, k_local, B);
+    if (st != LSA_OK) return st;
+    st = encode_kv_map(&tm_vl, v_local, B);
+    if (st != LSA_OK) return st;
+  } else {
+    tm_kl = tm_k;
+    tm_vl = tm_v;
+  }
   const size_t cnt_bytes = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
   int* counters = static_cast<int*>(workspace);
   float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cnt_bytes);
@@ -585,13 +650,33 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int kv_unchanged = (flags & LSA_ATTN_KV_UNCHANGED) ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, attn::sparse_decode_attn_kernel, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q),
-                         cu_kept, B, buf_chunks, scale_log2, out, counters, records, lsa_device_status_ptr(),
-                         kv_unchanged) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, attn::sparse_decode_attn_kernel, tm_k, tm_v, tm_kl, tm_vl,
+                         static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
+                         local ? local_len : static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records,
+                         lsa_device_status_ptr(), kv_unchanged) != cudaSuccess) {
     cudaGetLastError();
     return LSA_ERR_CUDA;
   }
   return launch_status();
+}
+}  // namespace
+
+extern "C" {
+
+int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
+                           const int32_t* cu_kept, int B, float softmax_scale, float* out, void* workspace,
+                           size_t workspace_bytes, unsigned int flags, void* stream) {
+  return attn_launch(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, nullptr, nullptr, nullptr, out,
+                     workspace, workspace_bytes, flags, stream);
+}
+
+int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
+                                 const int32_t* cu_kept, int B, float softmax_scale, const void* k_local,
+                                 const void* v_local, const int32_t* local_len, float* out, void* workspace,
+                                 size_t workspace_bytes, unsigned int flags, void* stream) {
+  if (!k_local) return LSA_ERR_INVALID_ARG;
+  return attn_launch(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, k_local, v_local, local_len, out,
+                     workspace, workspace_bytes, flags, stream);
 }
 
 }  // extern "C"
@@ -691,7 +776,7 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   }
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
-      tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks, scale_log2, out, counters, records,
-      lsa_device_status_ptr(), 0);
+      tm_k, tm_v, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
+      static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records, lsa_device_status_ptr(), 0);
   return launch_status();
 }

@@ -114,6 +114,30 @@ gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool
   }
 }
 
+// Appends one decoded token per sequence to its local chunk: K/V of the new
+// token ([B][8][128] each) go to position local_len[b] of k_local / v_local
+// ([B][8][64][128]), then local_len[b] is incremented.
+__global__ void __launch_bounds__(256)
+append_token_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_local,
+                    uint4* __restrict__ v_local, int32_t* __restrict__ local_len, unsigned* status) {
+  constexpr int kVecPerToken = kNumKVHeads * kHeadDim / 8;   // 128 x 16 B per token (all 8 heads)
+  constexpr int kVecPerRow = kHeadDim / 8;                   // 16 x 16 B per (head, token)
+  const int b = blockIdx.x;
+  const int pos = local_len[b];
+  if (pos < 0 || pos >= kChunkTokens) {
+    if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
+    return;
+  }
+  for (int i = threadIdx.x; i < 2 * kVecPerToken; i += blockDim.x) {
+    const int kv = i / kVecPerToken, r = i % kVecPerToken;
+    const int g = r / kVecPerRow, e = r % kVecPerRow;
+    const uint4 v = __ldg((kv ? v_new : k_new) + static_cast<int64_t>(b) * kVecPerToken + r);
+    (kv ? v_local : k_local)[((static_cast<int64_t>(b) * kNumKVHeads + g) * kChunkTokens + pos) * kVecPerRow + e] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) local_len[b] = pos + 1;
+}
+
 int check_common(const void* k_pool, const void* v_pool, int64_t n_slots, const int32_t* kept,
                  const int32_t* cu_kept, int B, int max_chunks, int max_kept, const void* k_buf, const void* v_buf,
                  int64_t buf_chunks) {
@@ -217,6 +241,19 @@ int lsa_fetch_from_host_delta(const void* host_k_pool, const void* host_v_pool, 
                           reused_chunks};
   return fetch_impl(host_k_pool, host_v_pool, n_slots, chunk_table, kept, cu_kept, B, max_chunks, max_kept, k_buf,
                     v_buf, buf_chunks, num_ctas, stream, done_event, prev);
+}
+
+int lsa_append_token(const void* k_new, const void* v_new, void* k_local, void* v_local, int32_t* local_len, int B,
+                     void* stream) {
+  using namespace lsa;
+  if (!k_new || !v_new || !k_local || !v_local || !local_len || B <= 0) return LSA_ERR_INVALID_ARG;
+  if (B > 65535) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_local) || !aligned16(v_local)) return LSA_ERR_MISALIGNED;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  gather::append_token_kernel<<<B, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_local),
+      static_cast<uint4*>(v_local), local_len, lsa_device_status_ptr());
+  return launch_status();
 }
 
 }  // extern "C"

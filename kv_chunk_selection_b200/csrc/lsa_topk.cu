@@ -35,14 +35,16 @@ __device__ __forceinline__ uint32_t desc_key(float s) {
   return ~ord;
 }
 
-// Kept count of one sequence, or 0 with *err set when its counts are invalid.
-__device__ __forceinline__ int kept_count(int n, int k, int max_chunks, int max_kept, unsigned* err) {
+// Kept count of one sequence (K chosen among the chunks before the latest
+// n_local, plus those n_local), or 0 with *err set when its counts are invalid.
+__device__ __forceinline__ int kept_count(int n, int k, int n_local, int max_chunks, int max_kept, unsigned* err) {
   if (n < 0 || n > max_chunks || k < 0) {
     *err |= LSA_DEV_ERR_BAD_COUNT;
     return 0;
   }
   if (n == 0) return 0;
-  const int nk = min(k, n - 1) + 1;
+  const int n_rec = min(n_local, n);
+  const int nk = min(k, n - n_rec) + n_rec;
   if (nk > max_kept) {
     *err |= LSA_DEV_ERR_CAPACITY;
     return 0;
@@ -228,7 +230,7 @@ __device__ void select_and_write(const float* __restrict__ sc, int cand, int kc,
 
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
-            const int32_t* __restrict__ k_per_seq, int B, int max_chunks, int max_kept,
+            const int32_t* __restrict__ k_per_seq, int n_local, int B, int max_chunks, int max_kept,
             int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, int32_t* __restrict__ cu_kept,
             unsigned* status) {
   __shared__ int hist[256];
@@ -241,12 +243,12 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   int part = 0;
   unsigned dummy = 0;
   for (int bb = tid; bb <= b; bb += kThreads)
-    part += kept_count(__ldg(n_chunks + bb), __ldg(k_per_seq + bb), max_chunks, max_kept, &dummy);
+    part += kept_count(__ldg(n_chunks + bb), __ldg(k_per_seq + bb), n_local, max_chunks, max_kept, &dummy);
   int tot = 0;
   block_exclusive_scan(part, warp_sums, &tot);
   unsigned err = 0;
   const int n = __ldg(n_chunks + b);
-  const int nk = kept_count(n, __ldg(k_per_seq + b), max_chunks, max_kept, &err);
+  const int nk = kept_count(n, __ldg(k_per_seq + b), n_local, max_chunks, max_kept, &err);
   if (tid == 0) {
     cu_kept[b + 1] = tot;
     if (b == 0) cu_kept[0] = 0;
@@ -255,13 +257,14 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   }
   if (nk == 0) return;
   int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
-  const int cand = n - 1;
-  const int kc = nk - 1;
+  const int n_rec = min(n_local, n);   // the recent chunks, always kept and last
+  const int cand = n - n_rec;
+  const int kc = nk - n_rec;
   if (kc == cand) {  // keep every chunk
     for (int c = tid; c < n; c += kThreads) out[c] = c;
     return;
   }
-  if (tid == 0) out[kc] = n - 1;  // the latest chunk, always last
+  for (int i = tid; i < n_rec; i += kThreads) out[kc + i] = cand + i;
   if (kc == 0) return;
   const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
   const int per = (cand + kThreads - 1) / kThreads;
@@ -274,19 +277,26 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
 }  // namespace topk
 }  // namespace lsa
 
-extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq, int B,
-                               int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
-                               void* stream) {
+extern "C" int lsa_topk_chunks_local(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq,
+                                     int n_local, int B, int max_chunks, int max_kept, int32_t* kept,
+                                     int32_t* n_kept, int32_t* cu_kept, void* stream) {
   using namespace lsa;
   if (!scores || !n_chunks || !k_per_seq || !kept || !n_kept || !cu_kept || B <= 0 || max_chunks <= 0 ||
-      max_kept <= 0)
+      max_kept <= 0 || n_local <= 0)
     return LSA_ERR_INVALID_ARG;
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   topk::topk_kernel<<<B, topk::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      scores, n_chunks, k_per_seq, B, max_chunks, max_kept, kept, n_kept, cu_kept, lsa_device_status_ptr());
+      scores, n_chunks, k_per_seq, n_local, B, max_chunks, max_kept, kept, n_kept, cu_kept, lsa_device_status_ptr());
   return launch_status();
+}
+
+extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq, int B,
+                               int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
+                               void* stream) {
+  return lsa_topk_chunks_local(scores, n_chunks, k_per_seq, 1, B, max_chunks, max_kept, kept, n_kept, cu_kept,
+                               stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -289,6 +289,83 @@ def test_attention_ragged_matches_oracle(n_kept):
     status_clean()
 
 
+@pytest.mark.parametrize("n_kept,local_len", [([0, 3, 150, 9], [0, 1, 17, 64]), ([5], [64]), ([0, 0], [3, 0]),
+                                               ([300, 1, 40], [63, 2, 32])])
+def test_attention_local_tokens_match_oracle(n_kept, local_len):
+    q, kb, vb, cu = ragged_buffers(n_kept, seed=41)
+    B = len(n_kept)
+    g = torch.Generator(device=DEV).manual_seed(42)
+    kl = torch.randn((B, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    vl = torch.randn((B, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    ll = torch.tensor(local_len, dtype=torch.int32, device=DEV)
+    out = torch.full((B, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_sparse_decode_attn_local(q, kb, vb, cu, kl, vl, ll, out, lsa.new_attn_workspace(B))
+    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), k_local=f64(kl), v_local=f64(vl),
+                                    local_len=local_len)
+    assert_attention_close(out, ref)
+    status_clean()
+
+
+def test_append_then_attend_is_causal():
+    """A window of decode steps: each step appends its token, then attends over the
+    kept chunks plus every token decoded so far (compared with the oracle)."""
+    n_kept = [7, 60]
+    q, kb, vb, cu = ragged_buffers(n_kept, seed=43)
+    B = len(n_kept)
+    g = torch.Generator(device=DEV).manual_seed(44)
+    steps = 6
+    k_new = torch.randn((steps, B, 8, 128), generator=g, device=DEV).to(torch.bfloat16)
+    v_new = torch.randn((steps, B, 8, 128), generator=g, device=DEV).to(torch.bfloat16)
+    qs = torch.randn((steps, B, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    kl = torch.zeros((B, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    vl = torch.zeros_like(kl)
+    ll = torch.zeros(B, dtype=torch.int32, device=DEV)
+    ws = lsa.new_attn_workspace(B)
+    outs = torch.empty((steps, B, 64, 128), device=DEV)
+    for t in range(steps):
+        lsa.lsa_append_token(k_new[t], v_new[t], kl, vl, ll)
+        lsa.lsa_sparse_decode_attn_local(qs[t], kb, vb, cu, kl, vl, ll, outs[t], ws, kv_unchanged=t > 0)
+    torch.cuda.synchronize()
+    assert i64(ll).tolist() == [steps] * B
+    for t in (0, steps - 1):
+        kloc = np.zeros((B, 8, 64, 128))
+        vloc = np.zeros((B, 8, 64, 128))
+        kloc[:, :, : t + 1] = f64(k_new[: t + 1]).transpose(1, 2, 0, 3)
+        vloc[:, :, : t + 1] = f64(v_new[: t + 1]).transpose(1, 2, 0, 3)
+        ref = oracle.sparse_decode_attn(f64(qs[t]), f64(kb), f64(vb), i64(cu), k_local=kloc, v_local=vloc,
+                                        local_len=[t + 1] * B)
+        assert_attention_close(outs[t], ref)
+    status_clean()
+
+
+def test_append_reports_full_local_chunk():
+    kl = torch.zeros((1, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    ll = torch.tensor([64], dtype=torch.int32, device=DEV)
+    tok = torch.ones((1, 8, 128), dtype=torch.bfloat16, device=DEV)
+    lsa.lsa_append_token(tok, tok, kl, kl, ll)
+    assert lsa.read_device_status() & 8
+    assert int(ll.item()) == 64 and int(kl.abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("n_local", [1, 4, 128])
+def test_topk_recent_window_matches_oracle(n_local):
+    inp = workloads.make_inputs("batched", DEV, pools=False, layers=1)
+    n, k = i64(inp.n_chunks), i64(inp.k_per_seq)
+    g = score_on_gpu(inp)
+    B = inp.batch
+    max_kept = int(k.max()) + n_local
+    kept = torch.full((B, max_kept), -7, dtype=torch.int32, device=DEV)
+    n_kept = torch.zeros(B, dtype=torch.int32, device=DEV)
+    cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_topk_chunks(g, inp.n_chunks, inp.k_per_seq, kept, n_kept, cu, n_local=n_local)
+    got = kept_from_gpu(kept, n_kept)
+    ref = oracle.topk_chunks(f64(g), n, k, n_local=n_local)
+    for b in range(B):
+        assert got[b] == list(ref[b]), f"seq {b}"
+    assert i64(cu).tolist() == oracle.cumulative_kept(ref).tolist()
+    status_clean()
+
+
 def test_attention_closed_forms():
     n_kept = [3, 70]
     q, kb, vb, cu = ragged_buffers(n_kept, seed=4)
