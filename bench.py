@@ -9,6 +9,10 @@ inputs (KV pools, indexer keys, queries of every window) are resident on the
 device before timing starts; the window's selection and its 64 attention
 launches are replayed from two captured CUDA graphs per window index.
 
+With ``--causal`` every decode step first appends its own token to the
+sequence's local chunk and then attends the kept chunks plus the tokens decoded
+so far in the window; ``--n-local L`` keeps the latest L chunks.
+
 Metric: decode tokens per second per layer (64 * B tokens per window and
 layer), with the achieved HBM bandwidth of the whole window and of the
 attention kernel against the measured copy bandwidth.
@@ -149,15 +153,24 @@ def copy_probe_gbs(device, nbytes=1 << 31, reps=10):
     return 2 * (nbytes // 2) * 2 / best / 1e9
 
 
-def window_bytes(n_chunks, kept_total, layers):
+TOKEN_KV_BYTES = 2 * 8 * 128 * 2     # K and V of one token, 8 KV heads, bf16
+
+
+def window_bytes(n_chunks, kept_total, layers, causal=False):
     """Algorithmic bytes of one window: indexer keys of every chunk once, and per
     decode step the kept K/V, the query and the fp32 output (gather excluded).
-    ``kept_total`` is the number of kept chunks the selection produced."""
+    ``kept_total`` is the number of kept chunks the selection produced.  A causal
+    window also appends one token per step (read + write) and attends on average
+    (TAU + 1) / 2 decoded tokens per step."""
     n = n_chunks.to(torch.int64).cpu()
     B = int(n.numel())
     keys = 256 * int(n.sum()) + B * 16 * 128 * 2 + 16 * 4
     attn_launch = int(round(kept_total * 2 * workloads.CHUNK_BYTES_ONE)) + B * (64 * 128 * 2 + 64 * 128 * 4)
-    per_layer = keys + workloads.TAU * attn_launch
+    append = 0
+    if causal:
+        attn_launch += int(round(B * (workloads.TAU + 1) / 2 * TOKEN_KV_BYTES))
+        append = B * 2 * TOKEN_KV_BYTES
+    per_layer = keys + workloads.TAU * (attn_launch + append)
     return per_layer * layers, attn_launch, int(n.sum())
 
 
@@ -318,9 +331,12 @@ def run_ours(args, rank, world, local_rank):
     B, layers, n_win = inp.batch, len(inp.layers), inp.workload.windows
     host_tier = inp.workload.host_pool
     lws = [LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev,
-                       selection=args.selection, threshold=args.threshold) for _ in range(layers)]
+                       selection=args.selection, threshold=args.threshold, n_local=args.n_local,
+                       causal=args.causal) for _ in range(layers)]
     outs = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
     stream = torch.cuda.Stream(device=dev)
+    decoded = [workloads.decoded_tokens(inp, l, dev, base_seed=workloads.BASE_SEED + rank) if args.causal else None
+               for l in range(layers)]
 
     def select_phase(w):
         for l, L in enumerate(inp.layers):
@@ -329,10 +345,14 @@ def run_ours(args, rank, world, local_rank):
                 lws[l].fetch(L.k_pool, L.v_pool, num_ctas=args.fetch_ctas)
             else:
                 lws[l].gather(L.k_pool, L.v_pool)
+            if args.causal:
+                lws[l].reset_local()
 
     def attn_phase(w):
         for t in range(workloads.TAU):
             for l, L in enumerate(inp.layers):
+                if args.causal:
+                    lws[l].append(decoded[l][0][w, t], decoded[l][1][w, t])
                 lws[l].attend(L.q[w, t], outs[l][t], kv_unchanged=t > 0)
 
     # warm every path once (and record the kept total of every window index,
@@ -411,7 +431,7 @@ def run_ours(args, rank, world, local_rank):
     elapsed, value = combine_ranks(elapsed, workloads.TAU * B * layers * args.steps, world, dev)
     # mean kept total over the timed windows (identical for every window with top-K)
     kept_total = sum(kept_totals[i % n_win] for i in range(args.steps)) / args.steps
-    wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers)
+    wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers, causal=args.causal)
     hbm_gbs = wbytes * args.steps / elapsed / 1e9
     n_attn = workloads.TAU * layers * args.steps
     attn_avg = att_s / n_attn
@@ -421,7 +441,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API, inputs from pinned host memory ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, inp, lws, dev, stream)
+        e2e = run_e2e(args, inp, lws, dev, stream, decoded)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -431,6 +451,9 @@ def run_ours(args, rank, world, local_rank):
             "workload": inp.workload.description, "name": args.workload, "batch": B, "layers": layers,
             "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
             "selection": args.selection if args.selection == "topk" else f"threshold {args.threshold}",
+            "recent_chunks": args.n_local,
+            "causal": ("each step appends its token to a local chunk and attends it with the kept chunks"
+                       if args.causal else False),
             "tau": workloads.TAU, "gqa": "64q/8kv/d128", "indexer": "16 heads x 128",
             "kv_dtype": "bf16", "softmax_accumulate": "fp32",
             "l2": ("inputs larger than L2: each attention launch streams "
@@ -442,6 +465,7 @@ def run_ours(args, rank, world, local_rank):
             "kernel": ATTN_KERNEL, "bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
             "frac": attn_gbs / peak, "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
             "algorithmic_bytes_per_launch": attn_bytes, "avg_launch_us": attn_avg * 1e6,
+            **({"timed_with": "the append launch before each attention launch"} if args.causal else {}),
         },
         "hbm": {"window_gbs": hbm_gbs, "frac_of_measured": hbm_gbs / peak,
                 "frac_of_nominal_8tbs": hbm_gbs / NOMINAL_HBM_GBS, "copy_probe_gbs": copy_gbs,
@@ -450,22 +474,28 @@ def run_ours(args, rank, world, local_rank):
         "stage_us": {"select_and_gather_per_window": sel_s / args.steps * 1e6,
                      "attention_per_decode_step": attn_avg * 1e6,
                      "attention_64_steps": att_s / args.steps * 1e6},
-        "gpu_launches": args.steps * layers * (3 + workloads.TAU),
+        "gpu_launches": args.steps * layers * (3 + workloads.TAU * (2 if args.causal else 1)),
         "clocks": clocks,
         "e2e": e2e,
     }
     return out
 
 
-def run_e2e(args, inp, lws, dev, stream):
-    """Same metric through the public API: every window copies its queries in from
-    pinned host memory and its 64 outputs back to pinned host memory."""
+def run_e2e(args, inp, lws, dev, stream, decoded=None):
+    """Same metric through the public API: every window copies its queries (and,
+    causal, its decoded tokens) in from pinned host memory and its 64 outputs back
+    to pinned host memory."""
     B, layers = inp.batch, len(inp.layers)
     n_win = inp.workload.windows
+    causal = decoded is not None and decoded[0] is not None
     host_q_idx = [[L.q_idx[w].cpu().pin_memory() for w in range(n_win)] for L in inp.layers]
     host_q = [[L.q[w].cpu().pin_memory() for w in range(n_win)] for L in inp.layers]
     dq_idx = [torch.empty_like(inp.layers[l].q_idx[0]) for l in range(layers)]
     dq = [torch.empty_like(inp.layers[l].q[0]) for l in range(layers)]
+    if causal:
+        host_kv = [[(decoded[l][0][w].cpu().pin_memory(), decoded[l][1][w].cpu().pin_memory())
+                    for w in range(n_win)] for l in range(layers)]
+        dkv = [(torch.empty_like(decoded[l][0][0]), torch.empty_like(decoded[l][1][0])) for l in range(layers)]
     douts = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
     hout = [torch.empty((workloads.TAU, B, 64, 128)).pin_memory() for _ in range(layers)]
     steps = max(1, min(args.steps, args.e2e_steps))
@@ -475,14 +505,21 @@ def run_e2e(args, inp, lws, dev, stream):
         for l, L in enumerate(inp.layers):
             dq_idx[l].copy_(host_q_idx[l][w], non_blocking=True)
             dq[l].copy_(host_q[l][w], non_blocking=True)
+            if causal:
+                dkv[l][0].copy_(host_kv[l][w][0], non_blocking=True)
+                dkv[l][1].copy_(host_kv[l][w][1], non_blocking=True)
         for l, L in enumerate(inp.layers):
             lws[l].select(dq_idx[l], L.w, L.chunk_keys)
             if inp.workload.host_pool:
                 lws[l].fetch(L.k_pool, L.v_pool, num_ctas=args.fetch_ctas)
             else:
                 lws[l].gather(L.k_pool, L.v_pool)
+            if causal:
+                lws[l].reset_local()
         for t in range(workloads.TAU):
             for l in range(layers):
+                if causal:
+                    lws[l].append(dkv[l][0][t], dkv[l][1][t])
                 lws[l].attend(dq[l][t], douts[l][t], kv_unchanged=t > 0)
         for l in range(layers):
             hout[l].copy_(douts[l], non_blocking=True)
@@ -499,7 +536,8 @@ def run_e2e(args, inp, lws, dev, stream):
         e.record(stream)
     torch.cuda.synchronize()
     el = s.elapsed_time(e) / 1e3
-    h2d = layers * (B * 16 * 128 * 2 + workloads.TAU * B * 64 * 128 * 2)
+    h2d = layers * (B * 16 * 128 * 2 + workloads.TAU * B * 64 * 128 * 2
+                    + (workloads.TAU * B * TOKEN_KV_BYTES if causal else 0))
     d2h = layers * workloads.TAU * B * 64 * 128 * 4
     return {"value": workloads.TAU * B * layers * steps / el, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "api": "kv_chunk_selection_b200.window.LayerWindow"}
@@ -568,7 +606,7 @@ def _blas_threads():
         return 1
 
 
-def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warmup=0):
+def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warmup=0, causal=False, n_local=1):
     """Times the fp64 oracle on a bounded sample of the workload.
 
     The sample is one full selection of window 0 of layer 0 (scoring of every
@@ -576,7 +614,8 @@ def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warm
     window, each over one KV head group (8 query heads), rotating over groups
     and steps until ``budget_s`` seconds (or ``group_steps`` steps) are spent.
     Throughput is extrapolated to whole windows: 64 * B tokens per
-    (selection + 64 steps x 8 groups).
+    (selection + 64 steps x 8 groups).  ``causal``: step t also attends the
+    t + 1 tokens decoded so far in the window.
     """
     import numpy as np
 
@@ -594,10 +633,16 @@ def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warm
     kpool = L.k_pool.view(torch.int16).cpu().numpy()
     vpool = L.v_pool.view(torch.int16).cpu().numpy()
     qs = L.q[0].float().cpu().numpy()
+    k_loc = v_loc = None
+    if causal:
+        # local chunk [B, 8, 64, 128]: the token of step t at position t
+        kn, vn = workloads.decoded_tokens(inp, 0, dev, windows=1)
+        k_loc = kn[0].permute(1, 2, 0, 3).float().cpu().numpy()
+        v_loc = vn[0].permute(1, 2, 0, 3).float().cpu().numpy()
     del inp, L
     t0 = time.perf_counter()
     scores = oracle.index_scores(q_idx, w, keys, table, n, int(table.shape[1]))
-    kept = oracle.topk_chunks(scores, n, k)
+    kept = oracle.topk_chunks(scores, n, k, n_local=n_local)
     kb_bits, vb_bits, cu = oracle.gather_chunks(kpool, vpool, table, kept, int(table.shape[1]))
     kb = oracle.bf16_bits_to_f64(kb_bits)
     vb = oracle.bf16_bits_to_f64(vb_bits)
@@ -611,7 +656,11 @@ def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warm
         t = (i * 7) % workloads.TAU
         heads = list(range(8 * g, 8 * g + 8))
         a = time.perf_counter()
-        oracle.sparse_decode_attn(qs[t], kb, vb, cu, heads=heads)
+        if causal:
+            oracle.sparse_decode_attn(qs[t], kb, vb, cu, heads=heads, k_local=k_loc, v_local=v_loc,
+                                      local_len=[t + 1] * B)
+        else:
+            oracle.sparse_decode_attn(qs[t], kb, vb, cu, heads=heads)
         if i >= warmup:
             times.append(time.perf_counter() - a)
         i += 1
@@ -625,7 +674,7 @@ def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warm
     sample = (f"{workload}: one selection of window 0 (score {int(n.sum())} chunks, top-K, gather "
               f"{int(cu[-1])} chunks) timed once ({t_sel:.2f} s) + {len(times)} decode-attention steps over one "
               f"KV-head group (8 query heads) each ({t_group * 1e3:.1f} ms mean); extrapolated to a window of "
-              f"64 steps x 8 groups")
+              f"64 steps x 8 groups" + ("; causal: step t also attends t + 1 decoded tokens" if causal else ""))
     return {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", "sample": sample,
             "window_s_extrapolated": window_s, "host_cpus": os.cpu_count()}, times, t_sel
 
@@ -635,7 +684,7 @@ def run_reference(args, rank, world):
         return None
     t_start = time.perf_counter()
     base, times, t_sel = oracle_sample(args.workload, budget_s=1e9, group_steps=args.steps + args.warmup,
-                                       warmup=0)
+                                       warmup=0, causal=args.causal, n_local=args.n_local)
     times = times[args.warmup:]
     import numpy as np
     t_group = float(np.mean(times))
@@ -648,6 +697,7 @@ def run_reference(args, rank, world):
         "warmup": args.warmup, "ms_per_step": t_group * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workloads.WORKLOADS[args.workload].description, "name": args.workload,
+                   "recent_chunks": args.n_local, "causal": bool(args.causal),
                    "step": "one decode-attention step over one KV-head group, selection timed once and "
                            "amortised over the 64-step window"},
         "cpu_baseline": base, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -676,12 +726,19 @@ def main():
     ap.add_argument("--selection", choices=["topk", "threshold"], default="topk",
                     help="chunk selection: fixed top-K budget (default) or the sigmoid threshold")
     ap.add_argument("--threshold", type=float, default=0.5)
+    ap.add_argument("--n-local", type=int, default=1, help="recent chunks always kept (top-K selection)")
+    ap.add_argument("--causal", action="store_true",
+                    help="append each step's token to a local chunk and attend it (decoded window)")
     ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
     ap.add_argument("--attn-only", action="store_true",
                     help="time attention launches alone on a random compact buffer (profiling case)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if (args.causal or args.n_local != 1) and workloads.WORKLOADS[args.workload].host_pool:
+        ap.error("--causal and --n-local apply to device-resident workloads, not the host tier")
+    if args.n_local != 1 and args.selection != "topk":
+        ap.error("--n-local applies to top-K selection")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -700,7 +757,8 @@ def main():
     # The oracle sample runs before any CUDA work of this process (rank 0, N = 1 only).
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu, _, _ = oracle_sample(args.workload, args.cpu_budget_s, on_gpu_inputs=True)
+        cpu, _, _ = oracle_sample(args.workload, args.cpu_budget_s, on_gpu_inputs=True, causal=args.causal,
+                                  n_local=args.n_local)
         torch.cuda.empty_cache()
 
     if world > 1:

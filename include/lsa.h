@@ -333,6 +333,14 @@ int lsa_append_token(const void* k_new, const void* v_new, void* k_local, void* 
                      int32_t* local_len, int B, void* stream);
 
 /*
+ * lsa_reset_local -- empties every sequence's local chunk at the start of a
+ * window: local_len (device int32 [B]) is set to 0, stream-ordered (a memset
+ * on `stream`, capturable in a CUDA graph; no kernel).  The local K/V rows
+ * are left as they are; the attention reads only the first local_len[b].
+ */
+int lsa_reset_local(int32_t* local_len, int B, void* stream);
+
+/*
  * lsa_sparse_decode_attn_local -- lsa_sparse_decode_attn over the kept chunks
  * and, after them, the first local_len[b] tokens of each sequence's local
  * chunk (every 8 query heads on their KV head, as for the kept tokens).  A

@@ -58,6 +58,7 @@ def _load():
         "lsa_topk_chunks": ([P, P, P, I, I, I, P, P, P, P], I),
         "lsa_topk_chunks_local": ([P, P, P, I, I, I, I, P, P, P, P], I),
         "lsa_append_token": ([P, P, P, P, P, I, P], I),
+        "lsa_reset_local": ([P, I, P], I),
         "lsa_sparse_decode_attn_local": ([P, P, P, I64, P, I, F, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
@@ -296,6 +297,12 @@ def lsa_append_token(k_new, v_new, k_local, v_local, local_len, stream=None):
         _ptr(k_new), _ptr(v_new), _ptr(k_local), _ptr(v_local), _ptr(local_len), B, _stream(stream)))
 
 
+def lsa_reset_local(local_len, stream=None):
+    """Sets local_len [B] to 0 (empties every local chunk), stream-ordered."""
+    _need(local_len, "local_len", torch.int32)
+    _check("lsa_reset_local", _load().lsa_reset_local(_ptr(local_len), local_len.shape[0], _stream(stream)))
+
+
 def lsa_sparse_decode_attn_local(q, k_buf, v_buf, cu_kept, k_local, v_local, local_len, out, workspace,
                                  softmax_scale=None, stream=None, kv_unchanged=False):
     """Attention over the kept chunks plus the first local_len[b] tokens of each local chunk."""
@@ -342,7 +349,7 @@ __all__ = [
     "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
     "lsa_threshold_chunks",
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
-    "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token",
+    "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token", "lsa_reset_local",
     "lsa_sparse_decode_attn_local", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

@@ -256,4 +256,17 @@ int lsa_append_token(const void* k_new, const void* v_new, void* k_local, void* 
   return launch_status();
 }
 
+int lsa_reset_local(int32_t* local_len, int B, void* stream) {
+  using namespace lsa;
+  if (!local_len || B <= 0) return LSA_ERR_INVALID_ARG;
+  if (B > 65535) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  if (cudaMemsetAsync(local_len, 0, sizeof(int32_t) * static_cast<size_t>(B), static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
+}
+
 }  // extern "C"

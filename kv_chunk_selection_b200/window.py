@@ -16,9 +16,9 @@ from typing import Optional
 
 import torch
 
-from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_attn_workspace_size,
-               lsa_fetch_from_host, lsa_gather_chunks, lsa_index_score, lsa_sparse_decode_attn,
-               lsa_threshold_chunks, lsa_topk_chunks)
+from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_append_token, lsa_attn_workspace_size,
+               lsa_fetch_from_host, lsa_gather_chunks, lsa_index_score, lsa_reset_local, lsa_sparse_decode_attn,
+               lsa_sparse_decode_attn_local, lsa_threshold_chunks, lsa_topk_chunks)
 
 TAU = 64
 
@@ -29,16 +29,22 @@ class LayerWindow:
     Selection is the fixed top-K budget (``selection="topk"``) or the pages'
     sigmoid threshold (``selection="threshold"``, keep a chunk when its weighted
     mean probability exceeds ``threshold``).  Sizes: with top-K, ``max_kept`` =
-    max_b K_b + 1 kept chunks per sequence row and the compact buffer holds
-    ``sum_b (K_b + 1)`` chunks (an upper bound of the kept total); with the
+    max_b K_b + n_local kept chunks per sequence row and the compact buffer
+    holds ``sum_b (K_b + n_local)`` chunks (an upper bound of the kept total); with the
     threshold the kept count depends on the data, so both are sized for every
     chunk.  With ``double_buffer`` two compact buffers alternate, so the
     selection of the next window can be fetched while the current one is read.
+
+    ``n_local`` (top-K only) keeps the latest ``n_local`` chunks beside the K
+    recalled ones.  With ``causal`` each sequence also has a local chunk of the
+    tokens decoded inside the window: ``append`` adds a step's token, and
+    ``attend`` then covers the kept chunks plus the tokens appended so far;
+    ``reset_local`` empties it when a window starts.
     """
 
     def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
                  max_chunks: int, device="cuda", double_buffer: bool = False, selection: str = "topk",
-                 threshold: float = 0.5):
+                 threshold: float = 0.5, n_local: int = 1, causal: bool = False):
         self.device = torch.device(device)
         self.n_chunks = n_chunks
         self.k_per_seq = k_per_seq
@@ -49,10 +55,13 @@ class LayerWindow:
             raise ValueError("selection must be 'topk' or 'threshold'")
         self.selection = selection
         self.threshold = float(threshold)
+        if n_local < 1 or (n_local != 1 and selection != "topk"):
+            raise ValueError("n_local must be >= 1, and above 1 only with top-K selection")
+        self.n_local = int(n_local)
         if selection == "topk":
             k_host = k_per_seq.to("cpu", torch.int64)
-            self.max_kept = int(k_host.max()) + 1
-            self.buf_chunks = int((k_host + 1).sum())
+            self.max_kept = int(k_host.max()) + self.n_local
+            self.buf_chunks = int((k_host + self.n_local).sum())
         else:
             n_host = n_chunks.to("cpu", torch.int64)
             self.max_kept = int(max_chunks)
@@ -67,13 +76,19 @@ class LayerWindow:
         self.cu_kept = [torch.zeros((self.B + 1,), dtype=torch.int32, device=self.device) for _ in range(nbuf)]
         self.workspace = torch.zeros(lsa_attn_workspace_size(self.B), dtype=torch.uint8, device=self.device)
         self.active = 0
+        self.causal = bool(causal)
+        if self.causal:
+            lshape = (self.B, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM)
+            self.k_local = torch.zeros(lshape, dtype=torch.bfloat16, device=self.device)
+            self.v_local = torch.zeros(lshape, dtype=torch.bfloat16, device=self.device)
+            self.local_len = torch.zeros((self.B,), dtype=torch.int32, device=self.device)
 
     def select(self, q_idx, w, chunk_keys, buf: int = 0, stream=None):
         """Indexer scores, then the selection (top-K or threshold) plus latest, into slot ``buf``."""
         lsa_index_score(q_idx, w, chunk_keys, self.chunk_table, self.n_chunks, self.scores, stream=stream)
         if self.selection == "topk":
             lsa_topk_chunks(self.scores, self.n_chunks, self.k_per_seq, self.kept[buf], self.n_kept[buf],
-                            self.cu_kept[buf], stream=stream)
+                            self.cu_kept[buf], stream=stream, n_local=self.n_local)
         else:
             lsa_threshold_chunks(self.scores, self.n_chunks, w, self.kept[buf], self.n_kept[buf], self.cu_kept[buf],
                                  threshold=self.threshold, stream=stream)
@@ -87,19 +102,42 @@ class LayerWindow:
                             self.max_chunks, self.k_bufs[buf], self.v_bufs[buf], num_ctas=num_ctas,
                             stream=stream, done_event=done_event)
 
+    def reset_local(self, stream=None):
+        """Empties every sequence's local chunk (start of a window; causal only)."""
+        lsa_reset_local(self.local_len, stream=stream)
+
+    def append(self, k_new, v_new, stream=None):
+        """Adds this step's token (k_new, v_new [B, 8, 128] bf16) to the local chunks (causal only)."""
+        lsa_append_token(k_new, v_new, self.k_local, self.v_local, self.local_len, stream=stream)
+
     def attend(self, q, out, buf: int = 0, stream=None, kv_unchanged: bool = False):
         """One decode step: out[B, 64, 128] fp32 from q[B, 64, 128] bf16.
 
         ``kv_unchanged``: the previous kernel on the stream did not write this
-        window's compact buffer or offsets (true for every step but the first)."""
-        lsa_sparse_decode_attn(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], out, self.workspace,
-                               stream=stream, kv_unchanged=kv_unchanged)
+        window's compact buffer or offsets (true for every step but the first).
+        With ``causal`` the tokens appended so far in the window are attended too."""
+        if self.causal:
+            lsa_sparse_decode_attn_local(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.k_local,
+                                         self.v_local, self.local_len, out, self.workspace, stream=stream,
+                                         kv_unchanged=kv_unchanged)
+        else:
+            lsa_sparse_decode_attn(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], out, self.workspace,
+                                   stream=stream, kv_unchanged=kv_unchanged)
 
-    def run_window(self, q_idx, w, chunk_keys, k_pool, v_pool, q_steps, outs, stream=None):
-        """Select, gather, then one attention call per step of ``q_steps`` [T, B, 64, 128]."""
+    def run_window(self, q_idx, w, chunk_keys, k_pool, v_pool, q_steps, outs, stream=None, k_new=None, v_new=None):
+        """Select, gather, then one attention call per step of ``q_steps`` [T, B, 64, 128].
+
+        Causal windows take the decoded tokens ``k_new``, ``v_new`` [T, B, 8, 128]:
+        step t appends its own token, then attends."""
+        if self.causal and (k_new is None or v_new is None):
+            raise ValueError("a causal window needs k_new and v_new")
         self.select(q_idx, w, chunk_keys, 0, stream)
         self.gather(k_pool, v_pool, 0, stream)
+        if self.causal:
+            self.reset_local(stream)
         for t in range(q_steps.shape[0]):
+            if self.causal:
+                self.append(k_new[t], v_new[t], stream)
             self.attend(q_steps[t], outs[t], 0, stream, kv_unchanged=t > 0)
 
     def kept_lists(self, buf: int = 0):

@@ -246,15 +246,32 @@ def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=No
 
 
 def decode_window(q_idx, w, chunk_keys, chunk_table, n_chunks, k_per_seq,
-                  k_pool, v_pool, q_steps, max_chunks=None, steps=None):
+                  k_pool, v_pool, q_steps, max_chunks=None, steps=None,
+                  n_local=1, k_new=None, v_new=None):
     """One lookahead window: score, select, gather, then attention for each step.
 
     q_steps [T, B, 64, 128]: the decode-step queries of the window.
+    n_local: recent chunks always kept (``topk_chunks``).
+    k_new, v_new [T, B, 8, 128] (optional): the token each step decodes.  When
+    given, the window is causal: step t first appends its own token to the
+    sequence's local chunk, then attends the kept chunks plus the t + 1 tokens
+    decoded so far in this window (FM-DS-V4 summary, 3 Experiments, the decoded
+    window; Reading: the local chunk starts empty at every window).
     Returns (scores, kept_lists, cu_kept, outputs[T, B, 64, 128]).
     """
     scores = index_scores(q_idx, w, chunk_keys, chunk_table, n_chunks, max_chunks)
-    kept = topk_chunks(scores, n_chunks, k_per_seq)
+    kept = topk_chunks(scores, n_chunks, k_per_seq, n_local=n_local)
     k_buf, v_buf, cu = gather_chunks(k_pool, v_pool, chunk_table, kept, max_chunks)
     steps = range(q_steps.shape[0]) if steps is None else steps
-    outs = {t: sparse_decode_attn(q_steps[t], k_buf, v_buf, cu) for t in steps}
+    if k_new is None:
+        outs = {t: sparse_decode_attn(q_steps[t], k_buf, v_buf, cu) for t in steps}
+        return scores, kept, cu, outs
+    T, B = q_steps.shape[0], q_steps.shape[1]
+    # local chunk [B, 8, 64, 128]: token t of the window at position t
+    k_loc = np.zeros((B, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM))
+    v_loc = np.zeros_like(k_loc)
+    k_loc[:, :, :T] = np.transpose(np.asarray(k_new, dtype=np.float64), (1, 2, 0, 3))
+    v_loc[:, :, :T] = np.transpose(np.asarray(v_new, dtype=np.float64), (1, 2, 0, 3))
+    outs = {t: sparse_decode_attn(q_steps[t], k_buf, v_buf, cu, k_local=k_loc, v_local=v_loc,
+                                  local_len=[t + 1] * B) for t in steps}
     return scores, kept, cu, outs

@@ -76,6 +76,8 @@ def test_host_checks_null_pointers(L):
     assert L.lsa_read_device_status(n, None) == INVALID
     assert L.lsa_topk_chunks_local(n, n, n, 1, 1, 1, 1, n, n, n, n) == INVALID
     assert L.lsa_append_token(n, n, n, n, n, 1, n) == INVALID
+    assert L.lsa_reset_local(n, 1, n) == INVALID
+    assert L.lsa_reset_local(ctypes.c_void_p(0x100000), 0, n) == INVALID
     assert L.lsa_sparse_decode_attn_local(n, n, n, 1, n, 1, ctypes.c_float(0.1), n, n, n, n, n, 0, 0, n) == INVALID
     assert L.lsa_selftest_bounded_wait(1, n, 1000, n) == INVALID      # mode 1 needs a flag
     assert L.lsa_selftest_bounded_wait(0, n, 0, n) == INVALID         # zero limit

@@ -399,3 +399,31 @@ def test_decode_window_composition():
     assert len(kept[0]) == K + 1 and kept[0][-1] == N - 1
     ref = oracle.sparse_decode_attn(qs[1], kp[kept[0]], vp[kept[0]], [0, K + 1])
     np.testing.assert_array_equal(outs[1], ref)
+
+
+def test_decode_window_causal_equals_dense_sdpa_over_kept_and_decoded_tokens():
+    """Causal window with a recent window of 2 chunks: step t attends exactly the
+    tokens of the kept chunks followed by the t + 1 tokens decoded so far.  The
+    reference is torch's fp64 scaled_dot_product_attention over that token list."""
+    rng = np.random.default_rng(41)
+    N, K, T = 10, 3, 5
+    keys = bf16_round(rng.standard_normal((N, 128)))
+    kp, vp = _rand_bufs(N, rng)
+    q_idx = bf16_round(rng.standard_normal((1, 16, 128)))
+    w = rng.uniform(0, 1, 16)
+    qs = bf16_round(rng.standard_normal((T, 1, 64, 128)))
+    k_new = bf16_round(rng.standard_normal((T, 1, 8, 128)))
+    v_new = bf16_round(rng.standard_normal((T, 1, 8, 128)))
+    scores, kept, cu, outs = oracle.decode_window(q_idx, w, keys, None, [N], [K], kp, vp, qs, max_chunks=N,
+                                                  n_local=2, k_new=k_new, v_new=v_new)
+    assert len(kept[0]) == K + 2 and list(kept[0][-2:]) == [N - 2, N - 1]
+    for t in (0, 2, T - 1):
+        Kc = torch.from_numpy(kp[kept[0]]).permute(1, 0, 2, 3).reshape(8, -1, 128)
+        Vc = torch.from_numpy(vp[kept[0]]).permute(1, 0, 2, 3).reshape(8, -1, 128)
+        Kd = torch.from_numpy(k_new[: t + 1, 0]).permute(1, 0, 2)       # [8, t+1, 128]
+        Vd = torch.from_numpy(v_new[: t + 1, 0]).permute(1, 0, 2)
+        Kall = torch.cat([Kc, Kd], dim=1).repeat_interleave(8, dim=0)
+        Vall = torch.cat([Vc, Vd], dim=1).repeat_interleave(8, dim=0)
+        Q = torch.from_numpy(qs[t, 0]).reshape(64, 1, 128)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, Kall, Vall).reshape(64, 128).numpy()
+        np.testing.assert_allclose(outs[t][0], ref, rtol=1e-12, atol=1e-14)

@@ -507,6 +507,49 @@ def test_window_tiny_full():
         assert_attention_close(outs[t], o_outs[t])
 
 
+def test_window_tiny_causal_recent_window():
+    """Causal window (every step appends its token, then attends) with the latest
+    2 chunks kept, all 64 steps, against the oracle's causal window; a second run
+    of the same window must reset the local chunk and repeat it bit for bit."""
+    inp = workloads.make_inputs("tiny", DEV)
+    L = inp.layers[0]
+    kn, vn = workloads.decoded_tokens(inp, 0, DEV)
+    lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, DEV, n_local=2, causal=True)
+    outs = torch.empty((64, 1, 64, 128), device=DEV)
+    lw.run_window(L.q_idx[0], L.w, L.chunk_keys, L.k_pool, L.v_pool, L.q[0], outs, k_new=kn[0], v_new=vn[0])
+    torch.cuda.synchronize()
+    status_clean()
+    assert int(lw.local_len[0]) == 64
+    scores, kept, cu, o_outs = oracle.decode_window(
+        f64(L.q_idx[0]), f64(L.w), f64(L.chunk_keys), i64(inp.chunk_table), i64(inp.n_chunks),
+        i64(inp.k_per_seq), f64(L.k_pool), f64(L.v_pool), f64(L.q[0]), inp.max_chunks,
+        n_local=2, k_new=f64(kn[0]), v_new=f64(vn[0]))
+    assert lw.kept_lists()[0] == list(kept[0])
+    for t in range(64):
+        assert_attention_close(outs[t], o_outs[t])
+    again = torch.empty_like(outs)
+    lw.run_window(L.q_idx[0], L.w, L.chunk_keys, L.k_pool, L.v_pool, L.q[0], again, k_new=kn[0], v_new=vn[0])
+    torch.cuda.synchronize()
+    status_clean()
+    assert torch.equal(outs, again)
+
+
+def test_reset_local_empties_the_local_chunk():
+    B = 3
+    kl = torch.zeros((B, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    vl = torch.zeros_like(kl)
+    ll = torch.tensor([5, 0, 64], dtype=torch.int32, device=DEV)
+    lsa.lsa_reset_local(ll)
+    assert ll.tolist() == [0, 0, 0]
+    g = torch.Generator(device=DEV).manual_seed(2)
+    kt = torch.randn((B, 8, 128), generator=g, device=DEV).to(torch.bfloat16)
+    vt = torch.randn((B, 8, 128), generator=g, device=DEV).to(torch.bfloat16)
+    lsa.lsa_append_token(kt, vt, kl, vl, ll)
+    assert ll.tolist() == [1, 1, 1]
+    assert torch.equal(kl[:, :, 0], kt) and torch.equal(vl[:, :, 0], vt)
+    status_clean()
+
+
 def test_window_128k_sampled_steps():
     window_parity("128k", steps=[0, 31, 63], window=1)
 

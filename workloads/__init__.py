@@ -85,7 +85,7 @@ WORKLOADS = {
 
 # Per-tensor seed offsets.
 _OFF = {"lengths": 1, "slots": 2, "w": 10, "keys": 20, "kpool": 30, "vpool": 40,
-        "qidx": 50, "q": 60, "planted": 70}
+        "qidx": 50, "q": 60, "planted": 70, "knew": 80, "vnew": 90}
 
 
 def _seed(base: int, name: str, layer: int = 0, extra: int = 0) -> int:
@@ -232,3 +232,11 @@ def make_inputs(name_or_wl, device="cuda", base_seed: int = BASE_SEED, layers: O
     return Inputs(wl, n_chunks.to(dev), k_per_seq.to(dev), table.to(dev), max_chunks, n_slots,
                   layer_list, steps)
 
+
+def decoded_tokens(inp: Inputs, layer: int, device, base_seed: int = BASE_SEED, windows: Optional[int] = None):
+    """K and V of the token each decode step produces, for the causal window:
+    two bf16 tensors [windows, TAU, B, 8, 128] drawn N(0, 1) like the pools."""
+    n_windows = inp.workload.windows if windows is None else windows
+    shape = (n_windows, inp.steps, inp.batch, NUM_KV_HEADS, HEAD_DIM)
+    return (randn_bf16(shape, _seed(base_seed, "knew", layer), device),
+            randn_bf16(shape, _seed(base_seed, "vnew", layer), device))
