@@ -6,4 +6,4 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 from .lsa_oracle import *  # noqa: F401,F403
 from .lsa_oracle import (attend_one, bf16_bits_to_f64, cumulative_kept, decode_window,  # noqa: F401
                          gather_chunks, index_scores, sparse_decode_attn, threshold_chunks,
-                         topk_chunks)
+                         topk_chunks, token_scores, topk_tokens, fine_decode_attn)

@@ -47,6 +47,13 @@ of the same paper (*FM-DS-V4 review*, with its section).
    3 Experiments) are appended before each step attends: attention then runs
    over the kept chunks plus the first local_len[b] tokens of the sequence's
    local chunk.
+8. ``token_scores`` / ``topk_tokens`` / ``fine_decode_attn`` -- the second,
+   token-level stage: native token-level scoring picks a fine-grained top-k of
+   entries inside the recalled subset instead of the whole context (FM-DS-V4
+   summary, 2.1 Architecture), k = 2048 tokens in the DSA lightning indexer
+   (search page "lightning indexer", the Multi-layer Indexer abstract).  Every
+   decode step scores each token of its sequence's recalled chunks with the
+   step's indexer query, keeps the k best, and attends only those.
 
 Readings taken where the pages are silent are listed in the design notes of
 this repository and marked "Reading:" at the point of use.
@@ -240,6 +247,83 @@ def sparse_decode_attn(q, k_buf, v_buf, cu_kept, scale=None, seqs=None, heads=No
             if n_loc:
                 K = np.concatenate([K, np.asarray(k_local[b, g, :n_loc], dtype=np.float64)])
                 V = np.concatenate([V, np.asarray(v_local[b, g, :n_loc], dtype=np.float64)])
+            for h in group_heads:
+                out[b, h] = attend_one(q[b, h], K, V, scale)
+    return out
+
+
+def token_scores(q_idx, w, token_keys, chunk_table, kept_lists, max_chunks=None):
+    """Token-level indexer scores inside the recalled chunks of each sequence.
+
+    q_idx      [B, H_I, d_I]         indexer query of the current decode step.
+    token_keys [n_slots, 64, d_I]    cached indexer key of every token, by chunk slot.
+    kept_lists                        recalled chunks of each sequence, ascending.
+    Returns one float64 array per sequence of length 64 * len(kept): position
+    p = 64 j + i is token i of the j-th recalled chunk (so positions follow
+    the context order), and
+        score[b, p] = sum_h w_h * sigmoid(q_idx[b, h] . key(p) / sqrt(d_I)).
+    Reading: the pages name the token-level stage but not its formula; it is
+    taken to be the indexer's own weighted-sigmoid form applied per token.
+    """
+    q_idx = np.asarray(q_idx, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    if max_chunks is None and chunk_table is not None:
+        max_chunks = chunk_table.shape[1]
+    out = []
+    for b, kept in enumerate(kept_lists):
+        if len(kept) == 0:
+            out.append(np.zeros(0, dtype=np.float64))
+            continue
+        rows = [np.asarray(token_keys[_slot(chunk_table, b, int(c), max_chunks)], dtype=np.float64)
+                for c in kept]
+        K = np.concatenate(rows)                                        # [64 * n_kept, d_I]
+        logits = q_idx[b] @ K.T / math.sqrt(INDEX_DIM)                  # [H_I, 64 * n_kept]
+        out.append(w @ (1.0 / (1.0 + np.exp(-logits))))
+    return out
+
+
+def topk_tokens(scores_list, k):
+    """The k best token positions of each sequence, by score descending then
+    position ascending, returned ascending; every position when there are at
+    most k (Reading: the same tie rule as the chunk selection)."""
+    out = []
+    for sc in scores_list:
+        n = len(sc)
+        if n <= k:
+            out.append(np.arange(n, dtype=np.int64))
+            continue
+        order = sorted(range(n), key=lambda p: (-sc[p], p))
+        out.append(np.sort(np.array(order[:k], dtype=np.int64)))
+    return out
+
+
+def fine_decode_attn(q, k_buf, v_buf, cu_kept, selected, scale=None, seqs=None, heads=None):
+    """GQA decode attention over the selected tokens only.
+
+    Token position p of sequence b is row p % 64 of compact chunk
+    cu_kept[b] + p // 64; every KV head attends the same selected positions
+    (one indexer score per token).  Other conventions as ``sparse_decode_attn``.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    q = np.asarray(q, dtype=np.float64)
+    B = q.shape[0]
+    out = np.full((B, NUM_Q_HEADS, HEAD_DIM), np.nan, dtype=np.float64)
+    seqs = range(B) if seqs is None else seqs
+    heads = range(NUM_Q_HEADS) if heads is None else heads
+    for b in seqs:
+        sel = np.asarray(selected[b], dtype=np.int64)
+        if sel.size == 0:
+            out[b, list(heads)] = 0.0
+            continue
+        chunk = int(cu_kept[b]) + sel // CHUNK_TOKENS
+        row = sel % CHUNK_TOKENS
+        for g in range(NUM_KV_HEADS):
+            group_heads = [h for h in heads if h // GROUP == g]
+            if not group_heads:
+                continue
+            K = np.asarray(k_buf[chunk, g, row], dtype=np.float64)       # [n_sel, 128]
+            V = np.asarray(v_buf[chunk, g, row], dtype=np.float64)
             for h in group_heads:
                 out[b, h] = attend_one(q[b, h], K, V, scale)
     return out

@@ -427,3 +427,100 @@ def test_decode_window_causal_equals_dense_sdpa_over_kept_and_decoded_tokens():
         Q = torch.from_numpy(qs[t, 0]).reshape(64, 1, 128)
         ref = torch.nn.functional.scaled_dot_product_attention(Q, Kall, Vall).reshape(64, 128).numpy()
         np.testing.assert_allclose(outs[t][0], ref, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------- token-level fine stage ---
+
+def _token_case(rng, n_slots=7, B=2, max_chunks=5):
+    tok_keys = bf16_round(rng.standard_normal((n_slots, 64, 128)))
+    table = np.array([[3, 0, 6, 1, 2], [5, 4, 0, 0, 0]], dtype=np.int64)[:B, :max_chunks]
+    kept = [np.array([0, 2, 4]), np.array([1])]
+    q_idx = bf16_round(rng.standard_normal((B, 16, 128)))
+    w = rng.uniform(0, 1, 16)
+    return tok_keys, table, kept, q_idx, w
+
+
+def test_token_scores_equal_chunk_scores_of_per_token_keys():
+    """Every token scored like a chunk whose indexer key is that token's key: the
+    pinned chunk scorer over a table that maps position p = 64 j + i to the flat
+    row 64 * slot(kept[j]) + i gives the same numbers."""
+    rng = np.random.default_rng(51)
+    tok_keys, table, kept, q_idx, w = _token_case(rng)
+    got = oracle.token_scores(q_idx, w, tok_keys, table, kept)
+    flat = tok_keys.reshape(-1, 128)
+    for b in range(2):
+        rows = np.array([64 * table[b, c] + i for c in kept[b] for i in range(64)])
+        ref = oracle.index_scores(q_idx[b:b + 1], w, flat, rows[None, :], [len(rows)])[0]
+        np.testing.assert_allclose(got[b], ref, rtol=1e-14, atol=0)
+
+
+def test_token_scores_brute_force_loops():
+    rng = np.random.default_rng(52)
+    tok_keys, table, kept, q_idx, w = _token_case(rng)
+    got = oracle.token_scores(q_idx, w, tok_keys, table, kept)
+    for b, p in ((0, 0), (0, 64 + 17), (0, 191), (1, 63)):
+        slot = table[b, kept[b][p // 64]]
+        key = tok_keys[slot, p % 64]
+        s = 0.0
+        for h in range(16):
+            dot = sum(float(q_idx[b, h, d]) * float(key[d]) for d in range(128))
+            s += float(w[h]) / (1.0 + math.exp(-dot / math.sqrt(128)))
+        assert abs(got[b][p] - s) <= 1e-12 * abs(s)
+    assert len(got[0]) == 192 and len(got[1]) == 64
+
+
+def test_token_scores_zero_query_is_half_weight_sum():
+    rng = np.random.default_rng(53)
+    tok_keys, table, kept, q_idx, w = _token_case(rng)
+    got = oracle.token_scores(np.zeros_like(q_idx), w, tok_keys, table, kept)
+    for b in range(2):
+        np.testing.assert_allclose(got[b], 0.5 * w.sum(), rtol=1e-15)
+
+
+@pytest.mark.parametrize("trial", range(4))
+def test_topk_tokens_matches_rank_count_definition(trial):
+    """Position p is selected iff fewer than k positions beat it, where q beats p
+    when s_q > s_p or (s_q == s_p and q < p); ties are frequent on purpose."""
+    rng = np.random.default_rng(60 + trial)
+    n = int(rng.integers(1, 300))
+    k = int(rng.integers(0, 320))
+    sc = np.round(rng.uniform(0, 1, n), 1)          # about 11 distinct values
+    got = oracle.topk_tokens([sc], k)[0]
+    beats = [(sc > sc[p]).sum() + (sc[:p] == sc[p]).sum() for p in range(n)]
+    ref = [p for p in range(n) if beats[p] < k]
+    assert list(got) == ref
+    assert len(got) == min(k, n)
+
+
+def test_fine_attention_keeping_every_token_is_chunk_attention():
+    rng = np.random.default_rng(54)
+    k_buf, v_buf = _rand_bufs(4, rng)
+    q = bf16_round(rng.standard_normal((2, 64, 128)))
+    cu = [0, 3, 4]
+    sel = [np.arange(192), np.arange(64)]
+    got = oracle.fine_decode_attn(q, k_buf, v_buf, cu, sel)
+    ref = oracle.sparse_decode_attn(q, k_buf, v_buf, cu)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-15)
+    empty = oracle.fine_decode_attn(q, k_buf, v_buf, cu, [np.arange(0), np.arange(64)])
+    assert np.all(empty[0] == 0)
+
+
+def test_fine_attention_equals_dense_sdpa_over_selected_rows():
+    """torch's fp64 SDPA over exactly the selected rows (KV repeated per group);
+    the order of the selected list does not matter."""
+    rng = np.random.default_rng(55)
+    k_buf, v_buf = _rand_bufs(5, rng)
+    q = bf16_round(rng.standard_normal((2, 64, 128)))
+    cu = [0, 3, 5]
+    sel = [np.sort(rng.choice(192, 70, replace=False)), np.sort(rng.choice(128, 9, replace=False))]
+    got = oracle.fine_decode_attn(q, k_buf, v_buf, cu, sel)
+    for b in range(2):
+        c = cu[b] + sel[b] // 64
+        r = sel[b] % 64
+        K = torch.from_numpy(k_buf[c, :, r]).permute(1, 0, 2).repeat_interleave(8, dim=0)   # [64, n, 128]
+        V = torch.from_numpy(v_buf[c, :, r]).permute(1, 0, 2).repeat_interleave(8, dim=0)
+        Q = torch.from_numpy(q[b]).reshape(64, 1, 128)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V).reshape(64, 128).numpy()
+        np.testing.assert_allclose(got[b], ref, rtol=1e-12, atol=1e-14)
+    shuffled = [rng.permutation(s) for s in sel]
+    np.testing.assert_allclose(oracle.fine_decode_attn(q, k_buf, v_buf, cu, shuffled), got, rtol=1e-12, atol=1e-15)
