@@ -11,7 +11,10 @@ launches are replayed from two captured CUDA graphs per window index.
 
 With ``--causal`` every decode step first appends its own token to the
 sequence's local chunk and then attends the kept chunks plus the tokens decoded
-so far in the window; ``--n-local L`` keeps the latest L chunks.
+so far in the window; ``--n-local L`` keeps the latest L chunks.  With
+``--fine-k k`` every step also runs the token-level fine stage (score every
+recalled token with the step's indexer query, keep the k best, pack them) and
+attends only those k tokens.
 
 Metric: decode tokens per second per layer (64 * B tokens per window and
 layer), with the achieved HBM bandwidth of the whole window and of the
@@ -156,16 +159,23 @@ def copy_probe_gbs(device, nbytes=1 << 31, reps=10):
 TOKEN_KV_BYTES = 2 * 8 * 128 * 2     # K and V of one token, 8 KV heads, bf16
 
 
-def window_bytes(n_chunks, kept_total, layers, causal=False):
+def window_bytes(n_chunks, kept_total, layers, causal=False, fine_tokens=None):
     """Algorithmic bytes of one window: indexer keys of every chunk once, and per
     decode step the kept K/V, the query and the fp32 output (gather excluded).
     ``kept_total`` is the number of kept chunks the selection produced.  A causal
     window also appends one token per step (read + write) and attends on average
-    (TAU + 1) / 2 decoded tokens per step."""
+    (TAU + 1) / 2 decoded tokens per step.  With the fine stage
+    (``fine_tokens`` = selected tokens summed over the batch) a step reads the
+    token indexer key of every recalled token and the K/V of the selected
+    tokens only (the packing copy excluded, like the gather)."""
     n = n_chunks.to(torch.int64).cpu()
     B = int(n.numel())
     keys = 256 * int(n.sum()) + B * 16 * 128 * 2 + 16 * 4
-    attn_launch = int(round(kept_total * 2 * workloads.CHUNK_BYTES_ONE)) + B * (64 * 128 * 2 + 64 * 128 * 4)
+    if fine_tokens is None:
+        kv = int(round(kept_total * 2 * workloads.CHUNK_BYTES_ONE))
+    else:
+        kv = int(round(kept_total * 64 * 256 + B * 16 * 128 * 2 + fine_tokens * TOKEN_KV_BYTES))
+    attn_launch = kv + B * (64 * 128 * 2 + 64 * 128 * 4)
     append = 0
     if causal:
         attn_launch += int(round(B * (workloads.TAU + 1) / 2 * TOKEN_KV_BYTES))
@@ -332,11 +342,13 @@ def run_ours(args, rank, world, local_rank):
     host_tier = inp.workload.host_pool
     lws = [LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev,
                        selection=args.selection, threshold=args.threshold, n_local=args.n_local,
-                       causal=args.causal) for _ in range(layers)]
+                       causal=args.causal, fine_k=args.fine_k) for _ in range(layers)]
     outs = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
     stream = torch.cuda.Stream(device=dev)
     decoded = [workloads.decoded_tokens(inp, l, dev, base_seed=workloads.BASE_SEED + rank) if args.causal else None
                for l in range(layers)]
+    fine = [workloads.fine_inputs(inp, l, dev, base_seed=workloads.BASE_SEED + rank) if args.fine_k else None
+            for l in range(layers)]
 
     def select_phase(w):
         for l, L in enumerate(inp.layers):
@@ -353,17 +365,22 @@ def run_ours(args, rank, world, local_rank):
             for l, L in enumerate(inp.layers):
                 if args.causal:
                     lws[l].append(decoded[l][0][w, t], decoded[l][1][w, t])
+                if args.fine_k:
+                    lws[l].fine_select(fine[l][1][w, t], L.w, fine[l][0])
                 lws[l].attend(L.q[w, t], outs[l][t], kv_unchanged=t > 0)
 
     # warm every path once (and record the kept total of every window index,
     # which the threshold selection makes data-dependent), then capture one pair
     # of graphs per window index
-    kept_totals = []
+    kept_totals, fine_totals = [], []
     with torch.cuda.stream(stream):
         for w in range(n_win):
             select_phase(w)
             torch.cuda.synchronize()
             kept_totals.append(sum(int(lw.cu_kept[0][-1].item()) for lw in lws) / layers)
+            if args.fine_k:
+                fine_totals.append(sum(min(args.fine_k, 64 * int(n)) for lw in lws for n in lw.n_kept[0].tolist())
+                                   / layers)
         attn_phase(n_win - 1)
     torch.cuda.synchronize()
     bits = lsa.read_device_status()
@@ -431,17 +448,20 @@ def run_ours(args, rank, world, local_rank):
     elapsed, value = combine_ranks(elapsed, workloads.TAU * B * layers * args.steps, world, dev)
     # mean kept total over the timed windows (identical for every window with top-K)
     kept_total = sum(kept_totals[i % n_win] for i in range(args.steps)) / args.steps
-    wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers, causal=args.causal)
+    fine_total = (sum(fine_totals[i % n_win] for i in range(args.steps)) / args.steps) if args.fine_k else None
+    wbytes, attn_bytes, total_chunks = window_bytes(inp.n_chunks, kept_total, layers, causal=args.causal,
+                                                    fine_tokens=fine_total)
     hbm_gbs = wbytes * args.steps / elapsed / 1e9
     n_attn = workloads.TAU * layers * args.steps
     attn_avg = att_s / n_attn
     attn_gbs = attn_bytes / attn_avg / 1e9
-    traffic = profiled_traffic(args.workload)
+    traffic = profiled_traffic(args.workload) if not (args.fine_k or args.causal) else None
+    fine_stages = fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total) if args.fine_k else None
 
     # ---- end to end through the public API, inputs from pinned host memory ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, inp, lws, dev, stream, decoded)
+        e2e = run_e2e(args, inp, lws, dev, stream, decoded, fine)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -452,6 +472,7 @@ def run_ours(args, rank, world, local_rank):
             "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
             "selection": args.selection if args.selection == "topk" else f"threshold {args.threshold}",
             "recent_chunks": args.n_local,
+            "fine_k": args.fine_k or None,
             "causal": ("each step appends its token to a local chunk and attends it with the kept chunks"
                        if args.causal else False),
             "tau": workloads.TAU, "gqa": "64q/8kv/d128", "indexer": "16 heads x 128",
@@ -474,14 +495,74 @@ def run_ours(args, rank, world, local_rank):
         "stage_us": {"select_and_gather_per_window": sel_s / args.steps * 1e6,
                      "attention_per_decode_step": attn_avg * 1e6,
                      "attention_64_steps": att_s / args.steps * 1e6},
-        "gpu_launches": args.steps * layers * (3 + workloads.TAU * (2 if args.causal else 1)),
+        "gpu_launches": args.steps * layers * (3 + workloads.TAU * (1 + int(args.causal) + 3 * bool(args.fine_k))),
         "clocks": clocks,
         "e2e": e2e,
     }
+    if fine_stages is not None:
+        out["fine_stages"] = fine_stages
+        out["roofline"]["timed_with"] = "the fine stage (token scores, token top-k, packing) before each launch"
     return out
 
 
-def run_e2e(args, inp, lws, dev, stream, decoded=None):
+def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=32, replays=10):
+    """Device time of each kernel of the fine step alone: a CUDA graph of `reps`
+    launches of that kernel on the inputs of window 0, step 0, layer 0, replayed
+    between CUDA events on the bench stream (inputs stay warm in L2 across the
+    repeats; the in-window step time is the timed region's).  Each kernel also
+    gets its algorithmic bytes per launch."""
+    import kv_chunk_selection_b200 as lsa
+    lw, L = lws[0], inp.layers[0]
+    keys, q_tok = fine[0]
+    B = inp.batch
+    out = torch.empty((B, 64, 128), device=lw.device)
+    calls = {
+        "token_score": lambda: lsa.lsa_token_score(q_tok[0, 0], L.w, keys, lw.chunk_table, lw.kept[0], lw.n_kept[0],
+                                                   lw.max_chunks, lw.tok_scores, lw.n_tokens),
+        "topk_tokens": lambda: lsa.lsa_topk_tokens(lw.tok_scores, lw.n_tokens, lw.fine_k, lw.sel, lw.n_sel,
+                                                   lw.cu_sel),
+        "gather_tokens": lambda: lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], lw.sel, lw.cu_sel,
+                                                       lw.k_fine, lw.v_fine, lw.cu_units),
+        "attention": lambda: lw.attend(L.q[0, 0], out),
+    }
+    with torch.cuda.stream(stream):
+        lw.select(L.q_idx[0], L.w, L.chunk_keys)
+        lw.gather(L.k_pool, L.v_pool)
+        for fn in calls.values():
+            fn()
+    torch.cuda.synchronize()
+    res = {}
+    tokens = kept_total * 64
+    nbytes = {"token_score": tokens * 256 + B * 16 * 128 * 2 + tokens * 4,
+              "topk_tokens": tokens * 4 + fine_total * 4,
+              "gather_tokens": 2 * fine_total * TOKEN_KV_BYTES,
+              "attention": fine_total * TOKEN_KV_BYTES + B * (64 * 128 * 2 + 64 * 128 * 4)}
+    for name, fn in calls.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fn()
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(replays):
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            with torch.cuda.stream(stream):
+                g.replay()
+            z.record(stream)
+            z.synchronize()
+            times.append(a.elapsed_time(z) / 1e3 / reps)
+        del g
+        t = statistics.median(times)
+        res[name] = {"us": t * 1e6, "bytes": int(nbytes[name]), "gbs": nbytes[name] / t / 1e9}
+    res.update({"timing": f"each kernel alone, graph of {reps} launches, median of {replays} replays",
+                "recalled_tokens": int(tokens), "selected_tokens": int(fine_total)})
+    return res
+
+
+def run_e2e(args, inp, lws, dev, stream, decoded=None, fine=None):
     """Same metric through the public API: every window copies its queries (and,
     causal, its decoded tokens) in from pinned host memory and its 64 outputs back
     to pinned host memory."""
@@ -496,6 +577,10 @@ def run_e2e(args, inp, lws, dev, stream, decoded=None):
         host_kv = [[(decoded[l][0][w].cpu().pin_memory(), decoded[l][1][w].cpu().pin_memory())
                     for w in range(n_win)] for l in range(layers)]
         dkv = [(torch.empty_like(decoded[l][0][0]), torch.empty_like(decoded[l][1][0])) for l in range(layers)]
+    use_fine = fine is not None and fine[0] is not None
+    if use_fine:
+        host_qt = [[fine[l][1][w].cpu().pin_memory() for w in range(n_win)] for l in range(layers)]
+        dqt = [torch.empty_like(fine[l][1][0]) for l in range(layers)]
     douts = [torch.empty((workloads.TAU, B, 64, 128), device=dev) for _ in range(layers)]
     hout = [torch.empty((workloads.TAU, B, 64, 128)).pin_memory() for _ in range(layers)]
     steps = max(1, min(args.steps, args.e2e_steps))
@@ -508,6 +593,8 @@ def run_e2e(args, inp, lws, dev, stream, decoded=None):
             if causal:
                 dkv[l][0].copy_(host_kv[l][w][0], non_blocking=True)
                 dkv[l][1].copy_(host_kv[l][w][1], non_blocking=True)
+            if use_fine:
+                dqt[l].copy_(host_qt[l][w], non_blocking=True)
         for l, L in enumerate(inp.layers):
             lws[l].select(dq_idx[l], L.w, L.chunk_keys)
             if inp.workload.host_pool:
@@ -520,6 +607,8 @@ def run_e2e(args, inp, lws, dev, stream, decoded=None):
             for l in range(layers):
                 if causal:
                     lws[l].append(dkv[l][0][t], dkv[l][1][t])
+                if use_fine:
+                    lws[l].fine_select(dqt[l][t], inp.layers[l].w, fine[l][0])
                 lws[l].attend(dq[l][t], douts[l][t], kv_unchanged=t > 0)
         for l in range(layers):
             hout[l].copy_(douts[l], non_blocking=True)
@@ -537,7 +626,8 @@ def run_e2e(args, inp, lws, dev, stream, decoded=None):
     torch.cuda.synchronize()
     el = s.elapsed_time(e) / 1e3
     h2d = layers * (B * 16 * 128 * 2 + workloads.TAU * B * 64 * 128 * 2
-                    + (workloads.TAU * B * TOKEN_KV_BYTES if causal else 0))
+                    + (workloads.TAU * B * TOKEN_KV_BYTES if causal else 0)
+                    + (workloads.TAU * B * 16 * 128 * 2 if use_fine else 0))
     d2h = layers * workloads.TAU * B * 64 * 128 * 4
     return {"value": workloads.TAU * B * layers * steps / el, "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "api": "kv_chunk_selection_b200.window.LayerWindow"}
@@ -727,6 +817,8 @@ def main():
                     help="chunk selection: fixed top-K budget (default) or the sigmoid threshold")
     ap.add_argument("--threshold", type=float, default=0.5)
     ap.add_argument("--n-local", type=int, default=1, help="recent chunks always kept (top-K selection)")
+    ap.add_argument("--fine-k", type=int, default=0,
+                    help="token-level fine stage: attend only the k best tokens of the recalled chunks (k %% 64 == 0)")
     ap.add_argument("--causal", action="store_true",
                     help="append each step's token to a local chunk and attend it (decoded window)")
     ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
@@ -739,6 +831,8 @@ def main():
         ap.error("--causal and --n-local apply to device-resident workloads, not the host tier")
     if args.n_local != 1 and args.selection != "topk":
         ap.error("--n-local applies to top-K selection")
+    if args.fine_k and (args.fine_k < 0 or args.fine_k % 64 or workloads.WORKLOADS[args.workload].host_pool):
+        ap.error("--fine-k must be a positive multiple of 64, on a device-resident workload")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -356,6 +356,72 @@ int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v
                                  const int32_t* local_len, float* out, void* workspace,
                                  size_t workspace_bytes, unsigned int flags, void* stream);
 
+/*
+ * Token-level fine stage.  Inside the recalled chunks, native token-level
+ * scoring keeps a fine-grained top-k of entries (summary page, 2.1
+ * Architecture; k = 2048 tokens for the DSA lightning indexer on the search
+ * page "lightning indexer").  Every decode step:
+ *   lsa_token_score   -> one score per token of the recalled chunks,
+ *   lsa_topk_tokens   -> the k best token positions,
+ *   lsa_gather_tokens -> those tokens packed into dense 64-token units,
+ *   lsa_sparse_decode_attn(_local) over the units (buf = k_out / v_out,
+ *   cu_kept = cu_units).
+ * Token position p of sequence b is token p % 64 of its recalled chunk
+ * p / 64 (kept[b*max_kept + p/64]); positions follow the context order.  All
+ * KV heads attend the same selected tokens (one score per token).
+ *
+ * lsa_token_score -- for p < 64 * n_kept[b]:
+ *   scores[b*64*max_kept + p] = sum_h w[h] * sigmoid(q_idx[b,h,:] . tok_key(p) / sqrt(128)),
+ *   tok_key(p) = token_keys[slot(b, kept[b*max_kept + p/64])][p % 64][:]
+ * (the indexer's own form at token granularity), and n_tokens[b] =
+ * 64 * n_kept[b].
+ *   q_idx      device bf16 [B][16][128], the current decode step's indexer query
+ *   w          device fp32 [16]
+ *   token_keys device bf16 [n_slots][64][128], per-token indexer keys by slot
+ *   chunk_table, kept, n_kept as for lsa_gather_chunks / lsa_topk_chunks
+ *   scores     device fp32 [B][64 * max_kept]; n_tokens device int32 [B]
+ * Device errors: BAD_COUNT (n_kept out of range: skipped, n_tokens 0),
+ * BAD_CHUNK / BAD_SLOT (that token's score is not written).
+ */
+int lsa_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                    const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
+                    int max_chunks, int max_kept, float* scores, int32_t* n_tokens, void* stream);
+
+/*
+ * lsa_topk_tokens -- the k best token positions of each sequence by (score
+ * descending, position ascending), every position when there are at most k;
+ * sel[b*max_sel + j], j < n_sel[b] = min(k, n_tokens[b]), ascending;
+ * cu_sel[0] = 0, cu_sel[b+1] = cu_sel[b] + n_sel[b].  Same key as
+ * lsa_topk_chunks (-0 equals +0, NaN last).
+ *   scores   device fp32 [B][max_tokens] (max_tokens = 64 * max_kept of lsa_token_score)
+ *   n_tokens device int32 [B]
+ *   k        > 0; a multiple of 64 when the result feeds lsa_gather_tokens
+ *   sel device int32 [B][max_sel]; n_sel device int32 [B]; cu_sel device int32 [B+1]
+ * Device errors: BAD_COUNT, CAPACITY (n_sel would exceed max_sel): that
+ * sequence selects nothing.
+ */
+int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int k, int B, int max_tokens,
+                    int max_sel, int32_t* sel, int32_t* n_sel, int32_t* cu_sel, void* stream);
+
+/*
+ * lsa_gather_tokens -- pack the selected tokens into dense units, bit for bit:
+ * for j < n_sel[b], with unit u = cu_sel[b]/64 + j/64 and row r = j % 64,
+ *   k_out[u][g][r][:] = k_buf[cu_kept[b] + p/64][g][p % 64][:],  p = sel[b*max_sel + j],
+ * for every KV head g, same for V; cu_units[b] = cu_sel[b] / 64.
+ *   k_buf, v_buf  device bf16 [buf_chunks][8][64][128] (the compact buffer)
+ *   cu_kept       device int32 [B+1]
+ *   sel, cu_sel   from lsa_topk_tokens; max_sel a multiple of 64
+ *   k_out, v_out  device bf16 [out_chunks][8][64][128]
+ *   cu_units      device int32 [B+1]
+ * Every count must be a multiple of 64 (k a multiple of 64 guarantees it).
+ * Device errors: BAD_COUNT (a count that is not, or bad cu_kept: skipped),
+ * CAPACITY (a unit beyond out_chunks: skipped), BAD_CHUNK (a position outside
+ * the sequence's recalled tokens: that row is written as zeros).
+ */
+int lsa_gather_tokens(const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
+                      const int32_t* sel, const int32_t* cu_sel, int B, int max_sel, void* k_out,
+                      void* v_out, int64_t out_chunks, int32_t* cu_units, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -59,6 +59,9 @@ def _load():
         "lsa_topk_chunks_local": ([P, P, P, I, I, I, I, P, P, P, P], I),
         "lsa_append_token": ([P, P, P, P, P, I, P], I),
         "lsa_reset_local": ([P, I, P], I),
+        "lsa_token_score": ([P, P, P, I64, P, P, P, I, I, I, P, P, P], I),
+        "lsa_topk_tokens": ([P, P, I, I, I, I, P, P, P, P], I),
+        "lsa_gather_tokens": ([P, P, I64, P, P, P, I, I, P, P, I64, P, P], I),
         "lsa_sparse_decode_attn_local": ([P, P, P, I64, P, I, F, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
@@ -325,6 +328,50 @@ def lsa_sparse_decode_attn_local(q, k_buf, v_buf, cu_kept, k_local, v_local, loc
         ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
 
 
+def lsa_token_score(q_idx, w, token_keys, chunk_table, kept, n_kept, max_chunks, scores, n_tokens, stream=None):
+    """Token-level scores inside the recalled chunks: scores[b, p] for p < 64 n_kept[b]
+    (token p % 64 of recalled chunk kept[b, p // 64]); n_tokens[b] = 64 n_kept[b]."""
+    _need(q_idx, "q_idx", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(token_keys, "token_keys", torch.bfloat16)
+    for t, n in ((kept, "kept"), (n_kept, "n_kept"), (n_tokens, "n_tokens")):
+        _need(t, n, torch.int32)
+    _need(scores, "scores", torch.float32)
+    if chunk_table is not None:
+        _need(chunk_table, "chunk_table", torch.int32)
+    B, max_kept = kept.shape
+    if tuple(q_idx.shape) != (B, INDEX_HEADS, INDEX_DIM) or tuple(scores.shape) != (B, CHUNK_TOKENS * max_kept):
+        raise ValueError("q_idx must be [B, 16, 128] and scores [B, 64 * max_kept]")
+    if token_keys.dim() != 3 or tuple(token_keys.shape[1:]) != (CHUNK_TOKENS, INDEX_DIM):
+        raise ValueError("token_keys must be [n_slots, 64, 128]")
+    _check("lsa_token_score", _load().lsa_token_score(
+        _ptr(q_idx), _ptr(w), _ptr(token_keys), token_keys.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(n_kept),
+        B, int(max_chunks), max_kept, _ptr(scores), _ptr(n_tokens), _stream(stream)))
+
+
+def lsa_topk_tokens(scores, n_tokens, k, sel, n_sel, cu_sel, stream=None):
+    """The k best token positions per sequence (score desc, position asc), ascending."""
+    _need(scores, "scores", torch.float32)
+    for t, n in ((n_tokens, "n_tokens"), (sel, "sel"), (n_sel, "n_sel"), (cu_sel, "cu_sel")):
+        _need(t, n, torch.int32)
+    B, max_tokens = scores.shape
+    _check("lsa_topk_tokens", _load().lsa_topk_tokens(
+        _ptr(scores), _ptr(n_tokens), int(k), B, max_tokens, sel.shape[1], _ptr(sel), _ptr(n_sel), _ptr(cu_sel),
+        _stream(stream)))
+
+
+def lsa_gather_tokens(k_buf, v_buf, cu_kept, sel, cu_sel, k_out, v_out, cu_units, stream=None):
+    """Packs the selected tokens into dense 64-token units (the attention's compact layout)."""
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf"), (k_out, "k_out"), (v_out, "v_out")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((cu_kept, "cu_kept"), (sel, "sel"), (cu_sel, "cu_sel"), (cu_units, "cu_units")):
+        _need(t, n, torch.int32)
+    B, max_sel = sel.shape
+    _check("lsa_gather_tokens", _load().lsa_gather_tokens(
+        _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), _ptr(sel), _ptr(cu_sel), B, max_sel,
+        _ptr(k_out), _ptr(v_out), k_out.shape[0], _ptr(cu_units), _stream(stream)))
+
+
 def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=None, stream=None):
     """lsa_sparse_decode_attn without a workspace argument, for callers that cannot
     allocate device memory; its scratch is a fixed array inside the library, shared
@@ -350,6 +397,7 @@ __all__ = [
     "lsa_threshold_chunks",
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token", "lsa_reset_local",
+    "lsa_token_score", "lsa_topk_tokens", "lsa_gather_tokens",
     "lsa_sparse_decode_attn_local", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

@@ -138,6 +138,73 @@ append_token_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v
   if (threadIdx.x == 0) local_len[b] = pos + 1;
 }
 
+// Token gather of the fine stage: the selected token positions of each
+// sequence (ascending; position p is row p % 64 of compact chunk
+// cu_kept[b] + p / 64) are packed into dense 64-token units in the same
+// [unit][KV head][64][128] layout as the compact buffer, so that the decode
+// attention runs over them unchanged.  One CTA copies one (unit, KV head):
+// 64 rows of K and of V, 256 B each, sixteen 16-byte loads per thread issued
+// before any store.  Counts are multiples of 64 (the budget is), so no unit is
+// partial; cu_units[b] = cu_sel[b] / 64.
+constexpr int kTokThreads = 128;
+constexpr int kRowVecs = kHeadDim * 2 / 16;                          // 16 x 16 B per row
+constexpr int kTokVecs = 2 * kChunkTokens * kRowVecs / kTokThreads;  // 16 per thread
+
+__global__ void __launch_bounds__(kTokThreads)
+gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ v_buf, int64_t buf_chunks,
+                     const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ sel,
+                     const int32_t* __restrict__ cu_sel, int max_sel, uint4* __restrict__ k_out,
+                     uint4* __restrict__ v_out, int64_t out_chunks, int32_t* __restrict__ cu_units,
+                     unsigned* status) {
+  const int b = blockIdx.y;
+  const int u = blockIdx.x / kNumKVHeads, g = blockIdx.x % kNumKVHeads;
+  const int tid = threadIdx.x;
+  const int s0 = __ldg(cu_sel + b), s1 = __ldg(cu_sel + b + 1);
+  const int n = s1 - s0;
+  const bool lead = blockIdx.x == 0 && tid == 0;
+  if (s0 < 0 || n < 0 || n > max_sel || (n % kChunkTokens) != 0 || (s0 % kChunkTokens) != 0) {
+    if (lead) set_status(status, LSA_DEV_ERR_BAD_COUNT);
+    return;
+  }
+  if (lead) {
+    cu_units[b + 1] = s1 / kChunkTokens;
+    if (b == 0) cu_units[0] = s0 / kChunkTokens;
+  }
+  if (u * kChunkTokens >= n) return;
+  const int64_t c0 = __ldg(cu_kept + b), c1 = __ldg(cu_kept + b + 1);
+  const int64_t ou = s0 / kChunkTokens + u;
+  if (c0 < 0 || c1 < c0 || c1 > buf_chunks || ou >= out_chunks) {
+    if (tid == 0) set_status(status, ou >= out_chunks ? LSA_DEV_ERR_CAPACITY : LSA_DEV_ERR_BAD_COUNT);
+    return;
+  }
+  const int64_t n_pos = (c1 - c0) * kChunkTokens;
+  const int32_t* my_sel = sel + static_cast<int64_t>(b) * max_sel + u * kChunkTokens;
+  uint4 v[kTokVecs];
+  bool ok[kTokVecs];
+#pragma unroll
+  for (int e = 0; e < kTokVecs; ++e) {
+    const int idx = tid + e * kTokThreads;
+    const int kv = idx / (kChunkTokens * kRowVecs), rem = idx % (kChunkTokens * kRowVecs);
+    const int r = rem / kRowVecs, x = rem % kRowVecs;
+    const int p = __ldg(my_sel + r);
+    ok[e] = p >= 0 && p < n_pos;
+    v[e] = make_uint4(0, 0, 0, 0);
+    if (ok[e]) {
+      const int64_t src = ((c0 + p / kChunkTokens) * kNumKVHeads + g) * kChunkTokens + p % kChunkTokens;
+      v[e] = __ldg((kv ? v_buf : k_buf) + src * kRowVecs + x);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < kTokVecs; ++e) {
+    const int idx = tid + e * kTokThreads;
+    const int kv = idx / (kChunkTokens * kRowVecs), rem = idx % (kChunkTokens * kRowVecs);
+    const int r = rem / kRowVecs, x = rem % kRowVecs;
+    const int64_t dst = (ou * kNumKVHeads + g) * kChunkTokens + r;
+    (kv ? v_out : k_out)[dst * kRowVecs + x] = v[e];
+    if (!ok[e] && x == 0) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
+  }
+}
+
 int check_common(const void* k_pool, const void* v_pool, int64_t n_slots, const int32_t* kept,
                  const int32_t* cu_kept, int B, int max_chunks, int max_kept, const void* k_buf, const void* v_buf,
                  int64_t buf_chunks) {
@@ -253,6 +320,26 @@ int lsa_append_token(const void* k_new, const void* v_new, void* k_local, void* 
   gather::append_token_kernel<<<B, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_local),
       static_cast<uint4*>(v_local), local_len, lsa_device_status_ptr());
+  return launch_status();
+}
+
+int lsa_gather_tokens(const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
+                      const int32_t* sel, const int32_t* cu_sel, int B, int max_sel, void* k_out, void* v_out,
+                      int64_t out_chunks, int32_t* cu_units, void* stream) {
+  using namespace lsa;
+  if (!k_buf || !v_buf || !cu_kept || !sel || !cu_sel || !k_out || !v_out || !cu_units || B <= 0 ||
+      max_sel <= 0 || buf_chunks <= 0 || out_chunks <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (max_sel % kChunkTokens != 0) return LSA_ERR_INVALID_ARG;
+  if (B > 65535 || static_cast<int64_t>(B) * max_sel >= (int64_t{1} << 31) ||
+      static_cast<int64_t>(max_sel / kChunkTokens) * kNumKVHeads > 0x7fffffff)
+    return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(k_buf) || !aligned16(v_buf) || !aligned16(k_out) || !aligned16(v_out)) return LSA_ERR_MISALIGNED;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  const dim3 grid((max_sel / kChunkTokens) * kNumKVHeads, B);
+  gather::gather_tokens_kernel<<<grid, gather::kTokThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_buf), static_cast<const uint4*>(v_buf), buf_chunks, cu_kept, sel, cu_sel, max_sel,
+      static_cast<uint4*>(k_out), static_cast<uint4*>(v_out), out_chunks, cu_units, lsa_device_status_ptr());
   return launch_status();
 }
 

@@ -18,6 +18,13 @@
 // thread issues the MMAs and commits them to an mbarrier; each warp then reads
 // its 32 TMEM lanes (one chunk per thread, 16 head logits) with tcgen05.ld and
 // applies the sigmoid and the weighted head sum in fp32.
+//
+// lsa_token_score is the second, token-level stage (summary page, 2.1
+// Architecture: native token-level scoring picks a fine-grained top-k inside
+// the recalled subset): the same form with the decode step's indexer query,
+// over every token of the recalled chunks.  Only the row source differs: tile
+// row r is token position p = 64 j + i (token i of the j-th recalled chunk),
+// whose key row is 64 * slot(kept[j]) + i of the per-token key pool.
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
@@ -40,15 +47,73 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int j, int rows) {
   return kb * rows * kKBlockBytes + r * kKBlockBytes + ((jj ^ (r & 7)) << 4);
 }
 
+// Row sources.  count(b) is the number of rows of sequence b (-1 when its
+// count is invalid), stride the row pitch of the score output, and key_row()
+// the key row of row c (false, with an error bit, when it is out of range).
+struct ChunkRows {
+  const int32_t* table;
+  const int32_t* n_chunks;
+  int max_chunks;
+  int64_t n_slots;
+  __device__ int count(int b) const {
+    const int n = __ldg(n_chunks + b);
+    return (n < 0 || n > max_chunks) ? -1 : n;
+  }
+  __device__ int64_t stride() const { return max_chunks; }
+  __device__ void on_count(int, int) const {}
+  __device__ bool key_row(int b, int c, int64_t* row, unsigned* err) const {
+    const int64_t slot =
+        table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
+    if (slot < 0 || slot >= n_slots) {
+      *err = LSA_DEV_ERR_BAD_SLOT;
+      return false;
+    }
+    *row = slot;
+    return true;
+  }
+};
+
+struct TokenRows {
+  const int32_t* table;
+  const int32_t* kept;
+  const int32_t* n_kept;
+  int max_chunks, max_kept;
+  int64_t n_slots;
+  int32_t* n_tokens;   // out: 64 * n_kept[b]
+  __device__ int count(int b) const {
+    const int n = __ldg(n_kept + b);
+    return (n < 0 || n > max_kept) ? -1 : n * kChunkTokens;
+  }
+  __device__ int64_t stride() const { return static_cast<int64_t>(max_kept) * kChunkTokens; }
+  __device__ void on_count(int b, int n) const { n_tokens[b] = n < 0 ? 0 : n; }
+  __device__ bool key_row(int b, int p, int64_t* row, unsigned* err) const {
+    const int j = p / kChunkTokens, i = p % kChunkTokens;
+    const int c = __ldg(kept + static_cast<int64_t>(b) * max_kept + j);
+    if (c < 0 || c >= max_chunks) {
+      *err = LSA_DEV_ERR_BAD_CHUNK;
+      return false;
+    }
+    const int64_t slot =
+        table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
+    if (slot < 0 || slot >= n_slots) {
+      *err = LSA_DEV_ERR_BAD_SLOT;
+      return false;
+    }
+    *row = slot * kChunkTokens + i;
+    return true;
+  }
+};
+
+template <class Rows>
 __global__ void __launch_bounds__(kThreads)
 index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restrict__ w,
-                   const __nv_bfloat16* __restrict__ keys, int64_t n_slots, const int32_t* __restrict__ table,
-                   const int32_t* __restrict__ n_chunks, int max_chunks, float* __restrict__ scores,
+                   const __nv_bfloat16* __restrict__ keys, Rows rows, float* __restrict__ scores,
                    float neg_scale_log2, unsigned* status) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int b = blockIdx.y;
-  const int n = __ldg(n_chunks + b);
-  if (n < 0 || n > max_chunks) {
+  const int n = rows.count(b);
+  if (blockIdx.x == 0 && threadIdx.x == 0) rows.on_count(b, n);
+  if (n < 0) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_BAD_COUNT);
     return;
   }
@@ -70,19 +135,19 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     mbar_fence_init();
   }
 
-  // A: key row of chunk base + tid, gathered through the chunk table.
+  // A: key row of row base + tid (a chunk, or a token of a recalled chunk).
   const int c = base + tid;
   bool ok = c < n;
-  int64_t slot = 0;
+  int64_t krow = 0;
   if (ok) {
-    slot = table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
-    if (slot < 0 || slot >= n_slots) {
-      set_status(status, LSA_DEV_ERR_BAD_SLOT);
+    unsigned err = 0;
+    if (!rows.key_row(b, c, &krow, &err)) {
+      set_status(status, err);
       ok = false;
     }
   }
   {
-    const uint4* src = reinterpret_cast<const uint4*>(keys + (ok ? slot : 0) * kIndexDim);
+    const uint4* src = reinterpret_cast<const uint4*>(keys + (ok ? krow : 0) * kIndexDim);
     uint4 v[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = ok ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
@@ -129,7 +194,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     float s = 0.f;
 #pragma unroll
     for (int h = 0; h < kIndexHeads; ++h) s += __ldg(w + h) * (1.f / (1.f + fast_exp2(logit[h] * neg_scale_log2)));
-    if (ok) scores[static_cast<int64_t>(b) * max_chunks + c] = s;
+    if (ok) scores[static_cast<int64_t>(b) * rows.stride() + c] = s;
   }
   tcgen05_fence_before();
   __syncthreads();
@@ -150,8 +215,32 @@ extern "C" int lsa_index_score(const void* q_idx, const float* w, const void* ch
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   const dim3 grid((max_chunks + score::kTile - 1) / score::kTile, B);
   const float neg_scale_log2 = -1.4426950408889634f / sqrtf(static_cast<float>(kIndexDim));
+  const score::ChunkRows rows{chunk_table, n_chunks, max_chunks, n_slots};
   score::index_score_kernel<<<grid, score::kThreads, score::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(chunk_keys), n_slots,
-      chunk_table, n_chunks, max_chunks, scores, neg_scale_log2, lsa_device_status_ptr());
+      static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(chunk_keys), rows, scores,
+      neg_scale_log2, lsa_device_status_ptr());
+  return launch_status();
+}
+
+extern "C" int lsa_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                               const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
+                               int max_chunks, int max_kept, float* scores, int32_t* n_tokens, void* stream) {
+  using namespace lsa;
+  if (!q_idx || !w || !token_keys || !kept || !n_kept || !scores || !n_tokens || B <= 0 || max_chunks <= 0 ||
+      max_kept <= 0 || n_slots <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (B > 65535) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(max_kept) * kChunkTokens >= (int64_t{1} << 31) ||
+      n_slots >= (int64_t{1} << 62) / kChunkTokens)
+    return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(token_keys)) return LSA_ERR_MISALIGNED;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  const int max_tokens = max_kept * kChunkTokens;
+  const dim3 grid((max_tokens + score::kTile - 1) / score::kTile, B);
+  const float neg_scale_log2 = -1.4426950408889634f / sqrtf(static_cast<float>(kIndexDim));
+  const score::TokenRows rows{chunk_table, kept, n_kept, max_chunks, max_kept, n_slots, n_tokens};
+  score::index_score_kernel<<<grid, score::kThreads, score::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(token_keys), rows, scores,
+      neg_scale_log2, lsa_device_status_ptr());
   return launch_status();
 }

@@ -15,6 +15,14 @@
 // digit passes, each a shared-memory histogram and a 256-bin scan.  The kept
 // set is then written in index order with two block-wide prefix scans, so the
 // output is ascending without a sort.
+//
+// Larger candidate sets (the token-level fine stage: 16K to 128K tokens per
+// sequence) take a cluster of 8 CTAs per sequence instead: 8192 threads keep
+// up to 16 keys each in registers; every radix pass builds one shared-memory
+// histogram per CTA, and each CTA sums the 8 histograms through distributed
+// shared memory, so all 8 reach the same boundary without touching global
+// memory; a last exchange of per-CTA (less, equal) counts gives each CTA its
+// output offset and its share of the boundary ties in index order.
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
@@ -230,9 +238,10 @@ __device__ void select_and_write(const float* __restrict__ sc, int cand, int kc,
 
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
-            const int32_t* __restrict__ k_per_seq, int n_local, int B, int max_chunks, int max_kept,
+            const int32_t* __restrict__ k_per_seq, int k_all, int n_local, int B, int max_chunks, int max_kept,
             int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, int32_t* __restrict__ cu_kept,
             unsigned* status) {
+  // k_per_seq == nullptr: every sequence has budget k_all.
   __shared__ int hist[256];
   __shared__ int warp_sums[32];
   __shared__ int sel[2];
@@ -243,12 +252,13 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   int part = 0;
   unsigned dummy = 0;
   for (int bb = tid; bb <= b; bb += kThreads)
-    part += kept_count(__ldg(n_chunks + bb), __ldg(k_per_seq + bb), n_local, max_chunks, max_kept, &dummy);
+    part += kept_count(__ldg(n_chunks + bb), k_per_seq ? __ldg(k_per_seq + bb) : k_all, n_local, max_chunks,
+                       max_kept, &dummy);
   int tot = 0;
   block_exclusive_scan(part, warp_sums, &tot);
   unsigned err = 0;
   const int n = __ldg(n_chunks + b);
-  const int nk = kept_count(n, __ldg(k_per_seq + b), n_local, max_chunks, max_kept, &err);
+  const int nk = kept_count(n, k_per_seq ? __ldg(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
   if (tid == 0) {
     cu_kept[b + 1] = tot;
     if (b == 0) cu_kept[0] = 0;
@@ -274,6 +284,204 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
     select_and_write<false>(sc, cand, kc, per, out, hist, warp_sums, sel);
 }
 
+// ---- cluster variant ------------------------------------------------------
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = kClusterCtas * kThreads;
+constexpr int kClusterMaxCand = kClusterThreads * kMaxPerThread;   // 131072
+// Candidate counts above this go to the cluster kernel (one CTA re-reads the
+// scores every pass beyond it).
+constexpr int kClusterMinCand = kThreads * kMaxPerThread;          // 16384
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
+topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
+                    const int32_t* __restrict__ k_per_seq, int k_all, int n_local, int B, int max_chunks,
+                    int max_kept, int32_t* __restrict__ kept, int32_t* __restrict__ n_kept,
+                    int32_t* __restrict__ cu_kept, unsigned* status) {
+  __shared__ int hist[256];
+  __shared__ int warp_sums[32];
+  __shared__ int sel[2];
+  __shared__ uint32_t xmm[2 * kClusterCtas];   // [rank] min key, [8 + rank] max key, pushed by each rank
+  __shared__ int xcnt[2 * kClusterCtas];       // [rank] keys below the boundary, [8 + rank] keys equal to it
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+
+  // Counts: identical in every CTA of the cluster, written by rank 0.  Every
+  // early return below depends on them only, so the whole cluster takes it.
+  int part = 0;
+  unsigned dummy = 0;
+  for (int bb = tid; bb <= b; bb += kThreads)
+    part += kept_count(__ldg(n_chunks + bb), k_per_seq ? __ldg(k_per_seq + bb) : k_all, n_local, max_chunks,
+                       max_kept, &dummy);
+  int tot = 0;
+  block_exclusive_scan(part, warp_sums, &tot);
+  unsigned err = 0;
+  const int n = __ldg(n_chunks + b);
+  const int nk = kept_count(n, k_per_seq ? __ldg(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
+  if (rank == 0 && tid == 0) {
+    cu_kept[b + 1] = tot;
+    if (b == 0) cu_kept[0] = 0;
+    n_kept[b] = nk;
+    if (err) set_status(status, err);
+  }
+  if (nk == 0) return;
+  int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
+  const int n_rec = min(n_local, n);
+  const int cand = n - n_rec;
+  const int kc = nk - n_rec;
+  const int gtid = static_cast<int>(rank) * kThreads + tid;
+  if (kc == cand) {
+    for (int c = gtid; c < n; c += kClusterThreads) out[c] = c;
+    return;
+  }
+  for (int i = gtid; i < n_rec; i += kClusterThreads) out[kc + i] = cand + i;
+  if (kc == 0) return;
+  const int per = (cand + kClusterThreads - 1) / kClusterThreads;
+  if (per > kMaxPerThread) {   // the host never launches this case
+    if (rank == 0 && tid == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
+    return;
+  }
+  const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
+  const int lo = min(cand, gtid * per), hi = min(cand, lo + per);
+  const int n_own = hi - lo;
+  uint32_t kr[kMaxPerThread];
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e) kr[e] = (e < n_own) ? desc_key(__ldg(sc + lo + e)) : 0u;
+
+  // ---- smallest and largest key of the whole cluster ------------------------
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e)
+    if (e < n_own) { kmin = min(kmin, kr[e]); kmax = max(kmax, kr[e]); }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+  }
+  if (lane == 0) { warp_sums[tid >> 5] = static_cast<int>(kmin); hist[tid >> 5] = static_cast<int>(kmax); }
+  __syncthreads();
+  if (tid < 32) {
+    uint32_t a = static_cast<uint32_t>(warp_sums[tid]), z = static_cast<uint32_t>(hist[tid]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, off));
+      z = max(z, __shfl_xor_sync(0xffffffffu, z, off));
+    }
+    if (tid < kClusterCtas) {   // push this CTA's extremes to every rank
+      st_cluster_u32(cluster_map(&xmm[rank], tid), a);
+      st_cluster_u32(cluster_map(&xmm[kClusterCtas + rank], tid), z);
+    }
+  }
+  cluster_sync_all();
+  kmin = 0xffffffffu;
+  kmax = 0u;
+#pragma unroll
+  for (int r = 0; r < kClusterCtas; ++r) {
+    kmin = min(kmin, xmm[r]);
+    kmax = max(kmax, xmm[kClusterCtas + r]);
+  }
+  const uint32_t diff = kmin ^ kmax;
+  int hi_bit = diff ? 31 - __clz(diff) : -1;
+  uint32_t mask = hi_bit >= 31 ? 0u : (0xffffffffu << (hi_bit + 1));
+  uint32_t prefix = kmin & mask;
+  int krem = kc;
+
+  // ---- radix select over the cluster ------------------------------------------
+  while (hi_bit >= 0) {
+    const int width = min(8, hi_bit + 1);
+    const int shift = hi_bit - width + 1;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kMaxPerThread; ++e)
+      if (e < n_own && (kr[e] & mask) == prefix) atomicAdd(&hist[(kr[e] >> shift) & dmask], 1);
+    cluster_sync_all();   // every rank's histogram is complete
+    int count = 0, incl = 0;
+    if (tid < 256) {
+#pragma unroll
+      for (int r = 0; r < kClusterCtas; ++r) count += static_cast<int>(ld_cluster_u32(cluster_map(&hist[tid], r)));
+      incl = count;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) warp_sums[tid >> 5] = incl;
+    }
+    __syncthreads();
+    if (tid < 256) {
+      for (int w = 0; w < (tid >> 5); ++w) incl += warp_sums[w];
+      const int excl = incl - count;
+      if (excl < krem && incl >= krem) {
+        sel[0] = tid;
+        sel[1] = krem - excl;
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel[0]) << shift;
+    mask |= dmask << shift;
+    krem = sel[1];
+    hi_bit -= width;
+    cluster_sync_all();   // no rank still reads a histogram that the next pass clears
+  }
+  const uint32_t boundary = prefix;   // the kc-th smallest key; krem of its ties are taken
+
+  // ---- offsets of this CTA: keys below the boundary and ties of lower ranks ---
+  int n_less = 0, n_eq = 0;
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e) {
+    n_less += (e < n_own && kr[e] < boundary);
+    n_eq += (e < n_own && kr[e] == boundary);
+  }
+  int cta_eq = 0, cta_less = 0;
+  const int eq_before = block_exclusive_scan(n_eq, warp_sums, &cta_eq);
+  block_exclusive_scan(n_less, warp_sums, &cta_less);
+  if (tid < kClusterCtas) {
+    st_cluster_u32(cluster_map(&xcnt[rank], tid), static_cast<uint32_t>(cta_less));
+    st_cluster_u32(cluster_map(&xcnt[kClusterCtas + rank], tid), static_cast<uint32_t>(cta_eq));
+  }
+  cluster_sync_all();   // the last cluster-wide step: only local reads follow
+  int eq_off = 0, out_off = 0;
+  for (int r = 0; r < static_cast<int>(rank); ++r) {
+    const int eq_r = xcnt[kClusterCtas + r];
+    out_off += xcnt[r] + min(max(krem - eq_off, 0), eq_r);
+    eq_off += eq_r;
+  }
+  int eq_seen = eq_off + eq_before, n_sel = 0;
+  bool take[kMaxPerThread];
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e) {
+    bool t = false;
+    if (e < n_own) {
+      if (kr[e] < boundary) t = true;
+      else if (kr[e] == boundary) t = (eq_seen++ < krem);
+    }
+    take[e] = t;
+    n_sel += t;
+  }
+  int pos = out_off + block_exclusive_scan(n_sel, warp_sums, nullptr);
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e)
+    if (take[e]) out[pos++] = lo + e;
+}
+
+// One CTA per sequence up to kClusterMinCand candidates, a cluster of 8 up to
+// kClusterMaxCand, one CTA re-reading the scores beyond.
+int launch_topk(const float* scores, const int32_t* n_count, const int32_t* k_per_seq, int k_all, int n_local,
+                int B, int max_count, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
+                cudaStream_t s) {
+  if (max_count > kClusterMinCand && max_count <= kClusterMaxCand) {
+    topk_cluster_kernel<<<dim3(kClusterCtas, B), kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B,
+                                                                    max_count, max_kept, kept, n_kept, cu_kept,
+                                                                    lsa_device_status_ptr());
+  } else {
+    topk_kernel<<<B, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count, max_kept, kept,
+                                        n_kept, cu_kept, lsa_device_status_ptr());
+  }
+  return launch_status();
+}
+
 }  // namespace topk
 }  // namespace lsa
 
@@ -287,9 +495,25 @@ extern "C" int lsa_topk_chunks_local(const float* scores, const int32_t* n_chunk
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
-  topk::topk_kernel<<<B, topk::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      scores, n_chunks, k_per_seq, n_local, B, max_chunks, max_kept, kept, n_kept, cu_kept, lsa_device_status_ptr());
-  return launch_status();
+  return topk::launch_topk(scores, n_chunks, k_per_seq, 0, n_local, B, max_chunks, max_kept, kept, n_kept, cu_kept,
+                           static_cast<cudaStream_t>(stream));
+}
+
+// Token-level fine top-k (summary page, 2.1 Architecture): the k best token
+// positions of each sequence's recalled chunks, same key and tie rule, no
+// recent window (every position is a candidate), ascending output.
+extern "C" int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int k, int B, int max_tokens,
+                               int max_sel, int32_t* sel, int32_t* n_sel, int32_t* cu_sel, void* stream) {
+  using namespace lsa;
+  if (!scores || !n_tokens || !sel || !n_sel || !cu_sel || B <= 0 || max_tokens <= 0 || max_sel <= 0 || k <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(B) * max_sel >= (int64_t{1} << 31) ||
+      static_cast<int64_t>(B) * max_tokens >= (int64_t{1} << 40))
+    return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  return topk::launch_topk(scores, n_tokens, nullptr, k, 0, B, max_tokens, max_sel, sel, n_sel, cu_sel,
+                           static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq, int B,

@@ -17,8 +17,9 @@ from typing import Optional
 import torch
 
 from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_append_token, lsa_attn_workspace_size,
-               lsa_fetch_from_host, lsa_gather_chunks, lsa_index_score, lsa_reset_local, lsa_sparse_decode_attn,
-               lsa_sparse_decode_attn_local, lsa_threshold_chunks, lsa_topk_chunks)
+               lsa_fetch_from_host, lsa_gather_chunks, lsa_gather_tokens, lsa_index_score, lsa_reset_local,
+               lsa_sparse_decode_attn, lsa_sparse_decode_attn_local, lsa_threshold_chunks, lsa_token_score,
+               lsa_topk_chunks, lsa_topk_tokens)
 
 TAU = 64
 
@@ -40,11 +41,16 @@ class LayerWindow:
     tokens decoded inside the window: ``append`` adds a step's token, and
     ``attend`` then covers the kept chunks plus the tokens appended so far;
     ``reset_local`` empties it when a window starts.
+
+    ``fine_k`` (a multiple of 64) adds the token-level fine stage: every step
+    ``fine_select`` scores each token of the recalled chunks with the step's
+    indexer query, keeps the ``fine_k`` best and packs them into dense units,
+    and ``attend`` then runs over those units instead of the whole recalled set.
     """
 
     def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
                  max_chunks: int, device="cuda", double_buffer: bool = False, selection: str = "topk",
-                 threshold: float = 0.5, n_local: int = 1, causal: bool = False):
+                 threshold: float = 0.5, n_local: int = 1, causal: bool = False, fine_k: int = 0):
         self.device = torch.device(device)
         self.n_chunks = n_chunks
         self.k_per_seq = k_per_seq
@@ -82,6 +88,20 @@ class LayerWindow:
             self.k_local = torch.zeros(lshape, dtype=torch.bfloat16, device=self.device)
             self.v_local = torch.zeros(lshape, dtype=torch.bfloat16, device=self.device)
             self.local_len = torch.zeros((self.B,), dtype=torch.int32, device=self.device)
+        self.fine_k = int(fine_k)
+        if self.fine_k:
+            if self.fine_k < 0 or self.fine_k % CHUNK_TOKENS:
+                raise ValueError("fine_k must be a positive multiple of 64")
+            dev = self.device
+            self.tok_scores = torch.empty((self.B, CHUNK_TOKENS * self.max_kept), dtype=torch.float32, device=dev)
+            self.n_tokens = torch.zeros((self.B,), dtype=torch.int32, device=dev)
+            self.sel = torch.zeros((self.B, self.fine_k), dtype=torch.int32, device=dev)
+            self.n_sel = torch.zeros((self.B,), dtype=torch.int32, device=dev)
+            self.cu_sel = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)
+            units = self.B * self.fine_k // CHUNK_TOKENS
+            self.k_fine = torch.empty((units, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+            self.v_fine = torch.empty_like(self.k_fine)
+            self.cu_units = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)
 
     def select(self, q_idx, w, chunk_keys, buf: int = 0, stream=None):
         """Indexer scores, then the selection (top-K or threshold) plus latest, into slot ``buf``."""
@@ -110,27 +130,44 @@ class LayerWindow:
         """Adds this step's token (k_new, v_new [B, 8, 128] bf16) to the local chunks (causal only)."""
         lsa_append_token(k_new, v_new, self.k_local, self.v_local, self.local_len, stream=stream)
 
+    def fine_select(self, q_tok, w, token_keys, buf: int = 0, stream=None):
+        """Token-level stage of one step: scores of the recalled tokens from the step's
+        indexer query q_tok [B, 16, 128], the fine_k best, packed into dense units."""
+        lsa_token_score(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf], self.max_chunks,
+                        self.tok_scores, self.n_tokens, stream=stream)
+        lsa_topk_tokens(self.tok_scores, self.n_tokens, self.fine_k, self.sel, self.n_sel, self.cu_sel, stream=stream)
+        lsa_gather_tokens(self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.sel, self.cu_sel, self.k_fine,
+                          self.v_fine, self.cu_units, stream=stream)
+
     def attend(self, q, out, buf: int = 0, stream=None, kv_unchanged: bool = False):
         """One decode step: out[B, 64, 128] fp32 from q[B, 64, 128] bf16.
 
         ``kv_unchanged``: the previous kernel on the stream did not write this
-        window's compact buffer or offsets (true for every step but the first).
+        window's compact buffer or offsets (true for every step but the first;
+        ignored with ``fine_k``, whose units change every step).
         With ``causal`` the tokens appended so far in the window are attended too."""
-        if self.causal:
-            lsa_sparse_decode_attn_local(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.k_local,
-                                         self.v_local, self.local_len, out, self.workspace, stream=stream,
-                                         kv_unchanged=kv_unchanged)
+        if self.fine_k:
+            kb, vb, cu, kv_unchanged = self.k_fine, self.v_fine, self.cu_units, False
         else:
-            lsa_sparse_decode_attn(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], out, self.workspace,
-                                   stream=stream, kv_unchanged=kv_unchanged)
+            kb, vb, cu = self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf]
+        if self.causal:
+            lsa_sparse_decode_attn_local(q, kb, vb, cu, self.k_local, self.v_local, self.local_len, out,
+                                         self.workspace, stream=stream, kv_unchanged=kv_unchanged)
+        else:
+            lsa_sparse_decode_attn(q, kb, vb, cu, out, self.workspace, stream=stream, kv_unchanged=kv_unchanged)
 
-    def run_window(self, q_idx, w, chunk_keys, k_pool, v_pool, q_steps, outs, stream=None, k_new=None, v_new=None):
+    def run_window(self, q_idx, w, chunk_keys, k_pool, v_pool, q_steps, outs, stream=None, k_new=None, v_new=None,
+                   q_tok=None, token_keys=None):
         """Select, gather, then one attention call per step of ``q_steps`` [T, B, 64, 128].
 
         Causal windows take the decoded tokens ``k_new``, ``v_new`` [T, B, 8, 128]:
-        step t appends its own token, then attends."""
+        step t appends its own token, then attends.  With ``fine_k`` every step
+        first runs the token stage with ``q_tok`` [T, B, 16, 128] over
+        ``token_keys`` [n_slots, 64, 128]."""
         if self.causal and (k_new is None or v_new is None):
             raise ValueError("a causal window needs k_new and v_new")
+        if self.fine_k and (q_tok is None or token_keys is None):
+            raise ValueError("the fine stage needs q_tok and token_keys")
         self.select(q_idx, w, chunk_keys, 0, stream)
         self.gather(k_pool, v_pool, 0, stream)
         if self.causal:
@@ -138,6 +175,8 @@ class LayerWindow:
         for t in range(q_steps.shape[0]):
             if self.causal:
                 self.append(k_new[t], v_new[t], stream)
+            if self.fine_k:
+                self.fine_select(q_tok[t], w, token_keys, 0, stream)
             self.attend(q_steps[t], outs[t], 0, stream, kv_unchanged=t > 0)
 
     def kept_lists(self, buf: int = 0):

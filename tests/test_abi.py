@@ -77,6 +77,14 @@ def test_host_checks_null_pointers(L):
     assert L.lsa_topk_chunks_local(n, n, n, 1, 1, 1, 1, n, n, n, n) == INVALID
     assert L.lsa_append_token(n, n, n, n, n, 1, n) == INVALID
     assert L.lsa_reset_local(n, 1, n) == INVALID
+    assert L.lsa_token_score(n, n, n, 1, n, n, n, 1, 1, 1, n, n, n) == INVALID
+    assert L.lsa_topk_tokens(n, n, 64, 1, 64, 64, n, n, n, n) == INVALID
+    assert L.lsa_gather_tokens(n, n, 1, n, n, n, 1, 64, n, n, 1, n, n) == INVALID
+    ok = ctypes.c_void_p(0x100000)
+    assert L.lsa_topk_tokens(ok, ok, 0, 1, 64, 64, ok, ok, ok, n) == INVALID                # k = 0
+    assert L.lsa_gather_tokens(ok, ok, 1, ok, ok, ok, 1, 100, ok, ok, 1, ok, n) == INVALID   # max_sel % 64
+    assert L.lsa_gather_tokens(ok, ok, 1, ok, ok, ok, 1, 64, ctypes.c_void_p(0x100008), ok, 1, ok, n) == MISALIGNED
+    assert L.lsa_token_score(ctypes.c_void_p(0x100002), ok, ok, 1, n, ok, ok, 1, 1, 1, ok, ok, n) == MISALIGNED
     assert L.lsa_reset_local(ctypes.c_void_p(0x100000), 0, n) == INVALID
     assert L.lsa_sparse_decode_attn_local(n, n, n, 1, n, 1, ctypes.c_float(0.1), n, n, n, n, n, 0, 0, n) == INVALID
     assert L.lsa_selftest_bounded_wait(1, n, 1000, n) == INVALID      # mode 1 needs a flag

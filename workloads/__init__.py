@@ -85,7 +85,7 @@ WORKLOADS = {
 
 # Per-tensor seed offsets.
 _OFF = {"lengths": 1, "slots": 2, "w": 10, "keys": 20, "kpool": 30, "vpool": 40,
-        "qidx": 50, "q": 60, "planted": 70, "knew": 80, "vnew": 90}
+        "qidx": 50, "q": 60, "planted": 70, "knew": 80, "vnew": 90, "tokkeys": 100, "qtok": 110}
 
 
 def _seed(base: int, name: str, layer: int = 0, extra: int = 0) -> int:
@@ -240,3 +240,14 @@ def decoded_tokens(inp: Inputs, layer: int, device, base_seed: int = BASE_SEED, 
     shape = (n_windows, inp.steps, inp.batch, NUM_KV_HEADS, HEAD_DIM)
     return (randn_bf16(shape, _seed(base_seed, "knew", layer), device),
             randn_bf16(shape, _seed(base_seed, "vnew", layer), device))
+
+
+def fine_inputs(inp: Inputs, layer: int, device, base_seed: int = BASE_SEED, windows: Optional[int] = None):
+    """Inputs of the token-level fine stage: per-token indexer keys by chunk slot,
+    bf16 [n_slots, 64, 128], and one indexer query per decode step, bf16
+    [windows, TAU, B, 16, 128]; both N(0, 1) like the chunk-level ones."""
+    n_windows = inp.workload.windows if windows is None else windows
+    keys = randn_bf16((inp.n_slots, CHUNK_TOKENS, INDEX_DIM), _seed(base_seed, "tokkeys", layer), device)
+    q_tok = randn_bf16((n_windows, inp.steps, inp.batch, INDEX_HEADS, INDEX_DIM), _seed(base_seed, "qtok", layer),
+                       device)
+    return keys, q_tok
