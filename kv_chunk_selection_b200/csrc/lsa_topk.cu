@@ -292,13 +292,21 @@ constexpr int kClusterMaxCand = kClusterThreads * kMaxPerThread;   // 131072
 // scores every pass beyond it).
 constexpr int kClusterMinCand = kThreads * kMaxPerThread;          // 16384
 
+// kPer: register slots per thread (4, 8 or 16), the smallest that holds the
+// candidates; dead slots still cost issue slots in every pass.
+template <int kPer>
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
 topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
                     const int32_t* __restrict__ k_per_seq, int k_all, int n_local, int B, int max_chunks,
                     int max_kept, int32_t* __restrict__ kept, int32_t* __restrict__ n_kept,
                     int32_t* __restrict__ cu_kept, unsigned* status) {
-  __shared__ int hist[256];
+  // Two histograms, alternating between passes: pass p clears the one that
+  // pass p-1's remote reads used two passes back, and the cluster barrier of
+  // pass p-1 orders those reads before this clear, so a pass needs one
+  // cluster barrier instead of two.
+  __shared__ int hist[2][256];
   __shared__ int warp_sums[32];
+  __shared__ uint32_t warp_max[32];
   __shared__ int sel[2];
   __shared__ uint32_t xmm[2 * kClusterCtas];   // [rank] min key, [8 + rank] max key, pushed by each rank
   __shared__ int xcnt[2 * kClusterCtas];       // [rank] keys below the boundary, [8 + rank] keys equal to it
@@ -337,40 +345,46 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   for (int i = gtid; i < n_rec; i += kClusterThreads) out[kc + i] = cand + i;
   if (kc == 0) return;
   const int per = (cand + kClusterThreads - 1) / kClusterThreads;
-  if (per > kMaxPerThread) {   // the host never launches this case
+  if (per > kPer) {   // the host never launches this case
     if (rank == 0 && tid == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
     return;
   }
+  // Past the last (cluster-uniform) return: announce this CTA to the cluster,
+  // load the keys, and wait for every CTA before the first remote store.
+  cluster_arrive_relaxed();
   const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
   const int lo = min(cand, gtid * per), hi = min(cand, lo + per);
   const int n_own = hi - lo;
-  uint32_t kr[kMaxPerThread];
+  uint32_t kr[kPer];
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e) kr[e] = (e < n_own) ? desc_key(__ldg(sc + lo + e)) : 0u;
+  for (int e = 0; e < kPer; ++e) kr[e] = (e < n_own) ? desc_key(__ldg(sc + lo + e)) : 0u;
 
   // ---- smallest and largest key of the whole cluster ------------------------
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e)
+  for (int e = 0; e < kPer; ++e)
     if (e < n_own) { kmin = min(kmin, kr[e]); kmax = max(kmax, kr[e]); }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
   }
-  if (lane == 0) { warp_sums[tid >> 5] = static_cast<int>(kmin); hist[tid >> 5] = static_cast<int>(kmax); }
+  if (lane == 0) { warp_sums[tid >> 5] = static_cast<int>(kmin); warp_max[tid >> 5] = kmax; }
   __syncthreads();
+  uint32_t cta_min = 0u, cta_max = 0u;   // valid in warp 0 (every lane, after the xor reduction)
   if (tid < 32) {
-    uint32_t a = static_cast<uint32_t>(warp_sums[tid]), z = static_cast<uint32_t>(hist[tid]);
+    cta_min = static_cast<uint32_t>(warp_sums[tid]);
+    cta_max = warp_max[tid];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      a = min(a, __shfl_xor_sync(0xffffffffu, a, off));
-      z = max(z, __shfl_xor_sync(0xffffffffu, z, off));
+      cta_min = min(cta_min, __shfl_xor_sync(0xffffffffu, cta_min, off));
+      cta_max = max(cta_max, __shfl_xor_sync(0xffffffffu, cta_max, off));
     }
-    if (tid < kClusterCtas) {   // push this CTA's extremes to every rank
-      st_cluster_u32(cluster_map(&xmm[rank], tid), a);
-      st_cluster_u32(cluster_map(&xmm[kClusterCtas + rank], tid), z);
-    }
+  }
+  cluster_wait();        // every CTA of the cluster is running
+  if (tid < kClusterCtas) {   // warp 0 pushes this CTA's extremes to every rank
+    st_cluster_u32(cluster_map(&xmm[rank], tid), cta_min);
+    st_cluster_u32(cluster_map(&xmm[kClusterCtas + rank], tid), cta_max);
   }
   cluster_sync_all();
   kmin = 0xffffffffu;
@@ -387,20 +401,22 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   int krem = kc;
 
   // ---- radix select over the cluster ------------------------------------------
+  int pass = 0;
   while (hi_bit >= 0) {
     const int width = min(8, hi_bit + 1);
     const int shift = hi_bit - width + 1;
     const uint32_t dmask = (1u << width) - 1u;
-    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    int* h = hist[pass & 1];
+    for (int i = tid; i < 256; i += kThreads) h[i] = 0;
     __syncthreads();
 #pragma unroll
-    for (int e = 0; e < kMaxPerThread; ++e)
-      if (e < n_own && (kr[e] & mask) == prefix) atomicAdd(&hist[(kr[e] >> shift) & dmask], 1);
-    cluster_sync_all();   // every rank's histogram is complete
+    for (int e = 0; e < kPer; ++e)
+      if (e < n_own && (kr[e] & mask) == prefix) atomicAdd(&h[(kr[e] >> shift) & dmask], 1);
+    cluster_sync_all();   // every rank's histogram of this pass is complete
     int count = 0, incl = 0;
     if (tid < 256) {
 #pragma unroll
-      for (int r = 0; r < kClusterCtas; ++r) count += static_cast<int>(ld_cluster_u32(cluster_map(&hist[tid], r)));
+      for (int r = 0; r < kClusterCtas; ++r) count += static_cast<int>(ld_cluster_u32(cluster_map(&h[tid], r)));
       incl = count;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -423,14 +439,15 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
     mask |= dmask << shift;
     krem = sel[1];
     hi_bit -= width;
-    cluster_sync_all();   // no rank still reads a histogram that the next pass clears
+    ++pass;
+    __syncthreads();   // sel is rewritten by the next pass
   }
   const uint32_t boundary = prefix;   // the kc-th smallest key; krem of its ties are taken
 
   // ---- offsets of this CTA: keys below the boundary and ties of lower ranks ---
   int n_less = 0, n_eq = 0;
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e) {
+  for (int e = 0; e < kPer; ++e) {
     n_less += (e < n_own && kr[e] < boundary);
     n_eq += (e < n_own && kr[e] == boundary);
   }
@@ -441,7 +458,9 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
     st_cluster_u32(cluster_map(&xcnt[rank], tid), static_cast<uint32_t>(cta_less));
     st_cluster_u32(cluster_map(&xcnt[kClusterCtas + rank], tid), static_cast<uint32_t>(cta_eq));
   }
-  cluster_sync_all();   // the last cluster-wide step: only local reads follow
+  // The last cluster-wide step: every remote read of a histogram above was
+  // consumed before this barrier, and only local reads follow it.
+  cluster_sync_all();
   int eq_off = 0, out_off = 0;
   for (int r = 0; r < static_cast<int>(rank); ++r) {
     const int eq_r = xcnt[kClusterCtas + r];
@@ -449,9 +468,9 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
     eq_off += eq_r;
   }
   int eq_seen = eq_off + eq_before, n_sel = 0;
-  bool take[kMaxPerThread];
+  bool take[kPer];
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e) {
+  for (int e = 0; e < kPer; ++e) {
     bool t = false;
     if (e < n_own) {
       if (kr[e] < boundary) t = true;
@@ -462,7 +481,7 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   }
   int pos = out_off + block_exclusive_scan(n_sel, warp_sums, nullptr);
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e)
+  for (int e = 0; e < kPer; ++e)
     if (take[e]) out[pos++] = lo + e;
 }
 
@@ -472,9 +491,17 @@ int launch_topk(const float* scores, const int32_t* n_count, const int32_t* k_pe
                 int B, int max_count, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
                 cudaStream_t s) {
   if (max_count > kClusterMinCand && max_count <= kClusterMaxCand) {
-    topk_cluster_kernel<<<dim3(kClusterCtas, B), kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B,
-                                                                    max_count, max_kept, kept, n_kept, cu_kept,
-                                                                    lsa_device_status_ptr());
+    const dim3 grid(kClusterCtas, B);
+    unsigned* st = lsa_device_status_ptr();
+    if (max_count <= kClusterThreads * 4)
+      topk_cluster_kernel<4><<<grid, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count,
+                                                       max_kept, kept, n_kept, cu_kept, st);
+    else if (max_count <= kClusterThreads * 8)
+      topk_cluster_kernel<8><<<grid, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count,
+                                                       max_kept, kept, n_kept, cu_kept, st);
+    else
+      topk_cluster_kernel<16><<<grid, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count,
+                                                        max_kept, kept, n_kept, cu_kept, st);
   } else {
     topk_kernel<<<B, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count, max_kept, kept,
                                         n_kept, cu_kept, lsa_device_status_ptr());
