@@ -324,6 +324,11 @@ int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, const void*
  * decoded since the window started, and a count local_len device int32 [B]
  * (0 at the start of a window; the caller resets it).
  *
+ * The local chunks must hold finite values in every row (zero them once when
+ * they are allocated): rows at or past local_len[b] are masked out of the
+ * softmax, but still enter the P.V product with weight 0, where a NaN or an
+ * infinity would poison the output.
+ *
  * lsa_append_token -- writes the new token of every sequence (k_new, v_new
  * device bf16 [B][8][128]) at position local_len[b] of its local chunk and
  * increments local_len[b].  Device error CAPACITY (the local chunk already

@@ -66,6 +66,8 @@ gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool
               const int32_t* __restrict__ table, const int32_t* __restrict__ kept, const int32_t* __restrict__ cu,
               int B, int max_chunks, int max_kept, uint4* __restrict__ k_buf, uint4* __restrict__ v_buf,
               int64_t buf_chunks, unsigned* status, PrevWindow prev) {
+  griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
+  griddep_wait();                 // the previous kernel on the stream has finished
   const int total = __ldg(cu + B);
   if (__ldg(cu) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
@@ -120,6 +122,8 @@ gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool
 __global__ void __launch_bounds__(256)
 append_token_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_local,
                     uint4* __restrict__ v_local, int32_t* __restrict__ local_len, unsigned* status) {
+  griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
+  griddep_wait();                 // the previous kernel on the stream has finished
   constexpr int kVecPerToken = kNumKVHeads * kHeadDim / 8;   // 128 x 16 B per token (all 8 heads)
   constexpr int kVecPerRow = kHeadDim / 8;                   // 16 x 16 B per (head, token)
   const int b = blockIdx.x;
@@ -156,6 +160,8 @@ gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ 
                      const int32_t* __restrict__ cu_sel, int max_sel, uint4* __restrict__ k_out,
                      uint4* __restrict__ v_out, int64_t out_chunks, int32_t* __restrict__ cu_units,
                      unsigned* status) {
+  griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
+  griddep_wait();                 // the previous kernel on the stream has finished
   const int b = blockIdx.y;
   const int u = blockIdx.x / kNumKVHeads, g = blockIdx.x % kNumKVHeads;
   const int tid = threadIdx.x;
@@ -231,10 +237,10 @@ int lsa_gather_chunks(const void* k_pool, const void* v_pool, int64_t n_slots, c
   if (st != LSA_OK) return st;
   const int sms = device_sm_count();
   if (sms <= 0) return LSA_ERR_NO_DEVICE;
-  gather::gather_kernel<<<sms * 8, gather::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k_pool), static_cast<const uint4*>(v_pool), n_slots, chunk_table, kept, cu_kept, B,
-      max_chunks, max_kept, static_cast<uint4*>(k_buf), static_cast<uint4*>(v_buf), buf_chunks,
-      lsa_device_status_ptr(), gather::PrevWindow{});
+  launch_pdl(false, gather::gather_kernel, dim3(sms * 8), dim3(gather::kThreads), 0, static_cast<cudaStream_t>(stream),
+             static_cast<const uint4*>(k_pool), static_cast<const uint4*>(v_pool), n_slots, chunk_table, kept,
+             cu_kept, B, max_chunks, max_kept, static_cast<uint4*>(k_buf), static_cast<uint4*>(v_buf), buf_chunks,
+             lsa_device_status_ptr(), gather::PrevWindow{});
   return launch_status();
 }
 
@@ -317,9 +323,9 @@ int lsa_append_token(const void* k_new, const void* v_new, void* k_local, void* 
   if (B > 65535) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_local) || !aligned16(v_local)) return LSA_ERR_MISALIGNED;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
-  gather::append_token_kernel<<<B, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_local),
-      static_cast<uint4*>(v_local), local_len, lsa_device_status_ptr());
+  launch_pdl(true, gather::append_token_kernel, dim3(B), dim3(256), 0, static_cast<cudaStream_t>(stream),
+             static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_local),
+             static_cast<uint4*>(v_local), local_len, lsa_device_status_ptr());
   return launch_status();
 }
 
@@ -337,9 +343,10 @@ int lsa_gather_tokens(const void* k_buf, const void* v_buf, int64_t buf_chunks, 
   if (!aligned16(k_buf) || !aligned16(v_buf) || !aligned16(k_out) || !aligned16(v_out)) return LSA_ERR_MISALIGNED;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   const dim3 grid((max_sel / kChunkTokens) * kNumKVHeads, B);
-  gather::gather_tokens_kernel<<<grid, gather::kTokThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k_buf), static_cast<const uint4*>(v_buf), buf_chunks, cu_kept, sel, cu_sel, max_sel,
-      static_cast<uint4*>(k_out), static_cast<uint4*>(v_out), out_chunks, cu_units, lsa_device_status_ptr());
+  launch_pdl(true, gather::gather_tokens_kernel, grid, dim3(gather::kTokThreads), 0, static_cast<cudaStream_t>(stream),
+             static_cast<const uint4*>(k_buf), static_cast<const uint4*>(v_buf), buf_chunks, cu_kept, sel, cu_sel,
+             max_sel, static_cast<uint4*>(k_out), static_cast<uint4*>(v_out), out_chunks, cu_units,
+             lsa_device_status_ptr());
   return launch_status();
 }
 

@@ -110,6 +110,8 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
                    const __nv_bfloat16* __restrict__ keys, Rows rows, float* __restrict__ scores,
                    float neg_scale_log2, unsigned* status) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
+  griddep_wait();                 // the previous kernel on the stream has finished
   const int b = blockIdx.y;
   const int n = rows.count(b);
   if (blockIdx.x == 0 && threadIdx.x == 0) rows.on_count(b, n);
@@ -216,9 +218,9 @@ extern "C" int lsa_index_score(const void* q_idx, const float* w, const void* ch
   const dim3 grid((max_chunks + score::kTile - 1) / score::kTile, B);
   const float neg_scale_log2 = -1.4426950408889634f / sqrtf(static_cast<float>(kIndexDim));
   const score::ChunkRows rows{chunk_table, n_chunks, max_chunks, n_slots};
-  score::index_score_kernel<<<grid, score::kThreads, score::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(chunk_keys), rows, scores,
-      neg_scale_log2, lsa_device_status_ptr());
+  launch_pdl(false, score::index_score_kernel<score::ChunkRows>, grid, dim3(score::kThreads), score::kSmemBytes,
+             static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(q_idx), w,
+             static_cast<const __nv_bfloat16*>(chunk_keys), rows, scores, neg_scale_log2, lsa_device_status_ptr());
   return launch_status();
 }
 
@@ -239,8 +241,8 @@ extern "C" int lsa_token_score(const void* q_idx, const float* w, const void* to
   const dim3 grid((max_tokens + score::kTile - 1) / score::kTile, B);
   const float neg_scale_log2 = -1.4426950408889634f / sqrtf(static_cast<float>(kIndexDim));
   const score::TokenRows rows{chunk_table, kept, n_kept, max_chunks, max_kept, n_slots, n_tokens};
-  score::index_score_kernel<<<grid, score::kThreads, score::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(token_keys), rows, scores,
-      neg_scale_log2, lsa_device_status_ptr());
+  launch_pdl(true, score::index_score_kernel<score::TokenRows>, grid, dim3(score::kThreads), score::kSmemBytes,
+             static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(q_idx), w,
+             static_cast<const __nv_bfloat16*>(token_keys), rows, scores, neg_scale_log2, lsa_device_status_ptr());
   return launch_status();
 }

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/lsa.h"
 
 namespace lsa {
@@ -26,6 +28,33 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encoder();
+
+// Launches `kernel` as a programmatic dependent launch on `s`: its grid may be
+// launched once every CTA of the previous kernel on the stream has signalled
+// griddepcontrol.launch_dependents, so its launch latency overlaps that
+// kernel's run.  Every kernel launched this way executes griddepcontrol.wait
+// before its first global-memory access, which orders it after the previous
+// kernel's completion and memory flush.
+//
+// With pdl == false it is an ordinary stream-ordered launch (the griddepcontrol
+// instructions are then no-ops).  The kernels of the per-step chain use PDL;
+// the once-per-window kernels do not: there, the next grid's CTAs waiting on
+// the SMs slowed the running selection more than the hidden launch saved.
+template <typename... KArgs, typename... Args>
+inline void launch_pdl(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace lsa
 

@@ -190,6 +190,7 @@ __device__ void select_and_write(const float* __restrict__ sc, int cand, int kc,
     __syncthreads();
   }
   const uint32_t boundary = prefix;  // the kc-th smallest key; take krem of its ties
+  griddep_launch_dependents();   // the rest is the output pass
 
   // ---- write the kept candidates in ascending index order ---------------------
   int n_eq = 0;
@@ -245,6 +246,7 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   __shared__ int hist[256];
   __shared__ int warp_sums[32];
   __shared__ int sel[2];
+  griddep_wait();   // the previous kernel on the stream has finished
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
 
@@ -310,6 +312,7 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   __shared__ int sel[2];
   __shared__ uint32_t xmm[2 * kClusterCtas];   // [rank] min key, [8 + rank] max key, pushed by each rank
   __shared__ int xcnt[2 * kClusterCtas];       // [rank] keys below the boundary, [8 + rank] keys equal to it
+  griddep_wait();   // the previous kernel on the stream has finished
   const int b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
@@ -443,6 +446,7 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
     __syncthreads();   // sel is rewritten by the next pass
   }
   const uint32_t boundary = prefix;   // the kc-th smallest key; krem of its ties are taken
+  griddep_launch_dependents();   // the rest is the count exchange and the output pass
 
   // ---- offsets of this CTA: keys below the boundary and ties of lower ranks ---
   int n_less = 0, n_eq = 0;
@@ -487,24 +491,20 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
 
 // One CTA per sequence up to kClusterMinCand candidates, a cluster of 8 up to
 // kClusterMaxCand, one CTA re-reading the scores beyond.
-int launch_topk(const float* scores, const int32_t* n_count, const int32_t* k_per_seq, int k_all, int n_local,
-                int B, int max_count, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
+int launch_topk(bool pdl, const float* scores, const int32_t* n_count, const int32_t* k_per_seq, int k_all,
+                int n_local, int B, int max_count, int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
                 cudaStream_t s) {
   if (max_count > kClusterMinCand && max_count <= kClusterMaxCand) {
     const dim3 grid(kClusterCtas, B);
     unsigned* st = lsa_device_status_ptr();
-    if (max_count <= kClusterThreads * 4)
-      topk_cluster_kernel<4><<<grid, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count,
-                                                       max_kept, kept, n_kept, cu_kept, st);
-    else if (max_count <= kClusterThreads * 8)
-      topk_cluster_kernel<8><<<grid, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count,
-                                                       max_kept, kept, n_kept, cu_kept, st);
-    else
-      topk_cluster_kernel<16><<<grid, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count,
-                                                        max_kept, kept, n_kept, cu_kept, st);
+    auto kernel = max_count <= kClusterThreads * 4   ? topk_cluster_kernel<4>
+                  : max_count <= kClusterThreads * 8 ? topk_cluster_kernel<8>
+                                                     : topk_cluster_kernel<16>;
+    launch_pdl(pdl, kernel, grid, dim3(kThreads), 0, s, scores, n_count, k_per_seq, k_all, n_local, B, max_count,
+               max_kept, kept, n_kept, cu_kept, st);
   } else {
-    topk_kernel<<<B, kThreads, 0, s>>>(scores, n_count, k_per_seq, k_all, n_local, B, max_count, max_kept, kept,
-                                        n_kept, cu_kept, lsa_device_status_ptr());
+    launch_pdl(pdl, topk_kernel, dim3(B), dim3(kThreads), 0, s, scores, n_count, k_per_seq, k_all, n_local, B, max_count,
+               max_kept, kept, n_kept, cu_kept, lsa_device_status_ptr());
   }
   return launch_status();
 }
@@ -522,8 +522,8 @@ extern "C" int lsa_topk_chunks_local(const float* scores, const int32_t* n_chunk
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
-  return topk::launch_topk(scores, n_chunks, k_per_seq, 0, n_local, B, max_chunks, max_kept, kept, n_kept, cu_kept,
-                           static_cast<cudaStream_t>(stream));
+  return topk::launch_topk(false, scores, n_chunks, k_per_seq, 0, n_local, B, max_chunks, max_kept, kept, n_kept,
+                           cu_kept, static_cast<cudaStream_t>(stream));
 }
 
 // Token-level fine top-k (summary page, 2.1 Architecture): the k best token
@@ -539,7 +539,7 @@ extern "C" int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int
       static_cast<int64_t>(B) * max_tokens >= (int64_t{1} << 40))
     return LSA_ERR_UNSUPPORTED_SHAPE;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
-  return topk::launch_topk(scores, n_tokens, nullptr, k, 0, B, max_tokens, max_sel, sel, n_sel, cu_sel,
+  return topk::launch_topk(true, scores, n_tokens, nullptr, k, 0, B, max_tokens, max_sel, sel, n_sel, cu_sel,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -568,6 +568,8 @@ threshold_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n
                  const float* __restrict__ w, float threshold, int max_chunks, int max_kept,
                  int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, unsigned* status) {
   __shared__ int warp_sums[32];
+  griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
+  griddep_wait();                 // the previous kernel on the stream has finished
   const int b = blockIdx.x, tid = threadIdx.x;
   const int n = __ldg(n_chunks + b);
   if (n < 0 || n > max_chunks) {
@@ -606,6 +608,8 @@ threshold_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n
 __global__ void __launch_bounds__(kThreads)
 offsets_kernel(const int32_t* __restrict__ n_kept, int B, int32_t* __restrict__ cu_kept) {
   __shared__ int warp_sums[32];
+  griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
+  griddep_wait();                 // the previous kernel on the stream has finished
   const int tid = threadIdx.x;
   constexpr int kPer = (LSA_MAX_BATCH + kThreads - 1) / kThreads;   // 4
   int v[kPer], s = 0;
@@ -639,10 +643,10 @@ extern "C" int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks
   if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  topk::threshold_kernel<<<B, topk::kThreads, 0, s>>>(scores, n_chunks, w, threshold, max_chunks, max_kept, kept,
-                                                       n_kept, lsa_device_status_ptr());
+  launch_pdl(false, topk::threshold_kernel, dim3(B), dim3(topk::kThreads), 0, s, scores, n_chunks, w, threshold, max_chunks,
+             max_kept, kept, n_kept, lsa_device_status_ptr());
   int st = launch_status();
   if (st != LSA_OK) return st;
-  topk::offsets_kernel<<<1, topk::kThreads, 0, s>>>(n_kept, B, cu_kept);
+  launch_pdl(false, topk::offsets_kernel, dim3(1), dim3(topk::kThreads), 0, s, n_kept, B, cu_kept);
   return launch_status();
 }
