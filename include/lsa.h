@@ -362,6 +362,27 @@ int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v
                                  size_t workspace_bytes, unsigned int flags, void* stream);
 
 /*
+ * lsa_sparse_decode_attn_append -- one causal decode step in one launch:
+ * lsa_append_token followed by lsa_sparse_decode_attn_local, fused.  With
+ * n = local_len_in[b], the step attends the kept chunks, tokens 0 .. n-1 of
+ * the local chunk and this step's own token (k_new, v_new device bf16
+ * [B][8][128]) as token n; it also writes that token to row n of the local
+ * chunk and sets local_len_out[b] = n + 1.  local_len_in is only read and
+ * local_len_out only written (they must be different arrays; a decode loop
+ * alternates the two), so no reader of this launch sees the count change.
+ * n == 64 (the local chunk is full) sets CAPACITY: the token is neither
+ * attended nor stored, and local_len_out[b] = 64.  Other arguments, the
+ * finiteness rule for the local chunks and LSA_ATTN_KV_UNCHANGED as for
+ * lsa_sparse_decode_attn_local.
+ */
+int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* v_buf,
+                                  int64_t buf_chunks, const int32_t* cu_kept, int B,
+                                  float softmax_scale, const void* k_new, const void* v_new,
+                                  void* k_local, void* v_local, const int32_t* local_len_in,
+                                  int32_t* local_len_out, float* out, void* workspace,
+                                  size_t workspace_bytes, unsigned int flags, void* stream);
+
+/*
  * Token-level fine stage.  Inside the recalled chunks, native token-level
  * scoring keeps a fine-grained top-k of entries (summary page, 2.1
  * Architecture; k = 2048 tokens for the DSA lightning indexer on the search

@@ -59,6 +59,7 @@ def _load():
         "lsa_topk_chunks_local": ([P, P, P, I, I, I, I, P, P, P, P], I),
         "lsa_append_token": ([P, P, P, P, P, I, P], I),
         "lsa_reset_local": ([P, I, P], I),
+        "lsa_sparse_decode_attn_append": ([P, P, P, I64, P, I, F, P, P, P, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_token_score": ([P, P, P, I64, P, P, P, I, I, I, P, P, P], I),
         "lsa_topk_tokens": ([P, P, I, I, I, I, P, P, P, P], I),
         "lsa_gather_tokens": ([P, P, I64, P, P, P, I, I, P, P, I64, P, P], I),
@@ -372,6 +373,34 @@ def lsa_gather_tokens(k_buf, v_buf, cu_kept, sel, cu_sel, k_out, v_out, cu_units
         _ptr(k_out), _ptr(v_out), k_out.shape[0], _ptr(cu_units), _stream(stream)))
 
 
+def lsa_sparse_decode_attn_append(q, k_buf, v_buf, cu_kept, k_new, v_new, k_local, v_local, local_len_in,
+                                  local_len_out, out, workspace, softmax_scale=None, stream=None,
+                                  kv_unchanged=False):
+    """One causal step in one launch: appends (k_new, v_new) [B, 8, 128] at row
+    local_len_in[b] of the local chunk, attends the kept chunks plus the local
+    tokens including it, and writes local_len_out[b] = local_len_in[b] + 1."""
+    _need(q, "q", torch.bfloat16)
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf"), (k_new, "k_new"), (v_new, "v_new"), (k_local, "k_local"),
+                 (v_local, "v_local")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((cu_kept, "cu_kept"), (local_len_in, "local_len_in"), (local_len_out, "local_len_out")):
+        _need(t, n, torch.int32)
+    _need(out, "out", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    B = q.shape[0]
+    if tuple(q.shape) != (B, NUM_Q_HEADS, HEAD_DIM) or tuple(out.shape) != (B, NUM_Q_HEADS, HEAD_DIM):
+        raise ValueError("q and out must be [B, 64, 128]")
+    if tuple(k_local.shape) != (B, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM) or k_local.shape != v_local.shape:
+        raise ValueError("k_local and v_local must be [B, 8, 64, 128]")
+    if tuple(k_new.shape) != (B, NUM_KV_HEADS, HEAD_DIM) or k_new.shape != v_new.shape:
+        raise ValueError("k_new and v_new must be [B, 8, 128]")
+    scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
+    _check("lsa_sparse_decode_attn_append", _load().lsa_sparse_decode_attn_append(
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(k_new), _ptr(v_new),
+        _ptr(k_local), _ptr(v_local), _ptr(local_len_in), _ptr(local_len_out), _ptr(out), _ptr(workspace),
+        workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
+
+
 def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=None, stream=None):
     """lsa_sparse_decode_attn without a workspace argument, for callers that cannot
     allocate device memory; its scratch is a fixed array inside the library, shared
@@ -397,7 +426,7 @@ __all__ = [
     "lsa_threshold_chunks",
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token", "lsa_reset_local",
-    "lsa_token_score", "lsa_topk_tokens", "lsa_gather_tokens",
+    "lsa_token_score", "lsa_topk_tokens", "lsa_gather_tokens", "lsa_sparse_decode_attn_append",
     "lsa_sparse_decode_attn_local", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

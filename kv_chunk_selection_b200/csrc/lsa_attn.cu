@@ -125,6 +125,18 @@ struct UnitCursor {
   }
 };
 
+// The decode step's own token, appended inside the step (all null otherwise):
+// position n = local_len[b] of the local chunk receives it and is attended as
+// token n; the new count n + 1 goes to a second array, so that no reader of
+// this grid sees the count change.
+struct AppendArgs {
+  const uint4* k_new;   // [B][8 KV heads][16 x 16 B]: one token
+  const uint4* v_new;
+  uint4* k_local;       // [B][8][64 tokens][16 x 16 B]: the local chunks
+  uint4* v_local;
+  int32_t* len_out;     // [B]
+};
+
 // Grid: kCtasPerSm CTAs per SM, capped at kMaxCtas.
 inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasPerSm : kMaxCtas; }
 
@@ -134,7 +146,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                           const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu, int B,
                           int64_t buf_chunks, const int32_t* __restrict__ local_len, float scale_log2,
                           float* __restrict__ out, int* __restrict__ counters, float* __restrict__ records,
-                          unsigned* status, int kv_unchanged) {
+                          unsigned* status, int kv_unchanged, AppendArgs app) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte TMA swizzle pattern repeats every 1024 bytes and the fragment
   // addressing below assumes each box starts on such a boundary.
@@ -365,13 +377,22 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     const int cb = __ldg(cu + b);
     const int n_kept_b = __ldg(cu + b + 1) - cb;
     const int n_b = n_kept_b + E;   // units of the pair
-    // Valid tokens of the pair's local unit (its last unit, when E = 1).
-    int valid_local = 64;
+    // Valid tokens of the pair's local unit (its last unit, when E = 1), and
+    // the row that receives this step's own token (-1: none).
+    int valid_local = 64, new_row = -1;
     if (E) {
       valid_local = __ldg(local_len + b);
       if (valid_local < 0 || valid_local > kChunkTokens) {
         if (tid == 0 && g == 0) set_status(status, LSA_DEV_ERR_BAD_COUNT);
         valid_local = min(max(valid_local, 0), kChunkTokens);
+      }
+      if (app.k_new) {
+        if (valid_local < kChunkTokens) {
+          new_row = valid_local;
+          valid_local += 1;
+        } else if (tid == 0 && g == 0) {
+          set_status(status, LSA_DEV_ERR_CAPACITY);   // the local chunk is full: the token is not appended
+        }
       }
     }
     const int j0 = cur.j;
@@ -408,6 +429,24 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       }
       if (ok) {
         const uint32_t sbase = smem_base + s * kStageBytes;
+        if (E && jj == n_kept_b && app.k_new) {
+          if (wig == 0 && lane == 0 && g == 0) app.len_out[b] = valid_local;   // one writer per sequence
+          if (new_row >= 0 && (new_row >> 4) == wig) {
+            // This warp owns row new_row: lanes 0-15 write the token's K row,
+            // lanes 16-31 its V row, into the tile (128-byte swizzle, as the
+            // ldmatrix offsets read it) and into the local chunk in memory.
+            const int kv = lane >> 4, x = lane & 15;
+            const int64_t pg = static_cast<int64_t>(b) * kNumKVHeads + g;
+            const uint4 val = __ldg((kv ? app.v_new : app.k_new) + pg * 16 + x);
+            const uint32_t off = (2 * kv + (x >> 3)) * kBoxBytes + new_row * 128 + (((x & 7) ^ (new_row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + off), "r"(val.x), "r"(val.y),
+                         "r"(val.z), "r"(val.w)
+                         : "memory");
+            (kv ? app.v_local : app.k_local)[(pg * kChunkTokens + new_row) * 16 + x] = val;
+            fence_proxy_async_smem();   // ordered before the TMA that refills this stage
+            __syncwarp();
+          }
+        }
         // ---- S^T[16 tokens x 8 heads] = K[16 x 128] Q^T[128 x 8] ----------
         float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -585,11 +624,12 @@ size_t lsa_attn_workspace_size(int B) {
 }  // extern "C"
 
 namespace {
-// Shared launcher of lsa_sparse_decode_attn and lsa_sparse_decode_attn_local
-// (k_local == nullptr: no local units).
+// Shared launcher of lsa_sparse_decode_attn, lsa_sparse_decode_attn_local
+// (k_local == nullptr: no local units) and lsa_sparse_decode_attn_append.
 int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
                 int B, float softmax_scale, const void* k_local, const void* v_local, const int32_t* local_len,
-                float* out, void* workspace, size_t workspace_bytes, unsigned int flags, void* stream) {
+                float* out, void* workspace, size_t workspace_bytes, unsigned int flags, void* stream,
+                const lsa::attn::AppendArgs& app = lsa::attn::AppendArgs{}) {
   using namespace lsa;
   if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
@@ -653,7 +693,7 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   if (cudaLaunchKernelEx(&cfg, attn::sparse_decode_attn_kernel, tm_k, tm_v, tm_kl, tm_vl,
                          static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
                          local ? local_len : static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records,
-                         lsa_device_status_ptr(), kv_unchanged) != cudaSuccess) {
+                         lsa_device_status_ptr(), kv_unchanged, app) != cudaSuccess) {
     cudaGetLastError();
     return LSA_ERR_CUDA;
   }
@@ -677,6 +717,21 @@ int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v
   if (!k_local) return LSA_ERR_INVALID_ARG;
   return attn_launch(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, k_local, v_local, local_len, out,
                      workspace, workspace_bytes, flags, stream);
+}
+
+int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
+                                  const int32_t* cu_kept, int B, float softmax_scale, const void* k_new,
+                                  const void* v_new, void* k_local, void* v_local, const int32_t* local_len_in,
+                                  int32_t* local_len_out, float* out, void* workspace, size_t workspace_bytes,
+                                  unsigned int flags, void* stream) {
+  using namespace lsa;
+  if (!k_local || !v_local || !k_new || !v_new || !local_len_in || !local_len_out) return LSA_ERR_INVALID_ARG;
+  if (static_cast<const void*>(local_len_in) == static_cast<const void*>(local_len_out)) return LSA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new)) return LSA_ERR_MISALIGNED;
+  const attn::AppendArgs app{static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                             static_cast<uint4*>(k_local), static_cast<uint4*>(v_local), local_len_out};
+  return attn_launch(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, k_local, v_local, local_len_in, out,
+                     workspace, workspace_bytes, flags, stream, app);
 }
 
 }  // extern "C"
@@ -777,6 +832,7 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
       tm_k, tm_v, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
-      static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records, lsa_device_status_ptr(), 0);
+      static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records, lsa_device_status_ptr(), 0,
+      attn::AppendArgs{});
   return launch_status();
 }

@@ -18,8 +18,8 @@ import torch
 
 from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_append_token, lsa_attn_workspace_size,
                lsa_fetch_from_host, lsa_gather_chunks, lsa_gather_tokens, lsa_index_score, lsa_reset_local,
-               lsa_sparse_decode_attn, lsa_sparse_decode_attn_local, lsa_threshold_chunks, lsa_token_score,
-               lsa_topk_chunks, lsa_topk_tokens)
+               lsa_sparse_decode_attn, lsa_sparse_decode_attn_append, lsa_sparse_decode_attn_local,
+               lsa_threshold_chunks, lsa_token_score, lsa_topk_chunks, lsa_topk_tokens)
 
 TAU = 64
 
@@ -38,9 +38,11 @@ class LayerWindow:
 
     ``n_local`` (top-K only) keeps the latest ``n_local`` chunks beside the K
     recalled ones.  With ``causal`` each sequence also has a local chunk of the
-    tokens decoded inside the window: ``append`` adds a step's token, and
-    ``attend`` then covers the kept chunks plus the tokens appended so far;
-    ``reset_local`` empties it when a window starts.
+    tokens decoded inside the window, emptied by ``reset_local`` when a window
+    starts.  ``attend_append`` runs one causal step in one launch (the step's
+    token is appended and attended together); ``append`` followed by ``attend``
+    does the same in two launches.  The token count lives in two arrays that
+    alternate between fused steps (one is read while the other is written).
 
     ``fine_k`` (a multiple of 64) adds the token-level fine stage: every step
     ``fine_select`` scores each token of the recalled chunks with the step's
@@ -87,7 +89,8 @@ class LayerWindow:
             lshape = (self.B, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM)
             self.k_local = torch.zeros(lshape, dtype=torch.bfloat16, device=self.device)
             self.v_local = torch.zeros(lshape, dtype=torch.bfloat16, device=self.device)
-            self.local_len = torch.zeros((self.B,), dtype=torch.int32, device=self.device)
+            self._lens = [torch.zeros((self.B,), dtype=torch.int32, device=self.device) for _ in range(2)]
+            self._phase = 0
         self.fine_k = int(fine_k)
         if self.fine_k:
             if self.fine_k < 0 or self.fine_k % CHUNK_TOKENS:
@@ -122,13 +125,36 @@ class LayerWindow:
                             self.max_chunks, self.k_bufs[buf], self.v_bufs[buf], num_ctas=num_ctas,
                             stream=stream, done_event=done_event)
 
+    @property
+    def local_len(self):
+        """Tokens in each local chunk [B] int32 (the array the next step reads)."""
+        return self._lens[self._phase]
+
     def reset_local(self, stream=None):
         """Empties every sequence's local chunk (start of a window; causal only)."""
-        lsa_reset_local(self.local_len, stream=stream)
+        self._phase = 0
+        lsa_reset_local(self._lens[0], stream=stream)
 
     def append(self, k_new, v_new, stream=None):
         """Adds this step's token (k_new, v_new [B, 8, 128] bf16) to the local chunks (causal only)."""
         lsa_append_token(k_new, v_new, self.k_local, self.v_local, self.local_len, stream=stream)
+
+    def _attn_buffers(self, buf):
+        if self.fine_k:
+            return self.k_fine, self.v_fine, self.cu_units
+        return self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf]
+
+    def attend_append(self, q, out, k_new, v_new, buf: int = 0, stream=None, kv_unchanged: bool = False):
+        """One causal step in one launch: the step's token (k_new, v_new [B, 8, 128])
+        joins the local chunks and is attended with the kept (or fine-selected)
+        tokens and the tokens decoded before it in this window."""
+        kb, vb, cu = self._attn_buffers(buf)
+        if self.fine_k:
+            kv_unchanged = False
+        lsa_sparse_decode_attn_append(q, kb, vb, cu, k_new, v_new, self.k_local, self.v_local,
+                                      self._lens[self._phase], self._lens[1 - self._phase], out, self.workspace,
+                                      stream=stream, kv_unchanged=kv_unchanged)
+        self._phase = 1 - self._phase
 
     def fine_select(self, q_tok, w, token_keys, buf: int = 0, stream=None):
         """Token-level stage of one step: scores of the recalled tokens from the step's
@@ -146,10 +172,9 @@ class LayerWindow:
         window's compact buffer or offsets (true for every step but the first;
         ignored with ``fine_k``, whose units change every step).
         With ``causal`` the tokens appended so far in the window are attended too."""
+        kb, vb, cu = self._attn_buffers(buf)
         if self.fine_k:
-            kb, vb, cu, kv_unchanged = self.k_fine, self.v_fine, self.cu_units, False
-        else:
-            kb, vb, cu = self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf]
+            kv_unchanged = False
         if self.causal:
             lsa_sparse_decode_attn_local(q, kb, vb, cu, self.k_local, self.v_local, self.local_len, out,
                                          self.workspace, stream=stream, kv_unchanged=kv_unchanged)
@@ -161,7 +186,7 @@ class LayerWindow:
         """Select, gather, then one attention call per step of ``q_steps`` [T, B, 64, 128].
 
         Causal windows take the decoded tokens ``k_new``, ``v_new`` [T, B, 8, 128]:
-        step t appends its own token, then attends.  With ``fine_k`` every step
+        step t appends its own token and attends it (one fused launch).  With ``fine_k`` every step
         first runs the token stage with ``q_tok`` [T, B, 16, 128] over
         ``token_keys`` [n_slots, 64, 128]."""
         if self.causal and (k_new is None or v_new is None):
@@ -173,11 +198,12 @@ class LayerWindow:
         if self.causal:
             self.reset_local(stream)
         for t in range(q_steps.shape[0]):
-            if self.causal:
-                self.append(k_new[t], v_new[t], stream)
             if self.fine_k:
                 self.fine_select(q_tok[t], w, token_keys, 0, stream)
-            self.attend(q_steps[t], outs[t], 0, stream, kv_unchanged=t > 0)
+            if self.causal:
+                self.attend_append(q_steps[t], outs[t], k_new[t], v_new[t], 0, stream, kv_unchanged=t > 0)
+            else:
+                self.attend(q_steps[t], outs[t], 0, stream, kv_unchanged=t > 0)
 
     def kept_lists(self, buf: int = 0):
         """Host copy of the kept chunk lists (for inspection and tests)."""

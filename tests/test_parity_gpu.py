@@ -338,6 +338,64 @@ def test_append_then_attend_is_causal():
     status_clean()
 
 
+def test_fused_append_step_matches_two_launch_path_and_oracle():
+    """lsa_sparse_decode_attn_append = lsa_append_token then the local attention,
+    bit for bit, and the oracle with the token at row n; the local chunk gets the
+    row, the other rows are untouched, and local_len_out = n + 1."""
+    n_kept, n_loc = [0, 3, 5, 1], [0, 5, 63, 17]
+    B = len(n_kept)
+    q, kb, vb, cu = ragged_buffers(n_kept, seed=91)
+    g = torch.Generator(device=DEV).manual_seed(92)
+    kl = torch.randn((B, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    vl = torch.randn((B, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    kn = torch.randn((B, 8, 128), generator=g, device=DEV).to(torch.bfloat16)
+    vn = torch.randn((B, 8, 128), generator=g, device=DEV).to(torch.bfloat16)
+    len_in = torch.tensor(n_loc, dtype=torch.int32, device=DEV)
+    len_out = torch.full((B,), -5, dtype=torch.int32, device=DEV)
+    kl_f, vl_f = kl.clone(), vl.clone()
+    out_f = torch.full((B, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_sparse_decode_attn_append(q, kb, vb, cu, kn, vn, kl_f, vl_f, len_in, len_out, out_f,
+                                      lsa.new_attn_workspace(B))
+    # two launches: append (in place), then the local attention
+    kl_t, vl_t, len_t = kl.clone(), vl.clone(), len_in.clone()
+    out_t = torch.full((B, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_append_token(kn, vn, kl_t, vl_t, len_t)
+    lsa.lsa_sparse_decode_attn_local(q, kb, vb, cu, kl_t, vl_t, len_t, out_t, lsa.new_attn_workspace(B))
+    torch.cuda.synchronize()
+    status_clean()
+    assert len_out.tolist() == [n + 1 for n in n_loc] == len_t.tolist()
+    assert torch.equal(kl_f, kl_t) and torch.equal(vl_f, vl_t)
+    for b, n in enumerate(n_loc):
+        assert torch.equal(kl_f[b, :, n], kn[b]) and torch.equal(vl_f[b, :, n], vn[b])
+    mask = torch.ones((B, 64), dtype=torch.bool, device=DEV)
+    mask[torch.arange(B), torch.tensor(n_loc)] = False
+    assert torch.equal(kl_f.permute(0, 2, 1, 3)[mask], kl.permute(0, 2, 1, 3)[mask])
+    assert torch.equal(out_f, out_t)
+    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), k_local=f64(kl_t), v_local=f64(vl_t),
+                                    local_len=[n + 1 for n in n_loc])
+    assert_attention_close(out_f, ref)
+
+
+def test_fused_append_full_local_chunk_reports_capacity():
+    n_kept = [2]
+    q, kb, vb, cu = ragged_buffers(n_kept, seed=93)
+    kl = torch.zeros((1, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    vl = torch.zeros_like(kl)
+    kl[:] = torch.randn((1, 8, 64, 128), generator=torch.Generator(device=DEV).manual_seed(94), device=DEV)
+    kn = torch.ones((1, 8, 128), dtype=torch.bfloat16, device=DEV)
+    len_in = torch.tensor([64], dtype=torch.int32, device=DEV)
+    len_out = torch.tensor([0], dtype=torch.int32, device=DEV)
+    before = kl.clone()
+    out = torch.empty((1, 64, 128), device=DEV)
+    lsa.lsa_sparse_decode_attn_append(q, kb, vb, cu, kn, kn, kl, vl, len_in, len_out, out, lsa.new_attn_workspace(1))
+    torch.cuda.synchronize()
+    assert lsa.read_device_status() & 8          # CAPACITY
+    assert len_out.tolist() == [64] and torch.equal(kl, before)
+    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), k_local=f64(kl), v_local=f64(vl),
+                                    local_len=[64])
+    assert_attention_close(out, ref)
+
+
 def test_append_reports_full_local_chunk():
     kl = torch.zeros((1, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
     ll = torch.tensor([64], dtype=torch.int32, device=DEV)
@@ -364,6 +422,57 @@ def test_topk_recent_window_matches_oracle(n_local):
         assert got[b] == list(ref[b]), f"seq {b}"
     assert i64(cu).tolist() == oracle.cumulative_kept(ref).tolist()
     status_clean()
+
+
+def test_max_batch_window_step():
+    """The largest batch the calls accept (4096 sequences), tiny ragged sequences,
+    some empty, through a paged table: score, select, gather and one attention
+    step.  Selection bit-exact on the GPU's scores, offsets exact, gathers exact,
+    attention on a sample of sequences and zeros for every empty one."""
+    B, M = 4096, 5
+    rng = np.random.default_rng(77)
+    n = rng.integers(0, M + 1, B)
+    n[:3] = [0, 1, M]
+    k = rng.integers(0, 3, B)
+    n_slots = int(n.sum())
+    perm = rng.permutation(n_slots)
+    table = np.zeros((B, M), dtype=np.int32)
+    off = 0
+    for b in range(B):
+        table[b, : n[b]] = perm[off: off + n[b]]
+        off += n[b]
+    g = torch.Generator(device=DEV).manual_seed(78)
+    k_pool = torch.randn((n_slots, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    v_pool = torch.randn((n_slots, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    keys = torch.randn((n_slots, 128), generator=g, device=DEV).to(torch.bfloat16)
+    w = torch.rand(16, generator=g, device=DEV)
+    q_idx = torch.randn((B, 16, 128), generator=g, device=DEV).to(torch.bfloat16)
+    q = torch.randn((B, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    n_t, k_t, tab = (torch.from_numpy(x.astype(np.int32)).to(DEV) for x in (n, k, table))
+    lw = LayerWindow(n_t, k_t, tab, M, DEV)
+    lw.select(q_idx, w, keys)
+    lw.gather(k_pool, v_pool)
+    out = torch.full((B, 64, 128), float("nan"), device=DEV)
+    lw.attend(q, out)
+    torch.cuda.synchronize()
+    status_clean()
+    sc = f64(lw.scores)
+    ref = oracle.topk_chunks(sc, n, k)
+    got = lw.kept_lists()
+    assert all(got[b] == list(ref[b]) for b in range(B))
+    cu = i64(lw.cu_kept[0])
+    assert cu.tolist() == oracle.cumulative_kept(ref).tolist()
+    for b in (1, 2, 4095, int(np.argmax(n))):
+        for j, c in enumerate(got[b]):
+            assert torch.equal(lw.k_bufs[0][cu[b] + j], k_pool[int(table[b, c])])
+    empty = [b for b in range(B) if n[b] == 0]
+    assert torch.all(out[empty] == 0)
+    seqs = sorted(set(rng.choice(B, 48, replace=False).tolist()) | {1, 2, 4095})
+    for b in seqs:   # one sequence at a time: only its own kept chunks go to the host
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        ref_o = oracle.sparse_decode_attn(f64(q[b: b + 1]), f64(lw.k_bufs[0][lo:hi]), f64(lw.v_bufs[0][lo:hi]),
+                                          [0, hi - lo])
+        assert_attention_close(out[b: b + 1], ref_o)
 
 
 def test_attention_closed_forms():
