@@ -690,6 +690,17 @@ def run_attn_only(args):
 
 # ---------------------------------------------------------- oracle (CPU) arm --
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -762,6 +773,16 @@ def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warm
         if group_steps is None and time.perf_counter() - start > budget_s and len(times) >= 1:
             break
     t_group = float(np.mean(times))
+    # the same step on one thread (BLAS limited to 1), for the per-core figure
+    t_one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            a = time.perf_counter()
+            oracle.sparse_decode_attn(qs[0], kb, vb, cu, heads=list(range(8)))
+            t_one = time.perf_counter() - a
+    except Exception:
+        pass
     window_s = t_sel + workloads.TAU * 8 * t_group
     value = workloads.TAU * B / window_s
     sample = (f"{workload}: one selection of window 0 (score {int(n.sum())} chunks, top-K, gather "
@@ -769,7 +790,9 @@ def oracle_sample(workload, budget_s, on_gpu_inputs=True, group_steps=None, warm
               f"KV-head group (8 query heads) each ({t_group * 1e3:.1f} ms mean); extrapolated to a window of "
               f"64 steps x 8 groups" + ("; causal: step t also attends t + 1 decoded tokens" if causal else ""))
     return {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", "sample": sample,
-            "window_s_extrapolated": window_s, "host_cpus": os.cpu_count()}, times, t_sel
+            "window_s_extrapolated": window_s, "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
+            "group_step_ms": t_group * 1e3,
+            "group_step_ms_1_thread": t_one * 1e3 if t_one is not None else None}, times, t_sel
 
 
 def run_reference(args, rank, world):
