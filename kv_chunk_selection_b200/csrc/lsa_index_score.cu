@@ -36,7 +36,7 @@ constexpr int kTile = 128;          // chunks per CTA (MMA M)
 constexpr int kKBlockBytes = 128;   // 64 bf16 per row per swizzle atom
 constexpr int kABytes = kTile * 2 * kKBlockBytes;          // 32 KiB: 2 K-blocks of [128 x 128 B]
 constexpr int kBBytes = kIndexHeads * 2 * kKBlockBytes;    // 4 KiB: 2 K-blocks of [16 x 128 B]
-constexpr int kSmemBytes = kABytes + kBBytes + 64;
+constexpr int kSmemBytes = kABytes + kBBytes + 16 + kTile * 9;   // + barrier, TMEM slot, row addresses and flags
 constexpr uint32_t kTmemCols = 32;  // allocation unit (>= 16 accumulator columns)
 constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kTile, kIndexHeads);
 
@@ -129,6 +129,8 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
   uint8_t* sb = smem + kABytes;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kABytes + kBBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  int64_t* row_at = reinterpret_cast<int64_t*>(smem + kABytes + kBBytes + 16);   // [kTile] key row or -1
+  bool* row_ok = reinterpret_cast<bool*>(row_at + kTile);                            // [kTile]
   const int tid = threadIdx.x, warp = tid >> 5;
 
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -137,24 +139,42 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     mbar_fence_init();
   }
 
-  // A: key row of row base + tid (a chunk, or a token of a recalled chunk).
-  const int c = base + tid;
-  bool ok = c < n;
-  int64_t krow = 0;
-  if (ok) {
-    unsigned err = 0;
-    if (!rows.key_row(b, c, &krow, &err)) {
-      set_status(status, err);
-      ok = false;
-    }
-  }
+  // A: the tile's 128 key rows (chunks, or tokens of recalled chunks).  Each
+  // thread first resolves one row's address (its lookup chain); then half a
+  // warp loads one 256-byte row, so a warp instruction reads two whole rows
+  // instead of 32 pieces of 32 different rows, all 16 loads of a thread issued
+  // before any store.  A row that is out of range or fails its lookup is zero
+  // and flagged, so its score is not written.
   {
-    const uint4* src = reinterpret_cast<const uint4*>(keys + (ok ? krow : 0) * kIndexDim);
+    const int c = base + tid;
+    bool okr = c < n;
+    int64_t krow = 0;
+    if (okr) {
+      unsigned err = 0;
+      if (!rows.key_row(b, c, &krow, &err)) {
+        set_status(status, err);
+        okr = false;
+      }
+    }
+    row_ok[tid] = okr;
+    row_at[tid] = okr ? krow : -1;
+  }
+  __syncthreads();
+  {
+    const int piece = tid & 15;
     uint4 v[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = ok ? __ldg(src + j) : make_uint4(0, 0, 0, 0);
+    for (int it = 0; it < 16; ++it) {
+      const int r = it * (kThreads / 16) + (tid >> 4);
+      const int64_t krow = row_at[r];
+      v[it] = krow >= 0 ? __ldg(reinterpret_cast<const uint4*>(keys + krow * kIndexDim) + piece)
+                        : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-    for (int j = 0; j < 16; ++j) *reinterpret_cast<uint4*>(sa + sw128_offset(tid, j, kTile)) = v[j];
+    for (int it = 0; it < 16; ++it) {
+      const int r = it * (kThreads / 16) + (tid >> 4);
+      *reinterpret_cast<uint4*>(sa + sw128_offset(r, piece, kTile)) = v[it];
+    }
   }
   // B: the 16 indexer query rows of sequence b (K-major, one row per head).
   {
@@ -196,7 +216,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     float s = 0.f;
 #pragma unroll
     for (int h = 0; h < kIndexHeads; ++h) s += __ldg(w + h) * (1.f / (1.f + fast_exp2(logit[h] * neg_scale_log2)));
-    if (ok) scores[static_cast<int64_t>(b) * rows.stride() + c] = s;
+    if (row_ok[tid]) scores[static_cast<int64_t>(b) * rows.stride() + base + tid] = s;
   }
   tcgen05_fence_before();
   __syncthreads();
