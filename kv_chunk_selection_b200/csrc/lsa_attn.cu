@@ -140,6 +140,17 @@ struct AppendArgs {
 // Grid: kCtasPerSm CTAs per SM, capped at kMaxCtas.
 inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasPerSm : kMaxCtas; }
 
+// Smallest share of units worth a CTA of its own.  A launch over few units
+// (the token-level fine stage: 32 units per KV head) runs on fewer CTAs, so
+// each (sequence, KV head) pair is split fewer ways and its merge folds fewer
+// partials; large launches keep one CTA per SM.
+constexpr int64_t kMinUnitsPerCta = 4;
+inline int grid_for_units(int sms, int64_t max_units) {
+  const int64_t want = (max_units + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+  const int full = grid_for(sms);
+  return want < 1 ? 1 : (want < full ? static_cast<int>(want) : full);
+}
+
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vl,
@@ -680,7 +691,8 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   // prologue (and, with LSA_ATTN_KV_UNCHANGED, its K/V stream) overlaps the
   // tail of that kernel; the kernel waits for it before touching its outputs.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(attn::grid_for(sms));
+  // buf_chunks bounds the kept total (cu_kept[B] lives on the device).
+  cfg.gridDim = dim3(attn::grid_for_units(sms, static_cast<int64_t>(kNumKVHeads) * (buf_chunks + (local ? B : 0))));
   cfg.blockDim = dim3(attn::kThreads);
   cfg.dynamicSmemBytes = attn::kSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
