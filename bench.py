@@ -497,7 +497,7 @@ def run_ours(args, rank, world, local_rank):
         "stage_us": {"select_and_gather_per_window": sel_s / args.steps * 1e6,
                      "attention_per_decode_step": attn_avg * 1e6,
                      "attention_64_steps": att_s / args.steps * 1e6},
-        "gpu_launches": args.steps * layers * (3 + workloads.TAU * (1 + 3 * bool(args.fine_k))),
+        "gpu_launches": args.steps * layers * (3 + workloads.TAU * (1 + (2 + int(args.causal)) * bool(args.fine_k))),
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -523,10 +523,11 @@ def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=
                                                    lw.max_chunks, lw.tok_scores, lw.n_tokens),
         "topk_tokens": lambda: lsa.lsa_topk_tokens(lw.tok_scores, lw.n_tokens, lw.fine_k, lw.sel, lw.n_sel,
                                                    lw.cu_sel),
-        "gather_tokens": lambda: lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], lw.sel, lw.cu_sel,
-                                                       lw.k_fine, lw.v_fine, lw.cu_units),
-        "attention": lambda: lw.attend(L.q[0, 0], out),
     }
+    if lw.packs:
+        calls["gather_tokens"] = lambda: lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], lw.sel,
+                                                               lw.cu_sel, lw.k_fine, lw.v_fine, lw.cu_units)
+    calls["attention"] = lambda: lw.attend(L.q[0, 0], out)
     with torch.cuda.stream(stream):
         lw.select(L.q_idx[0], L.w, L.chunk_keys)
         lw.gather(L.k_pool, L.v_pool)
@@ -535,6 +536,8 @@ def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=
     torch.cuda.synchronize()
     res = {}
     tokens = kept_total * 64
+    # (with the selected tokens read in place, the attention row is the kernel
+    # that copies them from the compact buffer itself)
     nbytes = {"token_score": tokens * 256 + B * 16 * 128 * 2 + tokens * 4,
               "topk_tokens": tokens * 4 + fine_total * 4,
               "gather_tokens": 2 * fine_total * TOKEN_KV_BYTES,

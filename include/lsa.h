@@ -362,6 +362,29 @@ int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v
                                  size_t workspace_bytes, unsigned int flags, void* stream);
 
 /*
+ * lsa_sparse_decode_attn_selected -- the decode attention of the token-level
+ * fine stage, read in place: for each sequence, the selected positions
+ * sel[b*max_sel + j], j < cu_sel[b+1] - cu_sel[b] (from lsa_topk_tokens;
+ * every count a multiple of 64), position p being token p % 64 of compact
+ * chunk cu_kept[b] + p / 64.  Equal to lsa_gather_tokens followed by
+ * lsa_sparse_decode_attn over the packed units, bit for bit, without the
+ * packed copy: the kernel copies the selected rows of k_buf / v_buf
+ * (bf16 [buf_chunks][8][64][128]) straight into its pipeline.
+ *   sel device int32 [B][max_sel], max_sel a multiple of 64;
+ *   cu_sel device int32 [B+1]; cu_kept device int32 [B+1]
+ * LSA_ATTN_KV_UNCHANGED additionally promises that sel and cu_sel were not
+ * written by the preceding kernel.  Device errors: CAPACITY (cu_sel
+ * inconsistent: nothing is computed), BAD_CHUNK (a position outside the
+ * sequence's recalled tokens: that row is read as zeros).  Workspace as for
+ * lsa_sparse_decode_attn.
+ */
+int lsa_sparse_decode_attn_selected(const void* q, const void* k_buf, const void* v_buf,
+                                    int64_t buf_chunks, const int32_t* cu_kept, const int32_t* sel,
+                                    const int32_t* cu_sel, int max_sel, int B, float softmax_scale,
+                                    float* out, void* workspace, size_t workspace_bytes,
+                                    unsigned int flags, void* stream);
+
+/*
  * lsa_sparse_decode_attn_append -- one causal decode step in one launch:
  * lsa_append_token followed by lsa_sparse_decode_attn_local, fused.  With
  * n = local_len_in[b], the step attends the kept chunks, tokens 0 .. n-1 of

@@ -60,6 +60,7 @@ def _load():
         "lsa_append_token": ([P, P, P, P, P, I, P], I),
         "lsa_reset_local": ([P, I, P], I),
         "lsa_sparse_decode_attn_append": ([P, P, P, I64, P, I, F, P, P, P, P, P, P, P, P, S, ctypes.c_uint, P], I),
+        "lsa_sparse_decode_attn_selected": ([P, P, P, I64, P, P, P, I, I, F, P, P, S, ctypes.c_uint, P], I),
         "lsa_token_score": ([P, P, P, I64, P, P, P, I, I, I, P, P, P], I),
         "lsa_topk_tokens": ([P, P, I, I, I, I, P, P, P, P], I),
         "lsa_gather_tokens": ([P, P, I64, P, P, P, I, I, P, P, I64, P, P], I),
@@ -373,6 +374,29 @@ def lsa_gather_tokens(k_buf, v_buf, cu_kept, sel, cu_sel, k_out, v_out, cu_units
         _ptr(k_out), _ptr(v_out), k_out.shape[0], _ptr(cu_units), _stream(stream)))
 
 
+def lsa_sparse_decode_attn_selected(q, k_buf, v_buf, cu_kept, sel, cu_sel, out, workspace, softmax_scale=None,
+                                    stream=None, kv_unchanged=False):
+    """Attention over the selected tokens (sel [B, max_sel] from lsa_topk_tokens), read
+    in place from the compact buffer: lsa_gather_tokens + lsa_sparse_decode_attn in one."""
+    _need(q, "q", torch.bfloat16)
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((cu_kept, "cu_kept"), (sel, "sel"), (cu_sel, "cu_sel")):
+        _need(t, n, torch.int32)
+    _need(out, "out", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    B = q.shape[0]
+    if tuple(q.shape) != (B, NUM_Q_HEADS, HEAD_DIM) or tuple(out.shape) != (B, NUM_Q_HEADS, HEAD_DIM):
+        raise ValueError("q and out must be [B, 64, 128]")
+    if sel.dim() != 2 or sel.shape[0] != B:
+        raise ValueError("sel must be [B, max_sel]")
+    scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
+    _check("lsa_sparse_decode_attn_selected", _load().lsa_sparse_decode_attn_selected(
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), _ptr(sel), _ptr(cu_sel), sel.shape[1], B,
+        scale, _ptr(out), _ptr(workspace), workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0,
+        _stream(stream)))
+
+
 def lsa_sparse_decode_attn_append(q, k_buf, v_buf, cu_kept, k_new, v_new, k_local, v_local, local_len_in,
                                   local_len_out, out, workspace, softmax_scale=None, stream=None,
                                   kv_unchanged=False):
@@ -427,6 +451,7 @@ __all__ = [
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token", "lsa_reset_local",
     "lsa_token_score", "lsa_topk_tokens", "lsa_gather_tokens", "lsa_sparse_decode_attn_append",
+    "lsa_sparse_decode_attn_selected",
     "lsa_sparse_decode_attn_local", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",
 ]

@@ -85,17 +85,24 @@ struct Partition {
   }
 };
 
+// Sequence offsets counted in 64-token units: an array of chunk offsets
+// (shift 0: cu_kept), or of token offsets that are multiples of 64 (shift 6:
+// cu_sel of the token-level fine stage, read without a packed copy).
+struct Offsets {
+  const int32_t* p;
+  int shift;
+  __device__ __forceinline__ int operator()(int i) const { return __ldg(p + i) >> shift; }
+};
+
 // Units of sequence b: its kept chunks plus E local chunks (E = 1 when the
 // window's decoded tokens are attended), for each of the 8 KV heads.  The
 // units of sequence b start at 8 * (cu[b] + E * b).
-__device__ __forceinline__ int64_t seq_unit_base(const int32_t* cu, int E, int b) {
-  return 8 * (static_cast<int64_t>(__ldg(cu + b)) + static_cast<int64_t>(E) * b);
+__device__ __forceinline__ int64_t seq_unit_base(Offsets cu, int E, int b) {
+  return 8 * (static_cast<int64_t>(cu(b)) + static_cast<int64_t>(E) * b);
 }
-__device__ __forceinline__ int units_of(const int32_t* cu, int E, int b) {
-  return __ldg(cu + b + 1) - __ldg(cu + b) + E;
-}
+__device__ __forceinline__ int units_of(Offsets cu, int E, int b) { return cu(b + 1) - cu(b) + E; }
 // Largest b in [0, B) whose units start at or before u (the sequence of unit u).
-__device__ __forceinline__ int seq_of_unit(const int32_t* cu, int E, int B, int64_t u) {
+__device__ __forceinline__ int seq_of_unit(Offsets cu, int E, int B, int64_t u) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -106,14 +113,14 @@ __device__ __forceinline__ int seq_of_unit(const int32_t* cu, int E, int B, int6
 
 struct UnitCursor {
   int b, g, j;
-  __device__ void start(const int32_t* cu, int E, int B, int64_t u) {
+  __device__ void start(Offsets cu, int E, int B, int64_t u) {
     b = seq_of_unit(cu, E, B, u);
     const int64_t r = u - seq_unit_base(cu, E, b);
     const int n = units_of(cu, E, b);
     g = static_cast<int>(r / n);
     j = static_cast<int>(r - static_cast<int64_t>(g) * n);
   }
-  __device__ void advance(const int32_t* cu, int E, int B, int n_b) {
+  __device__ void advance(Offsets cu, int E, int B, int n_b) {
     if (++j == n_b) {
       j = 0;
       if (++g == kNumKVHeads) {
@@ -137,6 +144,19 @@ struct AppendArgs {
   int32_t* len_out;     // [B]
 };
 
+// The token-level fine stage read in place (all null otherwise): unit j of
+// (b, g) holds the 64 selected positions sel[b][64 j .. 64 j + 63]; position
+// p is row p % 64 of compact chunk ck[b] + p / 64 of KV head g.  The producer
+// copies those rows straight into the stage instead of reading a packed copy.
+struct SelectArgs {
+  const int32_t* sel;   // [B][max_sel]
+  const int32_t* ck;    // [B + 1]: chunk offsets of the compact buffer (cu_kept)
+  int max_sel;
+  int64_t ck_chunks;    // chunks in the compact buffer
+  const uint4* k_buf;   // the compact buffer, [ck_chunks][8][64][16 x 16 B]
+  const uint4* v_buf;
+};
+
 // Grid: kCtasPerSm CTAs per SM, capped at kMaxCtas.
 inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasPerSm : kMaxCtas; }
 
@@ -154,10 +174,12 @@ inline int grid_for_units(int sms, int64_t max_units) {
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vl,
-                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu, int B,
+                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu_raw, int B,
                           int64_t buf_chunks, const int32_t* __restrict__ local_len, float scale_log2,
                           float* __restrict__ out, int* __restrict__ counters, float* __restrict__ records,
-                          unsigned* status, int kv_unchanged, AppendArgs app) {
+                          unsigned* status, int kv_unchanged, AppendArgs app, SelectArgs sa) {
+  const bool indexed = sa.sel != nullptr;
+  const Offsets cu{cu_raw, indexed ? 6 : 0};
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte TMA swizzle pattern repeats every 1024 bytes and the fragment
   // addressing below assumes each box starts on such a boundary.
@@ -182,9 +204,14 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   if (!kv_unchanged) griddep_wait();
 
   // ---- validate cu_kept (every thread reaches the same verdict) -------------
-  const int total = __ldg(cu + B);
-  int bad = (__ldg(cu) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) ? 1 : 0;
-  for (int b = tid; b < B; b += kThreads) bad |= (__ldg(cu + b + 1) < __ldg(cu + b));
+  // (Indexed: token offsets, multiples of 64, at most max_sel per sequence;
+  // buf_chunks is then the unit capacity B * max_sel / 64.)
+  const int total = cu(B);
+  int bad = (__ldg(cu_raw) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) ? 1 : 0;
+  for (int b = tid; b < B; b += kThreads) {
+    bad |= (cu(b + 1) < cu(b));
+    if (indexed) bad |= ((__ldg(cu_raw + b + 1) & 63) != 0) | (__ldg(cu_raw + b + 1) - __ldg(cu_raw + b) > sa.max_sel);
+  }
   bad = __syncthreads_or(bad);
   if (bad) {
     if (blockIdx.x == 0 && tid == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
@@ -214,7 +241,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], indexed ? 32 : 1);   // indexed: one cp.async arrival per producer lane
       mbar_init(&empty[s], kWarpsPerGroup);   // a stage is consumed by one warp group
     }
     flags[0] = 0;
@@ -224,6 +251,62 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   __syncthreads();
   griddep_launch_dependents();
   volatile int* abort_flag = flags;
+
+  if (warp == kConsumerWarps && indexed) {
+    // ============ producer warp, fine stage: selected rows in place ==========
+    // Each lane copies rows `lane` and `lane + 32` of the unit (K and V, 16
+    // pieces of 16 bytes each) to their swizzled places in the stage, then
+    // arrives on the stage's full barrier when its copies have landed.  A
+    // position outside the sequence's recalled tokens is written as zeros.
+    UnitCursor cur;
+    cur.start(cu, E, B, u0);
+    const int64_t n_units = u1 - u0;
+    int64_t issued = 0;
+    const uint32_t smem_base_p = smem_u32(smem);
+    for (int64_t i = 0; i < n_units; ++i) {
+      const int s = static_cast<int>(i % kStages);
+      if (i >= kStages) {
+        const unsigned par = static_cast<unsigned>(((i / kStages) - 1) & 1);
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait_bounded(&empty[s], par, abort_flag) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          if (lane == 0) {
+            if (!*abort_flag) set_status(status, LSA_DEV_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          break;
+        }
+      }
+      const int b = cur.b, g = cur.g, j = cur.j;
+      const int64_t ckb = __ldg(sa.ck + b);
+      const int64_t n_pos = (static_cast<int64_t>(__ldg(sa.ck + b + 1)) - ckb) * kChunkTokens;
+      const uint32_t st = smem_base_p + s * kStageBytes;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = lane + 32 * h;
+        const int p = __ldg(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + r);
+        const bool okp = p >= 0 && p < n_pos && ckb + p / kChunkTokens < sa.ck_chunks;
+        if (!okp) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
+        const int64_t row = okp ? ((ckb + p / kChunkTokens) * kNumKVHeads + g) * kChunkTokens + p % kChunkTokens : 0;
+        const uint4* ks = sa.k_buf + row * 16;
+        const uint4* vs = sa.v_buf + row * 16;
+        const uint32_t nb = okp ? 16u : 0u;
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const uint32_t off = (x >> 3) * kBoxBytes + r * 128 + (((x & 7) ^ (r & 7)) << 4);
+          cp_async_16_zfill(st + off, ks + x, nb);
+          cp_async_16_zfill(st + 2 * kBoxBytes + off, vs + x, nb);
+        }
+      }
+      cp_async_mbar_arrive_noinc(&full[s]);
+      issued = i + 1;
+      cur.advance(cu, E, B, units_of(cu, E, cur.b));
+    }
+    cp_async_wait_all();   // every copy this lane issued has landed before the warp leaves
+    (void)issued;
+    return;
+  }
 
   if (warp == kConsumerWarps) {
     // ====================== producer warp: TMA stream ========================
@@ -246,8 +329,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             break;
           }
         }
-        const int cb = __ldg(cu + cur.b);
-        const int n_kept_b = __ldg(cu + cur.b + 1) - cb;
+        const int cb = cu(cur.b);
+        const int n_kept_b = cu(cur.b + 1) - cb;
         const bool local = E && cur.j == n_kept_b;
         uint8_t* st = smem + s * kStageBytes;
         if (local && !waited) {
@@ -385,8 +468,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   int64_t unit_i = 0;
   while (u < u1) {
     const int b = cur.b, g = cur.g;
-    const int cb = __ldg(cu + b);
-    const int n_kept_b = __ldg(cu + b + 1) - cb;
+    const int cb = cu(b);
+    const int n_kept_b = cu(b + 1) - cb;
     const int n_b = n_kept_b + E;   // units of the pair
     // Valid tokens of the pair's local unit (its last unit, when E = 1), and
     // the row that receives this step's own token (-1: none).
@@ -640,7 +723,8 @@ namespace {
 int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
                 int B, float softmax_scale, const void* k_local, const void* v_local, const int32_t* local_len,
                 float* out, void* workspace, size_t workspace_bytes, unsigned int flags, void* stream,
-                const lsa::attn::AppendArgs& app = lsa::attn::AppendArgs{}) {
+                const lsa::attn::AppendArgs& app = lsa::attn::AppendArgs{},
+                const lsa::attn::SelectArgs& sa = lsa::attn::SelectArgs{}) {
   using namespace lsa;
   if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
@@ -705,7 +789,7 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   if (cudaLaunchKernelEx(&cfg, attn::sparse_decode_attn_kernel, tm_k, tm_v, tm_kl, tm_vl,
                          static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
                          local ? local_len : static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records,
-                         lsa_device_status_ptr(), kv_unchanged, app) != cudaSuccess) {
+                         lsa_device_status_ptr(), kv_unchanged, app, sa) != cudaSuccess) {
     cudaGetLastError();
     return LSA_ERR_CUDA;
   }
@@ -729,6 +813,25 @@ int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v
   if (!k_local) return LSA_ERR_INVALID_ARG;
   return attn_launch(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, k_local, v_local, local_len, out,
                      workspace, workspace_bytes, flags, stream);
+}
+
+int lsa_sparse_decode_attn_selected(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
+                                    const int32_t* cu_kept, const int32_t* sel, const int32_t* cu_sel, int max_sel,
+                                    int B, float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                    unsigned int flags, void* stream) {
+  using namespace lsa;
+  if (!sel || !cu_sel || !cu_kept || !k_buf || !v_buf || max_sel <= 0 || B <= 0 || buf_chunks <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (max_sel % kChunkTokens != 0) return LSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * max_sel >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(k_buf) || !aligned16(v_buf)) return LSA_ERR_MISALIGNED;
+  const attn::SelectArgs sa{sel, cu_kept, max_sel, buf_chunks, static_cast<const uint4*>(k_buf),
+                            static_cast<const uint4*>(v_buf)};
+  // The kernel walks units of 64 selected tokens (cu_sel / 64); their number
+  // is at most B * max_sel / 64, which stands in for the buffer size.
+  const int64_t unit_cap = static_cast<int64_t>(B) * (max_sel / kChunkTokens);
+  return attn_launch(q, k_buf, v_buf, unit_cap, cu_sel, B, softmax_scale, nullptr, nullptr, nullptr, out, workspace,
+                     workspace_bytes, flags, stream, attn::AppendArgs{}, sa);
 }
 
 int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
@@ -845,6 +948,6 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
       tm_k, tm_v, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
       static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records, lsa_device_status_ptr(), 0,
-      attn::AppendArgs{});
+      attn::AppendArgs{}, attn::SelectArgs{});
   return launch_status();
 }

@@ -19,7 +19,8 @@ import torch
 from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_append_token, lsa_attn_workspace_size,
                lsa_fetch_from_host, lsa_gather_chunks, lsa_gather_tokens, lsa_index_score, lsa_reset_local,
                lsa_sparse_decode_attn, lsa_sparse_decode_attn_append, lsa_sparse_decode_attn_local,
-               lsa_threshold_chunks, lsa_token_score, lsa_topk_chunks, lsa_topk_tokens)
+               lsa_sparse_decode_attn_selected, lsa_threshold_chunks, lsa_token_score, lsa_topk_chunks,
+               lsa_topk_tokens)
 
 TAU = 64
 
@@ -46,8 +47,10 @@ class LayerWindow:
 
     ``fine_k`` (a multiple of 64) adds the token-level fine stage: every step
     ``fine_select`` scores each token of the recalled chunks with the step's
-    indexer query, keeps the ``fine_k`` best and packs them into dense units,
-    and ``attend`` then runs over those units instead of the whole recalled set.
+    indexer query and keeps the ``fine_k`` best, and ``attend`` runs over those
+    tokens only, reading them in place from the compact buffer.  With
+    ``causal`` too, the selected tokens are first packed into dense units (the
+    fused append reads packed units).
     """
 
     def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
@@ -101,10 +104,13 @@ class LayerWindow:
             self.sel = torch.zeros((self.B, self.fine_k), dtype=torch.int32, device=dev)
             self.n_sel = torch.zeros((self.B,), dtype=torch.int32, device=dev)
             self.cu_sel = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)
-            units = self.B * self.fine_k // CHUNK_TOKENS
-            self.k_fine = torch.empty((units, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
-            self.v_fine = torch.empty_like(self.k_fine)
-            self.cu_units = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)
+            self.packs = self.causal   # the causal step reads packed units
+            if self.packs:
+                units = self.B * self.fine_k // CHUNK_TOKENS
+                self.k_fine = torch.empty((units, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM), dtype=torch.bfloat16,
+                                          device=dev)
+                self.v_fine = torch.empty_like(self.k_fine)
+                self.cu_units = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)
 
     def select(self, q_idx, w, chunk_keys, buf: int = 0, stream=None):
         """Indexer scores, then the selection (top-K or threshold) plus latest, into slot ``buf``."""
@@ -140,7 +146,7 @@ class LayerWindow:
         lsa_append_token(k_new, v_new, self.k_local, self.v_local, self.local_len, stream=stream)
 
     def _attn_buffers(self, buf):
-        if self.fine_k:
+        if self.fine_k and self.packs:
             return self.k_fine, self.v_fine, self.cu_units
         return self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf]
 
@@ -158,12 +164,14 @@ class LayerWindow:
 
     def fine_select(self, q_tok, w, token_keys, buf: int = 0, stream=None):
         """Token-level stage of one step: scores of the recalled tokens from the step's
-        indexer query q_tok [B, 16, 128], the fine_k best, packed into dense units."""
+        indexer query q_tok [B, 16, 128] and the fine_k best (packed into dense
+        units when the window is causal)."""
         lsa_token_score(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf], self.max_chunks,
                         self.tok_scores, self.n_tokens, stream=stream)
         lsa_topk_tokens(self.tok_scores, self.n_tokens, self.fine_k, self.sel, self.n_sel, self.cu_sel, stream=stream)
-        lsa_gather_tokens(self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.sel, self.cu_sel, self.k_fine,
-                          self.v_fine, self.cu_units, stream=stream)
+        if self.packs:
+            lsa_gather_tokens(self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.sel, self.cu_sel,
+                              self.k_fine, self.v_fine, self.cu_units, stream=stream)
 
     def attend(self, q, out, buf: int = 0, stream=None, kv_unchanged: bool = False):
         """One decode step: out[B, 64, 128] fp32 from q[B, 64, 128] bf16.
@@ -172,6 +180,10 @@ class LayerWindow:
         window's compact buffer or offsets (true for every step but the first;
         ignored with ``fine_k``, whose units change every step).
         With ``causal`` the tokens appended so far in the window are attended too."""
+        if self.fine_k and not self.packs:   # the selected tokens, read in place
+            lsa_sparse_decode_attn_selected(q, self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.sel,
+                                            self.cu_sel, out, self.workspace, stream=stream)
+            return
         kb, vb, cu = self._attn_buffers(buf)
         if self.fine_k:
             kv_unchanged = False

@@ -83,6 +83,9 @@ def test_host_checks_null_pointers(L):
     assert L.lsa_sparse_decode_attn_append(ok, ok, ok, 4, ok, 1, ctypes.c_float(0.1), n, ok, ok, ok, ok,
                                            ctypes.c_void_p(0x200000), ok, ok, 1 << 30, 0, n) == INVALID
     assert L.lsa_token_score(n, n, n, 1, n, n, n, 1, 1, 1, n, n, n) == INVALID
+    assert L.lsa_sparse_decode_attn_selected(n, n, n, 1, n, n, n, 64, 1, ctypes.c_float(0.1), n, n, 0, 0, n) == INVALID
+    assert L.lsa_sparse_decode_attn_selected(ok, ok, ok, 4, ok, ok, ok, 100, 1, ctypes.c_float(0.1), ok, ok,
+                                             1 << 30, 0, n) == INVALID   # max_sel % 64
     assert L.lsa_topk_tokens(n, n, 64, 1, 64, 64, n, n, n, n) == INVALID
     assert L.lsa_gather_tokens(n, n, 1, n, n, n, 1, 64, n, n, 1, n, n) == INVALID
     ok = ctypes.c_void_p(0x100000)

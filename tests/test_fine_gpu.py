@@ -265,3 +265,48 @@ def test_window_tiny_fine_and_causal():
         ref = oracle.sparse_decode_attn(f64(L.q[0, t]), units_k, units_v, [0, units_k.shape[0]], k_local=k_loc,
                                         v_local=v_loc, local_len=[t + 1])
         assert_attention_close(outs[t], ref)
+
+
+def test_selected_in_place_equals_packed_path():
+    """lsa_sparse_decode_attn_selected (the selected rows copied straight from the
+    compact buffer) equals lsa_gather_tokens + lsa_sparse_decode_attn bit for bit;
+    a position outside the recalled tokens reads as zeros and is reported."""
+    inp, L, lw, tok_keys, q_tok = recalled("batched", batch=6)
+    k = 1024
+    scores, n_tok = token_scores_gpu(lw, q_tok[0, 3], L.w, tok_keys)
+    sel, n_sel, cu_sel = topk_tokens_gpu(scores, n_tok, k)
+    B = lw.B
+    units = B * k // 64
+    k_out = torch.zeros((units, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    v_out = torch.zeros_like(k_out)
+    cu_units = torch.zeros((B + 1,), dtype=torch.int32, device=DEV)
+    lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], sel, cu_sel, k_out, v_out, cu_units)
+    q = L.q[0, 3]
+    out_p = torch.full((B, 64, 128), float("nan"), device=DEV)
+    out_s = torch.full((B, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_sparse_decode_attn(q, k_out, v_out, cu_units, out_p, lsa.new_attn_workspace(B))
+    lsa.lsa_sparse_decode_attn_selected(q, lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], sel, cu_sel, out_s,
+                                        lsa.new_attn_workspace(B))
+    torch.cuda.synchronize()
+    status_clean()
+    assert torch.equal(out_s, out_p)
+    # one corrupted position: its rows are zeros, the status says BAD_CHUNK
+    bad = sel.clone()
+    b0 = int(np.argmax(i64(n_sel)))
+    bad[b0, 5] = 10 ** 8
+    out_b = torch.full((B, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_sparse_decode_attn_selected(q, lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], bad, cu_sel, out_b,
+                                        lsa.new_attn_workspace(B))
+    torch.cuda.synchronize()
+    assert lsa.read_device_status() & 4          # BAD_CHUNK
+    cs, ck = i64(cu_sel), i64(lw.cu_kept[0])
+    n = int(cs[b0 + 1] - cs[b0])
+    p = sel[b0, :n].to(torch.int64)
+    K = f64(lw.k_bufs[0][int(ck[b0]) + p // 64, :, p % 64])    # [n, 8, 128], gathered on the GPU
+    V = f64(lw.v_bufs[0][int(ck[b0]) + p // 64, :, p % 64])
+    K[5] = 0.0
+    V[5] = 0.0
+    units_k = K.reshape(-1, 64, 8, 128).transpose(0, 2, 1, 3)
+    units_v = V.reshape(-1, 64, 8, 128).transpose(0, 2, 1, 3)
+    ref = oracle.sparse_decode_attn(f64(q[b0: b0 + 1]), units_k, units_v, [0, units_k.shape[0]])
+    assert_attention_close(out_b[b0: b0 + 1], ref)
