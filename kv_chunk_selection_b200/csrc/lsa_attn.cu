@@ -165,8 +165,9 @@ inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasP
 // each (sequence, KV head) pair is split fewer ways and its merge folds fewer
 // partials; large launches keep one CTA per SM.
 constexpr int64_t kMinUnitsPerCta = 4;
-inline int grid_for_units(int sms, int64_t max_units) {
-  const int64_t want = (max_units + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+constexpr int64_t kMinIndexedUnitsPerCta = 2;   // the in-place fine stage: more CTAs issue its row copies
+inline int grid_for_units(int sms, int64_t max_units, int64_t per_cta = kMinUnitsPerCta) {
+  const int64_t want = (max_units + per_cta - 1) / per_cta;
   const int full = grid_for(sms);
   return want < 1 ? 1 : (want < full ? static_cast<int>(want) : full);
 }
@@ -776,7 +777,8 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   // tail of that kernel; the kernel waits for it before touching its outputs.
   cudaLaunchConfig_t cfg = {};
   // buf_chunks bounds the kept total (cu_kept[B] lives on the device).
-  cfg.gridDim = dim3(attn::grid_for_units(sms, static_cast<int64_t>(kNumKVHeads) * (buf_chunks + (local ? B : 0))));
+  cfg.gridDim = dim3(attn::grid_for_units(sms, static_cast<int64_t>(kNumKVHeads) * (buf_chunks + (local ? B : 0)),
+                                           sa.sel ? attn::kMinIndexedUnitsPerCta : attn::kMinUnitsPerCta));
   cfg.blockDim = dim3(attn::kThreads);
   cfg.dynamicSmemBytes = attn::kSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);

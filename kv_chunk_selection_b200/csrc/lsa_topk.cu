@@ -9,8 +9,9 @@
 // a 32-bit key that orders scores descending (the float bits mapped to an
 // order-preserving unsigned and complemented); the chunk index breaks ties
 // among equal keys.  Each thread owns a contiguous run of candidates and keeps
-// their keys in registers (up to 16 per thread, N <= 16384; larger N re-reads
-// the scores).  The bits that every key shares (found from a block-wide min
+// their keys in registers (up to 16 per thread, N <= 16384; beyond that the
+// cluster kernel below takes over, and beyond 131072 this kernel re-reads the
+// scores).  The bits that every key shares (found from a block-wide min
 // and max) need no pass, so scores in a narrow range take 3 or fewer 8-bit
 // digit passes, each a shared-memory histogram and a 256-bin scan.  The kept
 // set is then written in index order with two block-wide prefix scans, so the

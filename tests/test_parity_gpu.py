@@ -475,6 +475,33 @@ def test_max_batch_window_step():
         assert_attention_close(out[b: b + 1], ref_o)
 
 
+@pytest.mark.parametrize("n_local", [1, 3])
+def test_topk_long_sequences_cluster_kernel(n_local):
+    """Chunk top-K beyond 16384 candidates runs on the 8-CTA cluster kernel, with a
+    per-sequence K and a recent window; ragged lengths, one sequence short, one
+    empty; bit-exact against the oracle's rule on the same scores."""
+    n = np.array([40000, 17000, 5, 0, 23456])
+    k = np.array([4000, 1700, 2, 3, 2345])
+    B, M = len(n), int(n.max())
+    g = torch.Generator(device=DEV).manual_seed(31 + n_local)
+    scores = torch.rand((B, M), generator=g, device=DEV)
+    scores[0, ::7] = 0.5                      # many exact ties
+    n_t = torch.from_numpy(n.astype(np.int32)).to(DEV)
+    k_t = torch.from_numpy(k.astype(np.int32)).to(DEV)
+    max_kept = int(k.max()) + n_local
+    kept = torch.full((B, max_kept), -7, dtype=torch.int32, device=DEV)
+    n_kept = torch.zeros(B, dtype=torch.int32, device=DEV)
+    cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_topk_chunks(scores, n_t, k_t, kept, n_kept, cu, n_local=n_local)
+    torch.cuda.synchronize()
+    status_clean()
+    got = kept_from_gpu(kept, n_kept)
+    ref = oracle.topk_chunks(f64(scores), n, k, n_local=n_local)
+    for b in range(B):
+        assert got[b] == list(ref[b]), f"seq {b}"
+    assert i64(cu).tolist() == oracle.cumulative_kept(ref).tolist()
+
+
 def test_attention_closed_forms():
     n_kept = [3, 70]
     q, kb, vb, cu = ragged_buffers(n_kept, seed=4)
