@@ -33,6 +33,11 @@
 // * Launched as a programmatic dependent of the previous kernel: when the
 //   caller states that K/V did not change, the producer starts streaming
 //   before the previous kernel has finished.
+// * Variants on the same pipeline: a per-sequence local chunk of decoded
+//   tokens as one more masked unit per KV head (with the step's own token
+//   optionally written into it by the consumer warp that owns its row), and
+//   units of 64 selected tokens (the token-level fine stage) whose rows the
+//   producer warp copies straight from the compact buffer with cp.async.
 #include <math.h>
 
 #include <mutex>
@@ -262,7 +267,6 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     UnitCursor cur;
     cur.start(cu, E, B, u0);
     const int64_t n_units = u1 - u0;
-    int64_t issued = 0;
     const uint32_t smem_base_p = smem_u32(smem);
     for (int64_t i = 0; i < n_units; ++i) {
       const int s = static_cast<int>(i % kStages);
@@ -301,11 +305,9 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
       }
       cp_async_mbar_arrive_noinc(&full[s]);
-      issued = i + 1;
       cur.advance(cu, E, B, units_of(cu, E, cur.b));
     }
     cp_async_wait_all();   // every copy this lane issued has landed before the warp leaves
-    (void)issued;
     return;
   }
 

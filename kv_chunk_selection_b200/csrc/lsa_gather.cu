@@ -16,6 +16,12 @@
 // small grid over the device alias of page-locked host memory: SMs pull the
 // scattered chunks over the host link directly, on the caller's side stream,
 // without a host loop or a device-to-host copy of the kept list.
+//
+// Also here: the copies of the NEXT rows. lsa_fetch_from_host_delta reuses
+// chunks already resident from the previous window. lsa_append_token writes
+// a decoded token into a sequence's local chunk, and lsa_reset_local empties
+// the local chunks. lsa_gather_tokens packs the fine stage's selected tokens
+// into dense units.
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
