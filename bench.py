@@ -39,6 +39,7 @@ import re
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -100,7 +101,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # raw samples (the JSON line carries their summary); LSA_CLOCKS_DIR picks the folder
+        self.path = os.path.join(os.environ.get("LSA_CLOCKS_DIR") or tempfile.gettempdir(),
+                                 f"lsa_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
