@@ -405,18 +405,21 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   int krem = kc;
 
   // ---- radix select over the cluster ------------------------------------------
+  // Buffer 0 is cleared here; buffer (p + 1) & 1 right after pass p's cluster
+  // barrier, which orders every remote read of it (made in pass p - 1) first.
+  if (tid < 256) hist[0][tid] = 0;
+  __syncthreads();
   int pass = 0;
   while (hi_bit >= 0) {
     const int width = min(8, hi_bit + 1);
     const int shift = hi_bit - width + 1;
     const uint32_t dmask = (1u << width) - 1u;
     int* h = hist[pass & 1];
-    for (int i = tid; i < 256; i += kThreads) h[i] = 0;
-    __syncthreads();
 #pragma unroll
     for (int e = 0; e < kPer; ++e)
       if (e < n_own && (kr[e] & mask) == prefix) atomicAdd(&h[(kr[e] >> shift) & dmask], 1);
     cluster_sync_all();   // every rank's histogram of this pass is complete
+    if (tid < 256) hist[(pass + 1) & 1][tid] = 0;   // published by the block barriers below
     int count = 0, incl = 0;
     if (tid < 256) {
 #pragma unroll
@@ -456,9 +459,12 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
     n_less += (e < n_own && kr[e] < boundary);
     n_eq += (e < n_own && kr[e] == boundary);
   }
-  int cta_eq = 0, cta_less = 0;
-  const int eq_before = block_exclusive_scan(n_eq, warp_sums, &cta_eq);
-  block_exclusive_scan(n_less, warp_sums, &cta_less);
+  // one block scan for both counts: equal keys in the high half, smaller ones
+  // in the low half (at most 16 per thread and 8192 per CTA each)
+  int cta_both = 0;
+  const int both_before = block_exclusive_scan((n_eq << 16) | n_less, warp_sums, &cta_both);
+  const int eq_before = both_before >> 16;
+  const int cta_eq = cta_both >> 16, cta_less = cta_both & 0xffff;
   if (tid < kClusterCtas) {
     st_cluster_u32(cluster_map(&xcnt[rank], tid), static_cast<uint32_t>(cta_less));
     st_cluster_u32(cluster_map(&xcnt[kClusterCtas + rank], tid), static_cast<uint32_t>(cta_eq));

@@ -310,3 +310,62 @@ def test_selected_in_place_equals_packed_path():
     units_v = V.reshape(-1, 64, 8, 128).transpose(0, 2, 1, 3)
     ref = oracle.sparse_decode_attn(f64(q[b0: b0 + 1]), units_k, units_v, [0, units_k.shape[0]])
     assert_attention_close(out_b[b0: b0 + 1], ref)
+
+
+@pytest.mark.slow
+def test_fine_stage_500k_full_size():
+    """The token-level stage on the 500K workload as the bench runs it (52480 recalled
+    tokens, k = 2048, selected tokens read in place), at steps 0 and 63: token
+    scores for every recalled token, the selection, and attention on sampled heads."""
+    inp = workloads.make_inputs("500k", DEV, layers=1, windows=1)
+    L = inp.layers[0]
+    tok_keys, q_tok = workloads.fine_inputs(inp, 0, DEV, windows=1)
+    lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, DEV, fine_k=2048)
+    lw.select(L.q_idx[0], L.w, L.chunk_keys)
+    lw.gather(L.k_pool, L.v_pool)
+    kept = lw.kept_lists()
+    keys32 = tok_keys.float().cpu().numpy()          # exact for bf16 values
+    total = int(lw.cu_kept[0][-1])
+    kb, vb = lw.k_bufs[0][:total].float().cpu().numpy(), lw.v_bufs[0][:total].float().cpu().numpy()
+    heads = [0, 9, 18, 27, 36, 45, 54, 63]
+    for t in (0, 63):
+        out = torch.empty((1, 64, 128), device=DEV)
+        lw.fine_select(q_tok[0, t], L.w, tok_keys)
+        lw.attend(L.q[0, t], out)
+        torch.cuda.synchronize()
+        status_clean()
+        ref_scores = oracle.token_scores(f64(q_tok[0, t]), f64(L.w), keys32, i64(inp.chunk_table), kept,
+                                         inp.max_chunks)
+        n = len(ref_scores[0])
+        g = f64(lw.tok_scores)[0, :n]
+        err = np.abs(g - ref_scores[0])
+        assert np.all(err <= SCORE_RTOL * np.abs(ref_scores[0])), f"step {t}: token scores off"
+        got = kept_from_gpu(lw.sel, lw.n_sel)
+        assert_token_selection(got, [g], ref_scores, 2048)
+        ref = oracle.fine_decode_attn(f64(L.q[0, t]), kb, vb, i64(lw.cu_kept[0]), got, heads=heads)
+        assert_attention_close(out, ref, heads=heads)
+
+
+@pytest.mark.slow
+def test_causal_window_500k_sampled_steps():
+    """A causal 500K window as the bench runs it (the step's token appended and
+    attended in one launch), all 64 steps on the GPU, steps 0 and 63 against the
+    oracle on sampled heads: the kept chunks plus the first t + 1 decoded tokens."""
+    inp = workloads.make_inputs("500k", DEV, layers=1, windows=1)
+    L = inp.layers[0]
+    kn, vn = workloads.decoded_tokens(inp, 0, DEV, windows=1)
+    lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, DEV, causal=True)
+    outs = torch.empty((64, 1, 64, 128), device=DEV)
+    lw.run_window(L.q_idx[0], L.w, L.chunk_keys, L.k_pool, L.v_pool, L.q[0], outs, k_new=kn[0], v_new=vn[0])
+    torch.cuda.synchronize()
+    status_clean()
+    assert int(lw.local_len[0]) == 64
+    total = int(lw.cu_kept[0][-1])
+    kb, vb = lw.k_bufs[0][:total].float().cpu().numpy(), lw.v_bufs[0][:total].float().cpu().numpy()
+    kl, vl = f64(lw.k_local), f64(lw.v_local)
+    assert np.array_equal(kl[0].transpose(1, 0, 2), f64(kn[0, :, 0]))   # token t at row t of the local chunk
+    heads = [0, 9, 18, 27, 36, 45, 54, 63]
+    for t in (0, 63):
+        ref = oracle.sparse_decode_attn(f64(L.q[0, t]), kb, vb, i64(lw.cu_kept[0]), heads=heads, k_local=kl,
+                                        v_local=vl, local_len=[t + 1])
+        assert_attention_close(outs[t], ref, heads=heads)
