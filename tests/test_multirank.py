@@ -57,3 +57,22 @@ def test_single_rank_needs_no_process_group():
     import bench
     t, v = bench.combine_ranks(0.25, 100.0, 1)
     assert t == 0.25 and v == pytest.approx(400.0)
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """`bench.py --impl reference` launched the driver's way for N = 2: rank 0 alone
+    runs the oracle and prints one JSON line; the other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "0", "--gpus", "2"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle"
