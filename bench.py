@@ -703,7 +703,7 @@ def run_attn_only(args):
     B = len(kept)
     cu = torch.tensor([0] + list(torch.tensor(kept).cumsum(0).tolist()), dtype=torch.int32, device=dev)
     total = int(sum(kept))
-    shape = (total, 8, 64, 128)
+    shape = (8, total, 64, 128)   # head-major compact buffer
     kbuf = workloads.randn_bf16(shape, 1, dev)
     vbuf = workloads.randn_bf16(shape, 2, dev)
     qs = workloads.randn_bf16((workloads.TAU, B, 64, 128), 3, dev)

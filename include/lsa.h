@@ -32,8 +32,12 @@
  *    chunks, 16 indexer heads of dim 128.  bf16 is IEEE-style bfloat16 stored
  *    as 2 bytes; all bf16 arrays must be 16-byte aligned.
  *  - Layouts (row-major, last index fastest):
- *      KV pool / compact buffer : bf16 [slot][8 kv heads][64 tokens][128]
+ *      KV pool                  : bf16 [slot][8 kv heads][64 tokens][128]
  *                                 (LSA_CHUNK_BYTES bytes per slot, per K or V)
+ *      compact buffer           : bf16 [8 kv heads][buf_chunks][64 tokens][128]
+ *                                 (head-major: the kept chunks of one KV head
+ *                                 are contiguous, so the attention streams one
+ *                                 contiguous range per (sequence, head))
  *      indexer keys             : bf16 [slot][128]
  *      indexer query            : bf16 [B][16][128]
  *      decode query             : bf16 [B][64][128]
@@ -183,9 +187,9 @@ int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks, const flo
 /*
  * lsa_gather_chunks -- copy every kept chunk from the device KV pools into the
  * compact buffers, bit for bit: for i = cu_kept[b] + j,
- *   k_buf[i] = k_pool[slot(b, kept[b*max_kept + j])], same for V.
+ *   k_buf[g][i] = k_pool[slot(b, kept[b*max_kept + j])][g] for every KV head g, same for V.
  *   k_pool, v_pool device bf16 [n_slots][8][64][128]
- *   k_buf,  v_buf  device bf16 [buf_chunks][8][64][128]
+ *   k_buf,  v_buf  device bf16 [8][buf_chunks][64][128]
  * Device errors: CAPACITY (cu_kept[B] > buf_chunks: nothing is copied),
  * BAD_CHUNK / BAD_SLOT (that chunk is not copied).
  */
@@ -229,7 +233,7 @@ int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_
  * is identical to lsa_fetch_from_host.
  *   prev_kept, prev_cu_kept  device int32 [B][prev_max_kept], [B+1]: the
  *                            previous window's selection (ascending lists)
- *   prev_k_buf, prev_v_buf   device bf16 [prev_buf_chunks][8][64][128]: its
+ *   prev_k_buf, prev_v_buf   device bf16 [8][prev_buf_chunks][64][128]: its
  *                            compact buffers (must not be k_buf / v_buf)
  *   reused_chunks            optional device int32 counter, incremented once
  *                            per chunk copied from the previous buffers
@@ -266,7 +270,7 @@ size_t lsa_attn_workspace_size(int B);
  * merged with their log-sum-exp weights in a fixed order, so repeated calls
  * are bit-identical.
  *   q            device bf16 [B][64][128]
- *   k_buf, v_buf device bf16 [buf_chunks][8][64][128]
+ *   k_buf, v_buf device bf16 [8][buf_chunks][64][128]
  *   cu_kept      device int32 [B+1]
  *   softmax_scale  usually 1/sqrt(128)
  *   out          device fp32 [B][64][128]
@@ -369,7 +373,7 @@ int lsa_sparse_decode_attn_local(const void* q, const void* k_buf, const void* v
  * chunk cu_kept[b] + p / 64.  Equal to lsa_gather_tokens followed by
  * lsa_sparse_decode_attn over the packed units, bit for bit, without the
  * packed copy: the kernel copies the selected rows of k_buf / v_buf
- * (bf16 [buf_chunks][8][64][128]) straight into its pipeline.
+ * (bf16 [8][buf_chunks][64][128]) straight into its pipeline.
  *   sel device int32 [B][max_sel], max_sel a multiple of 64;
  *   cu_sel device int32 [B+1]; cu_kept device int32 [B+1]
  * LSA_ATTN_KV_UNCHANGED additionally promises that sel and cu_sel were not
@@ -455,12 +459,12 @@ int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int k, int B, 
 /*
  * lsa_gather_tokens -- pack the selected tokens into dense units, bit for bit:
  * for j < n_sel[b], with unit u = cu_sel[b]/64 + j/64 and row r = j % 64,
- *   k_out[u][g][r][:] = k_buf[cu_kept[b] + p/64][g][p % 64][:],  p = sel[b*max_sel + j],
+ *   k_out[g][u][r][:] = k_buf[g][cu_kept[b] + p/64][p % 64][:],  p = sel[b*max_sel + j],
  * for every KV head g, same for V; cu_units[b] = cu_sel[b] / 64.
- *   k_buf, v_buf  device bf16 [buf_chunks][8][64][128] (the compact buffer)
+ *   k_buf, v_buf  device bf16 [8][buf_chunks][64][128] (the compact buffer)
  *   cu_kept       device int32 [B+1]
  *   sel, cu_sel   from lsa_topk_tokens; max_sel a multiple of 64
- *   k_out, v_out  device bf16 [out_chunks][8][64][128]
+ *   k_out, v_out  device bf16 [8][out_chunks][64][128] (the compact buffer's layout)
  *   cu_units      device int32 [B+1]
  * Every count must be a multiple of 64 (k a multiple of 64 guarantees it).
  * Device errors: BAD_COUNT (a count that is not, or bad cu_kept: skipped),

@@ -109,6 +109,13 @@ def _need(t: torch.Tensor, name: str, dtype, cuda=True):
         raise ValueError(f"{name} must be a CUDA tensor")
 
 
+def _buf_chunks(t: torch.Tensor, name: str) -> int:
+    """Chunks of a compact buffer, laid out head-major as [8 KV heads, chunks, 64, 128]."""
+    if t.dim() != 4 or t.shape[0] != NUM_KV_HEADS or tuple(t.shape[2:]) != (CHUNK_TOKENS, HEAD_DIM):
+        raise ValueError(f"{name} must be a compact buffer [8, chunks, 64, 128], got {tuple(t.shape)}")
+    return int(t.shape[1])
+
+
 def _check(fn: str, st: int):
     if st != 0:
         raise LsaError(fn, st)
@@ -196,7 +203,7 @@ def lsa_gather_chunks(k_pool, v_pool, chunk_table, kept, cu_kept, max_chunks, k_
     B, max_kept = kept.shape
     _check("lsa_gather_chunks", _load().lsa_gather_chunks(
         _ptr(k_pool), _ptr(v_pool), k_pool.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(cu_kept), B,
-        int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _stream(stream)))
+        int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _stream(stream)))
 
 
 def lsa_fetch_from_host(host_k_pool, host_v_pool, chunk_table, kept, cu_kept, max_chunks, k_buf, v_buf,
@@ -219,7 +226,7 @@ def lsa_fetch_from_host(host_k_pool, host_v_pool, chunk_table, kept, cu_kept, ma
         ev = ctypes.c_void_p(done_event.cuda_event)
     _check("lsa_fetch_from_host", _load().lsa_fetch_from_host(
         _ptr(host_k_pool), _ptr(host_v_pool), host_k_pool.shape[0], _ptr(chunk_table), _ptr(kept),
-        _ptr(cu_kept), B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], int(num_ctas),
+        _ptr(cu_kept), B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), int(num_ctas),
         _stream(stream), ev))
 
 
@@ -245,8 +252,8 @@ def lsa_fetch_from_host_delta(host_k_pool, host_v_pool, chunk_table, kept, cu_ke
         ev = ctypes.c_void_p(done_event.cuda_event)
     _check("lsa_fetch_from_host_delta", _load().lsa_fetch_from_host_delta(
         _ptr(host_k_pool), _ptr(host_v_pool), host_k_pool.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(cu_kept),
-        B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(prev_kept),
-        _ptr(prev_cu_kept), prev_kept.shape[1], _ptr(prev_k_buf), _ptr(prev_v_buf), prev_k_buf.shape[0],
+        B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(prev_kept),
+        _ptr(prev_cu_kept), prev_kept.shape[1], _ptr(prev_k_buf), _ptr(prev_v_buf), _buf_chunks(prev_k_buf, "prev_k_buf"),
         _ptr(reused_chunks), int(num_ctas), _stream(stream), ev))
 
 
@@ -285,7 +292,7 @@ def lsa_sparse_decode_attn(q, k_buf, v_buf, cu_kept, out, workspace, softmax_sca
         raise ValueError("bad shapes")
     scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
     _check("lsa_sparse_decode_attn", _load().lsa_sparse_decode_attn(
-        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(out),
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(cu_kept), B, scale, _ptr(out),
         _ptr(workspace), workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
 
 
@@ -325,7 +332,7 @@ def lsa_sparse_decode_attn_local(q, k_buf, v_buf, cu_kept, k_local, v_local, loc
         raise ValueError("k_local and v_local must be [B, 8, 64, 128]")
     scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
     _check("lsa_sparse_decode_attn_local", _load().lsa_sparse_decode_attn_local(
-        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(k_local),
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(cu_kept), B, scale, _ptr(k_local),
         _ptr(v_local), _ptr(local_len), _ptr(out), _ptr(workspace), workspace.numel(),
         ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
 
@@ -370,8 +377,8 @@ def lsa_gather_tokens(k_buf, v_buf, cu_kept, sel, cu_sel, k_out, v_out, cu_units
         _need(t, n, torch.int32)
     B, max_sel = sel.shape
     _check("lsa_gather_tokens", _load().lsa_gather_tokens(
-        _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), _ptr(sel), _ptr(cu_sel), B, max_sel,
-        _ptr(k_out), _ptr(v_out), k_out.shape[0], _ptr(cu_units), _stream(stream)))
+        _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(cu_kept), _ptr(sel), _ptr(cu_sel), B, max_sel,
+        _ptr(k_out), _ptr(v_out), _buf_chunks(k_out, "k_out"), _ptr(cu_units), _stream(stream)))
 
 
 def lsa_sparse_decode_attn_selected(q, k_buf, v_buf, cu_kept, sel, cu_sel, out, workspace, softmax_scale=None,
@@ -392,7 +399,7 @@ def lsa_sparse_decode_attn_selected(q, k_buf, v_buf, cu_kept, sel, cu_sel, out, 
         raise ValueError("sel must be [B, max_sel]")
     scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
     _check("lsa_sparse_decode_attn_selected", _load().lsa_sparse_decode_attn_selected(
-        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), _ptr(sel), _ptr(cu_sel), sel.shape[1], B,
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(cu_kept), _ptr(sel), _ptr(cu_sel), sel.shape[1], B,
         scale, _ptr(out), _ptr(workspace), workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0,
         _stream(stream)))
 
@@ -420,7 +427,7 @@ def lsa_sparse_decode_attn_append(q, k_buf, v_buf, cu_kept, k_new, v_new, k_loca
         raise ValueError("k_new and v_new must be [B, 8, 128]")
     scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
     _check("lsa_sparse_decode_attn_append", _load().lsa_sparse_decode_attn_append(
-        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(k_new), _ptr(v_new),
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(cu_kept), B, scale, _ptr(k_new), _ptr(v_new),
         _ptr(k_local), _ptr(v_local), _ptr(local_len_in), _ptr(local_len_out), _ptr(out), _ptr(workspace),
         workspace.numel(), ATTN_KV_UNCHANGED if kv_unchanged else 0, _stream(stream)))
 
@@ -442,7 +449,7 @@ def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=
         raise ValueError("bad shapes")
     scale = 1.0 / math.sqrt(HEAD_DIM) if softmax_scale is None else float(softmax_scale)
     _check("lsa_sparse_decode_attn_noalloc", _load().lsa_sparse_decode_attn_noalloc(
-        _ptr(q), _ptr(k_buf), _ptr(v_buf), k_buf.shape[0], _ptr(cu_kept), B, scale, _ptr(out), _stream(stream)))
+        _ptr(q), _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(cu_kept), B, scale, _ptr(out), _stream(stream)))
 
 
 __all__ = [

@@ -293,7 +293,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         const int p = __ldg(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + r);
         const bool okp = p >= 0 && p < n_pos && ckb + p / kChunkTokens < sa.ck_chunks;
         if (!okp) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
-        const int64_t row = okp ? ((ckb + p / kChunkTokens) * kNumKVHeads + g) * kChunkTokens + p % kChunkTokens : 0;
+        const int64_t row = okp ? (g * sa.ck_chunks + ckb + p / kChunkTokens) * kChunkTokens + p % kChunkTokens : 0;
         const uint4* ks = sa.k_buf + row * 16;
         const uint4* vs = sa.v_buf + row * 16;
         const uint32_t nb = okp ? 16u : 0u;
@@ -340,8 +340,9 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           griddep_wait();
           waited = true;
         }
+        // compact buffer: head-major rows (g, chunk, token); local chunks: (b, g, token)
         const int row = local ? (cur.b * kNumKVHeads + cur.g) * kChunkTokens
-                              : ((cb + cur.j) * kNumKVHeads + cur.g) * kChunkTokens;
+                              : (cur.g * static_cast<int>(buf_chunks) + cb + cur.j) * kChunkTokens;
         const CUtensorMap* mk = local ? &tm_kl : &tm_k;
         const CUtensorMap* mv = local ? &tm_vl : &tm_v;
         mbar_arrive_expect_tx(&full[s], kStageBytes);

@@ -108,12 +108,12 @@ gather_kernel(const uint4* __restrict__ k_pool, const uint4* __restrict__ v_pool
       if (pb >= 0 && pn > 0 && pn <= prev.max_kept && static_cast<int64_t>(pb) + pn <= prev.buf_chunks) {
         const int jp = find_sorted(prev.kept + static_cast<int64_t>(b) * prev.max_kept, pn, c);
         if (jp >= 0) {
-          src = (kv ? prev.v_buf : prev.k_buf) + (static_cast<int64_t>(pb) + jp) * tile + h * kVecPerTile;
+          src = (kv ? prev.v_buf : prev.k_buf) + (h * prev.buf_chunks + pb + jp) * kVecPerTile;
           if (prev.reused && kv == 0 && h == 0 && threadIdx.x == 0) atomicAdd(prev.reused, 1);
         }
       }
     }
-    uint4* dst = (kv ? v_buf : k_buf) + static_cast<int64_t>(i) * tile + h * kVecPerTile;
+    uint4* dst = (kv ? v_buf : k_buf) + (h * buf_chunks + i) * kVecPerTile;   // head-major compact buffer
     uint4 r[kVecPerThread];
 #pragma unroll
     for (int v = 0; v < kVecPerThread; ++v) r[v] = __ldcs(src + v * kThreads + threadIdx.x);
@@ -202,7 +202,7 @@ gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ 
     ok[e] = p >= 0 && p < n_pos;
     v[e] = make_uint4(0, 0, 0, 0);
     if (ok[e]) {
-      const int64_t src = ((c0 + p / kChunkTokens) * kNumKVHeads + g) * kChunkTokens + p % kChunkTokens;
+      const int64_t src = (g * buf_chunks + c0 + p / kChunkTokens) * kChunkTokens + p % kChunkTokens;
       v[e] = __ldg((kv ? v_buf : k_buf) + src * kRowVecs + x);
     }
   }
@@ -211,7 +211,7 @@ gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ 
     const int idx = tid + e * kTokThreads;
     const int kv = idx / (kChunkTokens * kRowVecs), rem = idx % (kChunkTokens * kRowVecs);
     const int r = rem / kRowVecs, x = rem % kRowVecs;
-    const int64_t dst = (ou * kNumKVHeads + g) * kChunkTokens + r;
+    const int64_t dst = (g * out_chunks + ou) * kChunkTokens + r;
     (kv ? v_out : k_out)[dst * kRowVecs + x] = v[e];
     if (!ok[e] && x == 0) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
   }

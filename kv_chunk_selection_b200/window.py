@@ -78,7 +78,7 @@ class LayerWindow:
             self.max_kept = int(max_chunks)
             self.buf_chunks = int(n_host.sum())
         nbuf = 2 if double_buffer else 1
-        shape = (self.buf_chunks, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM)
+        shape = (NUM_KV_HEADS, self.buf_chunks, CHUNK_TOKENS, HEAD_DIM)   # head-major compact buffer
         self.k_bufs = [torch.empty(shape, dtype=torch.bfloat16, device=self.device) for _ in range(nbuf)]
         self.v_bufs = [torch.empty(shape, dtype=torch.bfloat16, device=self.device) for _ in range(nbuf)]
         self.scores = torch.empty((self.B, self.max_chunks), dtype=torch.float32, device=self.device)
@@ -107,7 +107,7 @@ class LayerWindow:
             self.packs = self.causal   # the causal step reads packed units
             if self.packs:
                 units = self.B * self.fine_k // CHUNK_TOKENS
-                self.k_fine = torch.empty((units, NUM_KV_HEADS, CHUNK_TOKENS, HEAD_DIM), dtype=torch.bfloat16,
+                self.k_fine = torch.empty((NUM_KV_HEADS, units, CHUNK_TOKENS, HEAD_DIM), dtype=torch.bfloat16,
                                           device=dev)
                 self.v_fine = torch.empty_like(self.k_fine)
                 self.cu_units = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)

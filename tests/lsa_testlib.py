@@ -23,6 +23,15 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
+def cm(t: torch.Tensor) -> torch.Tensor:
+    """Chunk-major view [chunks, 8, 64, 128] of a head-major compact buffer [8, chunks, 64, 128].
+
+    The kernels keep compact buffers head-major; the oracle and the tests index them chunk first.
+    The permutation is its own inverse, so cm() also turns a chunk-major view back into the
+    head-major storage the kernels take."""
+    return t.permute(1, 0, 2, 3)
+
+
 def i64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.int64).numpy()
 

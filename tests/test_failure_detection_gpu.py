@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import kv_chunk_selection_b200 as lsa
-from lsa_testlib import assert_attention_close, f64
+from lsa_testlib import assert_attention_close, cm, f64
 import oracle
 
 pytestmark = pytest.mark.gpu
@@ -53,7 +53,7 @@ def test_context_usable_after_timeouts():
     n_kept = [3, 40]
     total = sum(n_kept)
     g = torch.Generator(device="cuda").manual_seed(1)
-    kb = torch.randn((total, 8, 64, 128), generator=g, device="cuda").to(torch.bfloat16)
+    kb = torch.randn((8, total, 64, 128), generator=g, device="cuda").to(torch.bfloat16)
     vb = torch.randn_like(kb, dtype=torch.float32).to(torch.bfloat16)
     cu = torch.tensor([0, 3, total], dtype=torch.int32, device="cuda")
     q = torch.randn((2, 64, 128), generator=g, device="cuda").to(torch.bfloat16)
@@ -61,7 +61,7 @@ def test_context_usable_after_timeouts():
     lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out, lsa.new_attn_workspace(2))
     torch.cuda.synchronize()
     assert lsa.read_device_status() == 0
-    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), cu.cpu().numpy())
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), cu.cpu().numpy())
     assert_attention_close(out, ref)
 
 

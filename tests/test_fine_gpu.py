@@ -18,7 +18,7 @@ import kv_chunk_selection_b200 as lsa
 import oracle
 import workloads
 from kv_chunk_selection_b200.window import LayerWindow
-from lsa_testlib import SCORE_RTOL, TIE_RTOL, assert_attention_close, f64, i64, kept_from_gpu
+from lsa_testlib import SCORE_RTOL, TIE_RTOL, assert_attention_close, cm, f64, i64, kept_from_gpu
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -151,7 +151,7 @@ def test_gather_tokens_bit_exact():
     k = 1024
     sel, n_sel, cu_sel = topk_tokens_gpu(scores, n_tok, k)
     units = lw.B * k // 64
-    k_out = torch.zeros((units, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    k_out = torch.zeros((8, units, 64, 128), dtype=torch.bfloat16, device=DEV)
     v_out = torch.zeros_like(k_out)
     cu_units = torch.full((lw.B + 1,), -1, dtype=torch.int32, device=DEV)
     lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], sel, cu_sel, k_out, v_out, cu_units)
@@ -164,12 +164,12 @@ def test_gather_tokens_bit_exact():
         p = torch.tensor(got[b], device=DEV, dtype=torch.int64)
         chunk = int(ck[b]) + p // 64
         row = p % 64
-        want_k = lw.k_bufs[0][chunk, :, row]                       # [n, 8, 128]
-        want_v = lw.v_bufs[0][chunk, :, row]
+        want_k = cm(lw.k_bufs[0])[chunk, :, row]                   # [n, 8, 128]
+        want_v = cm(lw.v_bufs[0])[chunk, :, row]
         u0 = int(cs[b]) // 64
         n = len(got[b])
-        have_k = k_out[u0: u0 + n // 64].permute(0, 2, 1, 3).reshape(n, 8, 128)
-        have_v = v_out[u0: u0 + n // 64].permute(0, 2, 1, 3).reshape(n, 8, 128)
+        have_k = cm(k_out)[u0: u0 + n // 64].permute(0, 2, 1, 3).reshape(n, 8, 128)
+        have_v = cm(v_out)[u0: u0 + n // 64].permute(0, 2, 1, 3).reshape(n, 8, 128)
         assert torch.equal(have_k, want_k) and torch.equal(have_v, want_v), f"seq {b}"
 
 
@@ -188,7 +188,7 @@ def test_fine_step_attention_matches_oracle(name, kw, k):
     status_clean()
     sel = kept_from_gpu(lw.sel, lw.n_sel)
     heads = None if lw.B == 1 else [0, 9, 18, 27, 36, 45, 54, 63]
-    ref = oracle.fine_decode_attn(f64(L.q[0, 7]), f64(lw.k_bufs[0]), f64(lw.v_bufs[0]), i64(lw.cu_kept[0]), sel,
+    ref = oracle.fine_decode_attn(f64(L.q[0, 7]), f64(cm(lw.k_bufs[0])), f64(cm(lw.v_bufs[0])), i64(lw.cu_kept[0]), sel,
                                   heads=heads)
     assert_attention_close(out, ref, heads=heads)
 
@@ -221,10 +221,10 @@ def test_fine_stage_short_and_empty_sequences():
     assert i64(lw.n_sel).tolist() == [0, 192, 256]
     sel = kept_from_gpu(lw.sel, lw.n_sel)
     assert sel[1] == list(range(192))
-    ref = oracle.fine_decode_attn(f64(q), f64(lw.k_bufs[0]), f64(lw.v_bufs[0]), i64(lw.cu_kept[0]), sel)
+    ref = oracle.fine_decode_attn(f64(q), f64(cm(lw.k_bufs[0])), f64(cm(lw.v_bufs[0])), i64(lw.cu_kept[0]), sel)
     assert_attention_close(out, ref)
     assert torch.all(out[0] == 0)
-    chunk_ref = oracle.sparse_decode_attn(f64(q), f64(lw.k_bufs[0]), f64(lw.v_bufs[0]), i64(lw.cu_kept[0]),
+    chunk_ref = oracle.sparse_decode_attn(f64(q), f64(cm(lw.k_bufs[0])), f64(cm(lw.v_bufs[0])), i64(lw.cu_kept[0]),
                                           seqs=[1])
     assert_attention_close(out[1:2], chunk_ref[1:2])
 
@@ -250,7 +250,7 @@ def test_window_tiny_fine_and_causal():
     torch.cuda.synchronize()
     status_clean()
     kept = lw.kept_lists()
-    kb, vb, cu = f64(lw.k_bufs[0]), f64(lw.v_bufs[0]), i64(lw.cu_kept[0])
+    kb, vb, cu = f64(cm(lw.k_bufs[0])), f64(cm(lw.v_bufs[0])), i64(lw.cu_kept[0])
     k_loc, v_loc = f64(lw.k_local), f64(lw.v_local)
     for t in range(64):
         ref_scores = oracle.token_scores(f64(q_tok[0, t]), f64(L.w), f64(tok_keys), i64(inp.chunk_table), kept,
@@ -277,7 +277,7 @@ def test_selected_in_place_equals_packed_path():
     sel, n_sel, cu_sel = topk_tokens_gpu(scores, n_tok, k)
     B = lw.B
     units = B * k // 64
-    k_out = torch.zeros((units, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    k_out = torch.zeros((8, units, 64, 128), dtype=torch.bfloat16, device=DEV)
     v_out = torch.zeros_like(k_out)
     cu_units = torch.zeros((B + 1,), dtype=torch.int32, device=DEV)
     lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], sel, cu_sel, k_out, v_out, cu_units)
@@ -302,8 +302,8 @@ def test_selected_in_place_equals_packed_path():
     cs, ck = i64(cu_sel), i64(lw.cu_kept[0])
     n = int(cs[b0 + 1] - cs[b0])
     p = sel[b0, :n].to(torch.int64)
-    K = f64(lw.k_bufs[0][int(ck[b0]) + p // 64, :, p % 64])    # [n, 8, 128], gathered on the GPU
-    V = f64(lw.v_bufs[0][int(ck[b0]) + p // 64, :, p % 64])
+    K = f64(cm(lw.k_bufs[0])[int(ck[b0]) + p // 64, :, p % 64])    # [n, 8, 128], gathered on the GPU
+    V = f64(cm(lw.v_bufs[0])[int(ck[b0]) + p // 64, :, p % 64])
     K[5] = 0.0
     V[5] = 0.0
     units_k = K.reshape(-1, 64, 8, 128).transpose(0, 2, 1, 3)
@@ -326,7 +326,7 @@ def test_fine_stage_500k_full_size():
     kept = lw.kept_lists()
     keys32 = tok_keys.float().cpu().numpy()          # exact for bf16 values
     total = int(lw.cu_kept[0][-1])
-    kb, vb = lw.k_bufs[0][:total].float().cpu().numpy(), lw.v_bufs[0][:total].float().cpu().numpy()
+    kb, vb = cm(lw.k_bufs[0])[:total].float().cpu().numpy(), cm(lw.v_bufs[0])[:total].float().cpu().numpy()
     heads = [0, 9, 18, 27, 36, 45, 54, 63]
     for t in (0, 63):
         out = torch.empty((1, 64, 128), device=DEV)
@@ -361,7 +361,7 @@ def test_causal_window_500k_sampled_steps():
     status_clean()
     assert int(lw.local_len[0]) == 64
     total = int(lw.cu_kept[0][-1])
-    kb, vb = lw.k_bufs[0][:total].float().cpu().numpy(), lw.v_bufs[0][:total].float().cpu().numpy()
+    kb, vb = cm(lw.k_bufs[0])[:total].float().cpu().numpy(), cm(lw.v_bufs[0])[:total].float().cpu().numpy()
     kl, vl = f64(lw.k_local), f64(lw.v_local)
     assert np.array_equal(kl[0].transpose(1, 0, 2), f64(kn[0, :, 0]))   # token t at row t of the local chunk
     heads = [0, 9, 18, 27, 36, 45, 54, 63]

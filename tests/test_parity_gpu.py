@@ -16,7 +16,7 @@ import kv_chunk_selection_b200 as lsa
 import oracle
 import workloads
 from kv_chunk_selection_b200.window import LayerWindow
-from lsa_testlib import (assert_attention_close, assert_kept_matches, assert_scores_close, f64, i64,
+from lsa_testlib import (assert_attention_close, assert_kept_matches, assert_scores_close, cm, f64, i64,
                          kept_from_gpu)
 
 pytestmark = pytest.mark.gpu
@@ -202,7 +202,7 @@ def test_threshold_window_attention():
     g = score_on_gpu(inp)
     kept, n_kept, cu = run_threshold(g, inp.n_chunks, L.w, 0.6, inp.max_chunks)
     total = int(cu[-1])
-    kb = torch.empty((total, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    kb = torch.empty((8, total, 64, 128), dtype=torch.bfloat16, device=DEV)
     vb = torch.empty_like(kb)
     lsa.lsa_gather_chunks(L.k_pool, L.v_pool, inp.chunk_table, kept, cu, inp.max_chunks, kb, vb)
     out = torch.empty((1, 64, 128), device=DEV)
@@ -210,8 +210,8 @@ def test_threshold_window_attention():
     lsa.lsa_sparse_decode_attn(L.q[0, 1], kb, vb, cu, out, ws)
     got = kept_from_gpu(kept, n_kept)
     assert_threshold_matches(got, f64(g), i64(inp.n_chunks), f64(L.w), 0.6)
-    assert torch.equal(kb, L.k_pool[torch.tensor(got[0], device=DEV)])
-    ref = oracle.sparse_decode_attn(f64(L.q[0, 1]), f64(kb), f64(vb), i64(cu))
+    assert torch.equal(cm(kb), L.k_pool[torch.tensor(got[0], device=DEV)])
+    ref = oracle.sparse_decode_attn(f64(L.q[0, 1]), f64(cm(kb)), f64(cm(vb)), i64(cu))
     assert_attention_close(out, ref)
     status_clean()
 
@@ -246,15 +246,15 @@ def test_gather_paged_bit_exact():
     tab = torch.from_numpy(table).to(DEV)
     kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
     buf_chunks = int((k + 1).sum())
-    kb = torch.zeros((buf_chunks,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    kb = torch.zeros((8, buf_chunks, 64, 128), dtype=torch.bfloat16, device=DEV)
     vb = torch.zeros_like(kb)
     lsa.lsa_gather_chunks(k_pool, v_pool, tab, kept, cu, M, kb, vb)
     kept_l = kept_from_gpu(kept, n_kept)
     rk, rv, rcu = oracle.gather_chunks(k_pool.view(torch.int16).cpu().numpy(), v_pool.view(torch.int16).cpu().numpy(),
                                        table, kept_l, M)
     total = int(rcu[-1])
-    assert np.array_equal(kb[:total].view(torch.int16).cpu().numpy(), rk)
-    assert np.array_equal(vb[:total].view(torch.int16).cpu().numpy(), rv)
+    assert np.array_equal(cm(kb)[:total].view(torch.int16).cpu().numpy(), rk)
+    assert np.array_equal(cm(vb)[:total].view(torch.int16).cpu().numpy(), rv)
     status_clean()
 
 
@@ -263,7 +263,7 @@ def test_gather_paged_bit_exact():
 def ragged_buffers(n_kept, seed=21):
     g = torch.Generator(device=DEV).manual_seed(seed)
     total = int(sum(n_kept))
-    shape = (max(total, 1), 8, 64, 128)
+    shape = (8, max(total, 1), 64, 128)   # head-major compact buffer
     kb = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
     vb = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
     cu = torch.tensor(np.concatenate([[0], np.cumsum(n_kept)]), dtype=torch.int32, device=DEV)
@@ -284,7 +284,7 @@ def run_attn(q, kb, vb, cu):
 def test_attention_ragged_matches_oracle(n_kept):
     q, kb, vb, cu = ragged_buffers(n_kept)
     out, _ = run_attn(q, kb, vb, cu)
-    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu))
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), i64(cu))
     assert_attention_close(out, ref)
     status_clean()
 
@@ -300,7 +300,7 @@ def test_attention_local_tokens_match_oracle(n_kept, local_len):
     ll = torch.tensor(local_len, dtype=torch.int32, device=DEV)
     out = torch.full((B, 64, 128), float("nan"), device=DEV)
     lsa.lsa_sparse_decode_attn_local(q, kb, vb, cu, kl, vl, ll, out, lsa.new_attn_workspace(B))
-    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), k_local=f64(kl), v_local=f64(vl),
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), i64(cu), k_local=f64(kl), v_local=f64(vl),
                                     local_len=local_len)
     assert_attention_close(out, ref)
     status_clean()
@@ -332,7 +332,7 @@ def test_append_then_attend_is_causal():
         vloc = np.zeros((B, 8, 64, 128))
         kloc[:, :, : t + 1] = f64(k_new[: t + 1]).transpose(1, 2, 0, 3)
         vloc[:, :, : t + 1] = f64(v_new[: t + 1]).transpose(1, 2, 0, 3)
-        ref = oracle.sparse_decode_attn(f64(qs[t]), f64(kb), f64(vb), i64(cu), k_local=kloc, v_local=vloc,
+        ref = oracle.sparse_decode_attn(f64(qs[t]), f64(cm(kb)), f64(cm(vb)), i64(cu), k_local=kloc, v_local=vloc,
                                         local_len=[t + 1] * B)
         assert_attention_close(outs[t], ref)
     status_clean()
@@ -371,7 +371,7 @@ def test_fused_append_step_matches_two_launch_path_and_oracle():
     mask[torch.arange(B), torch.tensor(n_loc)] = False
     assert torch.equal(kl_f.permute(0, 2, 1, 3)[mask], kl.permute(0, 2, 1, 3)[mask])
     assert torch.equal(out_f, out_t)
-    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), k_local=f64(kl_t), v_local=f64(vl_t),
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), i64(cu), k_local=f64(kl_t), v_local=f64(vl_t),
                                     local_len=[n + 1 for n in n_loc])
     assert_attention_close(out_f, ref)
 
@@ -391,7 +391,7 @@ def test_fused_append_full_local_chunk_reports_capacity():
     torch.cuda.synchronize()
     assert lsa.read_device_status() & 8          # CAPACITY
     assert len_out.tolist() == [64] and torch.equal(kl, before)
-    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), k_local=f64(kl), v_local=f64(vl),
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), i64(cu), k_local=f64(kl), v_local=f64(vl),
                                     local_len=[64])
     assert_attention_close(out, ref)
 
@@ -464,13 +464,13 @@ def test_max_batch_window_step():
     assert cu.tolist() == oracle.cumulative_kept(ref).tolist()
     for b in (1, 2, 4095, int(np.argmax(n))):
         for j, c in enumerate(got[b]):
-            assert torch.equal(lw.k_bufs[0][cu[b] + j], k_pool[int(table[b, c])])
+            assert torch.equal(cm(lw.k_bufs[0])[cu[b] + j], k_pool[int(table[b, c])])
     empty = [b for b in range(B) if n[b] == 0]
     assert torch.all(out[empty] == 0)
     seqs = sorted(set(rng.choice(B, 48, replace=False).tolist()) | {1, 2, 4095})
     for b in seqs:   # one sequence at a time: only its own kept chunks go to the host
         lo, hi = int(cu[b]), int(cu[b + 1])
-        ref_o = oracle.sparse_decode_attn(f64(q[b: b + 1]), f64(lw.k_bufs[0][lo:hi]), f64(lw.v_bufs[0][lo:hi]),
+        ref_o = oracle.sparse_decode_attn(f64(q[b: b + 1]), f64(cm(lw.k_bufs[0])[lo:hi]), f64(cm(lw.v_bufs[0])[lo:hi]),
                                           [0, hi - lo])
         assert_attention_close(out[b: b + 1], ref_o)
 
@@ -511,12 +511,12 @@ def test_attention_closed_forms():
     c = i64(cu)
     for b in range(2):
         for h in (0, 13, 63):
-            mean = f64(vb[c[b]: c[b + 1], h // 8]).reshape(-1, 128).mean(axis=0)
+            mean = f64(cm(vb)[c[b]: c[b + 1], h // 8]).reshape(-1, 128).mean(axis=0)
             np.testing.assert_allclose(o[b, h], mean, atol=2e-3, rtol=1e-3)
     # GQA mapping: V of KV head g is the constant g + 1
     q, kb, vb, cu = ragged_buffers(n_kept, seed=5)
     for g in range(8):
-        vb[:, g] = g + 1.0
+        vb[g] = g + 1.0                       # head-major: KV head g first
     out, _ = run_attn(q, kb, vb, cu)
     o = f64(out)
     for h in range(64):
@@ -549,7 +549,7 @@ def test_attention_overlapped_steps_match():
     scores = torch.rand((B, M), generator=g, device=DEV)
     kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
     buf = int((k + 1).sum())
-    kb = torch.empty((buf,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    kb = torch.empty((8, buf, 64, 128), dtype=torch.bfloat16, device=DEV)
     vb = torch.empty_like(kb)
     qs = torch.randn((6, B, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
     ws = lsa.new_attn_workspace(B)
@@ -566,7 +566,7 @@ def test_attention_overlapped_steps_match():
         lsa.lsa_sparse_decode_attn(qs[t], kb, vb, cu, got[t], ws, kv_unchanged=t > 0)
     torch.cuda.synchronize()
     assert torch.equal(ref, got)
-    o = oracle.sparse_decode_attn(f64(qs[3]), f64(kb), f64(vb), i64(cu))
+    o = oracle.sparse_decode_attn(f64(qs[3]), f64(cm(kb)), f64(cm(vb)), i64(cu))
     assert_attention_close(got[3], o)
     status_clean()
 
@@ -576,7 +576,7 @@ def test_attention_scale_argument():
     out = torch.empty((1, 64, 128), device=DEV)
     ws = lsa.new_attn_workspace(1)
     lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out, ws, softmax_scale=0.3)
-    ref = oracle.sparse_decode_attn(f64(q), f64(kb), f64(vb), i64(cu), scale=0.3)
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), i64(cu), scale=0.3)
     assert_attention_close(out, ref)
 
 
@@ -614,10 +614,10 @@ def window_parity(name, steps, layer=0, window=0, heads=None, seqs=None, **kw):
     # gather: every kept chunk equals its pool slot, bit for bit
     table = i64(inp.chunk_table)
     idx = torch.tensor([int(table[b, c]) for b in range(inp.batch) for c in got[b]], device=L.k_pool.device)
-    assert torch.equal(lw.k_bufs[0][:total], L.k_pool[idx].to(DEV))
-    assert torch.equal(lw.v_bufs[0][:total], L.v_pool[idx].to(DEV))
+    assert torch.equal(cm(lw.k_bufs[0])[:total], L.k_pool[idx].to(DEV))
+    assert torch.equal(cm(lw.v_bufs[0])[:total], L.v_pool[idx].to(DEV))
     # attention at the sampled steps: the oracle on the kept set the GPU chose
-    kb, vb = f32(lw.k_bufs[0][:total]), f32(lw.v_bufs[0][:total])
+    kb, vb = f32(cm(lw.k_bufs[0])[:total]), f32(cm(lw.v_bufs[0])[:total])
     errs = []
     for t in steps:
         ref = oracle.sparse_decode_attn(f64(L.q[window, t]), kb, vb, cu, heads=heads, seqs=seqs)
@@ -720,7 +720,7 @@ def test_fetch_from_host_equals_gather():
     n_t, k_t, tab = (torch.from_numpy(x).to(DEV) for x in (n, k, table))
     kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
     buf = int((k + 1).sum())
-    a_k = torch.zeros((buf,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    a_k = torch.zeros((8, buf, 64, 128), dtype=torch.bfloat16, device=DEV)
     a_v, b_k, b_v = torch.zeros_like(a_k), torch.zeros_like(a_k), torch.zeros_like(a_k)
     lsa.lsa_gather_chunks(k_dev, v_dev, tab, kept, cu, M, a_k, a_v)
     side = torch.cuda.Stream()
@@ -749,7 +749,7 @@ def test_fetch_delta_reuses_previous_window():
     ka, na, cua = run_topk(s_a, n_t, k_t, int(k.max()) + 1)
     kb_, nb, cub = run_topk(s_b, n_t, k_t, int(k.max()) + 1)
     buf = int((k + 1).sum())
-    ak = torch.zeros((buf,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    ak = torch.zeros((8, buf, 64, 128), dtype=torch.bfloat16, device=DEV)
     av = torch.zeros_like(ak)
     lsa.lsa_fetch_from_host(k_host, v_host, tab, ka, cua, M, ak, av)                 # window A
     bk, bv, rk, rv = (torch.zeros_like(ak) for _ in range(4))
@@ -768,7 +768,7 @@ def test_fetch_rejects_unpinned_pool():
     k_host = torch.zeros((4, 8, 64, 128), dtype=torch.bfloat16)     # pageable
     kept = torch.zeros((1, 2), dtype=torch.int32, device=DEV)
     cu = torch.tensor([0, 1], dtype=torch.int32, device=DEV)
-    buf = torch.zeros((2, 8, 64, 128), dtype=torch.bfloat16, device=DEV)
+    buf = torch.zeros((8, 2, 64, 128), dtype=torch.bfloat16, device=DEV)
     with pytest.raises(lsa.LsaError, match="NOT_PINNED"):
         lsa.lsa_fetch_from_host(k_host, k_host, None, kept, cu, 4, buf, buf)
 
@@ -778,7 +778,7 @@ def test_fetch_rejects_unpinned_pool():
 def test_device_errors_are_reported_not_trapped():
     shape = (4, 8, 64, 128)
     pool = torch.zeros(shape, dtype=torch.bfloat16, device=DEV)
-    buf = torch.zeros((2,) + shape[1:], dtype=torch.bfloat16, device=DEV)
+    buf = torch.zeros((8, 2, 64, 128), dtype=torch.bfloat16, device=DEV)
     kept = torch.tensor([[0, 9]], dtype=torch.int32, device=DEV)      # 9 >= max_chunks (4)
     cu = torch.tensor([0, 2], dtype=torch.int32, device=DEV)
     lsa.lsa_gather_chunks(pool, pool, None, kept, cu, 4, buf, buf)

@@ -41,7 +41,7 @@ def _p(t):
 def _inputs(n_kept, seed):
     g = torch.Generator(device=DEV).manual_seed(seed)
     total = int(sum(n_kept))
-    shape = (total, 8, 64, 128)
+    shape = (8, total, 64, 128)            # head-major compact buffer
     kb = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
     vb = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
     cu = torch.tensor(np.concatenate([[0], np.cumsum(n_kept)]), dtype=torch.int32, device=DEV)
@@ -60,12 +60,12 @@ def test_noalloc_matches_workspace_entry_point_twice(L):
 
     ref = torch.empty((B, 64, 128), device=DEV)
     ws = torch.zeros(L.lsa_attn_workspace_size(B), dtype=torch.uint8, device=DEV)
-    assert L.lsa_sparse_decode_attn(_p(q), _p(kb), _p(vb), kb.shape[0], _p(cu), B, scale, _p(ref), _p(ws),
+    assert L.lsa_sparse_decode_attn(_p(q), _p(kb), _p(vb), kb.shape[1], _p(cu), B, scale, _p(ref), _p(ws),
                                     ws.numel(), 0, stream) == 0
 
     for call in range(2):
         out = torch.full((B, 64, 128), float("nan"), device=DEV)
-        st = L.lsa_sparse_decode_attn_noalloc(_p(q), _p(kb), _p(vb), kb.shape[0], _p(cu), B, scale, _p(out),
+        st = L.lsa_sparse_decode_attn_noalloc(_p(q), _p(kb), _p(vb), kb.shape[1], _p(cu), B, scale, _p(out),
                                               stream)
         assert st == 0, f"call {call}: status {st}"
         torch.cuda.synchronize()
@@ -82,6 +82,6 @@ def test_noalloc_refuses_batch_beyond_its_scratch(L):
     q, kb, vb, cu = _inputs(n_kept, seed=78)
     out = torch.empty((len(n_kept), 64, 128), device=DEV)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    st = L.lsa_sparse_decode_attn_noalloc(_p(q), _p(kb), _p(vb), kb.shape[0], _p(cu), len(n_kept),
+    st = L.lsa_sparse_decode_attn_noalloc(_p(q), _p(kb), _p(vb), kb.shape[1], _p(cu), len(n_kept),
                                           1.0 / np.sqrt(128.0), _p(out), stream)
     assert st == UNSUPPORTED
