@@ -83,7 +83,7 @@ typedef enum {
 #define LSA_DEV_ERR_BAD_CHUNK 4u   /* kept chunk index outside [0, max_chunks)   */
 #define LSA_DEV_ERR_CAPACITY 8u    /* compact buffer or kept row too small        */
 #define LSA_DEV_ERR_TIMEOUT 16u    /* a bounded in-kernel wait ran out            */
-#define LSA_DEV_ERR_WORKSPACE 32u  /* attention workspace not zero-initialised    */
+#define LSA_DEV_ERR_WORKSPACE 32u  /* reserved: not raised by this version        */
 #define LSA_DEV_ERR_INTERNAL 64u   /* launch-layout assumption violated (a bug)    */
 
 /* Human-readable name of an lsa_status value. */
@@ -249,9 +249,9 @@ int lsa_fetch_from_host_delta(const void* host_k_pool, const void* host_v_pool, 
                               void* stream, void* done_event);
 
 /*
- * Bytes of workspace lsa_sparse_decode_attn needs for a batch of B sequences.
- * The workspace must be zero-filled once before its first use; every call
- * leaves it ready for the next one.
+ * Bytes of workspace lsa_sparse_decode_attn needs for a batch of B sequences:
+ * (B*8 + 1024) partial records of 1032 floats.  It needs no initialisation;
+ * each call writes the records it reads.
  */
 size_t lsa_attn_workspace_size(int B);
 
@@ -268,21 +268,23 @@ size_t lsa_attn_workspace_size(int B);
  * A sequence with no kept chunk gets zeros.  The work is split over all SMs
  * along the kept tokens (split-K flash decoding) and the partial results are
  * merged with their log-sum-exp weights in a fixed order, so repeated calls
- * are bit-identical.
+ * are bit-identical.  The call enqueues two kernels on `stream`: the
+ * attention grid and the merge of the pairs it split, a programmatic
+ * dependent of it.
  *   q            device bf16 [B][64][128]
  *   k_buf, v_buf device bf16 [8][buf_chunks][64][128]
  *   cu_kept      device int32 [B+1]
  *   softmax_scale  usually 1/sqrt(128)
  *   out          device fp32 [B][64][128]
- *   workspace    device, >= lsa_attn_workspace_size(B) bytes, zero-filled
- *                before first use.
+ *   workspace    device, >= lsa_attn_workspace_size(B) bytes; calls that
+ *                may overlap on the GPU need workspaces of their own.
  *   flags        0 or LSA_ATTN_KV_UNCHANGED.  The kernel is launched as a
  *                programmatic dependent of the preceding kernel on `stream`
  *                (its start overlaps that kernel's tail); it waits for that
  *                kernel before reading q or cu_kept (without the flag) and
  *                before writing out or the workspace.
  * B <= LSA_MAX_BATCH.  Device errors: CAPACITY (cu_kept[B] > buf_chunks or
- * cu_kept decreasing: nothing is computed), TIMEOUT, WORKSPACE.
+ * cu_kept decreasing: nothing is computed), TIMEOUT.
  */
 int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
                            int64_t buf_chunks, const int32_t* cu_kept, int B,
@@ -309,13 +311,12 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
  * and sets the kernel's shared-memory limit; make that first call before any
  * stream capture.  Every call on a device uses the same array: calls whose
  * work may overlap on the GPU (other streams, other host threads) race and
- * must be serialised by the caller.  Each call clears the array's counters on
- * `stream` before its kernel runs.
+ * must be serialised by the caller.
  */
 #define LSA_NOALLOC_MAX_BATCH 32
 #define LSA_NOALLOC_MAX_CTAS 512
-/* 1 KiB of counters + (32*8 + 512) partial records of 1032 floats. */
-#define LSA_NOALLOC_SCRATCH_BYTES 3171328
+/* (32*8 + 512) partial records of 1032 floats. */
+#define LSA_NOALLOC_SCRATCH_BYTES 3170304
 int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, const void* v_buf,
                                    int64_t buf_chunks, const int32_t* cu_kept, int B,
                                    float softmax_scale, float* out, void* stream);

@@ -262,11 +262,11 @@ def lsa_attn_workspace_size(B: int) -> int:
 
 
 def new_attn_workspace(B: int, device=None) -> torch.Tensor:
-    """A zero-filled workspace for lsa_sparse_decode_attn (zeroing is required once)."""
+    """A workspace for lsa_sparse_decode_attn (it needs no initialisation)."""
     n = lsa_attn_workspace_size(B)
     if n == 0:
         raise ValueError("unsupported batch")
-    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
 ATTN_KV_UNCHANGED = 1

@@ -26,10 +26,12 @@
 //   N = 8 heads, K = 16 tokens, V^T read once with ldmatrix.trans).
 // * At the end of each (b, g) segment the 8 warps combine their (max, sum,
 //   acc) in shared memory.  A segment that covers the whole pair writes the
-//   output; otherwise it writes a normalised partial and its log-sum-exp.  At
-//   the CTA's end it takes the tickets of its (at most two) partial pairs; the
-//   last CTA to finish a pair merges all partials of the pair in CTA order
-//   from shared memory, so the result does not depend on timing.
+//   output; otherwise it writes a normalised partial and its log-sum-exp, and
+//   the CTA is done: no tickets, fences or merges on the attention grid's
+//   tail.  A small second kernel, launched as a programmatic dependent, folds
+//   the partials of each split pair in CTA order once the grid has finished,
+//   spread over the SMs of the pair's contributors, so the result does not
+//   depend on timing.
 // * Launched as a programmatic dependent of the previous kernel: when the
 //   caller states that K/V did not change, the producer starts streaming
 //   before the previous kernel has finished.
@@ -68,9 +70,7 @@ constexpr int kStageBytes = 4 * kBoxBytes;   // K dims 0-63, K dims 64-127, V lo
 constexpr int kAccStride = 132;              // padded row of the combine buffer
 constexpr int kRecFloats = kGroup * kHeadDim + kGroup;  // partial o[8][128] + lse[8]
 constexpr int kMaxCtas = 1024;
-constexpr int kRecBytes = kRecFloats * 4;    // 4128, a multiple of 16
-// Partial records that fit in the stage ring plus the combine buffer.
-constexpr int kStagedRecs = (kStages * kStageBytes + kConsumerWarps * kGroup * kAccStride * 4) / kRecBytes;
+static_assert(kRecFloats * 4 % 16 == 0, "records are copied in 16-byte pieces");
 constexpr int kSmemBytes = kStages * kStageBytes +
                            kConsumerWarps * kGroup * kAccStride * 4 + 2 * kConsumerWarps * kGroup * 4 +
                            2 * kStages * 8 + 16;
@@ -93,11 +93,28 @@ struct Partition {
 // Sequence offsets counted in 64-token units: an array of chunk offsets
 // (shift 0: cu_kept), or of token offsets that are multiples of 64 (shift 6:
 // cu_sel of the token-level fine stage, read without a packed copy).
+// `l2` reads them through L2 only (a kernel that reads them before its grid
+// dependency wait, while another kernel may still be running on its SM).
 struct Offsets {
   const int32_t* p;
   int shift;
-  __device__ __forceinline__ int operator()(int i) const { return __ldg(p + i) >> shift; }
+  bool l2 = false;
+  __device__ __forceinline__ int raw(int i) const { return l2 ? __ldcg(p + i) : __ldg(p + i); }
+  __device__ __forceinline__ int operator()(int i) const { return raw(i) >> shift; }
 };
+
+// Verdict on the sequence offsets, the same in every thread of the block: the
+// first is 0, none decreases, the total fits `cap`; indexed offsets are token
+// offsets, multiples of 64 and at most max_sel apart.
+__device__ __forceinline__ bool offsets_bad(Offsets cu, int B, int64_t cap, bool indexed, int max_sel) {
+  const int total = cu(B);
+  int bad = (cu.raw(0) != 0 || total < 0 || static_cast<int64_t>(total) > cap) ? 1 : 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    bad |= (cu(b + 1) < cu(b));
+    if (indexed) bad |= ((cu.raw(b + 1) & 63) != 0) | (cu.raw(b + 1) - cu.raw(b) > max_sel);
+  }
+  return __syncthreads_or(bad) != 0;
+}
 
 // Units of sequence b: its kept chunks plus E local chunks (E = 1 when the
 // window's decoded tokens are attended), for each of the 8 KV heads.  The
@@ -158,7 +175,7 @@ struct SelectArgs {
   const int32_t* ck;    // [B + 1]: chunk offsets of the compact buffer (cu_kept)
   int max_sel;
   int64_t ck_chunks;    // chunks in the compact buffer
-  const uint4* k_buf;   // the compact buffer, [ck_chunks][8][64][16 x 16 B]
+  const uint4* k_buf;   // the compact buffer, head-major [8][ck_chunks][64][16 x 16 B]
   const uint4* v_buf;
 };
 
@@ -182,7 +199,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                           const __grid_constant__ CUtensorMap tm_kl, const __grid_constant__ CUtensorMap tm_vl,
                           const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ cu_raw, int B,
                           int64_t buf_chunks, const int32_t* __restrict__ local_len, float scale_log2,
-                          float* __restrict__ out, int* __restrict__ counters, float* __restrict__ records,
+                          float* __restrict__ out, float* __restrict__ records,
                           unsigned* status, int kv_unchanged, AppendArgs app, SelectArgs sa) {
   const bool indexed = sa.sel != nullptr;
   const Offsets cu{cu_raw, indexed ? 6 : 0};
@@ -199,7 +216,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   float* lbuf = mbuf + kConsumerWarps * kGroup;
   uint64_t* full = reinterpret_cast<uint64_t*>(lbuf + kConsumerWarps * kGroup);
   uint64_t* empty = full + kStages;
-  int* flags = reinterpret_cast<int*>(empty + kStages);  // [0] abort, [1] last-CTA
+  int* flags = reinterpret_cast<int*>(empty + kStages);  // [0] abort
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -212,19 +229,12 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   // ---- validate cu_kept (every thread reaches the same verdict) -------------
   // (Indexed: token offsets, multiples of 64, at most max_sel per sequence;
   // buf_chunks is then the unit capacity B * max_sel / 64.)
-  const int total = cu(B);
-  int bad = (__ldg(cu_raw) != 0 || total < 0 || static_cast<int64_t>(total) > buf_chunks) ? 1 : 0;
-  for (int b = tid; b < B; b += kThreads) {
-    bad |= (cu(b + 1) < cu(b));
-    if (indexed) bad |= ((__ldg(cu_raw + b + 1) & 63) != 0) | (__ldg(cu_raw + b + 1) - __ldg(cu_raw + b) > sa.max_sel);
-  }
-  bad = __syncthreads_or(bad);
-  if (bad) {
+  if (offsets_bad(cu, B, buf_chunks, indexed, sa.max_sel)) {
     if (blockIdx.x == 0 && tid == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
     return;
   }
   const int E = local_len ? 1 : 0;   // one local unit per (b, g) when decoded tokens are attended
-  const int T = 8 * (total + E * B);
+  const int T = 8 * (cu(B) + E * B);
   const int G = gridDim.x;
   const Partition part(T, G);
   const int64_t u0 = part.start(blockIdx.x), u1 = part.start(blockIdx.x + 1);
@@ -251,7 +261,6 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       mbar_init(&empty[s], kWarpsPerGroup);   // a stage is consumed by one warp group
     }
     flags[0] = 0;
-    flags[1] = 0;
     mbar_fence_init();
   }
   __syncthreads();
@@ -386,85 +395,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     vofs[t] = 2 * kBoxBytes + (t >> 2) * kBoxBytes + vrow * 128 + ((((t & 3) * 2 + vx) ^ (vrow & 7)) << 4);
   }
 
-  const int hh = tid >> 5;          // combine / merge: head within the group (warp-uniform)
+  const int hh = tid >> 5;          // combine: head within the group (warp-uniform)
   const int d0 = (tid & 31) * 4;    // 4 consecutive dims
-
-  // Merge of the partials of pair p in CTA order, run at the end of this CTA's
-  // work (the stage ring and the combine buffer are free).  Records of the
-  // contributing CTAs are contiguous (index p + c); whole batches of them are
-  // pulled into shared memory with asynchronous 16-byte copies (one L2 round
-  // trip per batch) and folded with a running log-sum-exp.  The log-sum-exp a
-  // thread reads is warp-uniform (one head per warp).
-  auto merge_pair = [&](int pp, int c_lo, int c_hi) {
-    const int n_rec = c_hi - c_lo + 1;
-    const char* gsrc = reinterpret_cast<const char*>(records + static_cast<int64_t>(pp + c_lo) * kRecFloats);
-    const float* srec = reinterpret_cast<const float*>(smem);
-    float lse_max = -INFINITY, den = 0.f;
-    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < n_rec; c0 += kStagedRecs) {
-      const int nc = min(kStagedRecs, n_rec - c0);
-      const char* gb = gsrc + static_cast<int64_t>(c0) * kRecBytes;
-      for (int i = tid; i < nc * (kRecBytes / 16); i += kConsumerThreads)
-        cp_async_16_cg(smem_base + i * 16, gb + static_cast<int64_t>(i) * 16);
-      cp_async_wait_all();
-      named_barrier(1, kConsumerThreads);
-      float m4[4] = {lse_max, lse_max, lse_max, lse_max};
-      int c = 0;
-      for (; c + 4 <= nc; c += 4) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], srec[(c + k) * kRecFloats + kGroup * kHeadDim + hh]);
-      }
-      for (; c < nc; ++c) m4[0] = fmaxf(m4[0], srec[c * kRecFloats + kGroup * kHeadDim + hh]);
-      const float m_new = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      const float mref = m_new == -INFINITY ? 0.f : m_new;   // all partials empty so far
-      const float resc = fast_exp2(lse_max - mref);           // 0 on the first batch
-      den *= resc;
-      r.x *= resc; r.y *= resc; r.z *= resc; r.w *= resc;
-      lse_max = m_new;
-#pragma unroll 4
-      for (int cc = 0; cc < nc; ++cc) {
-        const float* rc = srec + cc * kRecFloats;
-        const float wgt = fast_exp2(rc[kGroup * kHeadDim + hh] - mref);
-        const float4 x = *reinterpret_cast<const float4*>(rc + hh * kHeadDim + d0);
-        den += wgt;
-        r.x += wgt * x.x; r.y += wgt * x.y; r.z += wgt * x.z; r.w += wgt * x.w;
-      }
-      named_barrier(1, kConsumerThreads);
-    }
-    const float id = den > 0.f ? 1.f / den : 0.f;
-    const int bb = pp / kNumKVHeads, gg = pp % kNumKVHeads;
-    float* dst = out + (static_cast<int64_t>(bb) * kNumQHeads + gg * kGroup + hh) * kHeadDim + d0;
-    *reinterpret_cast<float4*>(dst) = make_float4(r.x * id, r.y * id, r.z * id, r.w * id);
-    if (tid == 0) counters[pp] = 0;   // ready for the next call
-  };
-
-  // Tickets of the deferred first segment (if any) and of the last segment
-  // (cur_p >= 0), taken by two threads in parallel after one fence over the
-  // records; the last contributor of a pair merges it.
-  int pend_p = -1, pend_lo = 0, pend_hi = 0;
-  auto settle = [&](int cur_p, int cur_lo, int cur_hi) {
-    __threadfence();
-    named_barrier(1, kConsumerThreads);
-    if (tid == 0 && pend_p >= 0) {
-      const int n_contrib = pend_hi - pend_lo + 1;   // every CTA in [lo, hi] owns part of the pair
-      const int old = atomicAdd(&counters[pend_p], 1);
-      if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
-      flags[2] = (old == n_contrib - 1);
-    }
-    if (tid == 32 && cur_p >= 0) {
-      const int n_contrib = cur_hi - cur_lo + 1;
-      const int old = atomicAdd(&counters[cur_p], 1);
-      if (old >= n_contrib) set_status(status, LSA_DEV_ERR_WORKSPACE);
-      flags[1] = (old == n_contrib - 1);
-    }
-    named_barrier(1, kConsumerThreads);
-    const bool m_pend = pend_p >= 0 && flags[2] != 0;
-    const bool m_cur = cur_p >= 0 && flags[1] != 0;
-    if (m_pend || m_cur) __threadfence();
-    if (m_pend) merge_pair(pend_p, pend_lo, pend_hi);
-    if (m_cur) merge_pair(cur_p, cur_lo, cur_hi);
-    pend_p = -1;
-  };
 
   UnitCursor cur;
   cur.start(cu, E, B, u0);
@@ -660,18 +592,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       float* rec = records + static_cast<int64_t>(p + blockIdx.x) * kRecFloats;
       *reinterpret_cast<float4*>(rec + hh * kHeadDim + d0) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
       if ((tid & 31) == 0) rec[kGroup * kHeadDim + hh] = M + __log2f(L);
-      // Contributing CTAs of pair p: those whose unit range meets [a_p, a_p + n_b).
-      const int a_p = static_cast<int>(seq_unit_base(cu, E, b)) + g * n_b;
-      const int c_lo = part.cta_of(a_p), c_hi = part.cta_of(a_p + n_b - 1);
-      if (u + (jend - j0) != u1) {
-        // Only a CTA's first segment can be partial without being its last:
-        // keep streaming and take this pair's ticket at the CTA's end.
-        pend_p = p;
-        pend_lo = c_lo;
-        pend_hi = c_hi;
-      } else {
-        settle(p, c_lo, c_hi);
-      }
+      // attn_merge_kernel folds the records of the pair once this grid is done.
     }
     named_barrier(1, kConsumerThreads);   // combine buffer free for the next segment
 
@@ -680,13 +601,141 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     cur.j = jend - 1;
     cur.advance(cu, E, B, n_b);
   }
-  if (pend_p >= 0) settle(-1, 0, 0);
 }
 
-// Workspace: int counters[B*8] (padded to 256 B), then fp32 records[(B*8 + kMaxCtas)][kRecFloats].
+// ---- split-K merge -----------------------------------------------------------
+// A (sequence, KV head) pair whose units the grid split over CTAs
+// [c_lo, c_hi] left one normalised partial per contributing CTA c (record
+// p + c: o[8 heads][128] and the log-sum-exp of each head).  attn_merge_kernel
+// runs as a programmatic dependent of the attention launch with the same grid
+// size G: its CTA c takes, for each split pair that attention CTA c
+// contributed to, the heads h with h = c - c_lo (mod n), n = c_hi - c_lo + 1,
+// so the 8 heads of a pair are folded on up to 8 SMs at once.  It fixes its
+// tasks from the offsets while the attention grid is still running, waits for
+// that grid, stages the needed rows of the records in shared memory with one
+// round of asynchronous copies and folds each (pair, head) in CTA order, so
+// the result does not depend on timing.  Small enough (256 threads, at most
+// 64 registers each, 33 KiB) to sit on an SM beside an attention CTA.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kMergeItems = 64;       // (task, record) rows staged per round
+// A CTA meets at most two split pairs (those of its first and last unit), and
+// takes at most 4 heads of each (a split pair has n >= 2 contributors): at
+// most 8 tasks, one per warp.
+constexpr int kMergeTasks = kMergeWarps;
+
+__global__ void __launch_bounds__(kMergeThreads, 4)
+attn_merge_kernel(const int32_t* __restrict__ cu_raw, int shift, int E, int B, int64_t cap, int max_sel,
+                  const float* __restrict__ records, float* __restrict__ out) {
+  __shared__ __align__(16) float4 s_o[kMergeItems * (kHeadDim / 4)];
+  __shared__ float s_l[kMergeItems];
+  __shared__ int t_rec[kMergeTasks], t_h[kMergeTasks], t_out[kMergeTasks], t_item0[kMergeTasks + 1];
+  __shared__ int s_ntasks;
+  griddep_launch_dependents();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // The offsets were final before the attention grid started (it waits for
+  // their writer before it lets this grid launch, or they did not change); they
+  // are read through L2 before the wait.
+  const Offsets cu{cu_raw, shift, true};
+  const bool bad = offsets_bad(cu, B, cap, shift != 0, max_sel);
+  if (tid == 0) {
+    int nt = 0, items = 0;
+    const int T = bad ? 0 : 8 * (cu(B) + E * B);
+    const Partition part(T, gridDim.x);
+    const int c = blockIdx.x;
+    const int u0 = part.start(c), u1 = part.start(c + 1);
+    int prev_a = -1;
+    for (int side = 0; side < 2 && u0 < u1; ++side) {
+      const int u = side == 0 ? u0 : u1 - 1;
+      const int b = seq_of_unit(cu, E, B, u);
+      const int base = static_cast<int>(seq_unit_base(cu, E, b));
+      const int n_b = units_of(cu, E, b);
+      const int g = (u - base) / n_b;
+      const int a_p = base + g * n_b;
+      if (a_p == prev_a) break;          // the same pair at both ends of the range
+      prev_a = a_p;
+      const int lo = part.cta_of(a_p), hi = part.cta_of(a_p + n_b - 1);
+      if (lo == hi) continue;            // whole in one CTA: written by the attention kernel
+      const int n = hi - lo + 1;
+      for (int h = c - lo; h < kGroup && nt < kMergeTasks; h += n) {
+        t_rec[nt] = (b * kNumKVHeads + g) + lo;
+        t_h[nt] = h;
+        t_out[nt] = b * kNumQHeads + g * kGroup + h;
+        t_item0[nt] = items;
+        items += n;
+        ++nt;
+      }
+    }
+    t_item0[nt] = items;
+    s_ntasks = nt;
+  }
+  __syncthreads();
+  griddep_wait();   // every CTA waits, so this grid never completes before the attention grid
+  const int nt = s_ntasks;
+  if (nt == 0) return;
+  const int items = t_item0[nt];
+  const int my0 = warp < nt ? t_item0[warp] : 0, my1 = warp < nt ? t_item0[warp + 1] : 0;
+  float m = -INFINITY, den = 0.f;
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < items; i0 += kMergeItems) {
+    const int ni = min(kMergeItems, items - i0);
+    for (int x = tid; x < ni * 33; x += kMergeThreads) {   // per row: 32 x 16 B of o, then its lse
+      const int it = x / 33, qd = x - it * 33;
+      const int gi = i0 + it;
+      int t = 0;
+      while (t + 1 < nt && t_item0[t + 1] <= gi) ++t;
+      const float* rec = records + static_cast<int64_t>(t_rec[t] + (gi - t_item0[t])) * kRecFloats;
+      if (qd < 32) cp_async_16_cg(smem_u32(s_o + it * 32 + qd), rec + t_h[t] * kHeadDim + qd * 4);
+      else s_l[it] = __ldcg(rec + kGroup * kHeadDim + t_h[t]);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // Warp t folds task t's rows of this round, in CTA order.
+    const int a = max(my0, i0), e = min(my1, i0 + ni);
+    for (int gi = a; gi < e; ++gi) {
+      const float l = s_l[gi - i0];
+      const float m_new = fmaxf(m, l);
+      const float mref = m_new == -INFINITY ? 0.f : m_new;   // every partial so far empty
+      const float sc = fast_exp2(m - mref), w = fast_exp2(l - mref);
+      const float4 x = s_o[(gi - i0) * 32 + lane];
+      den = den * sc + w;
+      r.x = r.x * sc + w * x.x;
+      r.y = r.y * sc + w * x.y;
+      r.z = r.z * sc + w * x.z;
+      r.w = r.w * sc + w * x.w;
+      m = m_new;
+    }
+    __syncthreads();
+  }
+  if (warp < nt) {
+    const float id = den > 0.f ? 1.f / den : 0.f;
+    reinterpret_cast<float4*>(out + static_cast<int64_t>(t_out[warp]) * kHeadDim)[lane] =
+        make_float4(r.x * id, r.y * id, r.z * id, r.w * id);
+  }
+}
+
+// Workspace: fp32 records[(B*8 + kMaxCtas)][kRecFloats], one slot per
+// (pair p, contributing CTA c) at index p + c.  Each launch writes the slots it
+// reads, so the contents left between calls do not matter.
 size_t workspace_bytes(int B) {
-  const size_t cnt = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
-  return cnt + (static_cast<size_t>(B) * kNumKVHeads + kMaxCtas) * kRecFloats * sizeof(float);
+  return (static_cast<size_t>(B) * kNumKVHeads + kMaxCtas) * kRecFloats * sizeof(float);
+}
+
+// The merge of split pairs, as a programmatic dependent of the attention
+// launch just issued on `stream` with `grid` CTAs.
+inline cudaError_t launch_merge(int grid, const int32_t* cu, int shift, int E, int B, int64_t cap, int max_sel,
+                                const float* records, float* out, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_merge_kernel, cu, shift, E, B, cap, max_sel, records, out);
 }
 
 }  // namespace attn
@@ -771,9 +820,7 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
     tm_kl = tm_k;
     tm_vl = tm_v;
   }
-  const size_t cnt_bytes = ((static_cast<size_t>(B) * kNumKVHeads * 4 + 255) / 256) * 256;
-  int* counters = static_cast<int*>(workspace);
-  float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + cnt_bytes);
+  float* records = static_cast<float*>(workspace);
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   // Launched as a programmatic dependent of the preceding kernel: its
   // prologue (and, with LSA_ATTN_KV_UNCHANGED, its K/V stream) overlaps the
@@ -793,8 +840,10 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   const int kv_unchanged = (flags & LSA_ATTN_KV_UNCHANGED) ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, attn::sparse_decode_attn_kernel, tm_k, tm_v, tm_kl, tm_vl,
                          static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
-                         local ? local_len : static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records,
-                         lsa_device_status_ptr(), kv_unchanged, app, sa) != cudaSuccess) {
+                         local ? local_len : static_cast<const int32_t*>(nullptr), scale_log2, out, records,
+                         lsa_device_status_ptr(), kv_unchanged, app, sa) != cudaSuccess ||
+      attn::launch_merge(static_cast<int>(cfg.gridDim.x), cu_kept, sa.sel ? 6 : 0, local ? 1 : 0, B, buf_chunks,
+                         sa.max_sel, records, out, cfg.stream) != cudaSuccess) {
     cudaGetLastError();
     return LSA_ERR_CUDA;
   }
@@ -863,7 +912,7 @@ int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* 
 // all device memory and forbids cudaMalloc once it has started), and some
 // cannot allocate at the moment they call (cudaMalloc may synchronise the
 // device, which a latency-critical decode loop must not do).  For them the
-// split-K scratch (ticket counters and partial results) lives in a fixed
+// split-K scratch (the partial results) lives in a fixed
 // array inside this library instead of a caller-provided workspace.
 //
 // The array is a file-scope __device__ variable of LSA_NOALLOC_SCRATCH_BYTES
@@ -873,15 +922,13 @@ int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* 
 // rejected with LSA_ERR_UNSUPPORTED_SHAPE.  All calls on a device share the
 // one array, so calls whose kernels may overlap on the GPU (different
 // streams, or different host threads) race with each other and must be
-// serialised by the caller.  The ticket counters are cleared on the stream
-// before every launch, so leftovers of an earlier call do not matter.
+// serialised by the caller.  Each launch writes the records it reads, so
+// leftovers of an earlier call do not matter.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr size_t kNoAllocCounterBytes =
-    ((static_cast<size_t>(LSA_NOALLOC_MAX_BATCH) * lsa::kNumKVHeads * 4 + 255) / 256) * 256;
 constexpr size_t kNoAllocScratchBytes =
-    kNoAllocCounterBytes + (static_cast<size_t>(LSA_NOALLOC_MAX_BATCH) * lsa::kNumKVHeads + LSA_NOALLOC_MAX_CTAS) *
-                               lsa::attn::kRecFloats * sizeof(float);
+    (static_cast<size_t>(LSA_NOALLOC_MAX_BATCH) * lsa::kNumKVHeads + LSA_NOALLOC_MAX_CTAS) * lsa::attn::kRecFloats *
+    sizeof(float);
 static_assert(kNoAllocScratchBytes == LSA_NOALLOC_SCRATCH_BYTES, "header constant out of date");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -943,16 +990,16 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   st = encode_kv_map(&tm_v, v_buf, buf_chunks);
   if (st != LSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* counters = static_cast<int*>(scratch);
-  float* records = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kNoAllocCounterBytes);
-  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(B) * kNumKVHeads * sizeof(int), s) != cudaSuccess) {
-    cudaGetLastError();
-    return LSA_ERR_CUDA;
-  }
+  float* records = static_cast<float*>(scratch);
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
       tm_k, tm_v, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
-      static_cast<const int32_t*>(nullptr), scale_log2, out, counters, records, lsa_device_status_ptr(), 0,
+      static_cast<const int32_t*>(nullptr), scale_log2, out, records, lsa_device_status_ptr(), 0,
       attn::AppendArgs{}, attn::SelectArgs{});
+  if (cudaGetLastError() != cudaSuccess ||
+      attn::launch_merge(grid, cu_kept, 0, 0, B, buf_chunks, 0, records, out, s) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
   return launch_status();
 }

@@ -61,8 +61,8 @@ def test_workspace_size(L):
     assert L.lsa_attn_workspace_size(4097) == 0
     s1, s32 = L.lsa_attn_workspace_size(1), L.lsa_attn_workspace_size(32)
     assert 0 < s1 < s32
-    # 8 counters (padded to 256 B) + (8 + 1024) partial records of 1032 floats
-    assert s1 == 256 + (8 + 1024) * 1032 * 4
+    # (8 + 1024) partial records of 1032 floats
+    assert s1 == (8 + 1024) * 1032 * 4
 
 
 def test_host_checks_null_pointers(L):
