@@ -373,6 +373,14 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   }
 
   // ========================= consumer warps ==================================
+  UnitCursor cur;
+  cur.start(cu, E, B, u0);
+  // While the previous kernel finishes, bring the first segment's 8 query rows
+  // (2 KiB) into L2, so that the loads after the wait hit L2.  A prefetch puts
+  // nothing in registers and L2 sees the previous kernel's stores, so this is
+  // safe even if that kernel writes q.
+  if (kv_unchanged && tid < 16)
+    prefetch_l2(q + (static_cast<int64_t>(cur.b) * kNumQHeads + cur.g * kGroup) * kHeadDim + tid * 64);
   if (kv_unchanged) griddep_wait();
   zero_empty(tid, kConsumerThreads);
   const int grp = warp / kWarpsPerGroup;   // takes the units with unit_i % 2 == grp
@@ -398,8 +406,6 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   const int hh = tid >> 5;          // combine: head within the group (warp-uniform)
   const int d0 = (tid & 31) * 4;    // 4 consecutive dims
 
-  UnitCursor cur;
-  cur.start(cu, E, B, u0);
   int64_t u = u0;
   int64_t unit_i = 0;
   while (u < u1) {
@@ -610,12 +616,13 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 // runs as a programmatic dependent of the attention launch with the same grid
 // size G: its CTA c takes, for each split pair that attention CTA c
 // contributed to, the heads h with h = c - c_lo (mod n), n = c_hi - c_lo + 1,
-// so the 8 heads of a pair are folded on up to 8 SMs at once.  It fixes its
-// tasks from the offsets while the attention grid is still running, waits for
-// that grid, stages the needed rows of the records in shared memory with one
-// round of asynchronous copies and folds each (pair, head) in CTA order, so
-// the result does not depend on timing.  Small enough (256 threads, at most
-// 64 registers each, 33 KiB) to sit on an SM beside an attention CTA.
+// so the 8 heads of a pair are folded on up to 8 SMs at once.  Its CTAs start
+// as attention CTAs exit and fix their tasks from the offsets while the
+// slowest attention CTAs still stream; then they wait for the grid, stage the
+// needed rows of the records in shared memory with one round of asynchronous
+// copies (the log-sum-exps too, so no thread stalls on a load while issuing)
+// and fold each (pair, head) in CTA order, so the result does not depend on
+// timing.  256 threads, at most 64 registers each, 34 KiB.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kMergeItems = 64;       // (task, record) rows staged per round
@@ -673,20 +680,24 @@ attn_merge_kernel(const int32_t* __restrict__ cu_raw, int shift, int E, int B, i
   griddep_wait();   // every CTA waits, so this grid never completes before the attention grid
   const int nt = s_ntasks;
   if (nt == 0) return;
+  // The code after the wait is kept short: it runs with cold instruction
+  // caches (the attention grid's stream evicts them between launches), and
+  // every further stretch of code costs a fetch round trip.
   const int items = t_item0[nt];
   const int my0 = warp < nt ? t_item0[warp] : 0, my1 = warp < nt ? t_item0[warp + 1] : 0;
   float m = -INFINITY, den = 0.f;
   float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int i0 = 0; i0 < items; i0 += kMergeItems) {
     const int ni = min(kMergeItems, items - i0);
-    for (int x = tid; x < ni * 33; x += kMergeThreads) {   // per row: 32 x 16 B of o, then its lse
+    // One round of asynchronous copies: per row its 32 x 16 B of o and its lse.
+    for (int x = tid; x < ni * 33; x += kMergeThreads) {
       const int it = x / 33, qd = x - it * 33;
       const int gi = i0 + it;
       int t = 0;
       while (t + 1 < nt && t_item0[t + 1] <= gi) ++t;
       const float* rec = records + static_cast<int64_t>(t_rec[t] + (gi - t_item0[t])) * kRecFloats;
       if (qd < 32) cp_async_16_cg(smem_u32(s_o + it * 32 + qd), rec + t_h[t] * kHeadDim + qd * 4);
-      else s_l[it] = __ldcg(rec + kGroup * kHeadDim + t_h[t]);
+      else cp_async_4(smem_u32(s_l + it), rec + kGroup * kHeadDim + t_h[t]);
     }
     cp_async_wait_all();
     __syncthreads();
@@ -719,6 +730,16 @@ attn_merge_kernel(const int32_t* __restrict__ cu_raw, int shift, int E, int B, i
 // reads, so the contents left between calls do not matter.
 size_t workspace_bytes(int B) {
   return (static_cast<size_t>(B) * kNumKVHeads + kMaxCtas) * kRecFloats * sizeof(float);
+}
+
+// Kernel attributes, set once per device.  The carve-out is left to the
+// driver: the one it picks for the attention CTA's 166 KB leaves no room for a
+// merge CTA beside it, so merge CTAs start as attention CTAs exit.  Asking for
+// the largest carve-out lets them sit side by side, which gained 0.1 us per
+// 500K step but cost 0.8 us per step of the token-level fine stage, whose next
+// kernels then also start early and wait on the SMs.
+inline cudaError_t set_kernel_attributes() {
+  return cudaFuncSetAttribute(sparse_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
 // The merge of split pairs, as a programmatic dependent of the attention
@@ -798,8 +819,7 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   {
     std::lock_guard<std::mutex> lk(g_attn_mu);
     if (dev < 64 && !g_attn_attr_set[dev]) {
-      if (cudaFuncSetAttribute(attn::sparse_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               attn::kSmemBytes) != cudaSuccess) {
+      if (attn::set_kernel_attributes() != cudaSuccess) {
         cudaGetLastError();
         return LSA_ERR_CUDA;
       }
@@ -951,8 +971,7 @@ int noalloc_setup(int dev, void** scratch) {
     g_noalloc_ptr[dev] = p;
   }
   if (!g_noalloc_attr_set[dev]) {
-    if (cudaFuncSetAttribute(lsa::attn::sparse_decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             lsa::attn::kSmemBytes) != cudaSuccess) {
+    if (lsa::attn::set_kernel_attributes() != cudaSuccess) {
       cudaGetLastError();
       return LSA_ERR_CUDA;
     }
