@@ -266,11 +266,23 @@ def run_host_tier(args, rank, world, local_rank):
             f1[w].record(side)
             ev_fetched[w].record(side)
 
+    def attend_steps(w):
+        for t in range(workloads.TAU):
+            lw.attend(L.q[w % n_win, t], out[t], buf=w % 2, kv_unchanged=t > 0)
+
+    # The 64 steps of a window are replayed from a CUDA graph per (buffer, query
+    # window), as in the main bench: launched one by one from the host, the two
+    # kernels of each attention call cost more host time than the window's fetch.
+    graphs = {}
+
     def attend(w):             # on the main stream: 64 steps over buffer w % 2
         main.wait_event(ev_fetched[w])
         with torch.cuda.stream(main):
-            for t in range(workloads.TAU):
-                lw.attend(L.q[w % n_win, t], out[t], buf=w % 2, kv_unchanged=t > 0)
+            g = graphs.get((w % 2, w % n_win))
+            if g is not None:
+                g.replay()
+            else:
+                attend_steps(w)
             ev_attn_done[w].record(main)
 
     probe = h2d_probe_gbs(dev)
@@ -281,6 +293,15 @@ def run_host_tier(args, rank, world, local_rank):
         prepare(w + 1)
         attend(w)
     torch.cuda.synchronize()
+    if args.graphs:
+        for w in range(2 * n_win):
+            key = (w % 2, w % n_win)
+            if key not in graphs:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=main):
+                    attend_steps(w)
+                graphs[key] = g
+        torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -319,7 +340,8 @@ def run_host_tier(args, rank, world, local_rank):
                    "stream overlaps the 64 attention steps of window w", "fetch_ctas": args.fetch_ctas,
                    "residency": "chunks kept by the previous window are copied from its device buffer"
                    if args.delta else "every kept chunk is fetched from the host pool",
-                   "l2": "inputs larger than L2 (host pool 8 GiB, 410 MiB per attention launch)"},
+                   "l2": "inputs larger than L2 (host pool 8 GiB, 410 MiB per attention launch)",
+                   "cuda_graphs": bool(args.graphs)},
         "roofline": {"kernel": "gather_kernel (host-tier fetch)", "bound": "pcie", "achieved": fetch_gbs,
                      "peak": probe, "unit": "GB/s", "frac": fetch_gbs / probe,
                      "peak_source": "same-run pinned H2D copy probe (cudaMemcpyAsync, 1 GiB)", "traffic": None,
