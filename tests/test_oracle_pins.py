@@ -361,6 +361,42 @@ def test_attention_large_logits_stay_finite():
     np.testing.assert_allclose(got[0, 63, :2], [1 / (1 + math.e), math.e / (1 + math.e)], rtol=1e-12)
 
 
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_attention_split_and_lse_merge_equal_one_pass(seed):
+    """Split-K invariant (rows a6 + a7): cutting the kept tokens of a (sequence,
+    KV head) pair at arbitrary points, normalising each part by its own softmax,
+    and folding the parts in order with base-2 log-sum-exp weights and a running
+    maximum (an empty part included) gives the oracle's one-pass attention to
+    rounding, for any number of parts, parts of one token among them."""
+    rng = np.random.default_rng(100 + seed)
+    n = 3
+    k_buf, v_buf = _rand_bufs(n, rng)
+    q = bf16_round(rng.standard_normal((1, 64, 128)))
+    ref = oracle.sparse_decode_attn(q, k_buf, v_buf, [0, n])
+    T = 64 * n
+    c = 1.0 / math.sqrt(128) / math.log(2.0)          # logits in base 2
+    for h in (0, 9, 63):
+        g = h // 8
+        K = k_buf[:, g].reshape(T, 128)
+        V = v_buf[:, g].reshape(T, 128)
+        cuts = sorted(set(rng.integers(1, T, 2 + 3 * seed).tolist()) | {1, T - 1})
+        bounds = [0] + cuts + [T]
+        parts = []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            s = (K[a:b] @ q[0, h]) * c
+            mx = s.max()
+            p = np.exp2(s - mx)
+            parts.append((mx + math.log2(p.sum()), (p @ V[a:b]) / p.sum()))
+        parts.insert(len(parts) // 2, (-math.inf, np.zeros(128)))   # a part with no valid token
+        m, den, acc = -math.inf, 0.0, np.zeros(128)
+        for lse, o in parts:
+            m_new = max(m, lse)
+            mref = 0.0 if m_new == -math.inf else m_new
+            sc, w = np.exp2(m - mref), np.exp2(lse - mref)
+            den, acc, m = den * sc + w, acc * sc + w * o, m_new
+        np.testing.assert_allclose(acc / den, ref[0, h], rtol=1e-12, atol=1e-14)
+
+
 def test_attention_chunk_permutation_invariance():
     rng = np.random.default_rng(10)
     k_buf, v_buf = _rand_bufs(4, rng)
