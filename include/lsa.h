@@ -278,11 +278,13 @@ size_t lsa_attn_workspace_size(int B);
  *   out          device fp32 [B][64][128]
  *   workspace    device, >= lsa_attn_workspace_size(B) bytes; calls that
  *                may overlap on the GPU need workspaces of their own.
- *   flags        0 or LSA_ATTN_KV_UNCHANGED.  The kernel is launched as a
- *                programmatic dependent of the preceding kernel on `stream`
- *                (its start overlaps that kernel's tail); it waits for that
- *                kernel before reading q or cu_kept (without the flag) and
- *                before writing out or the workspace.
+ *   flags        0 or LSA_ATTN_KV_UNCHANGED.  The attention grid is launched
+ *                as a programmatic dependent of the preceding kernel on
+ *                `stream` (its start overlaps that kernel's tail); it waits
+ *                for that kernel before reading q or cu_kept (without the
+ *                flag) and before writing out or the workspace.  The merge
+ *                grid waits for the attention grid before it reads the
+ *                workspace.
  * B <= LSA_MAX_BATCH.  Device errors: CAPACITY (cu_kept[B] > buf_chunks or
  * cu_kept decreasing: nothing is computed), TIMEOUT.
  */
@@ -390,8 +392,10 @@ int lsa_sparse_decode_attn_selected(const void* q, const void* k_buf, const void
                                     unsigned int flags, void* stream);
 
 /*
- * lsa_sparse_decode_attn_append -- one causal decode step in one launch:
- * lsa_append_token followed by lsa_sparse_decode_attn_local, fused.  With
+ * lsa_sparse_decode_attn_append -- one causal decode step with the append
+ * fused into the attention grid: lsa_append_token followed by
+ * lsa_sparse_decode_attn_local in one launch (plus the merge of split pairs
+ * that every attention call enqueues).  With
  * n = local_len_in[b], the step attends the kept chunks, tokens 0 .. n-1 of
  * the local chunk and this step's own token (k_new, v_new device bf16
  * [B][8][128]) as token n; it also writes that token to row n of the local
