@@ -634,8 +634,10 @@ constexpr int kMergeTasks = kMergeWarps;
 __global__ void __launch_bounds__(kMergeThreads, 4)
 attn_merge_kernel(const int32_t* __restrict__ cu_raw, int shift, int E, int B, int64_t cap, int max_sel,
                   const float* __restrict__ records, float* __restrict__ out) {
-  __shared__ __align__(16) float4 s_o[kMergeItems * (kHeadDim / 4)];
-  __shared__ float s_l[kMergeItems];
+  // Per staged row: 32 x 16 B of o, then the 16 B of the record that hold its
+  // log-sum-exp (4 heads' worth; the row's head picks one).
+  __shared__ __align__(16) float4 s_o[kMergeItems * 33];
+  __shared__ int s_off[kMergeItems], s_loff[kMergeItems];   // float4 offsets from `records`
   __shared__ int t_rec[kMergeTasks], t_h[kMergeTasks], t_out[kMergeTasks], t_item0[kMergeTasks + 1];
   __shared__ int s_ntasks;
   griddep_launch_dependents();
@@ -677,38 +679,59 @@ attn_merge_kernel(const int32_t* __restrict__ cu_raw, int shift, int E, int B, i
     s_ntasks = nt;
   }
   __syncthreads();
-  griddep_wait();   // every CTA waits, so this grid never completes before the attention grid
   const int nt = s_ntasks;
-  if (nt == 0) return;
-  // The code after the wait is kept short: it runs with cold instruction
-  // caches (the attention grid's stream evicts them between launches), and
-  // every further stretch of code costs a fetch round trip.
+  if (nt == 0) {
+    griddep_wait();   // every CTA waits, so this grid never completes before the attention grid
+    return;
+  }
   const int items = t_item0[nt];
-  const int my0 = warp < nt ? t_item0[warp] : 0, my1 = warp < nt ? t_item0[warp + 1] : 0;
-  float m = -INFINITY, den = 0.f;
-  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < items; i0 += kMergeItems) {
+  // Source offsets of the rows of round i0, in float4 units: the row's o and
+  // the 16-byte piece holding its log-sum-exp.
+  auto fill = [&](int i0) {
     const int ni = min(kMergeItems, items - i0);
-    // One round of asynchronous copies: per row its 32 x 16 B of o and its lse.
-    for (int x = tid; x < ni * 33; x += kMergeThreads) {
-      const int it = x / 33, qd = x - it * 33;
+    for (int it = tid; it < ni; it += kMergeThreads) {
       const int gi = i0 + it;
       int t = 0;
       while (t + 1 < nt && t_item0[t + 1] <= gi) ++t;
-      const float* rec = records + static_cast<int64_t>(t_rec[t] + (gi - t_item0[t])) * kRecFloats;
-      if (qd < 32) cp_async_16_cg(smem_u32(s_o + it * 32 + qd), rec + t_h[t] * kHeadDim + qd * 4);
-      else cp_async_4(smem_u32(s_l + it), rec + kGroup * kHeadDim + t_h[t]);
+      const int base = (t_rec[t] + (gi - t_item0[t])) * (kRecFloats / 4);
+      s_off[it] = base + t_h[t] * (kHeadDim / 4);
+      s_loff[it] = base + (kGroup * kHeadDim) / 4 + (t_h[t] >> 2);
+    }
+  };
+  // Everything that does not need the records is done before the wait: the
+  // code after it runs with cold instruction caches (the attention grid's
+  // stream evicts them between launches), and every further stretch of code
+  // costs a fetch round trip.
+  fill(0);
+  __syncthreads();
+  griddep_wait();   // every CTA waits, so this grid never completes before the attention grid
+  const float4* rec4 = reinterpret_cast<const float4*>(records);
+  const int my0 = warp < nt ? t_item0[warp] : 0, my1 = warp < nt ? t_item0[warp + 1] : 0;
+  const int hl = warp < nt ? (t_h[warp] & 3) : 0;   // this warp's log-sum-exp within its 16-byte piece
+  float m = -INFINITY, den = 0.f;
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < items; i0 += kMergeItems) {
+    if (i0 > 0) {   // rounds after the first (more than kMergeItems rows)
+      fill(i0);
+      __syncthreads();
+    }
+    const int ni = min(kMergeItems, items - i0);
+    // One round of asynchronous 16-byte copies: per row its o and its lse piece.
+    for (int x = tid; x < ni * 33; x += kMergeThreads) {
+      const int it = x / 33, qd = x - it * 33;
+      cp_async_16_cg(smem_u32(s_o + x), rec4 + (qd < 32 ? s_off[it] + qd : s_loff[it]));
     }
     cp_async_wait_all();
     __syncthreads();
     // Warp t folds task t's rows of this round, in CTA order.
     const int a = max(my0, i0), e = min(my1, i0 + ni);
     for (int gi = a; gi < e; ++gi) {
-      const float l = s_l[gi - i0];
+      const float4* row = s_o + (gi - i0) * 33;
+      const float l = reinterpret_cast<const float*>(row + 32)[hl];
       const float m_new = fmaxf(m, l);
       const float mref = m_new == -INFINITY ? 0.f : m_new;   // every partial so far empty
       const float sc = fast_exp2(m - mref), w = fast_exp2(l - mref);
-      const float4 x = s_o[(gi - i0) * 32 + lane];
+      const float4 x = row[lane];
       den = den * sc + w;
       r.x = r.x * sc + w * x.x;
       r.y = r.y * sc + w * x.y;
