@@ -239,6 +239,31 @@ def test_threshold_rule():
     assert list(got) == [1, 3, 4]                           # 0.6 and 0.505 pass; latest kept
 
 
+def test_threshold_extremes_and_nesting():
+    """The weighted mean of sigmoids lies strictly between 0 and 1, so threshold 0
+    keeps every chunk and threshold 1 keeps only the latest; a higher threshold
+    never keeps a chunk a lower one dropped; a sequence of one chunk keeps it and
+    an empty one keeps nothing.  Scores come from the oracle's own indexer on
+    random queries and keys."""
+    rng = np.random.default_rng(77)
+    B, N = 3, 40
+    q = bf16_round(rng.standard_normal((B, 16, 128)) * 3.0)
+    keys = bf16_round(rng.standard_normal((B * N, 128)))
+    w = rng.uniform(0, 1, 16)
+    n = [N, 1, 0]
+    s = oracle.index_scores(q, w, keys, None, n, max_chunks=N)
+    assert list(oracle.threshold_chunks(s, n, w, threshold=0.0)[0]) == list(range(N))
+    assert list(oracle.threshold_chunks(s, n, w, threshold=1.0)[0]) == [N - 1]
+    prev = set(range(N))
+    for t in np.linspace(0.05, 0.95, 19):
+        got = oracle.threshold_chunks(s, n, w, threshold=float(t))
+        assert list(got[1]) == [0] and list(got[2]) == []
+        cur = set(got[0].tolist())
+        assert N - 1 in cur and cur <= prev
+        prev = cur
+    assert len(prev) < N          # the random queries spread the scores across thresholds
+
+
 # ------------------------------------------------------------------ gather ---
 
 def test_gather_closed_form_positions():
