@@ -141,3 +141,13 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     with pytest.raises(RuntimeError, match="liblsa.so not found"):
         lsa.lib()
     importlib.reload(lsa)
+
+
+def test_binding_takes_head_major_compact_buffers():
+    """The binding reads the chunk count of a compact buffer from its head-major
+    shape [8, chunks, 64, 128] and rejects any other shape, a chunk-major
+    [chunks, 8, 64, 128] one included (it would pass a wrong size to the kernels)."""
+    assert lsa._buf_chunks(torch.empty((8, 20, 64, 128), dtype=torch.bfloat16), "k_buf") == 20
+    for bad in ((20, 8, 64, 128), (8, 20, 128, 64), (8, 20, 64), (4, 20, 64, 128)):
+        with pytest.raises(ValueError, match="k_buf"):
+            lsa._buf_chunks(torch.empty(bad, dtype=torch.bfloat16), "k_buf")
