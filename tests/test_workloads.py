@@ -1,0 +1,35 @@
+"""The seeded input recipe (CPU only).
+
+The pages measure on long-context benchmarks whose items are not used here;
+synthetic inputs stand in for them at the same context lengths.  The batched
+workload takes ragged lengths: each sequence's length is drawn uniformly in
+[32768, 262144] tokens and floored to whole 64-token chunks (never below
+32768), with K = floor(N / 8) kept chunks besides the latest one (the 12.5%
+recall ratio)."""
+import torch
+
+import workloads
+
+
+def test_batched_lengths_recipe():
+    wl = workloads.WORKLOADS["batched"]
+    n, k = workloads.lengths_for(wl)
+    assert n.numel() == wl.batch == 32
+    tokens = n.to(torch.int64) * 64
+    assert int(tokens.min()) >= 32768 and int(tokens.max()) <= 262144
+    assert torch.equal(k, torch.div(n, 8, rounding_mode="floor"))
+    assert int(n.min()) < int(n.max())                      # ragged
+
+
+def test_lengths_are_seeded():
+    wl = workloads.WORKLOADS["batched"]
+    n1, _ = workloads.lengths_for(wl)
+    n2, _ = workloads.lengths_for(wl)
+    n3, _ = workloads.lengths_for(wl, base_seed=workloads.BASE_SEED + 1)
+    assert torch.equal(n1, n2) and not torch.equal(n1, n3)
+
+
+def test_fixed_length_workloads():
+    for name, chunks, k in (("500k", 8192, 819), ("128k", 2048, 256), ("1m_host", 16384, 1638)):
+        n, kk = workloads.lengths_for(workloads.WORKLOADS[name])
+        assert n.tolist() == [chunks] and kk.tolist() == [k]
