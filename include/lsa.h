@@ -18,7 +18,10 @@
  * ---------------------------------
  *  - Pointers marked "device" are CUDA device (or managed) memory of the
  *    current device; "host" pointers are CPU memory.  The caller owns every
- *    buffer, stream and event.  The library allocates no device memory.
+ *    buffer, stream and event.  The library never calls cudaMalloc; its only
+ *    device memory is the static scratch array of
+ *    lsa_sparse_decode_attn_noalloc (LSA_NOALLOC_SCRATCH_BYTES per GPU that
+ *    loads the library) and the device status word.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every compute call only enqueues work on `stream` and returns.
  *  - Return value: LSA_OK (0) or a negative lsa_status.  Argument checks are
@@ -306,7 +309,10 @@ int lsa_sparse_decode_attn(const void* q, const void* k_buf, const void* v_buf,
  * (LSA_NOALLOC_SCRATCH_BYTES of device memory, held by every GPU that loads
  * the library until the process exits).  The caller still owns and passes q,
  * the compact buffers, cu_kept and out; arguments, results and device errors
- * are those of lsa_sparse_decode_attn.  Limits: B <= LSA_NOALLOC_MAX_BATCH
+ * are those of lsa_sparse_decode_attn, and so is the launch (the same grid,
+ * the same merge kernel, a programmatic dependent of the preceding kernel
+ * without LSA_ATTN_KV_UNCHANGED), so the output is bit-identical to
+ * lsa_sparse_decode_attn's on the same inputs.  Limits: B <= LSA_NOALLOC_MAX_BATCH
  * and a device of at most 512 SMs (one CTA per SM), otherwise
  * LSA_ERR_UNSUPPORTED_SHAPE.  The call allocates nothing (no cudaMalloc, no
  * cudaFree).  Its first call on a device looks up the array's device address

@@ -815,13 +815,17 @@ size_t lsa_attn_workspace_size(int B) {
 }  // extern "C"
 
 namespace {
-// Shared launcher of lsa_sparse_decode_attn, lsa_sparse_decode_attn_local
-// (k_local == nullptr: no local units) and lsa_sparse_decode_attn_append.
-int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
-                int B, float softmax_scale, const void* k_local, const void* v_local, const int32_t* local_len,
-                float* out, void* workspace, size_t workspace_bytes, unsigned int flags, void* stream,
-                const lsa::attn::AppendArgs& app = lsa::attn::AppendArgs{},
-                const lsa::attn::SelectArgs& sa = lsa::attn::SelectArgs{}) {
+// Shared launcher of every attention entry point: lsa_sparse_decode_attn,
+// lsa_sparse_decode_attn_local (k_local == nullptr: no local units),
+// lsa_sparse_decode_attn_append, lsa_sparse_decode_attn_selected and
+// lsa_sparse_decode_attn_noalloc.  `records` (records_bytes long) holds the
+// split-K partials: it must have room for (B * 8 + max_grid) records, and a
+// launch whose grid would exceed max_grid is refused.
+int attn_launch_records(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks,
+                        const int32_t* cu_kept, int B, float softmax_scale, const void* k_local, const void* v_local,
+                        const int32_t* local_len, float* out, float* records, size_t records_bytes, int max_grid,
+                        unsigned int flags, void* stream, const lsa::attn::AppendArgs& app,
+                        const lsa::attn::SelectArgs& sa) {
   using namespace lsa;
   if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
@@ -831,12 +835,18 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   // TMA row coordinates are 32-bit: (buf_chunks * 512) rows must fit.
   if (buf_chunks > (int64_t{1} << 22)) return LSA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out) || !aligned16(workspace))
+  if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out) || !aligned16(records))
     return LSA_ERR_MISALIGNED;
   if (local && (!aligned16(k_local) || !aligned16(v_local))) return LSA_ERR_MISALIGNED;
-  if (!workspace || workspace_bytes < attn::workspace_bytes(B)) return LSA_ERR_WORKSPACE;
+  const size_t need = (static_cast<size_t>(B) * kNumKVHeads + static_cast<size_t>(max_grid)) * attn::kRecFloats *
+                      sizeof(float);
+  if (!records || records_bytes < need) return LSA_ERR_WORKSPACE;
   const int sms = device_sm_count();
   if (sms <= 0) return LSA_ERR_NO_DEVICE;
+  // buf_chunks bounds the kept total (cu_kept[B] lives on the device).
+  const int grid = attn::grid_for_units(sms, static_cast<int64_t>(kNumKVHeads) * (buf_chunks + (local ? B : 0)),
+                                        sa.sel ? attn::kMinIndexedUnitsPerCta : attn::kMinUnitsPerCta);
+  if (grid > max_grid) return LSA_ERR_UNSUPPORTED_SHAPE;
   int dev = 0;
   cudaGetDevice(&dev);
   {
@@ -863,15 +873,12 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
     tm_kl = tm_k;
     tm_vl = tm_v;
   }
-  float* records = static_cast<float*>(workspace);
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   // Launched as a programmatic dependent of the preceding kernel: its
   // prologue (and, with LSA_ATTN_KV_UNCHANGED, its K/V stream) overlaps the
   // tail of that kernel; the kernel waits for it before touching its outputs.
   cudaLaunchConfig_t cfg = {};
-  // buf_chunks bounds the kept total (cu_kept[B] lives on the device).
-  cfg.gridDim = dim3(attn::grid_for_units(sms, static_cast<int64_t>(kNumKVHeads) * (buf_chunks + (local ? B : 0)),
-                                           sa.sel ? attn::kMinIndexedUnitsPerCta : attn::kMinUnitsPerCta));
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(attn::kThreads);
   cfg.dynamicSmemBytes = attn::kSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
@@ -891,6 +898,17 @@ int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf
     return LSA_ERR_CUDA;
   }
   return launch_status();
+}
+
+// The workspace entry points: the records live in the caller's workspace.
+int attn_launch(const void* q, const void* k_buf, const void* v_buf, int64_t buf_chunks, const int32_t* cu_kept,
+                int B, float softmax_scale, const void* k_local, const void* v_local, const int32_t* local_len,
+                float* out, void* workspace, size_t workspace_bytes, unsigned int flags, void* stream,
+                const lsa::attn::AppendArgs& app = lsa::attn::AppendArgs{},
+                const lsa::attn::SelectArgs& sa = lsa::attn::SelectArgs{}) {
+  return attn_launch_records(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, k_local, v_local, local_len,
+                             out, static_cast<float*>(workspace), workspace_bytes, lsa::attn::kMaxCtas, flags,
+                             stream, app, sa);
 }
 }  // namespace
 
@@ -978,7 +996,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64] = {};
-bool g_noalloc_attr_set[64] = {};
 
 // Device address of the scratch array for the current device.  The host-side
 // symbol is only a stand-in, so the address is looked up once per device
@@ -993,13 +1010,6 @@ int noalloc_setup(int dev, void** scratch) {
     }
     g_noalloc_ptr[dev] = p;
   }
-  if (!g_noalloc_attr_set[dev]) {
-    if (lsa::attn::set_kernel_attributes() != cudaSuccess) {
-      cudaGetLastError();
-      return LSA_ERR_CUDA;
-    }
-    g_noalloc_attr_set[dev] = true;
-  }
   *scratch = g_noalloc_ptr[dev];
   return LSA_OK;
 }
@@ -1012,36 +1022,18 @@ extern "C" int lsa_sparse_decode_attn_noalloc(const void* q, const void* k_buf, 
   if (!q || !k_buf || !v_buf || !cu_kept || !out || B <= 0 || buf_chunks <= 0) return LSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return LSA_ERR_INVALID_ARG;
   if (B > LSA_NOALLOC_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
-  if (buf_chunks > (int64_t{1} << 22)) return LSA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(q) || !aligned16(k_buf) || !aligned16(v_buf) || !aligned16(out)) return LSA_ERR_MISALIGNED;
-  const int sms = device_sm_count();
-  if (sms <= 0) return LSA_ERR_NO_DEVICE;
-  const int grid = attn::grid_for(sms);
-  if (grid > LSA_NOALLOC_MAX_CTAS) return LSA_ERR_UNSUPPORTED_SHAPE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return LSA_ERR_NO_DEVICE;
   }
   void* scratch = nullptr;
-  int st = noalloc_setup(dev, &scratch);
+  const int st = noalloc_setup(dev, &scratch);
   if (st != LSA_OK) return st;
-  CUtensorMap tm_k, tm_v;
-  st = encode_kv_map(&tm_k, k_buf, buf_chunks);
-  if (st != LSA_OK) return st;
-  st = encode_kv_map(&tm_v, v_buf, buf_chunks);
-  if (st != LSA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  float* records = static_cast<float*>(scratch);
-  const float scale_log2 = softmax_scale * 1.4426950408889634f;
-  attn::sparse_decode_attn_kernel<<<grid, attn::kThreads, attn::kSmemBytes, s>>>(
-      tm_k, tm_v, tm_k, tm_v, static_cast<const __nv_bfloat16*>(q), cu_kept, B, buf_chunks,
-      static_cast<const int32_t*>(nullptr), scale_log2, out, records, lsa_device_status_ptr(), 0,
-      attn::AppendArgs{}, attn::SelectArgs{});
-  if (cudaGetLastError() != cudaSuccess ||
-      attn::launch_merge(grid, cu_kept, 0, 0, B, buf_chunks, 0, records, out, s) != cudaSuccess) {
-    cudaGetLastError();
-    return LSA_ERR_CUDA;
-  }
-  return launch_status();
+  // The same launch as lsa_sparse_decode_attn (grid, programmatic dependent
+  // launch, merge), with the records in the static array; a grid beyond
+  // LSA_NOALLOC_MAX_CTAS (a device of more than 512 SMs) is refused.
+  return attn_launch_records(q, k_buf, v_buf, buf_chunks, cu_kept, B, softmax_scale, nullptr, nullptr, nullptr, out,
+                             static_cast<float*>(scratch), kNoAllocScratchBytes, LSA_NOALLOC_MAX_CTAS, 0, stream,
+                             attn::AppendArgs{}, attn::SelectArgs{});
 }

@@ -145,6 +145,29 @@ def test_token_topk_ties_and_signed_zero(n):
     assert got[2] == list(oracle.topk_tokens([finite], 128)[0])
 
 
+@pytest.mark.parametrize("n,k", [(131073, 2048), (200000, 128)])
+def test_token_topk_reread_path_random_scores(n, k):
+    """Beyond 131072 candidates the one-CTA kernel re-reads the scores from
+    memory.  Random scores (and scores quantised to 1/256, so the boundary
+    falls inside a long run of ties) must select exactly what the oracle's
+    rule selects on the same fp32 scores."""
+    g = torch.Generator(device=DEV).manual_seed(n + k)
+    s = torch.rand((3, n), generator=g, device=DEV)
+    s[1] = torch.floor(s[1] * 256.0) / 256.0
+    s[2] = torch.randn((n,), generator=g, device=DEV)
+    lens = [n, n - 77, n - 1]
+    n_tok = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    sel, n_sel, cu = topk_tokens_gpu(s, n_tok, k)
+    torch.cuda.synchronize()
+    status_clean()
+    got = kept_from_gpu(sel, n_sel)
+    host_scores = f64(s)
+    ref = oracle.topk_tokens([host_scores[b, : lens[b]] for b in range(3)], k)
+    for b in range(3):
+        assert got[b] == list(ref[b]), f"seq {b}"
+    assert i64(cu).tolist() == [0, k, 2 * k, 3 * k]
+
+
 def test_gather_tokens_bit_exact():
     inp, L, lw, tok_keys, q_tok = recalled("batched", batch=6)
     scores, n_tok = token_scores_gpu(lw, q_tok[0, 1], L.w, tok_keys)

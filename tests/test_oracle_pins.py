@@ -585,3 +585,65 @@ def test_fine_attention_equals_dense_sdpa_over_selected_rows():
         np.testing.assert_allclose(got[b], ref, rtol=1e-12, atol=1e-14)
     shuffled = [rng.permutation(s) for s in sel]
     np.testing.assert_allclose(oracle.fine_decode_attn(q, k_buf, v_buf, cu, shuffled), got, rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------------- unit-signature closed form ---
+# The full-size GPU tests of the split-K partition use zero keys and one-hot
+# values (tests/unit_signature.py), where attention is a ratio of token counts.
+# These pins tie that closed form to the oracle's attention.
+
+def _signature_case(n_kept, seed):
+    import unit_signature as us
+    cu = np.concatenate([[0], np.cumsum(n_kept)]).astype(np.int64)
+    total = int(cu[-1])
+    off = us.offsets(max(total, 1), seed)
+    v_hm = us.compact_v(off[:, :total], "cpu").to(torch.float64)             # [8, total, 64, 128]
+    v_buf = v_hm.permute(1, 0, 2, 3).numpy()                                  # chunk-major for the oracle
+    k_buf = np.zeros_like(v_buf)
+    q = bf16_round(np.random.default_rng(seed).standard_normal((len(n_kept), 64, 128)))
+    return us, cu, off, k_buf, v_buf, q
+
+
+@pytest.mark.parametrize("n_kept", [[1], [3, 0, 2], [5, 1]])
+def test_unit_signature_closed_form_equals_oracle(n_kept):
+    us, cu, off, k_buf, v_buf, q = _signature_case(n_kept, seed=sum(n_kept) + 7)
+    got = oracle.sparse_decode_attn(q, k_buf, v_buf, cu)
+    want = us.expected_chunks(off, cu)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-15)
+    us.assert_signature(got, want)
+
+
+def test_unit_signature_closed_form_with_local_tokens_equals_oracle():
+    us, cu, off, k_buf, v_buf, q = _signature_case([2, 0, 1], seed=31)
+    B = 3
+    offl = us.local_offsets(B, 32)
+    v_loc = us.one_hot_rows(torch.from_numpy(offl)).to(torch.float64).numpy()  # [B, 8, 64, 128]
+    k_loc = np.zeros_like(v_loc)
+    ll = [5, 17, 0]
+    got = oracle.sparse_decode_attn(q, k_buf, v_buf, cu, k_local=k_loc, v_local=v_loc, local_len=ll)
+    want = us.expected_chunks(off, cu, local_off=offl, local_len=ll)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-15)
+
+
+def test_unit_signature_closed_form_selected_equals_oracle():
+    us, cu, off, k_buf, v_buf, q = _signature_case([3, 2], seed=41)
+    rng = np.random.default_rng(42)
+    sel = [np.sort(rng.choice(192, 128, replace=False)), np.sort(rng.choice(128, 64, replace=False))]
+    got = oracle.fine_decode_attn(q, k_buf, v_buf, cu, sel)
+    want = us.expected_selected(off, cu, sel)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-15)
+
+
+def test_unit_signature_detects_a_missing_or_repeated_unit():
+    """The closed form separates the right unit set from one with a unit dropped
+    or read twice by far more than its tolerance (mistakes planted on the CPU)."""
+    import pytest as _pt
+    us, cu, off, k_buf, v_buf, q = _signature_case([40], seed=51)
+    want = us.expected_chunks(off, cu)
+    dropped = oracle.sparse_decode_attn(q, k_buf[:39], v_buf[:39], [0, 39])
+    with _pt.raises(AssertionError):
+        us.assert_signature(dropped, want)
+    twice = np.concatenate([k_buf, k_buf[7:8]]), np.concatenate([v_buf, v_buf[7:8]])
+    repeated = oracle.sparse_decode_attn(q, twice[0], twice[1], [0, 41])
+    with _pt.raises(AssertionError):
+        us.assert_signature(repeated, want)
