@@ -20,6 +20,11 @@ Metric: decode tokens per second per layer (64 * B tokens per window and
 layer), with the achieved HBM bandwidth of the whole window and of the
 attention kernel against the measured copy bandwidth.
 
+On one GPU with the default workload, the other configurations of the metric
+(128K, the 1M host tier, the batched workload, and the 500K fine-stage and
+causal modes) then run for ``--config-steps`` windows each and appear as
+compact lines under ``configs``; ``--no-configs`` skips them.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 500k]
     python bench.py --impl reference ...   # the fp64 oracle on the host cores
 
@@ -96,21 +101,78 @@ def profiled_traffic(workload):
     return float(m_b.group(1))
 
 
+_REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+            ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+            ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+            ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+            ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+
+def summarise_clocks(sm, mx, reasons):
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled while the timed region runs.
+
+    A thread queries NVML every ``interval_s`` (read-only queries: nothing of the
+    GPU's settings is touched), so a timed region of a few tens of milliseconds
+    still carries several samples of its own.  Without NVML it falls back to
+    ``nvidia-smi -lms 20``."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_s: float = 0.005):
         self.gpu = gpu_index
+        self.interval = interval_s
         self.proc = None
-        # raw samples (the JSON line carries their summary); LSA_CLOCKS_DIR picks the folder
+        self.thread = None
+        self.nvml = None
+        # raw samples of the nvidia-smi fallback; LSA_CLOCKS_DIR picks the folder
         self.path = os.path.join(os.environ.get("LSA_CLOCKS_DIR") or tempfile.gettempdir(),
                                  f"lsa_clocks_gpu{gpu_index}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:   # the CUDA device's own PCI address (CUDA and NVML may number GPUs differently)
+            p = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
     def start(self):
+        import threading
+        try:
+            self.nvml, self.handle = self._nvml_handle()
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            nv, h = self.nvml, self.handle
+            self.samples = []
+            self.stop_evt = threading.Event()
+            bits = [(name, getattr(nv, attr, 0)) for name, attr in _REASONS]
+            max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+            def loop():
+                while not self.stop_evt.is_set():
+                    try:
+                        mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((mhz, max_mhz, [n for n, b in bits if b and (r & b)]))
+                    except Exception:
+                        pass
+                    self.stop_evt.wait(self.interval)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            while not self.samples and self.thread.is_alive():   # the first sample precedes the timed region
+                time.sleep(self.interval / 5)
+            return
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
@@ -121,8 +183,17 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            sm = [float(m) for m, _, _ in self.samples]
+            mx = [float(x) for _, x, _ in self.samples]
+            reasons = {n for _, _, rs in self.samples for n in rs}
+            out = summarise_clocks(sm, mx, reasons)
+            out["source"] = f"NVML every {self.interval * 1e3:.0f} ms"
+            return out
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -143,8 +214,9 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        out = summarise_clocks(sm, mx, reasons)
+        out["source"] = "nvidia-smi -lms 20"
+        return out
 
 
 def copy_probe_gbs(device, nbytes=1 << 31, reps=10):
@@ -538,6 +610,60 @@ def run_ours(args, rank, world, local_rank):
         out["fine_stages"] = fine_stages
         out["roofline"]["timed_with"] = "the fine stage (token scores, token top-k, packing) before each launch"
     return out
+
+
+# The other configurations of the metric, each run for a few windows after the
+# headline and reported as a compact line under "configs": (name, overrides).
+EXTRA_CONFIGS = (
+    ("128k", {"workload": "128k"}),
+    ("1m_host", {"workload": "1m_host"}),
+    ("batched", {"workload": "batched"}),
+    ("500k_fine_k2048", {"workload": "500k", "fine_k": 2048}),
+    ("500k_causal", {"workload": "500k", "causal": True}),
+)
+
+
+def compact_line(name, out):
+    """The fields of a full line that describe one configuration's result."""
+    keep = {"name": name, "workload": out["config"]["workload"], "value": out["value"], "unit": out["unit"],
+            "steps": out["steps"], "warmup": out["warmup"], "ms_per_step": out["ms_per_step"],
+            "kept_chunks_total": out["config"]["kept_chunks_total"],
+            "frac_of_measured": out["hbm"]["frac_of_measured"], "roofline": out["roofline"],
+            "clocks": out["clocks"]}
+    for k in ("l2", "fine_k", "causal", "schedule"):
+        if out["config"].get(k):
+            keep[k] = out["config"][k]
+    for k in ("fine_stages", "pcie", "stage_us"):
+        if out.get(k) is not None:
+            keep[k] = out[k]
+    return keep
+
+
+def run_extra_configs(args, rank, world, local_rank):
+    """Every other configuration of the metric for a few windows (N = 1 only)."""
+    import gc
+    lines = []
+    for name, over in EXTRA_CONFIGS:
+        sub = argparse.Namespace(**vars(args))
+        sub.fine_k, sub.causal, sub.delta = 0, False, False
+        sub.selection, sub.n_local = "topk", 1
+        sub.no_e2e, sub.no_cpu_baseline = True, True
+        sub.steps, sub.warmup = args.config_steps, 3
+        for k, v in over.items():
+            setattr(sub, k, v)
+        gc.collect()
+        torch.cuda.empty_cache()
+        try:
+            if workloads.WORKLOADS[sub.workload].host_pool:
+                out = run_host_tier(sub, rank, world, local_rank)
+            else:
+                out = run_ours(sub, rank, world, local_rank)
+            lines.append(compact_line(name, out))
+        except Exception as e:   # one configuration failing must not lose the headline line
+            lines.append({"name": name, "error": f"{type(e).__name__}: {e}"[:300]})
+        gc.collect()
+        torch.cuda.empty_cache()
+    return lines
 
 
 def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=32, replays=10):
@@ -934,6 +1060,9 @@ def main():
     ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
     ap.add_argument("--attn-only", action="store_true",
                     help="time attention launches alone on a random compact buffer (profiling case)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations after the headline (one GPU, default workload only)")
+    ap.add_argument("--config-steps", type=int, default=8, help="timed windows of each other configuration")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -978,6 +1107,10 @@ def main():
         if world > 1:
             torch.distributed.barrier()
     out["cpu_baseline"] = cpu
+    headline_only = (args.fine_k or args.causal or args.delta or args.selection != "topk" or args.n_local != 1
+                     or args.workload != DEFAULT_WORKLOAD)
+    if world == 1 and not args.no_configs and not headline_only:
+        out["configs"] = run_extra_configs(args, rank, world, local_rank)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -427,9 +427,12 @@ int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* 
  * page "lightning indexer").  Every decode step:
  *   lsa_token_score   -> one score per token of the recalled chunks,
  *   lsa_topk_tokens   -> the k best token positions,
- *   lsa_gather_tokens -> those tokens packed into dense 64-token units,
- *   lsa_sparse_decode_attn(_local) over the units (buf = k_out / v_out,
- *   cu_kept = cu_units).
+ *   lsa_sparse_decode_attn_selected -> attention over those tokens, whose
+ *                        rows it reads in place from the compact buffer.
+ * A causal step (lsa_sparse_decode_attn_append, which attends whole units)
+ * first packs the selected tokens into dense 64-token units with
+ * lsa_gather_tokens and attends the units (buf = k_out / v_out,
+ * cu_kept = cu_units).
  * Token position p of sequence b is token p % 64 of its recalled chunk
  * p / 64 (kept[b*max_kept + p/64]); positions follow the context order.  All
  * KV heads attend the same selected tokens (one score per token).
