@@ -154,11 +154,17 @@ def topk_chunks(scores, n_chunks, k_per_seq, n_local=1):
     return out
 
 
-def threshold_chunks(scores, n_chunks, w, threshold=0.5):
+def threshold_chunks(scores, n_chunks, w, threshold=0.5, cap=None):
     """The pages' sigmoid-threshold selection (FM-DS-V4 summary, 2.1 and 2.4).
 
     Reading: a chunk is recalled when its weighted mean sigmoid probability
     score_c / sum_h w_h exceeds the threshold; the latest chunk is always kept.
+
+    ``cap`` (one budget per sequence, optional): the pages want the resident
+    KV cut to about a tenth (FM-DS-V4 summary, Abstract) but give the threshold
+    no bound.  Reading: when more than cap[b] chunks pass, the cap[b] passing
+    chunks with the highest scores are kept, by score descending then chunk
+    index ascending (the tie rule of ``topk_chunks``), listed ascending.
     """
     scores = np.asarray(scores, dtype=np.float64)
     wsum = float(np.sum(np.asarray(w, dtype=np.float64)))
@@ -170,6 +176,9 @@ def threshold_chunks(scores, n_chunks, w, threshold=0.5):
             continue
         cand = np.arange(n - 1, dtype=np.int64)
         chosen = cand[scores[b, : n - 1] / wsum > threshold]
+        if cap is not None and len(chosen) > int(cap[b]):
+            ranked = sorted(chosen.tolist(), key=lambda c: (-scores[b, c], c))
+            chosen = np.sort(np.array(ranked[: int(cap[b])], dtype=np.int64))
         out.append(np.concatenate([chosen, np.array([n - 1], dtype=np.int64)]))
     return out
 

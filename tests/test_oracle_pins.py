@@ -264,6 +264,46 @@ def test_threshold_extremes_and_nesting():
     assert len(prev) < N          # the random queries spread the scores across thresholds
 
 
+@pytest.mark.parametrize("trial", range(6))
+def test_threshold_cap_matches_full_sort(trial):
+    """Under a budget the capped rule keeps the cap best passing chunks: a full
+    Python sort of the passing chunks by (score descending, index ascending),
+    on random scores with heavy ties; a cap at or above the passing count
+    changes nothing, and cap 0 keeps only the latest chunk."""
+    rng = np.random.default_rng(300 + trial)
+    B, N = 5, 60
+    w = rng.uniform(0, 1, 16)
+    s = rng.integers(0, 9, size=(B, N)) * (w.sum() / 8.0)     # score / sum(w) in {0, 1/8, ..., 1}: ties
+    n = [60, 45, 2, 1, 0]
+    t = 0.3
+    plain = oracle.threshold_chunks(s, n, w, threshold=t)
+    for cap in ([0, 0, 0, 0, 0], [7, 3, 1, 5, 2], [100] * 5, [len(p) - 1 for p in plain]):
+        cap = [max(c, 0) for c in cap]
+        got = oracle.threshold_chunks(s, n, w, threshold=t, cap=cap)
+        for b in range(B):
+            if n[b] == 0:
+                assert list(got[b]) == []
+                continue
+            passing = [c for c in range(n[b] - 1) if s[b, c] / w.sum() > t]
+            best = sorted(passing, key=lambda c: (-s[b, c], c))[: cap[b]]
+            assert list(got[b]) == sorted(best) + [n[b] - 1]
+            if cap[b] >= len(passing):
+                assert list(got[b]) == list(plain[b])
+
+
+def test_threshold_cap_is_topk_when_the_budget_binds():
+    """Every passing chunk outscores every other, so when more pass than the
+    budget the capped rule equals the top-K rule with K = cap."""
+    rng = np.random.default_rng(310)
+    w = rng.uniform(0, 1, 16)
+    s = rng.uniform(0.0, w.sum(), size=(3, 200))
+    n, cap = [200, 150, 90], [20, 5, 60]
+    got = oracle.threshold_chunks(s, n, w, threshold=0.2, cap=cap)
+    ref = oracle.topk_chunks(s, n, cap)
+    for b in range(3):
+        assert list(got[b]) == list(ref[b])
+
+
 # ------------------------------------------------------------------ gather ---
 
 def test_gather_closed_form_positions():
