@@ -317,6 +317,12 @@ def run_host_tier(args, rank, world, local_rank):
     f1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_total + 1)]
 
     reused = torch.zeros(n_total + 1, dtype=torch.int32, device=dev)
+    copy_engine = args.fetch == "copy"
+    if copy_engine:   # the copy-engine fetch plans its copies from a host copy of the selection
+        kept_h = [torch.empty_like(lw.kept[i], device="cpu").pin_memory() for i in range(2)]
+        cu_h = [torch.empty_like(lw.cu_kept[i], device="cpu").pin_memory() for i in range(2)]
+        table_h = inp.chunk_table.cpu()
+        ev_sel = torch.cuda.Event()
 
     def prepare(w):            # on the side stream: select + fetch window w into buffer w % 2
         buf = w % 2
@@ -333,6 +339,15 @@ def run_host_tier(args, rank, world, local_rank):
                                               inp.max_chunks, lw.k_bufs[buf], lw.v_bufs[buf], lw.kept[pb],
                                               lw.cu_kept[pb], lw.k_bufs[pb], lw.v_bufs[pb], reused[w:w + 1],
                                               num_ctas=args.fetch_ctas, stream=side)
+            elif copy_engine:
+                # the selection comes to the host (two small copies), which then enqueues one
+                # 2-D copy per kept chunk and per K/V on the side stream
+                kept_h[buf].copy_(lw.kept[buf], non_blocking=True)
+                cu_h[buf].copy_(lw.cu_kept[buf], non_blocking=True)
+                ev_sel.record(side)
+                ev_sel.synchronize()
+                lsa.lsa_fetch_from_host_copy(L.k_pool, L.v_pool, table_h, kept_h[buf], cu_h[buf], inp.max_chunks,
+                                             lw.k_bufs[buf], lw.v_bufs[buf], stream=side)
             else:
                 lw.fetch(L.k_pool, L.v_pool, buf=buf, num_ctas=args.fetch_ctas)
             f1[w].record(side)
@@ -360,10 +375,19 @@ def run_host_tier(args, rank, world, local_rank):
     probe = h2d_probe_gbs(dev)
     copy_gbs = copy_probe_gbs(dev)
     peak, peak_kind = measured_peaks()
+    def window(w):
+        # The copy-engine fetch blocks the host until window w + 1's selection is
+        # known, so window w's attention is enqueued first and overlaps that wait.
+        if copy_engine:
+            attend(w)
+            prepare(w + 1)
+        else:
+            prepare(w + 1)
+            attend(w)
+
     prepare(0)
     for w in range(args.warmup):
-        prepare(w + 1)
-        attend(w)
+        window(w)
     torch.cuda.synchronize()
     if args.graphs:
         for w in range(2 * n_win):
@@ -382,8 +406,7 @@ def run_host_tier(args, rank, world, local_rank):
     torch.cuda.synchronize()
     t0.record(main)
     for w in range(args.warmup, n_total):
-        prepare(w + 1)
-        attend(w)
+        window(w)
     t1.record(main)
     torch.cuda.synchronize()
     if world > 1:
@@ -412,9 +435,12 @@ def run_host_tier(args, rank, world, local_rank):
                    "stream overlaps the 64 attention steps of window w", "fetch_ctas": args.fetch_ctas,
                    "residency": "chunks kept by the previous window are copied from its device buffer"
                    if args.delta else "every kept chunk is fetched from the host pool",
+                   "fetch": ("copy engines: the selection is copied to the host, then one 2-D copy per kept chunk "
+                             "and per K/V" if copy_engine else "SM threads reading mapped page-locked memory"),
                    "l2": "inputs larger than L2 (host pool 8 GiB, 410 MiB per attention launch)",
                    "cuda_graphs": bool(args.graphs)},
-        "roofline": {"kernel": "gather_kernel (host-tier fetch)", "bound": "pcie", "achieved": fetch_gbs,
+        "roofline": {"kernel": "cudaMemcpy2DAsync (copy engines)" if copy_engine else "gather_kernel (host-tier fetch)",
+                     "bound": "pcie", "achieved": fetch_gbs,
                      "peak": probe, "unit": "GB/s", "frac": fetch_gbs / probe,
                      "peak_source": "same-run pinned H2D copy probe (cudaMemcpyAsync, 1 GiB)", "traffic": None,
                      "algorithmic_bytes_per_launch": fetch_bytes, "avg_launch_us": statistics.median(fetch_s) * 1e6},
@@ -424,7 +450,7 @@ def run_host_tier(args, rank, world, local_rank):
                  "window_bound_by_fetch_ms": fetch_bytes / probe / 1e6, "delta": bool(args.delta),
                  "reused_chunks_per_window": reuse, "host_link_bytes_per_window": link_bytes,
                  "host_link_gbs": link_bytes / statistics.median(fetch_s) / 1e9},
-        "gpu_launches": args.steps * (3 + workloads.TAU * ATTN_LAUNCHES),
+        "gpu_launches": args.steps * (3 - int(copy_engine) + workloads.TAU * ATTN_LAUNCHES),
         "clocks": clocks, "e2e": None,
     }
 
@@ -576,7 +602,9 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": inp.workload.description, "name": args.workload, "batch": B, "layers": layers,
             "chunks_per_seq": int(inp.n_chunks.max()), "kept_chunks_total": kept_total,
-            "selection": args.selection if args.selection == "topk" else f"threshold {args.threshold}",
+            "selection": args.selection if args.selection == "topk" else
+            f"threshold {args.threshold}, at most the top-K budget K_b per sequence",
+            "compact_buffer_chunks": lws[0].buf_chunks,
             "recent_chunks": args.n_local,
             "fine_k": args.fine_k or None,
             "causal": ("each step appends its token to a local chunk and attends it with the kept chunks"
@@ -1049,6 +1077,8 @@ def main():
     ap.add_argument("--fetch-ctas", type=int, default=64)
     ap.add_argument("--delta", action="store_true",
                     help="host tier: reuse chunks the previous window kept from its device buffer")
+    ap.add_argument("--fetch", choices=["sm", "copy"], default="sm",
+                    help="host tier: SM threads over mapped memory (default) or the copy engines")
     ap.add_argument("--selection", choices=["topk", "threshold"], default="topk",
                     help="chunk selection: fixed top-K budget (default) or the sigmoid threshold")
     ap.add_argument("--threshold", type=float, default=0.5)
@@ -1068,6 +1098,8 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if (args.causal or args.n_local != 1) and workloads.WORKLOADS[args.workload].host_pool:
         ap.error("--causal and --n-local apply to device-resident workloads, not the host tier")
+    if args.fetch == "copy" and (args.delta or not workloads.WORKLOADS[args.workload].host_pool):
+        ap.error("--fetch copy applies to the host-tier workload, without --delta")
     if args.n_local != 1 and args.selection != "topk":
         ap.error("--n-local applies to top-K selection")
     if args.fine_k and (args.fine_k < 0 or args.fine_k % 64 or workloads.WORKLOADS[args.workload].host_pool):
@@ -1108,6 +1140,7 @@ def main():
             torch.distributed.barrier()
     out["cpu_baseline"] = cpu
     headline_only = (args.fine_k or args.causal or args.delta or args.selection != "topk" or args.n_local != 1
+                     or args.fetch != "sm"
                      or args.workload != DEFAULT_WORKLOAD)
     if world == 1 and not args.no_configs and not headline_only:
         out["configs"] = run_extra_configs(args, rank, world, local_rank)

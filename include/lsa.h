@@ -188,6 +188,22 @@ int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks, const flo
                          int32_t* cu_kept, void* stream);
 
 /*
+ * lsa_threshold_chunks_capped -- lsa_threshold_chunks under a memory budget.
+ * The point of the recall step is the cut in resident KV (summary page,
+ * Abstract: the GPU KV cache shrinks by about 90%), while the threshold alone
+ * can keep any number of chunks.  With cap (device int32 [B], each >= 0):
+ * when more than cap[b] candidates pass the threshold, the cap[b] best passing
+ * chunks are kept (score descending, chunk index ascending), plus the latest
+ * chunk; otherwise the result is lsa_threshold_chunks'.  n_kept[b] is then at
+ * most cap[b] + 1, so buffers sized for the budget suffice.  cap == NULL is
+ * lsa_threshold_chunks.  Device errors as lsa_threshold_chunks, plus
+ * BAD_COUNT for a negative cap (that sequence keeps nothing).
+ */
+int lsa_threshold_chunks_capped(const float* scores, const int32_t* n_chunks, const float* w, float threshold,
+                                const int32_t* cap, int B, int max_chunks, int max_kept, int32_t* kept,
+                                int32_t* n_kept, int32_t* cu_kept, void* stream);
+
+/*
  * lsa_gather_chunks -- copy every kept chunk from the device KV pools into the
  * compact buffers, bit for bit: for i = cu_kept[b] + j,
  *   k_buf[g][i] = k_pool[slot(b, kept[b*max_kept + j])][g] for every KV head g, same for V.
@@ -220,6 +236,38 @@ int lsa_fetch_from_host(const void* host_k_pool, const void* host_v_pool, int64_
                         const int32_t* chunk_table, const int32_t* kept, const int32_t* cu_kept,
                         int B, int max_chunks, int max_kept, void* k_buf, void* v_buf,
                         int64_t buf_chunks, int num_ctas, void* stream, void* done_event);
+
+/*
+ * lsa_fetch_from_host_copy -- the same copy as lsa_fetch_from_host, through
+ * the GPU's copy engines instead of SM threads (host-to-device prefetch over
+ * the host link, handbook page, "The Neural Memory Indexer", item 3 and its
+ * closing paragraph on PCIe/NVLink bandwidth).  The copies are planned on the
+ * host, so the selection must be there: kept_host and cu_kept_host are host
+ * int32 copies of kept [B][max_kept] and cu_kept [B+1] (for instance one small
+ * device-to-host copy after lsa_topk_chunks), and chunk_table_host a host copy
+ * of the chunk table or NULL.  Each kept chunk is one cudaMemcpy2DAsync per K
+ * and V (its 8 head tiles of 16 KiB into the head-major compact buffer); a run
+ * of 8 or more chunks adjacent in the pool takes 8 per-head copies instead.
+ * The call returns once every copy is enqueued on `stream`; done_event, when
+ * given, is recorded after them.  Unlike lsa_fetch_from_host it cannot be
+ * captured in a CUDA graph with a selection that changes (the copies depend on
+ * host data).  Host errors: LSA_ERR_INVALID_ARG for a count, chunk index or
+ * slot out of range (checked before any copy), LSA_ERR_NOT_PINNED.
+ */
+int lsa_fetch_from_host_copy(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                             const int32_t* chunk_table_host, const int32_t* kept_host,
+                             const int32_t* cu_kept_host, int B, int max_chunks, int max_kept, void* k_buf,
+                             void* v_buf, int64_t buf_chunks, void* stream, void* done_event);
+
+/*
+ * lsa_debug_fail_fetch -- host-side fault injection for the host tier: the
+ * next `calls` calls of lsa_fetch_from_host, lsa_fetch_from_host_delta and
+ * lsa_fetch_from_host_copy return `status` (a negative lsa_status, normally
+ * LSA_ERR_CUDA: a failed transfer) after their argument checks, without
+ * touching the device.  calls = 0 disarms it.  Process-wide; for tests of the
+ * caller's error handling.  Not part of the decode path.
+ */
+int lsa_debug_fail_fetch(int calls, int status);
 
 /* Flags of lsa_sparse_decode_attn. */
 /* The kernel that ran just before this call on `stream` did not write k_buf,

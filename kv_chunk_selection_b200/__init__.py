@@ -66,9 +66,12 @@ def _load():
         "lsa_gather_tokens": ([P, P, I64, P, P, P, I, I, P, P, I64, P, P], I),
         "lsa_sparse_decode_attn_local": ([P, P, P, I64, P, I, F, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
+        "lsa_threshold_chunks_capped": ([P, P, P, F, P, I, I, I, P, P, P, P], I),
         "lsa_gather_chunks": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P], I),
         "lsa_fetch_from_host": ([P, P, I64, P, P, P, I, I, I, P, P, I64, I, P, P], I),
         "lsa_fetch_from_host_delta": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P, P, I, P, P, I64, P, I, P, P], I),
+        "lsa_fetch_from_host_copy": ([P, P, I64, P, P, P, I, I, I, P, P, I64, P, P], I),
+        "lsa_debug_fail_fetch": ([I, I], I),
         "lsa_attn_workspace_size": ([I], S),
         "lsa_sparse_decode_attn": ([P, P, P, I64, P, I, F, P, P, S, ctypes.c_uint, P], I),
         "lsa_sparse_decode_attn_noalloc": ([P, P, P, I64, P, I, F, P, P], I),
@@ -177,8 +180,11 @@ def lsa_topk_chunks(scores, n_chunks, k_per_seq, kept, n_kept, cu_kept, stream=N
         _ptr(n_kept), _ptr(cu_kept), _stream(stream)))
 
 
-def lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu_kept, threshold=0.5, stream=None):
-    """Sigmoid-threshold selection: chunks with score / sum(w) > threshold, plus the latest, ascending."""
+def lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu_kept, threshold=0.5, stream=None, cap=None):
+    """Sigmoid-threshold selection: chunks with score / sum(w) > threshold, plus the latest, ascending.
+
+    ``cap`` (int32 [B], optional) is a per-sequence budget: when more chunks
+    pass, the ``cap[b]`` best passing chunks are kept (lsa_threshold_chunks_capped)."""
     _need(scores, "scores", torch.float32)
     _need(w, "w", torch.float32)
     for t, n in ((n_chunks, "n_chunks"), (kept, "kept"), (n_kept, "n_kept"), (cu_kept, "cu_kept")):
@@ -187,8 +193,12 @@ def lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu_kept, threshold=0
     max_kept = kept.shape[1]
     if kept.shape[0] != B or cu_kept.numel() != B + 1 or n_kept.numel() != B:
         raise ValueError("bad shapes")
-    _check("lsa_threshold_chunks", _load().lsa_threshold_chunks(
-        _ptr(scores), _ptr(n_chunks), _ptr(w), float(threshold), B, max_chunks, max_kept, _ptr(kept),
+    if cap is not None:
+        _need(cap, "cap", torch.int32)
+        if cap.numel() != B:
+            raise ValueError("cap must have one entry per sequence")
+    _check("lsa_threshold_chunks_capped", _load().lsa_threshold_chunks_capped(
+        _ptr(scores), _ptr(n_chunks), _ptr(w), float(threshold), _ptr(cap), B, max_chunks, max_kept, _ptr(kept),
         _ptr(n_kept), _ptr(cu_kept), _stream(stream)))
 
 
@@ -255,6 +265,38 @@ def lsa_fetch_from_host_delta(host_k_pool, host_v_pool, chunk_table, kept, cu_ke
         B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"), _ptr(prev_kept),
         _ptr(prev_cu_kept), prev_kept.shape[1], _ptr(prev_k_buf), _ptr(prev_v_buf), _buf_chunks(prev_k_buf, "prev_k_buf"),
         _ptr(reused_chunks), int(num_ctas), _stream(stream), ev))
+
+
+def lsa_fetch_from_host_copy(host_k_pool, host_v_pool, chunk_table_host, kept_host, cu_kept_host, max_chunks, k_buf,
+                             v_buf, stream=None, done_event: Optional[torch.cuda.Event] = None):
+    """lsa_fetch_from_host through the copy engines: the selection (kept_host
+    [B, max_kept], cu_kept_host [B+1], chunk_table_host [B, max_chunks] or None)
+    is read on the host, and each kept chunk is one 2-D copy per K and V."""
+    for t, n in ((host_k_pool, "host_k_pool"), (host_v_pool, "host_v_pool")):
+        _need(t, n, torch.bfloat16, cuda=False)
+    for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((kept_host, "kept_host"), (cu_kept_host, "cu_kept_host")):
+        _need(t, n, torch.int32, cuda=False)
+    if chunk_table_host is not None:
+        _need(chunk_table_host, "chunk_table_host", torch.int32, cuda=False)
+    B, max_kept = kept_host.shape
+    if cu_kept_host.numel() != B + 1:
+        raise ValueError("cu_kept_host must have B + 1 entries")
+    ev = None
+    if done_event is not None:
+        if not done_event.cuda_event:
+            done_event.record(stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream())
+        ev = ctypes.c_void_p(done_event.cuda_event)
+    _check("lsa_fetch_from_host_copy", _load().lsa_fetch_from_host_copy(
+        _ptr(host_k_pool), _ptr(host_v_pool), host_k_pool.shape[0], _ptr(chunk_table_host), _ptr(kept_host),
+        _ptr(cu_kept_host), B, int(max_chunks), max_kept, _ptr(k_buf), _ptr(v_buf), _buf_chunks(k_buf, "k_buf"),
+        _stream(stream), ev))
+
+
+def lsa_debug_fail_fetch(calls: int, status: int = -4):
+    """Host-side fault injection: the next ``calls`` host-tier fetch calls fail with ``status``."""
+    _check("lsa_debug_fail_fetch", _load().lsa_debug_fail_fetch(int(calls), int(status)))
 
 
 def lsa_attn_workspace_size(B: int) -> int:
@@ -455,7 +497,8 @@ def lsa_sparse_decode_attn_noalloc(q, k_buf, v_buf, cu_kept, out, softmax_scale=
 __all__ = [
     "LsaError", "lib", "read_device_status", "decode_status", "lsa_index_score", "lsa_topk_chunks",
     "lsa_threshold_chunks",
-    "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_attn_workspace_size", "new_attn_workspace",
+    "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_fetch_from_host_copy",
+    "lsa_debug_fail_fetch", "lsa_attn_workspace_size", "new_attn_workspace", "lsa_threshold_chunks",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token", "lsa_reset_local",
     "lsa_token_score", "lsa_topk_tokens", "lsa_gather_tokens", "lsa_sparse_decode_attn_append",
     "lsa_sparse_decode_attn_selected",

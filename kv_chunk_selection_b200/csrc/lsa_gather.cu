@@ -22,6 +22,9 @@
 // a decoded token into a sequence's local chunk, and lsa_reset_local empties
 // the local chunks. lsa_gather_tokens packs the fine stage's selected tokens
 // into dense units.
+#include <atomic>
+#include <vector>
+
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
@@ -253,6 +256,20 @@ int lsa_gather_chunks(const void* k_pool, const void* v_pool, int64_t n_slots, c
 }  // extern "C"
 
 namespace {
+// Host-side fault injection of the fetch (lsa_debug_fail_fetch): the next
+// g_fetch_fail_calls fetch calls return g_fetch_fail_status after their
+// argument checks, before anything touches the device.
+std::atomic<int> g_fetch_fail_calls{0};
+std::atomic<int> g_fetch_fail_status{LSA_ERR_CUDA};
+
+int injected_fetch_failure() {
+  int n = g_fetch_fail_calls.load();
+  while (n > 0) {
+    if (g_fetch_fail_calls.compare_exchange_weak(n, n - 1)) return g_fetch_fail_status.load();
+  }
+  return LSA_OK;
+}
+
 int fetch_impl(const void* host_k_pool, const void* host_v_pool, int64_t n_slots, const int32_t* chunk_table,
                const int32_t* kept, const int32_t* cu_kept, int B, int max_chunks, int max_kept, void* k_buf,
                void* v_buf, int64_t buf_chunks, int num_ctas, void* stream, void* done_event,
@@ -261,6 +278,7 @@ int fetch_impl(const void* host_k_pool, const void* host_v_pool, int64_t n_slots
   const int st = gather::check_common(host_k_pool, host_v_pool, n_slots, kept, cu_kept, B, max_chunks, max_kept,
                                       k_buf, v_buf, buf_chunks);
   if (st != LSA_OK) return st;
+  if (const int inj = injected_fetch_failure()) return inj;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   // The pools must be page-locked host memory; use their device aliases.
   void* dk = nullptr;
@@ -363,6 +381,117 @@ int lsa_reset_local(int32_t* local_len, int B, void* stream) {
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   if (cudaMemsetAsync(local_len, 0, sizeof(int32_t) * static_cast<size_t>(B), static_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// lsa_fetch_from_host_copy: the host-tier fetch through the copy engines.  The
+// kept list is read on the host, and every kept chunk becomes one 2-D copy per
+// K and V: 8 rows (its KV heads) of 16 KiB, from its pool slot (rows 16 KiB
+// apart) to its column of the head-major compact buffer (rows buf_chunks *
+// 16 KiB apart).  A run of at least 8 chunks that are adjacent both in the
+// pool and in the buffer is copied per head instead (one 2-D copy of the run's
+// tiles of that head), which takes fewer calls.  Nothing runs on the SMs.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kRunPerHead = 8;   // a run this long takes 8 per-head copies instead of 1 per chunk
+
+cudaError_t copy_run(const uint8_t* pool, uint8_t* buf, int64_t slot0, int64_t c0, int r, int64_t buf_chunks,
+                     cudaStream_t s) {
+  const size_t tile = lsa::kTileBytes;                        // one (chunk, KV head) tile
+  const size_t slot_bytes = tile * lsa::kNumKVHeads;
+  if (r >= kRunPerHead) {
+    for (int g = 0; g < lsa::kNumKVHeads; ++g) {
+      const cudaError_t e = cudaMemcpy2DAsync(buf + (g * buf_chunks + c0) * tile, tile,
+                                              pool + slot0 * slot_bytes + g * tile, slot_bytes, tile, r,
+                                              cudaMemcpyHostToDevice, s);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  for (int i = 0; i < r; ++i) {
+    const cudaError_t e = cudaMemcpy2DAsync(buf + (c0 + i) * tile, buf_chunks * tile,
+                                            pool + (slot0 + i) * slot_bytes, tile, tile, lsa::kNumKVHeads,
+                                            cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+}  // namespace
+
+extern "C" {
+
+int lsa_debug_fail_fetch(int calls, int status) {
+  if (calls < 0 || status >= 0 || status < LSA_ERR_NO_DEVICE) return LSA_ERR_INVALID_ARG;
+  g_fetch_fail_status.store(status);
+  g_fetch_fail_calls.store(calls);
+  return LSA_OK;
+}
+
+int lsa_fetch_from_host_copy(const void* host_k_pool, const void* host_v_pool, int64_t n_slots,
+                             const int32_t* chunk_table_host, const int32_t* kept_host, const int32_t* cu_kept_host,
+                             int B, int max_chunks, int max_kept, void* k_buf, void* v_buf, int64_t buf_chunks,
+                             void* stream, void* done_event) {
+  using namespace lsa;
+  if (!host_k_pool || !host_v_pool || !kept_host || !cu_kept_host || !k_buf || !v_buf || B <= 0 ||
+      max_chunks <= 0 || max_kept <= 0 || n_slots <= 0 || buf_chunks <= 0)
+    return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(host_k_pool) || !aligned16(host_v_pool) || !aligned16(k_buf) || !aligned16(v_buf))
+    return LSA_ERR_MISALIGNED;
+  // The selection, read on the host: every count and slot is checked before
+  // the first copy is issued.
+  if (cu_kept_host[0] != 0 || cu_kept_host[B] > buf_chunks) return LSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b) {
+    const int n = cu_kept_host[b + 1] - cu_kept_host[b];
+    if (n < 0 || n > max_kept) return LSA_ERR_INVALID_ARG;
+    for (int j = 0; j < n; ++j) {
+      const int c = kept_host[static_cast<int64_t>(b) * max_kept + j];
+      if (c < 0 || c >= max_chunks) return LSA_ERR_INVALID_ARG;
+      const int64_t slot = chunk_table_host ? chunk_table_host[static_cast<int64_t>(b) * max_chunks + c]
+                                            : static_cast<int64_t>(b) * max_chunks + c;
+      if (slot < 0 || slot >= n_slots) return LSA_ERR_INVALID_ARG;
+    }
+  }
+  if (const int inj = injected_fetch_failure()) return inj;
+  if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  cudaPointerAttributes ak, av;
+  if (cudaPointerGetAttributes(&ak, host_k_pool) != cudaSuccess ||
+      cudaPointerGetAttributes(&av, host_v_pool) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_NOT_PINNED;
+  }
+  if (ak.type != cudaMemoryTypeHost || av.type != cudaMemoryTypeHost) return LSA_ERR_NOT_PINNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* pk = static_cast<const uint8_t*>(host_k_pool);
+  const uint8_t* pv = static_cast<const uint8_t*>(host_v_pool);
+  uint8_t* bk = static_cast<uint8_t*>(k_buf);
+  uint8_t* bv = static_cast<uint8_t*>(v_buf);
+  for (int b = 0; b < B; ++b) {
+    const int c0 = cu_kept_host[b], n = cu_kept_host[b + 1] - c0;
+    const int32_t* kb = kept_host + static_cast<int64_t>(b) * max_kept;
+    auto slot_of = [&](int j) -> int64_t {
+      return chunk_table_host ? chunk_table_host[static_cast<int64_t>(b) * max_chunks + kb[j]]
+                              : static_cast<int64_t>(b) * max_chunks + kb[j];
+    };
+    for (int j = 0; j < n;) {
+      const int64_t s0 = slot_of(j);
+      int r = 1;
+      while (j + r < n && slot_of(j + r) == s0 + r) ++r;   // adjacent in the pool (and in the buffer)
+      if (copy_run(pk, bk, s0, c0 + j, r, buf_chunks, s) != cudaSuccess ||
+          copy_run(pv, bv, s0, c0 + j, r, buf_chunks, s) != cudaSuccess) {
+        cudaGetLastError();
+        return LSA_ERR_CUDA;
+      }
+      j += r;
+    }
+  }
+  if (done_event && cudaEventRecord(static_cast<cudaEvent_t>(done_event), s) != cudaSuccess) {
     cudaGetLastError();
     return LSA_ERR_CUDA;
   }

@@ -90,21 +90,27 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
 
 constexpr int kMaxPerThread = 16;   // candidates kept in registers per thread (N <= 16384)
 
+// Key of candidate i: the descending key of its score.
+struct ScoreKey {
+  const float* sc;
+  __device__ __forceinline__ uint32_t operator()(int i) const { return desc_key(__ldg(sc + i)); }
+};
+
 // Selects the kc smallest keys among candidates 0..cand-1 (kc < cand) and
 // writes their indices in ascending order to out[0..kc).  Thread t owns the
 // contiguous candidates [t*per, (t+1)*per); with kCached their keys live in
-// registers for all passes, otherwise they are re-read from the scores.
-template <bool kCached>
-__device__ void select_and_write(const float* __restrict__ sc, int cand, int kc, int per, int32_t* __restrict__ out,
+// registers for all passes, otherwise they are re-read through key_at.
+template <bool kCached, class KeyAt>
+__device__ void select_and_write(KeyAt key_at, int cand, int kc, int per, int32_t* __restrict__ out,
                                  int* hist, int* warp_sums, int* sel) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int lo = min(cand, tid * per), hi = min(cand, lo + per);
   uint32_t kr[kCached ? kMaxPerThread : 1];
   if (kCached) {
 #pragma unroll
-    for (int e = 0; e < kMaxPerThread; ++e) kr[e] = (lo + e < hi) ? desc_key(__ldg(sc + lo + e)) : 0u;
+    for (int e = 0; e < kMaxPerThread; ++e) kr[e] = (lo + e < hi) ? key_at(lo + e) : 0u;
   }
-  auto key_of = [&](int e) -> uint32_t { return kCached ? kr[e] : desc_key(__ldg(sc + lo + e)); };
+  auto key_of = [&](int e) -> uint32_t { return kCached ? kr[e] : key_at(lo + e); };
   const int n_own = hi - lo;
 
   // Bits shared by every candidate key need no pass: start below the highest
@@ -279,12 +285,12 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   }
   for (int i = tid; i < n_rec; i += kThreads) out[kc + i] = cand + i;
   if (kc == 0) return;
-  const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
+  const ScoreKey key{scores + static_cast<int64_t>(b) * max_chunks};
   const int per = (cand + kThreads - 1) / kThreads;
   if (per <= kMaxPerThread)
-    select_and_write<true>(sc, cand, kc, per, out, hist, warp_sums, sel);
+    select_and_write<true>(key, cand, kc, per, out, hist, warp_sums, sel);
   else
-    select_and_write<false>(sc, cand, kc, per, out, hist, warp_sums, sel);
+    select_and_write<false>(key, cand, kc, per, out, hist, warp_sums, sel);
 }
 
 // ---- cluster variant ------------------------------------------------------
@@ -570,11 +576,26 @@ extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, con
 namespace lsa {
 namespace topk {
 
+// Key of candidate i for the capped threshold rule: a chunk that passes the
+// threshold keeps its descending score key; one that does not gets the largest
+// key, which only NaN scores share (and NaN never passes), so every passing
+// chunk ranks before every other one.
+struct PassKey {
+  const float* sc;
+  float wsum, threshold;
+  __device__ __forceinline__ uint32_t operator()(int i) const {
+    const float s = __ldg(sc + i);
+    return (s / wsum > threshold) ? desc_key(s) : 0xffffffffu;
+  }
+};
+
 __global__ void __launch_bounds__(kThreads)
 threshold_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
-                 const float* __restrict__ w, float threshold, int max_chunks, int max_kept,
-                 int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, unsigned* status) {
+                 const float* __restrict__ w, float threshold, const int32_t* __restrict__ cap, int max_chunks,
+                 int max_kept, int32_t* __restrict__ kept, int32_t* __restrict__ n_kept, unsigned* status) {
   __shared__ int warp_sums[32];
+  __shared__ int hist[256];
+  __shared__ int sel[2];
   griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
   griddep_wait();                 // the previous kernel on the stream has finished
   const int b = blockIdx.x, tid = threadIdx.x;
@@ -598,11 +619,33 @@ threshold_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n
   for (int i = lo; i < hi; ++i) cnt += (__ldg(sc + i) / wsum > threshold);
   int total = 0;
   int pos = block_exclusive_scan(cnt, warp_sums, &total);
-  if (total + 1 > max_kept) {
+  const int cap_b = cap ? __ldg(cap + b) : total;
+  if (cap_b < 0) {
+    if (tid == 0) { n_kept[b] = 0; set_status(status, LSA_DEV_ERR_BAD_COUNT); }
+    return;
+  }
+  if (min(total, cap_b) + 1 > max_kept) {
     if (tid == 0) { n_kept[b] = 0; set_status(status, LSA_DEV_ERR_CAPACITY); }
     return;
   }
   int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
+  if (total > cap_b) {
+    // More chunks pass than the budget allows: keep the cap_b best passing
+    // chunks (score descending, chunk index ascending), in index order.
+    if (cap_b > 0) {
+      const PassKey key{sc, wsum, threshold};
+      const int per_t = (cand + kThreads - 1) / kThreads;
+      if (per_t <= kMaxPerThread)
+        select_and_write<true>(key, cand, cap_b, per_t, out, hist, warp_sums, sel);
+      else
+        select_and_write<false>(key, cand, cap_b, per_t, out, hist, warp_sums, sel);
+    }
+    if (tid == 0) {
+      out[cap_b] = n - 1;
+      n_kept[b] = cap_b + 1;
+    }
+    return;
+  }
   for (int i = lo; i < hi; ++i)
     if (__ldg(sc + i) / wsum > threshold) out[pos++] = i;
   if (tid == 0) {
@@ -642,6 +685,14 @@ offsets_kernel(const int32_t* __restrict__ n_kept, int B, int32_t* __restrict__ 
 extern "C" int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks, const float* w, float threshold,
                                     int B, int max_chunks, int max_kept, int32_t* kept, int32_t* n_kept,
                                     int32_t* cu_kept, void* stream) {
+  return lsa_threshold_chunks_capped(scores, n_chunks, w, threshold, nullptr, B, max_chunks, max_kept, kept,
+                                     n_kept, cu_kept, stream);
+}
+
+extern "C" int lsa_threshold_chunks_capped(const float* scores, const int32_t* n_chunks, const float* w,
+                                           float threshold, const int32_t* cap, int B, int max_chunks,
+                                           int max_kept, int32_t* kept, int32_t* n_kept, int32_t* cu_kept,
+                                           void* stream) {
   using namespace lsa;
   if (!scores || !n_chunks || !w || !kept || !n_kept || !cu_kept || B <= 0 || max_chunks <= 0 || max_kept <= 0)
     return LSA_ERR_INVALID_ARG;
@@ -650,8 +701,8 @@ extern "C" int lsa_threshold_chunks(const float* scores, const int32_t* n_chunks
   if (static_cast<int64_t>(B) * max_kept >= (int64_t{1} << 31)) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  launch_pdl(false, topk::threshold_kernel, dim3(B), dim3(topk::kThreads), 0, s, scores, n_chunks, w, threshold, max_chunks,
-             max_kept, kept, n_kept, lsa_device_status_ptr());
+  launch_pdl(false, topk::threshold_kernel, dim3(B), dim3(topk::kThreads), 0, s, scores, n_chunks, w, threshold, cap,
+             max_chunks, max_kept, kept, n_kept, lsa_device_status_ptr());
   int st = launch_status();
   if (st != LSA_OK) return st;
   launch_pdl(false, topk::offsets_kernel, dim3(1), dim3(topk::kThreads), 0, s, n_kept, B, cu_kept);

@@ -32,10 +32,13 @@ class LayerWindow:
     sigmoid threshold (``selection="threshold"``, keep a chunk when its weighted
     mean probability exceeds ``threshold``).  Sizes: with top-K, ``max_kept`` =
     max_b K_b + n_local kept chunks per sequence row and the compact buffer
-    holds ``sum_b (K_b + n_local)`` chunks (an upper bound of the kept total); with the
-    threshold the kept count depends on the data, so both are sized for every
-    chunk.  With ``double_buffer`` two compact buffers alternate, so the
-    selection of the next window can be fetched while the current one is read.
+    holds ``sum_b (K_b + n_local)`` chunks (an upper bound of the kept total).
+    The threshold keeps a data-dependent number of chunks; with
+    ``threshold_cap`` (the default) it is held to the same budget, K_b best
+    passing chunks at most, so the buffers have the top-K sizes; without it
+    both are sized for every chunk.  With ``double_buffer`` two compact buffers
+    alternate, so the selection of the next window can be fetched while the
+    current one is read.
 
     ``n_local`` (top-K only) keeps the latest ``n_local`` chunks beside the K
     recalled ones.  With ``causal`` each sequence also has a local chunk of the
@@ -55,7 +58,8 @@ class LayerWindow:
 
     def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
                  max_chunks: int, device="cuda", double_buffer: bool = False, selection: str = "topk",
-                 threshold: float = 0.5, n_local: int = 1, causal: bool = False, fine_k: int = 0):
+                 threshold: float = 0.5, n_local: int = 1, causal: bool = False, fine_k: int = 0,
+                 threshold_cap: bool = True):
         self.device = torch.device(device)
         self.n_chunks = n_chunks
         self.k_per_seq = k_per_seq
@@ -69,7 +73,8 @@ class LayerWindow:
         if n_local < 1 or (n_local != 1 and selection != "topk"):
             raise ValueError("n_local must be >= 1, and above 1 only with top-K selection")
         self.n_local = int(n_local)
-        if selection == "topk":
+        self.threshold_cap = bool(threshold_cap) and selection == "threshold"
+        if selection == "topk" or self.threshold_cap:
             k_host = k_per_seq.to("cpu", torch.int64)
             self.max_kept = int(k_host.max()) + self.n_local
             self.buf_chunks = int((k_host + self.n_local).sum())
@@ -120,7 +125,8 @@ class LayerWindow:
                             self.cu_kept[buf], stream=stream, n_local=self.n_local)
         else:
             lsa_threshold_chunks(self.scores, self.n_chunks, w, self.kept[buf], self.n_kept[buf], self.cu_kept[buf],
-                                 threshold=self.threshold, stream=stream)
+                                 threshold=self.threshold, stream=stream,
+                                 cap=self.k_per_seq if self.threshold_cap else None)
 
     def gather(self, k_pool, v_pool, buf: int = 0, stream=None):
         lsa_gather_chunks(k_pool, v_pool, self.chunk_table, self.kept[buf], self.cu_kept[buf], self.max_chunks,

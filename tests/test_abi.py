@@ -124,6 +124,51 @@ def test_host_checks_sizes_and_alignment(L):
 LSA_MAX_BATCH = 4096
 
 
+def test_fetch_fault_injection_returns_the_injected_status(L):
+    """The host-side injection hook makes the host-tier fetch report a failed
+    transfer without touching the device: argument errors still come first and
+    do not use up an armed failure; after the armed calls the fetch goes on to
+    its device checks (no device here, or an address that is not page-locked)."""
+    ok = ctypes.c_void_p(0x100000)
+    fetch = (ok, ok, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, 0, None, None)
+    prev = ctypes.c_void_p(0x200000)      # the previous window's buffers: not the target's
+    delta = (ok, ok, 4, None, ok, ok, 1, 4, 2, ok, ok, 2, ok, ok, 2, prev, prev, 2, None, 0, None, None)
+    kept = (ctypes.c_int32 * 2)(0, 1)
+    cu = (ctypes.c_int32 * 2)(0, 2)
+    copy = (ok, ok, 4, None, ctypes.cast(kept, ctypes.c_void_p), ctypes.cast(cu, ctypes.c_void_p), 1, 4, 2, ok, ok,
+            2, None, None)
+    try:
+        assert L.lsa_debug_fail_fetch(3, CUDA) == OK
+        assert L.lsa_fetch_from_host(*fetch) == CUDA
+        assert L.lsa_fetch_from_host(None, *fetch[1:]) == INVALID          # argument check first, not counted
+        assert L.lsa_fetch_from_host_delta(*delta) == CUDA
+        assert L.lsa_fetch_from_host_copy(*copy) == CUDA
+        assert L.lsa_fetch_from_host(*fetch) in (NO_DEVICE, NOT_PINNED)     # disarmed after three calls
+        assert L.lsa_debug_fail_fetch(1, NOT_PINNED) == OK
+        assert L.lsa_fetch_from_host(*fetch) == NOT_PINNED
+        for calls, status in ((-1, CUDA), (1, OK), (1, 5), (1, NO_DEVICE - 1)):
+            assert L.lsa_debug_fail_fetch(calls, status) == INVALID
+    finally:
+        L.lsa_debug_fail_fetch(0, CUDA)
+
+
+def test_copy_engine_fetch_checks_the_selection_on_the_host(L):
+    ok = ctypes.c_void_p(0x100000)
+
+    def call(kept_vals, cu_vals, table=None, max_chunks=4, n_slots=4, buf=2):
+        kept = (ctypes.c_int32 * len(kept_vals))(*kept_vals)
+        cu = (ctypes.c_int32 * len(cu_vals))(*cu_vals)
+        tb = None if table is None else ctypes.cast((ctypes.c_int32 * len(table))(*table), ctypes.c_void_p)
+        return L.lsa_fetch_from_host_copy(ok, ok, n_slots, tb, ctypes.cast(kept, ctypes.c_void_p),
+                                          ctypes.cast(cu, ctypes.c_void_p), 1, max_chunks, 2, ok, ok, buf, None, None)
+
+    assert call([0, 4], [0, 2]) == INVALID                     # chunk index past max_chunks
+    assert call([0, 1], [0, 3]) == INVALID                     # more chunks than the buffer holds
+    assert call([0, 1], [1, 2]) == INVALID                     # cu_kept[0] != 0
+    assert call([0, 3], [0, 2], table=[0, 1, 2, 9]) == INVALID  # slot past n_slots
+    assert call([0, 1], [0, 2]) in (NO_DEVICE, NOT_PINNED)     # valid: on to the device checks
+
+
 @pytest.mark.skipif(not NO_GPU, reason="asserts the answer on a machine without a GPU")
 def test_no_device_answer(L):
     ok = ctypes.c_void_p(0x100000)

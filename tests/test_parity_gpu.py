@@ -195,6 +195,71 @@ def test_threshold_edge_cases():
     assert i64(n_kept).tolist()[2] == 0 and i64(n_kept).tolist()[1] == 1
 
 
+def run_threshold_capped(scores, n_chunks, w, threshold, cap, max_kept):
+    B = scores.shape[0]
+    kept = torch.full((B, max_kept), -7, dtype=torch.int32, device=DEV)
+    n_kept = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_threshold_chunks(scores, n_chunks, w, kept, n_kept, cu, threshold=threshold, cap=cap)
+    return kept, n_kept, cu
+
+
+def assert_capped_matches(got, scores64, n, w64, t, cap):
+    """The oracle's capped rule on the same scores, exactly, unless a chunk lies
+    within 1e-6 (relative) of the threshold, where fp32 and fp64 may differ on
+    whether it passes."""
+    ref = oracle.threshold_chunks(scores64, n, w64, t, cap=cap)
+    wsum = float(np.sum(w64))
+    for b in range(len(n)):
+        if got[b] == list(ref[b]):
+            continue
+        near = np.abs(scores64[b, : max(int(n[b]) - 1, 0)] / wsum - t) <= 1e-6 * abs(t)
+        assert near.any(), f"seq {b}: capped selection differs with no chunk at the threshold"
+
+
+@pytest.mark.parametrize("name,t", [("128k", 0.5), ("128k", 0.6), ("batched", 0.55), ("500k", 0.5)])
+def test_threshold_capped_matches_oracle(name, t):
+    """The budget is the top-K budget K_b: at 0.5 about half the chunks pass, so
+    it binds; at 0.6 fewer pass than it allows, and the result is the plain rule."""
+    inp = workloads.make_inputs(name, DEV, pools=False, layers=1)
+    n, cap = i64(inp.n_chunks), i64(inp.k_per_seq)
+    g = score_on_gpu(inp)
+    kept, n_kept, cu = run_threshold_capped(g, inp.n_chunks, inp.layers[0].w, t, inp.k_per_seq, int(cap.max()) + 1)
+    status_clean()
+    got = kept_from_gpu(kept, n_kept)
+    assert all(len(got[b]) <= cap[b] + 1 for b in range(len(n)))
+    assert_capped_matches(got, f64(g), n, f64(inp.layers[0].w), t, cap)
+    assert i64(cu).tolist() == oracle.cumulative_kept(got).tolist()
+
+
+def test_threshold_capped_edge_cases():
+    """Budget 0 keeps only the latest chunk; a budget above the passing count
+    changes nothing; ties at the budget go to the lower index; 20000 candidates
+    take the path that re-reads the scores; a negative budget is BAD_COUNT."""
+    w = torch.full((16,), 0.5, device=DEV)                     # sum(w) = 8
+    N = 20001
+    n = torch.tensor([0, 1, 40, 40, 40, N, N], dtype=torch.int32, device=DEV)
+    cap = torch.tensor([3, 3, 0, 100, 5, 1500, 3000], dtype=torch.int32, device=DEV)
+    s = torch.zeros((7, N), device=DEV)
+    s[2:5, :40] = torch.linspace(0, 8, 40, device=DEV)
+    s[4, 30:36] = 7.0                                          # six equal passing scores, budget 5
+    g = torch.Generator(device=DEV).manual_seed(9)
+    s[5] = torch.rand(N, generator=g, device=DEV) * 8.0
+    s[6] = torch.floor(torch.rand(N, generator=g, device=DEV) * 16.0) * 0.5   # heavy ties
+    kept, n_kept, cu = run_threshold_capped(s, n, w, 0.5, cap, 20001)
+    status_clean()
+    got = kept_from_gpu(kept, n_kept)
+    ref = oracle.threshold_chunks(f64(s), i64(n), f64(w), 0.5, cap=i64(cap))
+    for b in range(7):
+        assert got[b] == list(ref[b]), f"seq {b}"
+    assert got[2] == [39] and got[4] == [30, 31, 36, 37, 38, 39]   # 36-38 score higher than the six ties
+    assert got[3] == list(oracle.threshold_chunks(f64(s), i64(n), f64(w), 0.5)[3])
+    assert i64(cu).tolist() == oracle.cumulative_kept(got).tolist()
+    bad = torch.tensor([3, -1, 0, 100, 5, 1500, 3000], dtype=torch.int32, device=DEV)   # on a sequence with a chunk
+    run_threshold_capped(s, n, w, 0.5, bad, 20001)
+    assert lsa.read_device_status() == 1                      # LSA_DEV_ERR_BAD_COUNT
+
+
 def test_threshold_window_attention():
     """Threshold selection feeds the same gather and attention: whole step vs the oracle."""
     inp = workloads.make_inputs("128k", DEV, layers=1, windows=1, steps=2)
@@ -732,6 +797,73 @@ def test_fetch_from_host_equals_gather():
     lsa.lsa_fetch_from_host(k_host, v_host, tab, kept, cu, M, b_k, b_v, num_ctas=16, stream=side, done_event=ev)
     torch.cuda.current_stream().wait_event(ev)
     assert torch.equal(a_k, b_k) and torch.equal(a_v, b_v)
+    status_clean()
+
+
+@pytest.mark.parametrize("table_kind", ["paged", "identity_runs"])
+def test_fetch_copy_engine_equals_gather(table_kind):
+    """The copy-engine fetch (selection read on the host, one 2-D copy per kept
+    chunk and per K/V, per-head copies for runs of adjacent slots) is byte-equal
+    to the device gather.  The identity table with a budget of most chunks makes
+    long runs of adjacent slots."""
+    if table_kind == "paged":
+        n, k, table, n_slots = paged_case(B=4, seed=19, max_chunks=30)
+    else:
+        n = np.array([40, 25, 64])
+        k = np.array([36, 3, 60])
+        table = np.zeros((3, 64), dtype=np.int32)
+        off = 0
+        for b in range(3):
+            table[b, : n[b]] = np.arange(off, off + n[b])
+            off += int(n[b])
+        n_slots = off
+        n, k = n.astype(np.int32), k.astype(np.int32)
+    B, M = table.shape
+    g = torch.Generator(device=DEV).manual_seed(13)
+    shape = (n_slots, 8, 64, 128)
+    k_dev = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    v_dev = torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
+    k_host, v_host = k_dev.cpu().pin_memory(), v_dev.cpu().pin_memory()
+    scores = torch.rand((B, M), generator=g, device=DEV)
+    n_t, k_t, tab = (torch.from_numpy(np.ascontiguousarray(x)).to(DEV) for x in (n, k, table))
+    kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
+    buf = int((k + 1).sum()) + 3
+    a_k = torch.zeros((8, buf, 64, 128), dtype=torch.bfloat16, device=DEV)
+    a_v, b_k, b_v = torch.zeros_like(a_k), torch.zeros_like(a_k), torch.zeros_like(a_k)
+    lsa.lsa_gather_chunks(k_dev, v_dev, tab, kept, cu, M, a_k, a_v)
+    side = torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    kept_h, cu_h = kept.cpu(), cu.cpu()
+    side.wait_stream(torch.cuda.current_stream())
+    lsa.lsa_fetch_from_host_copy(k_host, v_host, tab.cpu(), kept_h, cu_h, M, b_k, b_v, stream=side, done_event=ev)
+    torch.cuda.current_stream().wait_event(ev)
+    assert torch.equal(a_k, b_k) and torch.equal(a_v, b_v)
+    status_clean()
+
+
+def test_fetch_injected_failure_reaches_the_caller():
+    """An injected transfer failure comes back from the binding as an error
+    (nothing is launched), and the next fetch works."""
+    n, k, table, n_slots = paged_case(B=2, seed=21, max_chunks=12)
+    B, M = table.shape
+    g = torch.Generator(device=DEV).manual_seed(14)
+    k_dev = torch.randn((n_slots, 8, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    k_host = k_dev.cpu().pin_memory()
+    scores = torch.rand((B, M), generator=g, device=DEV)
+    n_t, k_t, tab = (torch.from_numpy(x).to(DEV) for x in (n, k, table))
+    kept, n_kept, cu = run_topk(scores, n_t, k_t, int(k.max()) + 1)
+    buf = int((k + 1).sum())
+    a_k = torch.zeros((8, buf, 64, 128), dtype=torch.bfloat16, device=DEV)
+    b_k, b_v = torch.zeros_like(a_k), torch.zeros_like(a_k)
+    lsa.lsa_gather_chunks(k_dev, k_dev, tab, kept, cu, M, a_k, torch.zeros_like(a_k))
+    lsa.lsa_debug_fail_fetch(1, -4)
+    with pytest.raises(lsa.LsaError) as err:
+        lsa.lsa_fetch_from_host(k_host, k_host, tab, kept, cu, M, b_k, b_v)
+    assert err.value.status == -4
+    assert torch.count_nonzero(b_k) == 0
+    lsa.lsa_fetch_from_host(k_host, k_host, tab, kept, cu, M, b_k, b_v)
+    torch.cuda.synchronize()
+    assert torch.equal(a_k, b_k)
     status_clean()
 
 
