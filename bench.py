@@ -631,6 +631,7 @@ def run_ours(args, rank, world, local_rank):
                      "attention_64_steps": att_s / args.steps * 1e6},
         "gpu_launches": args.steps * layers * (3 + workloads.TAU * (ATTN_LAUNCHES +
                                                                     (2 + int(args.causal)) * bool(args.fine_k))),
+        # (the fine step's selection is two kernels either way: scorer + top-k, or scorer + bin-driven selection)
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -711,6 +712,8 @@ def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=
         "topk_tokens": lambda: lsa.lsa_topk_tokens(lw.tok_scores, lw.n_tokens, lw.fine_k, lw.sel, lw.n_sel,
                                                    lw.cu_sel),
     }
+    if lw.fused_select:   # the step's selection call: scorer with bin counts, then the bin-driven selection
+        calls["select_tokens"] = lambda: lw.fine_select(q_tok[0, 0], L.w, keys)
     if lw.packs:
         calls["gather_tokens"] = lambda: lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], lw.sel,
                                                                lw.cu_sel, lw.k_fine, lw.v_fine, lw.cu_units)
@@ -727,6 +730,7 @@ def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=
     # that copies them from the compact buffer itself)
     nbytes = {"token_score": tokens * 256 + B * 16 * 128 * 2 + tokens * 4,
               "topk_tokens": tokens * 4 + fine_total * 4,
+              "select_tokens": tokens * 256 + B * 16 * 128 * 2 + tokens * 4 + fine_total * 4,
               "gather_tokens": 2 * fine_total * TOKEN_KV_BYTES,
               "attention": fine_total * TOKEN_KV_BYTES + B * (64 * 128 * 2 + 64 * 128 * 4)}
     for name, fn in calls.items():

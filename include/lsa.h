@@ -474,7 +474,8 @@ int lsa_sparse_decode_attn_append(const void* q, const void* k_buf, const void* 
  * Architecture; k = 2048 tokens for the DSA lightning indexer on the search
  * page "lightning indexer").  Every decode step:
  *   lsa_token_score   -> one score per token of the recalled chunks,
- *   lsa_topk_tokens   -> the k best token positions,
+ *   lsa_topk_tokens   -> the k best token positions
+ *                        (or both in one call: lsa_select_tokens),
  *   lsa_sparse_decode_attn_selected -> attention over those tokens, whose
  *                        rows it reads in place from the compact buffer.
  * A causal step (lsa_sparse_decode_attn_append, which attends whole units)
@@ -517,6 +518,36 @@ int lsa_token_score(const void* q_idx, const float* w, const void* token_keys, i
  */
 int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int k, int B, int max_tokens,
                     int max_sel, int32_t* sel, int32_t* n_sel, int32_t* cu_sel, void* stream);
+
+/*
+ * lsa_select_tokens -- lsa_token_score followed by lsa_topk_tokens in one
+ * call, with the same outputs bit for bit (scores, n_tokens, sel, n_sel,
+ * cu_sel; arguments as those two calls, k and max_sel as for lsa_topk_tokens).
+ * The scorer also counts each sequence's scores in 4096 bins of equal width
+ * over [0, sum_h w[h]), so the selection knows the bin of the k-th best score
+ * before it reads a score again: a cluster of 8 CTAs per sequence reads every
+ * score once, keeps the tokens above that bin and ranks the few inside it
+ * exactly.  Inputs where that does not pay (many tokens in one bin, ties
+ * everywhere, more than 131072 tokens in a sequence) take the exact radix
+ * select of lsa_topk_tokens inside the same launch.  The counts take the
+ * scorer shared memory, which pays only when its grid (B * max_kept / 2 CTAs)
+ * fits in one wave of 4 CTAs per SM; larger batches run lsa_token_score and
+ * lsa_topk_tokens instead (the workspace is then not touched).  Two kernels
+ * either way, both programmatic dependents of their predecessor.
+ *   workspace  device, >= lsa_select_tokens_workspace_size(B) bytes (64 KiB
+ *              per sequence: 4 copies of the counts, so fewer of the scorer's
+ *              atomic adds meet on one address), 16-byte aligned, zero before the first call
+ *              (zero it once when it is allocated): the bin counts; every
+ *              call leaves it zero again.  Calls that may overlap on the GPU
+ *              need workspaces of their own.
+ * Device errors as lsa_token_score and lsa_topk_tokens.
+ */
+size_t lsa_select_tokens_workspace_size(int B);
+int lsa_select_tokens(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                      const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
+                      int max_chunks, int max_kept, int k, float* scores, int32_t* n_tokens, int32_t* sel,
+                      int32_t* n_sel, int32_t* cu_sel, int max_sel, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 /*
  * lsa_gather_tokens -- pack the selected tokens into dense units, bit for bit:

@@ -63,6 +63,8 @@ def _load():
         "lsa_sparse_decode_attn_selected": ([P, P, P, I64, P, P, P, I, I, F, P, P, S, ctypes.c_uint, P], I),
         "lsa_token_score": ([P, P, P, I64, P, P, P, I, I, I, P, P, P], I),
         "lsa_topk_tokens": ([P, P, I, I, I, I, P, P, P, P], I),
+        "lsa_select_tokens_workspace_size": ([I], S),
+        "lsa_select_tokens": ([P, P, P, I64, P, P, P, I, I, I, I, P, P, P, P, P, I, P, S, P], I),
         "lsa_gather_tokens": ([P, P, I64, P, P, P, I, I, P, P, I64, P, P], I),
         "lsa_sparse_decode_attn_local": ([P, P, P, I64, P, I, F, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
@@ -411,6 +413,41 @@ def lsa_topk_tokens(scores, n_tokens, k, sel, n_sel, cu_sel, stream=None):
         _stream(stream)))
 
 
+def new_select_tokens_workspace(B: int, device=None) -> torch.Tensor:
+    """The bin-count workspace of lsa_select_tokens, zeroed (every call leaves it zero)."""
+    n = int(_load().lsa_select_tokens_workspace_size(int(B)))
+    if n == 0:
+        raise ValueError("unsupported batch")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def lsa_select_tokens(q_idx, w, token_keys, chunk_table, kept, n_kept, max_chunks, k, scores, n_tokens, sel, n_sel,
+                      cu_sel, workspace, stream=None):
+    """lsa_token_score then lsa_topk_tokens in one call (same outputs), the
+    selection driven by the scorer's score-bin counts."""
+    _need(q_idx, "q_idx", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(token_keys, "token_keys", torch.bfloat16)
+    for t, n in ((kept, "kept"), (n_kept, "n_kept"), (n_tokens, "n_tokens"), (sel, "sel"), (n_sel, "n_sel"),
+                 (cu_sel, "cu_sel")):
+        _need(t, n, torch.int32)
+    _need(scores, "scores", torch.float32)
+    _need(workspace, "workspace", torch.uint8)
+    if chunk_table is not None:
+        _need(chunk_table, "chunk_table", torch.int32)
+    B, max_kept = kept.shape
+    if tuple(q_idx.shape) != (B, INDEX_HEADS, INDEX_DIM) or tuple(scores.shape) != (B, CHUNK_TOKENS * max_kept):
+        raise ValueError("q_idx must be [B, 16, 128] and scores [B, 64 * max_kept]")
+    if token_keys.dim() != 3 or tuple(token_keys.shape[1:]) != (CHUNK_TOKENS, INDEX_DIM):
+        raise ValueError("token_keys must be [n_slots, 64, 128]")
+    if sel.dim() != 2 or sel.shape[0] != B or cu_sel.numel() != B + 1 or n_sel.numel() != B:
+        raise ValueError("sel must be [B, max_sel], n_sel [B] and cu_sel [B + 1]")
+    _check("lsa_select_tokens", _load().lsa_select_tokens(
+        _ptr(q_idx), _ptr(w), _ptr(token_keys), token_keys.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(n_kept), B,
+        int(max_chunks), max_kept, int(k), _ptr(scores), _ptr(n_tokens), _ptr(sel), _ptr(n_sel), _ptr(cu_sel),
+        sel.shape[1], _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
 def lsa_gather_tokens(k_buf, v_buf, cu_kept, sel, cu_sel, k_out, v_out, cu_units, stream=None):
     """Packs the selected tokens into dense 64-token units (the attention's compact layout)."""
     for t, n in ((k_buf, "k_buf"), (v_buf, "v_buf"), (k_out, "k_out"), (v_out, "v_out")):
@@ -500,7 +537,7 @@ __all__ = [
     "lsa_gather_chunks", "lsa_fetch_from_host", "lsa_fetch_from_host_delta", "lsa_fetch_from_host_copy",
     "lsa_debug_fail_fetch", "lsa_attn_workspace_size", "new_attn_workspace", "lsa_threshold_chunks",
     "lsa_sparse_decode_attn", "lsa_sparse_decode_attn_noalloc", "lsa_append_token", "lsa_reset_local",
-    "lsa_token_score", "lsa_topk_tokens", "lsa_gather_tokens", "lsa_sparse_decode_attn_append",
+    "lsa_token_score", "lsa_topk_tokens", "lsa_select_tokens", "new_select_tokens_workspace", "lsa_gather_tokens", "lsa_sparse_decode_attn_append",
     "lsa_sparse_decode_attn_selected",
     "lsa_sparse_decode_attn_local", "NUM_Q_HEADS", "NUM_KV_HEADS", "HEAD_DIM", "CHUNK_TOKENS", "INDEX_HEADS",
     "INDEX_DIM", "CHUNK_BYTES",

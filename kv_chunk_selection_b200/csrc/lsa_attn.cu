@@ -269,10 +269,14 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 
   if (warp == kConsumerWarps && indexed) {
     // ============ producer warp, fine stage: selected rows in place ==========
-    // Each lane copies rows `lane` and `lane + 32` of the unit (K and V, 16
-    // pieces of 16 bytes each) to their swizzled places in the stage, then
-    // arrives on the stage's full barrier when its copies have landed.  A
-    // position outside the sequence's recalled tokens is written as zeros.
+    // Lane l resolves the addresses of rows l and l + 32 of the unit; then the
+    // warp copies two rows per instruction, lanes 0-15 the 16 pieces of 16
+    // bytes of one row and lanes 16-31 those of the next (each row's address
+    // taken from the lane that resolved it), so one instruction touches two
+    // 256-byte rows instead of 32 scattered pieces.  The pieces land at their
+    // swizzled places in the stage; each lane arrives on the stage's full
+    // barrier when its copies have landed.  A position outside the sequence's
+    // recalled tokens is written as zeros.
     UnitCursor cur;
     cur.start(cu, E, B, u0);
     const int64_t n_units = u1 - u0;
@@ -296,22 +300,24 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       const int64_t ckb = __ldg(sa.ck + b);
       const int64_t n_pos = (static_cast<int64_t>(__ldg(sa.ck + b + 1)) - ckb) * kChunkTokens;
       const uint32_t st = smem_base_p + s * kStageBytes;
+      int64_t row_of[2];   // rows lane and lane + 32: compact-buffer row, or -1 (zeros)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int r = lane + 32 * h;
-        const int p = __ldg(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + r);
+        const int p = __ldg(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + lane + 32 * h);
         const bool okp = p >= 0 && p < n_pos && ckb + p / kChunkTokens < sa.ck_chunks;
         if (!okp) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
-        const int64_t row = okp ? (g * sa.ck_chunks + ckb + p / kChunkTokens) * kChunkTokens + p % kChunkTokens : 0;
-        const uint4* ks = sa.k_buf + row * 16;
-        const uint4* vs = sa.v_buf + row * 16;
-        const uint32_t nb = okp ? 16u : 0u;
+        row_of[h] = okp ? (g * sa.ck_chunks + ckb + p / kChunkTokens) * kChunkTokens + p % kChunkTokens : -1;
+      }
+      const int x = lane & 15;   // this lane's 16-byte piece of its row
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const uint32_t off = (x >> 3) * kBoxBytes + r * 128 + (((x & 7) ^ (r & 7)) << 4);
-          cp_async_16_zfill(st + off, ks + x, nb);
-          cp_async_16_zfill(st + 2 * kBoxBytes + off, vs + x, nb);
-        }
+      for (int it = 0; it < kChunkTokens / 2; ++it) {
+        const int r = 2 * it + (lane >> 4);                       // the row this lane copies
+        const int64_t row = __shfl_sync(0xffffffffu, row_of[it >> 4], r & 31);   // rows 0-31 in h = 0
+        const uint32_t nb = row >= 0 ? 16u : 0u;
+        const int64_t src = row >= 0 ? row * 16 + x : 0;
+        const uint32_t off = (x >> 3) * kBoxBytes + r * 128 + (((x & 7) ^ (r & 7)) << 4);
+        cp_async_16_zfill(st + off, sa.k_buf + src, nb);
+        cp_async_16_zfill(st + 2 * kBoxBytes + off, sa.v_buf + src, nb);
       }
       cp_async_mbar_arrive_noinc(&full[s]);
       cur.advance(cu, E, B, units_of(cu, E, cur.b));

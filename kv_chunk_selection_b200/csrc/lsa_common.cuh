@@ -25,6 +25,35 @@ constexpr int kTileBytes = kTileElems * 2;  // 16 KiB
 constexpr int64_t kChunkElems = (int64_t)kNumKVHeads * kTileElems;
 static_assert(kChunkElems * 2 == LSA_CHUNK_BYTES, "chunk size");
 
+// Score bins of the token-level selection: 4096 bins of equal width over
+// [0, sum_h w_h), the range of the indexer's weighted sigmoid sum.  The token
+// scorer counts its scores per bin and the selection kernel recomputes the bin
+// of each stored score with the same fp32 expression, so both agree bit for
+// bit.  The bin is a non-decreasing function of the score (a product with a
+// positive constant, then a floor), so a token in a higher bin outscores every
+// token in a lower one.  Anything below 0 (and NaN) falls in bin 0, anything
+// at or above the top in the last bin; a scale of 0 (sum of w not positive or
+// not finite) puts every token in bin 0.
+constexpr int kScoreBins = 4096;
+// Copies of each sequence's bin counts: the scorer's CTA x adds to copy
+// x % kScoreBinReplicas, so the hot bins near the middle of the score range
+// see a quarter of the atomic adds each; the selection sums the copies.
+constexpr int kScoreBinReplicas = 4;
+
+__device__ __forceinline__ float score_bin_scale(const float* w) {
+  float wsum = 0.f;   // head order, as every kernel that needs it
+#pragma unroll
+  for (int h = 0; h < kIndexHeads; ++h) wsum += __ldg(w + h);
+  return (wsum > 0.f && wsum < 3.0e38f) ? static_cast<float>(kScoreBins) / wsum : 0.f;
+}
+
+__device__ __forceinline__ int score_bin(float s, float scale) {
+  const float x = s * scale;
+  if (!(x >= 0.f)) return 0;
+  if (x >= static_cast<float>(kScoreBins - 1)) return kScoreBins - 1;
+  return static_cast<int>(x);
+}
+
 // Upper bound of any in-kernel spin: 1 s of wall time (globaltimer, ns).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 

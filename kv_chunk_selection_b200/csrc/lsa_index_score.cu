@@ -25,6 +25,8 @@
 // over every token of the recalled chunks.  Only the row source differs: tile
 // row r is token position p = 64 j + i (token i of the j-th recalled chunk),
 // whose key row is 64 * slot(kept[j]) + i of the per-token key pool.
+#include <mutex>
+
 #include "lsa_common.cuh"
 #include "lsa_runtime.cuh"
 
@@ -37,6 +39,8 @@ constexpr int kKBlockBytes = 128;   // 64 bf16 per row per swizzle atom
 constexpr int kABytes = kTile * 2 * kKBlockBytes;          // 32 KiB: 2 K-blocks of [128 x 128 B]
 constexpr int kBBytes = kIndexHeads * 2 * kKBlockBytes;    // 4 KiB: 2 K-blocks of [16 x 128 B]
 constexpr int kSmemBytes = kABytes + kBBytes + 16 + kTile * 9;   // + barrier, TMEM slot, row addresses and flags
+constexpr int kHistOffset = (kSmemBytes + 15) / 16 * 16;         // score-bin counts of the tile (token selection)
+constexpr int kSmemBytesHist = kHistOffset + kScoreBins * 4;
 constexpr uint32_t kTmemCols = 32;  // allocation unit (>= 16 accumulator columns)
 constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kTile, kIndexHeads);
 
@@ -61,6 +65,7 @@ struct ChunkRows {
   }
   __device__ int64_t stride() const { return max_chunks; }
   __device__ void on_count(int, int) const {}
+  __device__ int32_t* hist_of(int) const { return nullptr; }
   __device__ bool key_row(int b, int c, int64_t* row, unsigned* err) const {
     const int64_t slot =
         table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
@@ -80,6 +85,11 @@ struct TokenRows {
   int max_chunks, max_kept;
   int64_t n_slots;
   int32_t* n_tokens;   // out: 64 * n_kept[b]
+  int32_t* hist;       // optional [B][kScoreBinReplicas][kScoreBins]: score-bin counts, added to (lsa_select_tokens)
+  __device__ int32_t* hist_of(int b) const {
+    return hist ? hist + (static_cast<int64_t>(b) * kScoreBinReplicas + blockIdx.x % kScoreBinReplicas) * kScoreBins
+                : nullptr;
+  }
   __device__ int count(int b) const {
     const int n = __ldg(n_kept + b);
     return (n < 0 || n > max_kept) ? -1 : n * kChunkTokens;
@@ -132,8 +142,14 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
   int64_t* row_at = reinterpret_cast<int64_t*>(smem + kABytes + kBBytes + 16);   // [kTile] key row or -1
   bool* row_ok = reinterpret_cast<bool*>(row_at + kTile);                            // [kTile]
   const int tid = threadIdx.x, warp = tid >> 5;
+  int32_t* const ghist = rows.hist_of(b);                                            // block-uniform
+  int* const shist = reinterpret_cast<int*>(smem + kHistOffset);                      // [kScoreBins] when ghist
 
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  if (ghist) {   // cleared here; the barrier before the MMA publishes it
+#pragma unroll
+    for (int i = tid; i < kScoreBins / 4; i += kThreads) reinterpret_cast<int4*>(shist)[i] = make_int4(0, 0, 0, 0);
+  }
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
@@ -208,6 +224,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
   // warp-uniform, so the .sync.aligned TMEM load below never diverges
   const bool done = __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0, &never));
   tcgen05_fence_after();
+  int bin = -1;         // this row's score bin, when it is the first of the tile in that bin
   if (!done) {
     if (tid == 0) set_status(status, LSA_DEV_ERR_TIMEOUT);
   } else {
@@ -216,11 +233,19 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     float s = 0.f;
 #pragma unroll
     for (int h = 0; h < kIndexHeads; ++h) s += __ldg(w + h) * (1.f / (1.f + fast_exp2(logit[h] * neg_scale_log2)));
-    if (row_ok[tid]) scores[static_cast<int64_t>(b) * rows.stride() + base + tid] = s;
+    if (row_ok[tid]) {
+      scores[static_cast<int64_t>(b) * rows.stride() + base + tid] = s;
+      if (ghist) {
+        const int bi = score_bin(s, score_bin_scale(w));
+        if (atomicAdd(&shist[bi], 1) == 0) bin = bi;
+      }
+    }
   }
   tcgen05_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  // One global add per bin this tile touched, by the row that touched it first.
+  if (bin >= 0) atomicAdd(ghist + bin, shist[bin]);
 }
 
 }  // namespace score
@@ -244,10 +269,13 @@ extern "C" int lsa_index_score(const void* q_idx, const float* w, const void* ch
   return launch_status();
 }
 
-extern "C" int lsa_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
-                               const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
-                               int max_chunks, int max_kept, float* scores, int32_t* n_tokens, void* stream) {
-  using namespace lsa;
+namespace lsa {
+namespace score {
+// The token scorer's launch, shared by lsa_token_score (hist == nullptr) and
+// lsa_select_tokens (hist: [B][kScoreBins] counts to add to).
+int launch_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                       const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B, int max_chunks,
+                       int max_kept, float* scores, int32_t* n_tokens, int32_t* hist, cudaStream_t stream) {
   if (!q_idx || !w || !token_keys || !kept || !n_kept || !scores || !n_tokens || B <= 0 || max_chunks <= 0 ||
       max_kept <= 0 || n_slots <= 0)
     return LSA_ERR_INVALID_ARG;
@@ -257,12 +285,38 @@ extern "C" int lsa_token_score(const void* q_idx, const float* w, const void* to
     return LSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q_idx) || !aligned16(token_keys)) return LSA_ERR_MISALIGNED;
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
+  const int smem = hist ? kSmemBytesHist : kSmemBytes;
+  if (hist) {   // the histogram needs more than the default 48 KB of dynamic shared memory
+    static std::mutex mu;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+      if (cudaFuncSetAttribute(index_score_kernel<TokenRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemBytesHist) != cudaSuccess) {
+        cudaGetLastError();
+        return LSA_ERR_CUDA;
+      }
+      attr_set[dev] = true;
+    }
+  }
   const int max_tokens = max_kept * kChunkTokens;
-  const dim3 grid((max_tokens + score::kTile - 1) / score::kTile, B);
+  const dim3 grid((max_tokens + kTile - 1) / kTile, B);
   const float neg_scale_log2 = -1.4426950408889634f / sqrtf(static_cast<float>(kIndexDim));
-  const score::TokenRows rows{chunk_table, kept, n_kept, max_chunks, max_kept, n_slots, n_tokens};
-  launch_pdl(true, score::index_score_kernel<score::TokenRows>, grid, dim3(score::kThreads), score::kSmemBytes,
-             static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(q_idx), w,
-             static_cast<const __nv_bfloat16*>(token_keys), rows, scores, neg_scale_log2, lsa_device_status_ptr());
+  TokenRows rows{chunk_table, kept, n_kept, max_chunks, max_kept, n_slots, n_tokens};
+  rows.hist = hist;
+  launch_pdl(true, index_score_kernel<TokenRows>, grid, dim3(kThreads), smem, stream,
+             static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(token_keys), rows, scores,
+             neg_scale_log2, lsa_device_status_ptr());
   return launch_status();
+}
+}  // namespace score
+}  // namespace lsa
+
+extern "C" int lsa_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                               const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
+                               int max_chunks, int max_kept, float* scores, int32_t* n_tokens, void* stream) {
+  return lsa::score::launch_token_score(q_idx, w, token_keys, n_slots, chunk_table, kept, n_kept, B, max_chunks,
+                                        max_kept, scores, n_tokens, nullptr, static_cast<cudaStream_t>(stream));
 }

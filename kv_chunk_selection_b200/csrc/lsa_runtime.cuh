@@ -56,6 +56,14 @@ inline void launch_pdl(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block
   cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+namespace score {
+// The token scorer's launch (lsa_index_score.cu); with hist != nullptr it also
+// adds each sequence's score-bin counts to hist[b][kScoreBins].
+int launch_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                       const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B, int max_chunks,
+                       int max_kept, float* scores, int32_t* n_tokens, int32_t* hist, cudaStream_t stream);
+}  // namespace score
+
 }  // namespace lsa
 
 unsigned* lsa_device_status_ptr();

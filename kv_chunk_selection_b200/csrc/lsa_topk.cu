@@ -301,14 +301,14 @@ constexpr int kClusterMaxCand = kClusterThreads * kMaxPerThread;   // 131072
 // scores every pass beyond it).
 constexpr int kClusterMinCand = kThreads * kMaxPerThread;          // 16384
 
-// kPer: register slots per thread (4, 8 or 16), the smallest that holds the
-// candidates; dead slots still cost issue slots in every pass.
+// The cluster's exact radix select: the kc smallest keys of candidates
+// 0 .. cand-1 (kc < cand, cand <= 8192 * kPer) of the scores at sc, written to
+// out[0 .. kc) in ascending index order.  Every thread of every CTA of the
+// cluster calls it; rank r's threads own the contiguous candidates
+// [gtid * per, (gtid + 1) * per), gtid = r * 1024 + thread, with their keys
+// in registers.
 template <int kPer>
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
-topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
-                    const int32_t* __restrict__ k_per_seq, int k_all, int n_local, int B, int max_chunks,
-                    int max_kept, int32_t* __restrict__ kept, int32_t* __restrict__ n_kept,
-                    int32_t* __restrict__ cu_kept, unsigned* status) {
+__device__ void cluster_select_and_write(const float* __restrict__ sc, int cand, int kc, int32_t* __restrict__ out) {
   // Two histograms, alternating between passes: pass p clears the one that
   // pass p-1's remote reads used two passes back, and the cluster barrier of
   // pass p-1 orders those reads before this clear, so a pass needs one
@@ -319,50 +319,13 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   __shared__ int sel[2];
   __shared__ uint32_t xmm[2 * kClusterCtas];   // [rank] min key, [8 + rank] max key, pushed by each rank
   __shared__ int xcnt[2 * kClusterCtas];       // [rank] keys below the boundary, [8 + rank] keys equal to it
-  griddep_wait();   // the previous kernel on the stream has finished
-  const int b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
-
-  // Counts: identical in every CTA of the cluster, written by rank 0.  Every
-  // early return below depends on them only, so the whole cluster takes it.
-  int part = 0;
-  unsigned dummy = 0;
-  for (int bb = tid; bb <= b; bb += kThreads)
-    part += kept_count(__ldg(n_chunks + bb), k_per_seq ? __ldg(k_per_seq + bb) : k_all, n_local, max_chunks,
-                       max_kept, &dummy);
-  int tot = 0;
-  block_exclusive_scan(part, warp_sums, &tot);
-  unsigned err = 0;
-  const int n = __ldg(n_chunks + b);
-  const int nk = kept_count(n, k_per_seq ? __ldg(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
-  if (rank == 0 && tid == 0) {
-    cu_kept[b + 1] = tot;
-    if (b == 0) cu_kept[0] = 0;
-    n_kept[b] = nk;
-    if (err) set_status(status, err);
-  }
-  if (nk == 0) return;
-  int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
-  const int n_rec = min(n_local, n);
-  const int cand = n - n_rec;
-  const int kc = nk - n_rec;
   const int gtid = static_cast<int>(rank) * kThreads + tid;
-  if (kc == cand) {
-    for (int c = gtid; c < n; c += kClusterThreads) out[c] = c;
-    return;
-  }
-  for (int i = gtid; i < n_rec; i += kClusterThreads) out[kc + i] = cand + i;
-  if (kc == 0) return;
   const int per = (cand + kClusterThreads - 1) / kClusterThreads;
-  if (per > kPer) {   // the host never launches this case
-    if (rank == 0 && tid == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
-    return;
-  }
-  // Past the last (cluster-uniform) return: announce this CTA to the cluster,
-  // load the keys, and wait for every CTA before the first remote store.
+  // Announce this CTA to the cluster, load the keys, and wait for every CTA
+  // before the first remote store.
   cluster_arrive_relaxed();
-  const float* sc = scores + static_cast<int64_t>(b) * max_chunks;
   const int lo = min(cand, gtid * per), hi = min(cand, lo + per);
   const int n_own = hi - lo;
   uint32_t kr[kPer];
@@ -502,6 +465,283 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
     if (take[e]) out[pos++] = lo + e;
 }
 
+
+// kPer: register slots per thread (4, 8 or 16), the smallest that holds the
+// candidates; dead slots still cost issue slots in every pass.
+template <int kPer>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads)
+topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chunks,
+                    const int32_t* __restrict__ k_per_seq, int k_all, int n_local, int B, int max_chunks,
+                    int max_kept, int32_t* __restrict__ kept, int32_t* __restrict__ n_kept,
+                    int32_t* __restrict__ cu_kept, unsigned* status) {
+  __shared__ int warp_sums[32];
+  griddep_wait();   // the previous kernel on the stream has finished
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x;
+  const uint32_t rank = cluster_ctarank();
+
+  // Counts: identical in every CTA of the cluster, written by rank 0.  Every
+  // early return below depends on them only, so the whole cluster takes it.
+  int part = 0;
+  unsigned dummy = 0;
+  for (int bb = tid; bb <= b; bb += kThreads)
+    part += kept_count(__ldg(n_chunks + bb), k_per_seq ? __ldg(k_per_seq + bb) : k_all, n_local, max_chunks,
+                       max_kept, &dummy);
+  int tot = 0;
+  block_exclusive_scan(part, warp_sums, &tot);
+  unsigned err = 0;
+  const int n = __ldg(n_chunks + b);
+  const int nk = kept_count(n, k_per_seq ? __ldg(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
+  if (rank == 0 && tid == 0) {
+    cu_kept[b + 1] = tot;
+    if (b == 0) cu_kept[0] = 0;
+    n_kept[b] = nk;
+    if (err) set_status(status, err);
+  }
+  if (nk == 0) return;
+  int32_t* out = kept + static_cast<int64_t>(b) * max_kept;
+  const int n_rec = min(n_local, n);
+  const int cand = n - n_rec;
+  const int kc = nk - n_rec;
+  const int gtid = static_cast<int>(rank) * kThreads + tid;
+  if (kc == cand) {
+    for (int c = gtid; c < n; c += kClusterThreads) out[c] = c;
+    return;
+  }
+  for (int i = gtid; i < n_rec; i += kClusterThreads) out[kc + i] = cand + i;
+  if (kc == 0) return;
+  const int per = (cand + kClusterThreads - 1) / kClusterThreads;
+  if (per > kPer) {   // the host never launches this case
+    if (rank == 0 && tid == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
+    return;
+  }
+  cluster_select_and_write<kPer>(scores + static_cast<int64_t>(b) * max_chunks, cand, kc, out);
+}
+
+// ---- token selection from the scorer's score-bin counts ---------------------
+// lsa_select_tokens: the token scorer also counts every sequence's scores in
+// kScoreBins bins of equal width (lsa_common.cuh), in kScoreBinReplicas copies
+// so that fewer of its atomic adds meet on one address; the bin that holds
+// the k-th best score is then known before any score is read again.  A
+// cluster of 8 CTAs per sequence, each owning an eighth of the positions:
+//   1. right after the grid dependency wait every thread issues its loads at
+//      once: up to kPer scores of its CTA's slice (in registers), four bins of
+//      the counts, the token counts and the head weights;
+//   2. every CTA sums the count copies and finds that boundary bin b* (one
+//      block scan; all reach the same answer from the same counts);
+//   3. each CTA classifies its slice: a token in a bin above b* is selected
+//      (its bit is set in the CTA's bitmap, one ballot per 32 positions), a
+//      token in b* is a candidate (key and position; the bins are narrow, so
+//      there are few);
+//   4. each CTA pushes its count of selected tokens and its candidates into
+//      every CTA's shared memory, and one cluster barrier publishes them; then
+//      every CTA ranks all candidates by (key, position) the same way, takes
+//      the r best (r = k - tokens above b*), and knows its own output offset;
+//   5. each CTA writes its slice's positions in ascending order.
+// Every token above b* outscores every token in or below it, so this is the
+// exact top-k.  When the counts cannot be trusted (they do not add up to the
+// sequence's tokens, or b* does not split the tokens at k), the candidates do
+// not fit the lists, or the sequence is longer than the slices, the cluster
+// runs the exact radix select instead (one CTA re-reading the scores beyond
+// 131072 tokens).  The result is the same either way.
+constexpr int kSelMaxTokens = kClusterMaxCand;                       // 131072: 16 per thread
+constexpr int kSelSliceWords = kSelMaxTokens / kClusterCtas / 32;    // 512 bitmap words per CTA
+constexpr int kSelMaxCand = 128;                                     // candidates of one CTA
+static_assert(kThreads * 4 == kScoreBins, "one int4 of bin counts per thread");
+static_assert(kScoreBinReplicas * kScoreBins / 4 == kClusterCtas * 512, "each CTA clears 512 int4 of the counts");
+
+template <int kPer>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads, 1)
+select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_tokens,
+                     const float* __restrict__ w, int k, int max_tokens, int max_sel, int32_t* __restrict__ hist,
+                     int32_t* __restrict__ sel, int32_t* __restrict__ n_sel, int32_t* __restrict__ cu_sel,
+                     unsigned* status) {
+  __shared__ uint32_t bits[kSelSliceWords];
+  __shared__ uint32_t all_key[kClusterCtas * kSelMaxCand];   // [rank r][i]: CTA r's candidates, pushed by r
+  __shared__ int all_pos[kClusterCtas * kSelMaxCand];
+  __shared__ int x_above[kClusterCtas], x_cand[kClusterCtas];  // pushed by each rank
+  __shared__ int warp_sums[32];
+  __shared__ int hist_s[256];
+  __shared__ int sel2[2];
+  __shared__ int s_bstar, s_above, s_ncand;
+  griddep_wait();   // the scorer has finished: scores, n_tokens and the bin counts are final
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = cluster_ctarank();
+  const float* sc = scores + static_cast<int64_t>(b) * max_tokens;
+  int4* hrow = reinterpret_cast<int4*>(hist + static_cast<int64_t>(b) * kScoreBinReplicas * kScoreBins);
+
+  // ---- 1. every load at once ------------------------------------------------------
+  // This CTA's slice of positions, in whole bitmap words, sized from the row
+  // length (so the loads need not wait for the token count): thread t holds
+  // positions lo + j * 1024 + t, j < kPer.
+  const int slice = ((max_tokens + kClusterCtas - 1) / kClusterCtas + 31) / 32 * 32;
+  const int lo = min(max_tokens, static_cast<int>(rank) * slice);
+  const int hi_row = min(max_tokens, lo + slice);
+  const bool sliced = slice <= kPer * kThreads;                      // the slice fits the registers
+  float v[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int p = lo + j * kThreads + tid;
+    v[j] = (sliced && p < hi_row) ? __ldg(sc + p) : 0.f;
+  }
+  int c4[4] = {0, 0, 0, 0};   // bins 4 tid .. 4 tid + 3, summed over the copies
+#pragma unroll
+  for (int rep = 0; rep < kScoreBinReplicas; ++rep) {
+    const int4 x = hrow[rep * (kScoreBins / 4) + tid];
+    c4[0] += x.x; c4[1] += x.y; c4[2] += x.z; c4[3] += x.w;
+  }
+  const float scale = score_bin_scale(w);
+  auto clear_counts = [&]() {   // this CTA's eighth of the counts, zero for the next call
+    if (tid < 512) hrow[rank * 512 + tid] = make_int4(0, 0, 0, 0);
+  };
+
+  // Offsets and counts, as lsa_topk_tokens: min(k, n) positions per sequence
+  // (identical in every CTA of the cluster, written by rank 0).
+  int part = 0;
+  unsigned dummy = 0;
+  for (int bb = tid; bb <= b; bb += kThreads) part += kept_count(__ldg(n_tokens + bb), k, 0, max_tokens, max_sel, &dummy);
+  int tot = 0;
+  block_exclusive_scan(part, warp_sums, &tot);
+  unsigned err = 0;
+  const int n = __ldg(n_tokens + b);
+  const int nk = kept_count(n, k, 0, max_tokens, max_sel, &err);
+  if (rank == 0 && tid == 0) {
+    cu_sel[b + 1] = tot;
+    if (b == 0) cu_sel[0] = 0;
+    n_sel[b] = nk;
+    if (err) set_status(status, err);
+  }
+  int32_t* out = sel + static_cast<int64_t>(b) * max_sel;
+  if (nk == 0 || nk == n) {   // nothing, or every position (cluster-uniform: no count is needed)
+    clear_counts();
+    for (int c = static_cast<int>(rank) * kThreads + tid; c < nk; c += kClusterThreads) out[c] = c;
+    return;
+  }
+  cluster_arrive_relaxed();   // (A) this CTA runs; waited on before the first remote store
+
+  // ---- 2. the boundary bin ----------------------------------------------------------
+  const int own = c4[0] + c4[1] + c4[2] + c4[3];
+  int total = 0;
+  const int below = block_exclusive_scan(own, warp_sums, &total);   // tokens in bins under 4 tid
+  if (tid == 0) { s_bstar = -1; s_above = 0; s_ncand = 0; }
+  __syncthreads();
+  if (total == n && sliced && scale > 0.f) {                         // cluster-uniform
+    int above = total - below - own;                                 // tokens in bins over 4 tid + 3
+#pragma unroll
+    for (int j = 3; j >= 0; --j) {
+      if (above < nk && above + c4[j] >= nk) s_bstar = 4 * tid + j;
+      above += c4[j];
+    }
+  }
+  __syncthreads();
+  const int bstar = s_bstar;
+  bool fast = bstar >= 0;                                            // cluster-uniform
+  const int hi = min(n, hi_row);
+
+  // ---- 3. classify this CTA's slice -------------------------------------------------
+  if (fast) {
+    int above_w = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (lo + j * kThreads < hi) {   // block-uniform
+        const int p = lo + j * kThreads + tid;
+        const int bi = p < hi ? score_bin(v[j], scale) : -1;
+        const uint32_t up = __ballot_sync(0xffffffffu, bi > bstar);
+        const uint32_t eq = __ballot_sync(0xffffffffu, bi == bstar);
+        if (lane == 0) bits[j * (kThreads / 32) + warp] = up;
+        above_w += __popc(up);
+        if (eq) {
+          int base = 0;
+          if (lane == 0) base = atomicAdd(&s_ncand, __popc(eq));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if ((eq >> lane) & 1u) {
+            const int slot = base + __popc(eq & ((1u << lane) - 1u));
+            if (slot < kSelMaxCand) {
+              all_key[rank * kSelMaxCand + slot] = desc_key(v[j]);
+              all_pos[rank * kSelMaxCand + slot] = p;
+            }
+          }
+        }
+      }
+    }
+    if (lane == 0 && above_w) atomicAdd(&s_above, above_w);
+  }
+  __syncthreads();
+
+  // ---- 4. push counts and candidates to every CTA; one barrier publishes them -------
+  cluster_wait();   // (A): every CTA of the cluster runs
+  if (fast) {
+    const int m_own = min(s_ncand, kSelMaxCand);
+    if (tid < kClusterCtas) {
+      st_cluster_u32(cluster_map(&x_above[rank], tid), static_cast<uint32_t>(s_above));
+      st_cluster_u32(cluster_map(&x_cand[rank], tid), static_cast<uint32_t>(s_ncand));
+    }
+    for (int t = tid; t < kClusterCtas * m_own; t += kThreads) {
+      const int r = t / m_own, i = t - r * m_own;
+      if (r != static_cast<int>(rank)) {
+        st_cluster_u32(cluster_map(&all_key[rank * kSelMaxCand + i], r), all_key[rank * kSelMaxCand + i]);
+        st_cluster_u32(cluster_map(&all_pos[rank * kSelMaxCand + i], r),
+                       static_cast<uint32_t>(all_pos[rank * kSelMaxCand + i]));
+      }
+    }
+  }
+  cluster_sync_all();   // #1: every push is visible, and every CTA has read the counts
+  clear_counts();
+
+  if (fast) {
+    int mt = 0, above_all = 0, off = 0;
+#pragma unroll
+    for (int r = 0; r < kClusterCtas; ++r) {
+      fast = fast && x_cand[r] <= kSelMaxCand;
+      mt += x_cand[r];
+      above_all += x_above[r];
+      if (r < static_cast<int>(rank)) off += x_above[r];
+    }
+    const int r_take = nk - above_all;
+    fast = fast && r_take >= 0 && r_take <= mt;                      // cluster-uniform
+    if (fast) {
+      // Candidate t = (CTA r, index i) of the slotted lists, ranked against all.
+      bool taken = false, earlier = false;
+      if (tid < kClusterCtas * kSelMaxCand) {
+        const int r = tid / kSelMaxCand, i = tid - r * kSelMaxCand;
+        if (i < x_cand[r]) {
+          const uint32_t ki = all_key[tid];
+          const int pi = all_pos[tid];
+          int rnk = 0;
+          for (int rr = 0; rr < kClusterCtas; ++rr)
+            for (int jj = 0; jj < x_cand[rr]; ++jj) {
+              const uint32_t kj = all_key[rr * kSelMaxCand + jj];
+              rnk += (kj < ki) || (kj == ki && all_pos[rr * kSelMaxCand + jj] < pi);
+            }
+          taken = rnk < r_take;
+          earlier = taken && r < static_cast<int>(rank);
+          if (taken && r == static_cast<int>(rank)) atomicOr(&bits[(pi - lo) >> 5], 1u << ((pi - lo) & 31));
+        }
+      }
+      off += __syncthreads_count(earlier);   // also publishes the bits
+      // ---- 5. this slice's positions, ascending ---------------------------------------
+      griddep_launch_dependents();
+      const int words = hi > lo ? (hi - lo + 31) >> 5 : 0;
+      const uint32_t x0 = tid < words ? bits[tid] : 0u;
+      int pos = off + block_exclusive_scan(__popc(x0), warp_sums, nullptr);
+      uint32_t x = x0;
+      while (x) {
+        out[pos++] = lo + (tid << 5) + (__ffs(x) - 1);
+        x &= x - 1u;
+      }
+      return;
+    }
+  }
+
+  // ---- the exact path --------------------------------------------------------------
+  if (n <= kClusterThreads * kPer) {
+    cluster_select_and_write<kPer>(sc, n, nk, out);
+  } else if (rank == 0) {   // beyond the cluster's registers: one CTA re-reads the scores
+    select_and_write<false>(ScoreKey{sc}, n, nk, (n + kThreads - 1) / kThreads, out, hist_s, warp_sums, sel2);
+  }
+}
+
 // One CTA per sequence up to kClusterMinCand candidates, a cluster of 8 up to
 // kClusterMaxCand, one CTA re-reading the scores beyond.
 int launch_topk(bool pdl, const float* scores, const int32_t* n_count, const int32_t* k_per_seq, int k_all,
@@ -554,6 +794,56 @@ extern "C" int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int
   if (device_sm_count() <= 0) return LSA_ERR_NO_DEVICE;
   return topk::launch_topk(true, scores, n_tokens, nullptr, k, 0, B, max_tokens, max_sel, sel, n_sel, cu_sel,
                            static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t lsa_select_tokens_workspace_size(int B) {
+  if (B <= 0 || B > LSA_MAX_BATCH) return 0;
+  return static_cast<size_t>(B) * lsa::kScoreBinReplicas * lsa::kScoreBins * sizeof(int32_t);
+}
+
+// lsa_token_score followed by lsa_topk_tokens, with the selection driven by
+// the scorer's score-bin counts (summary page, 2.1 Architecture: native
+// token-level scoring keeps a fine-grained top-k inside the recalled subset).
+extern "C" int lsa_select_tokens(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
+                                 const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
+                                 int max_chunks, int max_kept, int k, float* scores, int32_t* n_tokens, int32_t* sel,
+                                 int32_t* n_sel, int32_t* cu_sel, int max_sel, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  using namespace lsa;
+  // Every check of both kernels comes before the first launch.
+  if (!sel || !n_sel || !cu_sel || k <= 0 || max_sel <= 0 || B <= 0 || max_kept <= 0) return LSA_ERR_INVALID_ARG;
+  if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(B) * max_sel >= (int64_t{1} << 31) ||
+      static_cast<int64_t>(max_kept) * kChunkTokens >= (int64_t{1} << 31))
+    return LSA_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || workspace_bytes < lsa_select_tokens_workspace_size(B)) return LSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LSA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = device_sm_count();
+  if (sms <= 0) return LSA_ERR_NO_DEVICE;
+  const int max_tokens = max_kept * kChunkTokens;
+  // The bin counts cost the scorer shared memory (four CTAs per SM instead of
+  // five), which only pays when its grid runs in one wave: then the step waits
+  // on the selection's latency, which the counts cut.  Larger grids take the
+  // scorer without counts and the radix select (lsa_token_score +
+  // lsa_topk_tokens), with the same result.
+  const int64_t score_ctas = static_cast<int64_t>(B) * ((max_tokens + 127) / 128);
+  if (score_ctas > static_cast<int64_t>(4) * sms) {
+    const int st = score::launch_token_score(q_idx, w, token_keys, n_slots, chunk_table, kept, n_kept, B, max_chunks,
+                                             max_kept, scores, n_tokens, nullptr, s);
+    if (st != LSA_OK) return st;
+    return topk::launch_topk(true, scores, n_tokens, nullptr, k, 0, B, max_tokens, max_sel, sel, n_sel, cu_sel, s);
+  }
+  int32_t* hist = static_cast<int32_t*>(workspace);
+  const int st = score::launch_token_score(q_idx, w, token_keys, n_slots, chunk_table, kept, n_kept, B, max_chunks,
+                                           max_kept, scores, n_tokens, hist, s);
+  if (st != LSA_OK) return st;
+  auto kernel = max_tokens <= topk::kClusterThreads * 4   ? topk::select_tokens_kernel<4>
+                : max_tokens <= topk::kClusterThreads * 8 ? topk::select_tokens_kernel<8>
+                                                          : topk::select_tokens_kernel<16>;
+  launch_pdl(true, kernel, dim3(topk::kClusterCtas, B), dim3(topk::kThreads), 0, s, scores, n_tokens, w, k,
+             max_tokens, max_sel, hist, sel, n_sel, cu_sel, lsa_device_status_ptr());
+  return launch_status();
 }
 
 extern "C" int lsa_topk_chunks(const float* scores, const int32_t* n_chunks, const int32_t* k_per_seq, int B,

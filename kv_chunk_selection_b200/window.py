@@ -19,8 +19,8 @@ import torch
 from . import (CHUNK_TOKENS, HEAD_DIM, NUM_KV_HEADS, NUM_Q_HEADS, lsa_append_token, lsa_attn_workspace_size,
                lsa_fetch_from_host, lsa_gather_chunks, lsa_gather_tokens, lsa_index_score, lsa_reset_local,
                lsa_sparse_decode_attn, lsa_sparse_decode_attn_append, lsa_sparse_decode_attn_local,
-               lsa_sparse_decode_attn_selected, lsa_threshold_chunks, lsa_token_score, lsa_topk_chunks,
-               lsa_topk_tokens)
+               lsa_sparse_decode_attn_selected, lsa_select_tokens, lsa_threshold_chunks, lsa_token_score,
+               lsa_topk_chunks, lsa_topk_tokens, new_select_tokens_workspace)
 
 TAU = 64
 
@@ -53,13 +53,15 @@ class LayerWindow:
     indexer query and keeps the ``fine_k`` best, and ``attend`` runs over those
     tokens only, reading them in place from the compact buffer.  With
     ``causal`` too, the selected tokens are first packed into dense units (the
-    fused append reads packed units).
+    fused append reads packed units).  ``fused_select`` (the default) scores and
+    selects with lsa_select_tokens; without it, lsa_token_score and
+    lsa_topk_tokens run one after the other (the same result).
     """
 
     def __init__(self, n_chunks: torch.Tensor, k_per_seq: torch.Tensor, chunk_table: Optional[torch.Tensor],
                  max_chunks: int, device="cuda", double_buffer: bool = False, selection: str = "topk",
                  threshold: float = 0.5, n_local: int = 1, causal: bool = False, fine_k: int = 0,
-                 threshold_cap: bool = True):
+                 threshold_cap: bool = True, fused_select: bool = True):
         self.device = torch.device(device)
         self.n_chunks = n_chunks
         self.k_per_seq = k_per_seq
@@ -109,6 +111,9 @@ class LayerWindow:
             self.sel = torch.zeros((self.B, self.fine_k), dtype=torch.int32, device=dev)
             self.n_sel = torch.zeros((self.B,), dtype=torch.int32, device=dev)
             self.cu_sel = torch.zeros((self.B + 1,), dtype=torch.int32, device=dev)
+            self.fused_select = bool(fused_select)
+            if self.fused_select:
+                self.sel_workspace = new_select_tokens_workspace(self.B, dev)
             self.packs = self.causal   # the causal step reads packed units
             if self.packs:
                 units = self.B * self.fine_k // CHUNK_TOKENS
@@ -172,9 +177,15 @@ class LayerWindow:
         """Token-level stage of one step: scores of the recalled tokens from the step's
         indexer query q_tok [B, 16, 128] and the fine_k best (packed into dense
         units when the window is causal)."""
-        lsa_token_score(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf], self.max_chunks,
-                        self.tok_scores, self.n_tokens, stream=stream)
-        lsa_topk_tokens(self.tok_scores, self.n_tokens, self.fine_k, self.sel, self.n_sel, self.cu_sel, stream=stream)
+        if self.fused_select:
+            lsa_select_tokens(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf],
+                              self.max_chunks, self.fine_k, self.tok_scores, self.n_tokens, self.sel, self.n_sel,
+                              self.cu_sel, self.sel_workspace, stream=stream)
+        else:
+            lsa_token_score(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf],
+                            self.max_chunks, self.tok_scores, self.n_tokens, stream=stream)
+            lsa_topk_tokens(self.tok_scores, self.n_tokens, self.fine_k, self.sel, self.n_sel, self.cu_sel,
+                            stream=stream)
         if self.packs:
             lsa_gather_tokens(self.k_bufs[buf], self.v_bufs[buf], self.cu_kept[buf], self.sel, self.cu_sel,
                               self.k_fine, self.v_fine, self.cu_units, stream=stream)

@@ -168,6 +168,114 @@ def test_token_topk_reread_path_random_scores(n, k):
     assert i64(cu).tolist() == [0, k, 2 * k, 3 * k]
 
 
+def two_call_selection(lw, q, w, tok_keys, k, max_sel=None):
+    scores, n_tok = token_scores_gpu(lw, q, w, tok_keys)
+    sel, n_sel, cu = topk_tokens_gpu(scores, n_tok, k, max_sel)
+    return scores, n_tok, sel, n_sel, cu
+
+
+def fused_selection(lw, q, w, tok_keys, k, ws, max_sel=None):
+    B = lw.B
+    max_sel = k if max_sel is None else max_sel
+    scores = torch.full((B, 64 * lw.max_kept), float("nan"), device=DEV)
+    n_tok = torch.full((B,), -1, dtype=torch.int32, device=DEV)
+    sel = torch.full((B, max_sel), -7, dtype=torch.int32, device=DEV)
+    n_sel = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
+    lsa.lsa_select_tokens(q, w, tok_keys, lw.chunk_table, lw.kept[0], lw.n_kept[0], lw.max_chunks, k, scores, n_tok,
+                          sel, n_sel, cu, ws)
+    return scores, n_tok, sel, n_sel, cu
+
+
+def assert_same_selection(a, b):
+    for x, y, name in zip(a, b, ("scores", "n_tokens", "sel", "n_sel", "cu_sel")):
+        if name == "sel":   # entries past n_sel are not written
+            n = a[3].cpu().tolist()
+            for i, m in enumerate(n):
+                assert torch.equal(x[i, :m], y[i, :m]), f"sel of sequence {i}"
+        else:
+            assert torch.equal(torch.nan_to_num(x, nan=-9.0) if x.is_floating_point() else x,
+                               torch.nan_to_num(y, nan=-9.0) if y.is_floating_point() else y), name
+
+
+@pytest.mark.parametrize("name,kw,k", [("128k", {}, 2048), ("500k", {}, 2048), ("batched", {"batch": 2}, 1024),
+                                       ("batched", {"batch": 2}, 64), ("batched", {"batch": 8}, 1024),
+                                       ("tiny", {}, 2048)])
+def test_select_tokens_equals_score_then_topk(name, kw, k):
+    """lsa_select_tokens (scores counted into bins, the selection driven by the
+    counts) gives the two-call path's outputs bit for bit, twice in a row (the
+    bin counts are left zeroed), and the oracle's rule on its own scores.  A
+    batch of 8 has a scorer grid of more than one wave and takes the two-call
+    path inside the library."""
+    inp, L, lw, tok_keys, q_tok = recalled(name, **kw)
+    ws = lsa.new_select_tokens_workspace(lw.B)
+    ref = two_call_selection(lw, q_tok[0, 3], L.w, tok_keys, k)
+    for call in range(2):
+        got = fused_selection(lw, q_tok[0, 3], L.w, tok_keys, k, ws)
+        torch.cuda.synchronize()
+        status_clean()
+        assert_same_selection(got, ref)
+        assert int(torch.count_nonzero(ws)) == 0, f"call {call}: the bin counts must be left zeroed"
+    kept = lw.kept_lists()
+    g = f64(got[0])
+    sel = kept_from_gpu(got[2], got[3])
+    same = oracle.topk_tokens([g[b, : 64 * len(kept[b])] for b in range(lw.B)], k)
+    for b in range(lw.B):
+        assert sel[b] == list(same[b]), f"seq {b}"
+
+
+def test_select_tokens_exact_path_on_ties():
+    """A zero indexer query makes every token score sum(w)/2: one bin holds
+    every token, so the selection takes its exact radix-select path, and keeps
+    the first k positions."""
+    inp, L, lw, tok_keys, q_tok = recalled("batched", batch=2)
+    ws = lsa.new_select_tokens_workspace(lw.B)
+    zero_q = torch.zeros_like(q_tok[0, 0])
+    got = fused_selection(lw, zero_q, L.w, tok_keys, 512, ws)
+    ref = two_call_selection(lw, zero_q, L.w, tok_keys, 512)
+    torch.cuda.synchronize()
+    status_clean()
+    assert_same_selection(got, ref)
+    for b, s in enumerate(kept_from_gpu(got[2], got[3])):
+        assert s == list(range(len(s))), f"seq {b}"
+    assert int(torch.count_nonzero(ws)) == 0
+
+
+def test_select_tokens_crowded_boundary_bin():
+    """An indexer query a thousand times smaller puts nearly every score in one
+    or two bins: the boundary bin overflows the candidate lists and the cluster
+    takes its exact path, with the two-call path's result."""
+    inp, L, lw, tok_keys, q_tok = recalled("128k")
+    ws = lsa.new_select_tokens_workspace(lw.B)
+    small_q = (q_tok[0, 2].float() * 1e-3).to(torch.bfloat16)
+    got = fused_selection(lw, small_q, L.w, tok_keys, 2048, ws)
+    ref = two_call_selection(lw, small_q, L.w, tok_keys, 2048)
+    torch.cuda.synchronize()
+    status_clean()
+    assert_same_selection(got, ref)
+    assert int(torch.count_nonzero(ws)) == 0
+
+
+def test_select_tokens_beyond_the_bitmap():
+    """131136 recalled tokens (2049 chunks): the scorer's grid is more than one
+    wave, so the library runs the two-call path; same result."""
+    n_chunks = torch.tensor([2050], dtype=torch.int32, device=DEV)
+    lw = LayerWindow(n_chunks, torch.tensor([2048], dtype=torch.int32, device=DEV), None, 2050, DEV, fine_k=2048)
+    lw.kept[0][0] = torch.arange(2049, dtype=torch.int32, device=DEV)
+    lw.n_kept[0][0] = 2049
+    tok_keys = workloads.randn_bf16((2050, 64, 128), 123, DEV)
+    q = workloads.randn_bf16((1, 16, 128), 124, DEV)
+    w = torch.rand(16, generator=torch.Generator(device=DEV).manual_seed(125), device=DEV)
+    ws = lsa.new_select_tokens_workspace(1)
+    got = fused_selection(lw, q, w, tok_keys, 2048, ws)
+    ref = two_call_selection(lw, q, w, tok_keys, 2048)
+    torch.cuda.synchronize()
+    status_clean()
+    assert int(got[1][0]) == 2049 * 64
+    assert_same_selection(got, ref)
+    assert int(torch.count_nonzero(ws)) == 0
+
+
 def test_gather_tokens_bit_exact():
     inp, L, lw, tok_keys, q_tok = recalled("batched", batch=6)
     scores, n_tok = token_scores_gpu(lw, q_tok[0, 1], L.w, tok_keys)
