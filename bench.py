@@ -930,6 +930,72 @@ def run_attn_only(args):
             "peak_source": kind, "device_status": bits, "source_digest": source_digest()}
 
 
+def run_fine_only(args):
+    """The fine step alone (token scoring and selection, then attention over the
+    selected tokens read in place) over a random recalled set of the workload's
+    kept size, without the KV pools: the small case for kernel profiling."""
+    import kv_chunk_selection_b200 as lsa
+    from kv_chunk_selection_b200.window import LayerWindow
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = workloads.WORKLOADS[args.workload]
+    n, k = workloads.lengths_for(wl)
+    kept = [min(int(kb), int(nb) - 1) + 1 if int(nb) > 0 else 0 for nb, kb in zip(n, k)]
+    B, total = len(kept), int(sum(kept))
+    # the recalled chunks are slots 0 .. total-1, sequence by sequence
+    n_t = torch.tensor(kept, dtype=torch.int32, device=dev)
+    table = torch.zeros((B, max(kept)), dtype=torch.int32)
+    off = 0
+    for b, m in enumerate(kept):
+        table[b, :m] = torch.arange(off, off + m, dtype=torch.int32)
+        off += m
+    lw = LayerWindow(n_t, n_t - 1, table.to(dev), max(kept), dev, fine_k=args.fine_k or 2048)
+    for b, m in enumerate(kept):
+        lw.kept[0][b, :m] = torch.arange(m, dtype=torch.int32, device=dev)
+    lw.n_kept[0].copy_(n_t)
+    lw.cu_kept[0].copy_(torch.tensor([0] + torch.tensor(kept).cumsum(0).tolist(), dtype=torch.int32, device=dev))
+    lw.k_bufs[0].copy_(workloads.randn_bf16(tuple(lw.k_bufs[0].shape), 1, dev))
+    lw.v_bufs[0].copy_(workloads.randn_bf16(tuple(lw.v_bufs[0].shape), 2, dev))
+    tok_keys = workloads.randn_bf16((total, 64, 128), 3, dev)
+    q_tok = workloads.randn_bf16((workloads.TAU, B, 16, 128), 4, dev)
+    qs = workloads.randn_bf16((workloads.TAU, B, 64, 128), 5, dev)
+    w = torch.rand(16, generator=torch.Generator(device=dev).manual_seed(6), device=dev)
+    out = torch.empty((B, 64, 128), device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        lw.fine_select(q_tok[i % workloads.TAU], w, tok_keys)
+        lw.attend(qs[i % workloads.TAU], out)
+
+    with torch.cuda.stream(stream):
+        step(0)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            step(i)
+    for _ in range(max(1, args.warmup // max(1, args.steps))):
+        graph.replay()
+    torch.cuda.synchronize()
+    per_step = []
+    for _ in range(args.repeats):
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        with torch.cuda.stream(stream):
+            graph.replay()
+        b_.record(stream)
+        b_.synchronize()
+        per_step.append(a.elapsed_time(b_) / 1e3 / args.steps)
+    torch.cuda.synchronize()
+    bits = lsa.read_device_status()
+    med = sorted(per_step)[len(per_step) // 2]
+    sel_tokens = sum(min(lw.fine_k, 64 * m) for m in kept)
+    nbytes = 64 * total * 256 + B * 16 * 128 * 2 + sel_tokens * TOKEN_KV_BYTES + B * (64 * 128 * 2 + 64 * 128 * 4)
+    return {"mode": "fine-only", "workload": args.workload, "recalled_chunks": total, "selected_tokens": sel_tokens,
+            "steps_per_replay": args.steps, "replays": args.repeats, "median_us_per_step": med * 1e6,
+            "bytes_per_step": nbytes, "device_status": bits}
+
+
 # ---------------------------------------------------------- oracle (CPU) arm --
 
 def _cpu_model():
@@ -1094,6 +1160,8 @@ def main():
     ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
     ap.add_argument("--attn-only", action="store_true",
                     help="time attention launches alone on a random compact buffer (profiling case)")
+    ap.add_argument("--fine-only", action="store_true",
+                    help="time fine steps alone over a random recalled set of the workload's kept size (profiling case)")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other configurations after the headline (one GPU, default workload only)")
     ap.add_argument("--config-steps", type=int, default=8, help="timed windows of each other configuration")
@@ -1115,6 +1183,9 @@ def main():
 
     if args.attn_only:
         print(json.dumps(run_attn_only(args)), flush=True)
+        return
+    if args.fine_only:
+        print(json.dumps(run_fine_only(args)), flush=True)
         return
 
     if args.impl == "reference":
