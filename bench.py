@@ -21,8 +21,8 @@ layer), with the achieved HBM bandwidth of the whole window and of the
 attention kernel against the measured copy bandwidth.
 
 On one GPU with the default workload, the other configurations of the metric
-(128K, the 1M host tier, the batched workload, and the 500K fine-stage and
-causal modes) then run for ``--config-steps`` windows each and appear as
+(128K, 1M with the pool in HBM, the 1M host tier, the batched workload, the
+500K and batched fine-stage modes and the 500K causal mode) then run for ``--config-steps`` windows each and appear as
 compact lines under ``configs``; ``--no-configs`` skips them.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 500k]
@@ -645,9 +645,11 @@ def run_ours(args, rank, world, local_rank):
 # headline and reported as a compact line under "configs": (name, overrides).
 EXTRA_CONFIGS = (
     ("128k", {"workload": "128k"}),
+    ("1m", {"workload": "1m"}),
     ("1m_host", {"workload": "1m_host"}),
     ("batched", {"workload": "batched"}),
     ("500k_fine_k2048", {"workload": "500k", "fine_k": 2048}),
+    ("batched_fine_k2048", {"workload": "batched", "fine_k": 2048}),
     ("500k_causal", {"workload": "500k", "causal": True}),
 )
 

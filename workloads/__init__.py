@@ -16,6 +16,7 @@ tiny       1     64             8           1        parity case
 128k       1     2048           256         4        16 planted chunks
 500k       1     8192           819         2        2 GiB pool in HBM
 1m_host    1     16384          1638        2        4 GiB pool, pinned host
+1m         1     16384          1638        2        4 GiB pool in HBM
 batched    32    512..4096      N_b // 8    2        4 layers, paged table
 =========  ====  =============  ==========  =======  ======================
 
@@ -76,6 +77,11 @@ WORKLOADS = {
         "1m_host", "1M decode with host-tier KV pool, 1 layer: B=1, L=1048576 (16384 chunks), "
         "K=1638 + latest, 2 windows, KV pool in pinned host memory", batch=1, chunks=16384,
         k_fraction=None, k_fixed=1638, windows=2, host_pool=True),
+    # The 1M sizes with the pool resident in HBM (4 GiB per K/V): the HBM side of
+    # the 1M decode step, beside the host tier that the host link bounds.
+    "1m": Workload(
+        "1m", "1M decode, 1 layer: B=1, L=1048576 (16384 chunks), K=1638 + latest, 2 windows, "
+        "pool resident in HBM", batch=1, chunks=16384, k_fraction=None, k_fixed=1638, windows=2),
     "batched": Workload(
         "batched", "batched ragged serving, 4 layers: B=32, L~U[32K,256K] rounded down to 64, "
         "K_b = floor(0.125 N_b) + latest, paged chunk table, 2 windows",
