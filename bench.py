@@ -290,6 +290,14 @@ def h2d_probe_gbs(device, nbytes=1 << 30, reps=5):
     return nbytes / best / 1e9
 
 
+def inp_windows(args):
+    """Distinct query windows of the host-tier run: the workload's own, or with
+    --query-drift one per timed and warm-up window (a drifting sequence, not a
+    cycle of two)."""
+    wl = workloads.WORKLOADS[args.workload]
+    return wl.windows if args.query_drift is None else args.steps + args.warmup + 1
+
+
 def run_host_tier(args, rank, world, local_rank):
     """Host-tier window pipeline: while the main stream runs the 64 attention
     steps of window w over compact buffer w % 2, a side stream scores and selects
@@ -303,10 +311,12 @@ def run_host_tier(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     lsa.lib()
-    inp = workloads.make_inputs(args.workload, dev, base_seed=workloads.BASE_SEED + rank)
+    n_win = max(inp_windows(args), 1)
+    inp = workloads.make_inputs(args.workload, dev, base_seed=workloads.BASE_SEED + rank, windows=n_win,
+                                query_drift=args.query_drift)
     assert len(inp.layers) == 1
     L = inp.layers[0]
-    B, n_win = inp.batch, inp.workload.windows
+    B = inp.batch
     lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, dev, double_buffer=True)
     out = torch.empty((workloads.TAU, B, 64, 128), device=dev)
     main, side = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -435,6 +445,7 @@ def run_host_tier(args, rank, world, local_rank):
                    "stream overlaps the 64 attention steps of window w", "fetch_ctas": args.fetch_ctas,
                    "residency": "chunks kept by the previous window are copied from its device buffer"
                    if args.delta else "every kept chunk is fetched from the host pool",
+                   "query_drift": args.query_drift,
                    "fetch": ("copy engines: the selection is copied to the host, then one 2-D copy per kept chunk "
                              "and per K/V" if copy_engine else "SM threads reading mapped page-locked memory"),
                    "l2": "inputs larger than L2 (host pool 8 GiB, 410 MiB per attention launch)",
@@ -1149,6 +1160,8 @@ def main():
     ap.add_argument("--fetch-ctas", type=int, default=64)
     ap.add_argument("--delta", action="store_true",
                     help="host tier: reuse chunks the previous window kept from its device buffer")
+    ap.add_argument("--query-drift", type=float, default=None,
+                    help="host tier: correlate consecutive windows' indexer queries (d in (0, 1]; 1 = independent)")
     ap.add_argument("--fetch", choices=["sm", "copy"], default="sm",
                     help="host tier: SM threads over mapped memory (default) or the copy engines")
     ap.add_argument("--selection", choices=["topk", "threshold"], default="topk",
@@ -1172,6 +1185,9 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if (args.causal or args.n_local != 1) and workloads.WORKLOADS[args.workload].host_pool:
         ap.error("--causal and --n-local apply to device-resident workloads, not the host tier")
+    if args.query_drift is not None and (not 0.0 < args.query_drift <= 1.0
+                                         or not workloads.WORKLOADS[args.workload].host_pool):
+        ap.error("--query-drift takes d in (0, 1] and applies to the host-tier workload")
     if args.fetch == "copy" and (args.delta or not workloads.WORKLOADS[args.workload].host_pool):
         ap.error("--fetch copy applies to the host-tier workload, without --delta")
     if args.n_local != 1 and args.selection != "topk":
@@ -1217,7 +1233,7 @@ def main():
             torch.distributed.barrier()
     out["cpu_baseline"] = cpu
     headline_only = (args.fine_k or args.causal or args.delta or args.selection != "topk" or args.n_local != 1
-                     or args.fetch != "sm"
+                     or args.fetch != "sm" or args.query_drift is not None
                      or args.workload != DEFAULT_WORKLOAD)
     if world == 1 and not args.no_configs and not headline_only:
         out["configs"] = run_extra_configs(args, rank, world, local_rank)

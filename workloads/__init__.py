@@ -170,10 +170,18 @@ def lengths_for(wl: Workload, base_seed: int = BASE_SEED):
 
 def make_inputs(name_or_wl, device="cuda", base_seed: int = BASE_SEED, layers: Optional[int] = None,
                 windows: Optional[int] = None, steps: int = TAU, chunks: Optional[int] = None,
-                k: Optional[int] = None, batch: Optional[int] = None, pools: bool = True) -> Inputs:
+                k: Optional[int] = None, batch: Optional[int] = None, pools: bool = True,
+                query_drift: Optional[float] = None) -> Inputs:
     """Draw every input of a workload.  ``chunks``/``k``/``batch`` override the
     sizes (used for reduced parity cases with the same distributions); with
-    ``pools=False`` the KV pools are left out (scoring and selection only)."""
+    ``pools=False`` the KV pools are left out (scoring and selection only).
+
+    ``query_drift`` d in [0, 1] correlates the indexer queries of consecutive
+    windows: the query of window w > 0 is sqrt(1 - d^2) times that of window
+    w - 1 plus d times a fresh N(0, 1) draw (in float32, then rounded to bf16),
+    so every element stays N(0, 1) and d = 1 (or None) gives independent windows.
+    Small d stands in for the temporal locality of real decoding, where the
+    hidden state moves little from one window to the next."""
     wl = WORKLOADS[name_or_wl] if isinstance(name_or_wl, str) else name_or_wl
     if chunks is not None or k is not None or batch is not None:
         wl = dataclasses.replace(
@@ -203,6 +211,12 @@ def make_inputs(name_or_wl, device="cuda", base_seed: int = BASE_SEED, layers: O
         gw = _gen(_seed(base_seed, "w", l), "cpu")
         w = torch.rand((INDEX_HEADS,), generator=gw, dtype=torch.float32).to(device)
         q_idx = randn_bf16((n_windows, B, INDEX_HEADS, INDEX_DIM), _seed(base_seed, "qidx", l), device)
+        if query_drift is not None and query_drift < 1.0:
+            d = float(query_drift)
+            prev = q_idx[0].float()
+            for wi in range(1, n_windows):
+                prev = math.sqrt(1.0 - d * d) * prev + d * q_idx[wi].float()
+                q_idx[wi] = prev.to(torch.bfloat16)
         q = randn_bf16((n_windows, steps, B, NUM_Q_HEADS, HEAD_DIM), _seed(base_seed, "q", l), device)
         planted = None
         if wl.planted:
