@@ -100,6 +100,27 @@ def test_host_checks_null_pointers(L):
     assert L.lsa_selftest_bounded_wait(5, n, 1000, n) == INVALID      # unknown mode
 
 
+def test_host_checks_of_the_later_entry_points(L):
+    n, ok = None, ctypes.c_void_p(0x100000)
+    f = ctypes.c_float(0.5)
+    # capped threshold: null pointers; a NULL cap is allowed (it is the plain rule)
+    assert L.lsa_threshold_chunks_capped(n, n, n, f, n, 1, 1, 1, n, n, n, n) == INVALID
+    assert L.lsa_threshold_chunks_capped(ok, ok, ok, ctypes.c_float(float("nan")), n, 1, 4, 2, ok, ok, ok, n) == INVALID
+    # fused token selection: missing outputs, k <= 0, no or a small workspace, a misaligned one
+    ws = L.lsa_select_tokens_workspace_size(1)
+    assert ws == 4 * 4096 * 4 and L.lsa_select_tokens_workspace_size(0) == 0
+    sel_args = lambda k, w, wb: (ok, ok, ok, 4, n, ok, ok, 1, 4, 2, k, ok, ok, ok, ok, ok, 128, w, wb, n)
+    assert L.lsa_select_tokens(*sel_args(0, ok, ws)) == INVALID
+    assert L.lsa_select_tokens(*sel_args(64, n, ws)) == WORKSPACE
+    assert L.lsa_select_tokens(*sel_args(64, ok, ws - 16)) == WORKSPACE
+    assert L.lsa_select_tokens(*sel_args(64, ctypes.c_void_p(0x100008), ws)) == MISALIGNED
+    assert L.lsa_select_tokens(ok, ok, ok, 4, n, ok, ok, LSA_MAX_BATCH + 1, 4, 2, 64, ok, ok, ok, ok, ok, 128, ok,
+                               1 << 40, n) == UNSUPPORTED
+    # copy-engine fetch: null pointers, misaligned pools
+    assert L.lsa_fetch_from_host_copy(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, n, n) == INVALID
+    assert L.lsa_fetch_from_host_copy(ctypes.c_void_p(0x1001), ok, 4, n, ok, ok, 1, 4, 2, ok, ok, 2, n, n) == MISALIGNED
+
+
 def test_host_checks_sizes_and_alignment(L):
     odd = ctypes.c_void_p(0x1001)         # misaligned, never dereferenced
     ok = ctypes.c_void_p(0x100000)        # aligned, never dereferenced (checks fail first)

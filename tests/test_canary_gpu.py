@@ -265,6 +265,24 @@ def test_canaries_fine_stage_k_beyond_recalled_tokens():
     assert ns == [min(kk, x) for x in nt]
     assert tails_untouched(sel.bytes(), ns), "sel past n_sel"
 
+    # the same step through lsa_select_tokens (scores counted into bins, the selection driven by the counts)
+    tok2 = Guarded((B, 64 * max_kept), torch.float32)
+    n_tok2 = Guarded((B,), torch.int32)
+    sel2, n_sel2, cu_sel2 = Guarded((B, kk), torch.int32), Guarded((B,), torch.int32), Guarded((B + 1,), torch.int32)
+    ws_sel = Guarded((lsa.lib().lsa_select_tokens_workspace_size(B),), torch.uint8)
+    ws_sel.t.zero_()
+    lsa.lsa_select_tokens(q_tok, w, tok_keys, table, kept, n_kept, max_chunks, kk, tok2.t, n_tok2.t, sel2.t, n_sel2.t,
+                          cu_sel2.t, ws_sel.t)
+    torch.cuda.synchronize()
+    assert status() == 0
+    for g, name in ((tok2, "fused token scores"), (n_tok2, "fused n_tokens"), (sel2, "fused sel"),
+                    (n_sel2, "fused n_sel"), (cu_sel2, "fused cu_sel"), (ws_sel, "selection counts")):
+        g.check(name)
+    assert tails_untouched(tok2.bytes(), nt), "fused token scores past a sequence's tokens"
+    assert tails_untouched(sel2.bytes(), ns), "fused sel past n_sel"
+    assert int(torch.count_nonzero(ws_sel.t)) == 0, "the counts are left zeroed"
+    assert torch.equal(n_sel2.t, n_sel.t) and torch.equal(cu_sel2.t, cu_sel.t)
+
     units = sum(ns) // 64
     k_out = Guarded((8, units + 2, 64, 128), torch.bfloat16)
     v_out = Guarded((8, units + 2, 64, 128), torch.bfloat16)
