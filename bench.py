@@ -502,8 +502,8 @@ def run_ours(args, rank, world, local_rank):
     def attn_phase(w):
         for t in range(workloads.TAU):
             for l, L in enumerate(inp.layers):
-                if args.fine_k:
-                    lws[l].fine_select(fine[l][1][w, t], L.w, fine[l][0])
+                if args.fine_k:   # the kept lists and token keys are unchanged after the window's first step
+                    lws[l].fine_select(fine[l][1][w, t], L.w, fine[l][0], keys_unchanged=t > 0)
                 if args.causal:   # the step's token is appended and attended in one launch
                     lws[l].attend_append(L.q[w, t], outs[l][t], decoded[l][0][w, t], decoded[l][1][w, t],
                                          kv_unchanged=t > 0)
@@ -726,7 +726,7 @@ def fine_stage_times(args, lws, inp, fine, stream, kept_total, fine_total, reps=
                                                    lw.cu_sel),
     }
     if lw.fused_select:   # the step's selection call: scorer with bin counts, then the bin-driven selection
-        calls["select_tokens"] = lambda: lw.fine_select(q_tok[0, 0], L.w, keys)
+        calls["select_tokens"] = lambda: lw.fine_select(q_tok[0, 0], L.w, keys, keys_unchanged=True)
     if lw.packs:
         calls["gather_tokens"] = lambda: lsa.lsa_gather_tokens(lw.k_bufs[0], lw.v_bufs[0], lw.cu_kept[0], lw.sel,
                                                                lw.cu_sel, lw.k_fine, lw.v_fine, lw.cu_units)
@@ -977,7 +977,7 @@ def run_fine_only(args):
     stream = torch.cuda.Stream(device=dev)
 
     def step(i):
-        lw.fine_select(q_tok[i % workloads.TAU], w, tok_keys)
+        lw.fine_select(q_tok[i % workloads.TAU], w, tok_keys, keys_unchanged=i > 0)
         lw.attend(qs[i % workloads.TAU], out)
 
     with torch.cuda.stream(stream):

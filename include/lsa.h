@@ -540,14 +540,21 @@ int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int k, int B, 
  *              (zero it once when it is allocated): the bin counts; every
  *              call leaves it zero again.  Calls that may overlap on the GPU
  *              need workspaces of their own.
+ *   flags      0 or LSA_TOKENS_UNCHANGED: the kernel that ran just before this
+ *              call on `stream` wrote none of token_keys, chunk_table, kept
+ *              and n_kept (true for every decode step of a window after the
+ *              first).  The scorer then looks up and loads its key rows while
+ *              that kernel is still finishing; it reads q_idx and writes its
+ *              outputs only after it.  Without the flag it waits first.
  * Device errors as lsa_token_score and lsa_topk_tokens.
  */
+#define LSA_TOKENS_UNCHANGED 1u
 size_t lsa_select_tokens_workspace_size(int B);
 int lsa_select_tokens(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
                       const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
                       int max_chunks, int max_kept, int k, float* scores, int32_t* n_tokens, int32_t* sel,
                       int32_t* n_sel, int32_t* cu_sel, int max_sel, void* workspace, size_t workspace_bytes,
-                      void* stream);
+                      unsigned int flags, void* stream);
 
 /*
  * lsa_gather_tokens -- pack the selected tokens into dense units, bit for bit:

@@ -64,7 +64,7 @@ def _load():
         "lsa_token_score": ([P, P, P, I64, P, P, P, I, I, I, P, P, P], I),
         "lsa_topk_tokens": ([P, P, I, I, I, I, P, P, P, P], I),
         "lsa_select_tokens_workspace_size": ([I], S),
-        "lsa_select_tokens": ([P, P, P, I64, P, P, P, I, I, I, I, P, P, P, P, P, I, P, S, P], I),
+        "lsa_select_tokens": ([P, P, P, I64, P, P, P, I, I, I, I, P, P, P, P, P, I, P, S, ctypes.c_uint, P], I),
         "lsa_gather_tokens": ([P, P, I64, P, P, P, I, I, P, P, I64, P, P], I),
         "lsa_sparse_decode_attn_local": ([P, P, P, I64, P, I, F, P, P, P, P, P, S, ctypes.c_uint, P], I),
         "lsa_threshold_chunks": ([P, P, P, F, I, I, I, P, P, P, P], I),
@@ -421,10 +421,18 @@ def new_select_tokens_workspace(B: int, device=None) -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
+TOKENS_UNCHANGED = 1
+
+
 def lsa_select_tokens(q_idx, w, token_keys, chunk_table, kept, n_kept, max_chunks, k, scores, n_tokens, sel, n_sel,
-                      cu_sel, workspace, stream=None):
+                      cu_sel, workspace, stream=None, keys_unchanged=False):
     """lsa_token_score then lsa_topk_tokens in one call (same outputs), the
-    selection driven by the scorer's score-bin counts."""
+    selection driven by the scorer's score-bin counts.
+
+    ``keys_unchanged=True`` tells the library that the kernel just before this
+    call on the stream wrote none of token_keys, chunk_table, kept and n_kept
+    (every decode step of a window after the first), so the scorer may load its
+    key rows while that kernel finishes."""
     _need(q_idx, "q_idx", torch.bfloat16)
     _need(w, "w", torch.float32)
     _need(token_keys, "token_keys", torch.bfloat16)
@@ -445,7 +453,8 @@ def lsa_select_tokens(q_idx, w, token_keys, chunk_table, kept, n_kept, max_chunk
     _check("lsa_select_tokens", _load().lsa_select_tokens(
         _ptr(q_idx), _ptr(w), _ptr(token_keys), token_keys.shape[0], _ptr(chunk_table), _ptr(kept), _ptr(n_kept), B,
         int(max_chunks), max_kept, int(k), _ptr(scores), _ptr(n_tokens), _ptr(sel), _ptr(n_sel), _ptr(cu_sel),
-        sel.shape[1], _ptr(workspace), workspace.numel(), _stream(stream)))
+        sel.shape[1], _ptr(workspace), workspace.numel(), TOKENS_UNCHANGED if keys_unchanged else 0,
+        _stream(stream)))
 
 
 def lsa_gather_tokens(k_buf, v_buf, cu_kept, sel, cu_sel, k_out, v_out, cu_units, stream=None):

@@ -118,17 +118,26 @@ template <class Rows>
 __global__ void __launch_bounds__(kThreads)
 index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restrict__ w,
                    const __nv_bfloat16* __restrict__ keys, Rows rows, float* __restrict__ scores,
-                   float neg_scale_log2, unsigned* status) {
+                   float neg_scale_log2, unsigned* status, int keys_unchanged) {
   extern __shared__ __align__(1024) uint8_t smem[];
   griddep_launch_dependents();   // let the next kernel launch; its CTAs wait for this grid
-  griddep_wait();                 // the previous kernel on the stream has finished
+  // With keys_unchanged the caller guarantees that the preceding kernel on the
+  // stream wrote none of the keys, the chunk table and the kept lists (true for
+  // every decode step of a window after the first), so the key rows are
+  // resolved and loaded while that kernel finishes; the query, which it may
+  // have written, and every output wait for it.
+  if (!keys_unchanged) griddep_wait();
   const int b = blockIdx.y;
   const int n = rows.count(b);
-  if (blockIdx.x == 0 && threadIdx.x == 0) rows.on_count(b, n);
   if (n < 0) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_BAD_COUNT);
+    if (keys_unchanged) griddep_wait();
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      rows.on_count(b, n);
+      set_status(status, LSA_DEV_ERR_BAD_COUNT);
+    }
     return;
   }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !keys_unchanged) rows.on_count(b, n);
   const int base = blockIdx.x * kTile;
   if (base >= n) return;
   if (smem_u32(smem) & 1023u) {   // the swizzle atoms assume 1024-byte alignment
@@ -191,6 +200,10 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
       const int r = it * (kThreads / 16) + (tid >> 4);
       *reinterpret_cast<uint4*>(sa + sw128_offset(r, piece, kTile)) = v[it];
     }
+  }
+  if (keys_unchanged) {
+    griddep_wait();   // the query and the outputs: after the preceding kernel
+    if (blockIdx.x == 0 && threadIdx.x == 0) rows.on_count(b, n);
   }
   // B: the 16 indexer query rows of sequence b (K-major, one row per head).
   {
@@ -265,7 +278,7 @@ extern "C" int lsa_index_score(const void* q_idx, const float* w, const void* ch
   const score::ChunkRows rows{chunk_table, n_chunks, max_chunks, n_slots};
   launch_pdl(false, score::index_score_kernel<score::ChunkRows>, grid, dim3(score::kThreads), score::kSmemBytes,
              static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(q_idx), w,
-             static_cast<const __nv_bfloat16*>(chunk_keys), rows, scores, neg_scale_log2, lsa_device_status_ptr());
+             static_cast<const __nv_bfloat16*>(chunk_keys), rows, scores, neg_scale_log2, lsa_device_status_ptr(), 0);
   return launch_status();
 }
 
@@ -275,7 +288,8 @@ namespace score {
 // lsa_select_tokens (hist: [B][kScoreBins] counts to add to).
 int launch_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
                        const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B, int max_chunks,
-                       int max_kept, float* scores, int32_t* n_tokens, int32_t* hist, cudaStream_t stream) {
+                       int max_kept, float* scores, int32_t* n_tokens, int32_t* hist, int keys_unchanged,
+                       cudaStream_t stream) {
   if (!q_idx || !w || !token_keys || !kept || !n_kept || !scores || !n_tokens || B <= 0 || max_chunks <= 0 ||
       max_kept <= 0 || n_slots <= 0)
     return LSA_ERR_INVALID_ARG;
@@ -308,7 +322,7 @@ int launch_token_score(const void* q_idx, const float* w, const void* token_keys
   rows.hist = hist;
   launch_pdl(true, index_score_kernel<TokenRows>, grid, dim3(kThreads), smem, stream,
              static_cast<const __nv_bfloat16*>(q_idx), w, static_cast<const __nv_bfloat16*>(token_keys), rows, scores,
-             neg_scale_log2, lsa_device_status_ptr());
+             neg_scale_log2, lsa_device_status_ptr(), keys_unchanged);
   return launch_status();
 }
 }  // namespace score
@@ -318,5 +332,5 @@ extern "C" int lsa_token_score(const void* q_idx, const float* w, const void* to
                                const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
                                int max_chunks, int max_kept, float* scores, int32_t* n_tokens, void* stream) {
   return lsa::score::launch_token_score(q_idx, w, token_keys, n_slots, chunk_table, kept, n_kept, B, max_chunks,
-                                        max_kept, scores, n_tokens, nullptr, static_cast<cudaStream_t>(stream));
+                                        max_kept, scores, n_tokens, nullptr, 0, static_cast<cudaStream_t>(stream));
 }

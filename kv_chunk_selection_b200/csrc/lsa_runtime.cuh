@@ -61,7 +61,8 @@ namespace score {
 // adds each sequence's score-bin counts to hist[b][kScoreBins].
 int launch_token_score(const void* q_idx, const float* w, const void* token_keys, int64_t n_slots,
                        const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B, int max_chunks,
-                       int max_kept, float* scores, int32_t* n_tokens, int32_t* hist, cudaStream_t stream);
+                       int max_kept, float* scores, int32_t* n_tokens, int32_t* hist, int keys_unchanged,
+                       cudaStream_t stream);
 }  // namespace score
 
 }  // namespace lsa

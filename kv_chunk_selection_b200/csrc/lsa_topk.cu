@@ -808,10 +808,12 @@ extern "C" int lsa_select_tokens(const void* q_idx, const float* w, const void* 
                                  const int32_t* chunk_table, const int32_t* kept, const int32_t* n_kept, int B,
                                  int max_chunks, int max_kept, int k, float* scores, int32_t* n_tokens, int32_t* sel,
                                  int32_t* n_sel, int32_t* cu_sel, int max_sel, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+                                 size_t workspace_bytes, unsigned int flags, void* stream) {
   using namespace lsa;
   // Every check of both kernels comes before the first launch.
   if (!sel || !n_sel || !cu_sel || k <= 0 || max_sel <= 0 || B <= 0 || max_kept <= 0) return LSA_ERR_INVALID_ARG;
+  if (flags & ~static_cast<unsigned>(LSA_TOKENS_UNCHANGED)) return LSA_ERR_INVALID_ARG;
+  const int keys_unchanged = (flags & LSA_TOKENS_UNCHANGED) ? 1 : 0;
   if (B > LSA_MAX_BATCH) return LSA_ERR_UNSUPPORTED_SHAPE;
   if (static_cast<int64_t>(B) * max_sel >= (int64_t{1} << 31) ||
       static_cast<int64_t>(max_kept) * kChunkTokens >= (int64_t{1} << 31))
@@ -830,13 +832,13 @@ extern "C" int lsa_select_tokens(const void* q_idx, const float* w, const void* 
   const int64_t score_ctas = static_cast<int64_t>(B) * ((max_tokens + 127) / 128);
   if (score_ctas > static_cast<int64_t>(4) * sms) {
     const int st = score::launch_token_score(q_idx, w, token_keys, n_slots, chunk_table, kept, n_kept, B, max_chunks,
-                                             max_kept, scores, n_tokens, nullptr, s);
+                                             max_kept, scores, n_tokens, nullptr, keys_unchanged, s);
     if (st != LSA_OK) return st;
     return topk::launch_topk(true, scores, n_tokens, nullptr, k, 0, B, max_tokens, max_sel, sel, n_sel, cu_sel, s);
   }
   int32_t* hist = static_cast<int32_t*>(workspace);
   const int st = score::launch_token_score(q_idx, w, token_keys, n_slots, chunk_table, kept, n_kept, B, max_chunks,
-                                           max_kept, scores, n_tokens, hist, s);
+                                           max_kept, scores, n_tokens, hist, keys_unchanged, s);
   if (st != LSA_OK) return st;
   auto kernel = max_tokens <= topk::kClusterThreads * 4   ? topk::select_tokens_kernel<4>
                 : max_tokens <= topk::kClusterThreads * 8 ? topk::select_tokens_kernel<8>

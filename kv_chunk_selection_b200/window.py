@@ -173,14 +173,16 @@ class LayerWindow:
                                       stream=stream, kv_unchanged=kv_unchanged)
         self._phase = 1 - self._phase
 
-    def fine_select(self, q_tok, w, token_keys, buf: int = 0, stream=None):
+    def fine_select(self, q_tok, w, token_keys, buf: int = 0, stream=None, keys_unchanged: bool = False):
         """Token-level stage of one step: scores of the recalled tokens from the step's
         indexer query q_tok [B, 16, 128] and the fine_k best (packed into dense
-        units when the window is causal)."""
+        units when the window is causal).  ``keys_unchanged``: the previous kernel
+        on the stream wrote neither the token keys nor this window's kept lists
+        (true for every step but the first)."""
         if self.fused_select:
             lsa_select_tokens(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf],
                               self.max_chunks, self.fine_k, self.tok_scores, self.n_tokens, self.sel, self.n_sel,
-                              self.cu_sel, self.sel_workspace, stream=stream)
+                              self.cu_sel, self.sel_workspace, stream=stream, keys_unchanged=keys_unchanged)
         else:
             lsa_token_score(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf],
                             self.max_chunks, self.tok_scores, self.n_tokens, stream=stream)
@@ -228,7 +230,7 @@ class LayerWindow:
             self.reset_local(stream)
         for t in range(q_steps.shape[0]):
             if self.fine_k:
-                self.fine_select(q_tok[t], w, token_keys, 0, stream)
+                self.fine_select(q_tok[t], w, token_keys, 0, stream, keys_unchanged=t > 0)
             if self.causal:
                 self.attend_append(q_steps[t], outs[t], k_new[t], v_new[t], 0, stream, kv_unchanged=t > 0)
             else:

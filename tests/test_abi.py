@@ -109,13 +109,14 @@ def test_host_checks_of_the_later_entry_points(L):
     # fused token selection: missing outputs, k <= 0, no or a small workspace, a misaligned one
     ws = L.lsa_select_tokens_workspace_size(1)
     assert ws == 4 * 4096 * 4 and L.lsa_select_tokens_workspace_size(0) == 0
-    sel_args = lambda k, w, wb: (ok, ok, ok, 4, n, ok, ok, 1, 4, 2, k, ok, ok, ok, ok, ok, 128, w, wb, n)
+    sel_args = lambda k, w, wb, fl=0: (ok, ok, ok, 4, n, ok, ok, 1, 4, 2, k, ok, ok, ok, ok, ok, 128, w, wb, fl, n)
     assert L.lsa_select_tokens(*sel_args(0, ok, ws)) == INVALID
     assert L.lsa_select_tokens(*sel_args(64, n, ws)) == WORKSPACE
     assert L.lsa_select_tokens(*sel_args(64, ok, ws - 16)) == WORKSPACE
     assert L.lsa_select_tokens(*sel_args(64, ctypes.c_void_p(0x100008), ws)) == MISALIGNED
+    assert L.lsa_select_tokens(*sel_args(64, ok, ws, 2)) == INVALID                       # unknown flag
     assert L.lsa_select_tokens(ok, ok, ok, 4, n, ok, ok, LSA_MAX_BATCH + 1, 4, 2, 64, ok, ok, ok, ok, ok, 128, ok,
-                               1 << 40, n) == UNSUPPORTED
+                               1 << 40, 0, n) == UNSUPPORTED
     # copy-engine fetch: null pointers, misaligned pools
     assert L.lsa_fetch_from_host_copy(n, n, 1, n, n, n, 1, 1, 1, n, n, 1, n, n) == INVALID
     assert L.lsa_fetch_from_host_copy(ctypes.c_void_p(0x1001), ok, 4, n, ok, ok, 1, 4, 2, ok, ok, 2, n, n) == MISALIGNED

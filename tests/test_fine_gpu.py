@@ -174,7 +174,7 @@ def two_call_selection(lw, q, w, tok_keys, k, max_sel=None):
     return scores, n_tok, sel, n_sel, cu
 
 
-def fused_selection(lw, q, w, tok_keys, k, ws, max_sel=None):
+def fused_selection(lw, q, w, tok_keys, k, ws, max_sel=None, keys_unchanged=False):
     B = lw.B
     max_sel = k if max_sel is None else max_sel
     scores = torch.full((B, 64 * lw.max_kept), float("nan"), device=DEV)
@@ -183,7 +183,7 @@ def fused_selection(lw, q, w, tok_keys, k, ws, max_sel=None):
     n_sel = torch.full((B,), -7, dtype=torch.int32, device=DEV)
     cu = torch.full((B + 1,), -7, dtype=torch.int32, device=DEV)
     lsa.lsa_select_tokens(q, w, tok_keys, lw.chunk_table, lw.kept[0], lw.n_kept[0], lw.max_chunks, k, scores, n_tok,
-                          sel, n_sel, cu, ws)
+                          sel, n_sel, cu, ws, keys_unchanged=keys_unchanged)
     return scores, n_tok, sel, n_sel, cu
 
 
@@ -210,8 +210,8 @@ def test_select_tokens_equals_score_then_topk(name, kw, k):
     inp, L, lw, tok_keys, q_tok = recalled(name, **kw)
     ws = lsa.new_select_tokens_workspace(lw.B)
     ref = two_call_selection(lw, q_tok[0, 3], L.w, tok_keys, k)
-    for call in range(2):
-        got = fused_selection(lw, q_tok[0, 3], L.w, tok_keys, k, ws)
+    for call in range(2):   # the second call loads its keys before the preceding kernel ends
+        got = fused_selection(lw, q_tok[0, 3], L.w, tok_keys, k, ws, keys_unchanged=call > 0)
         torch.cuda.synchronize()
         status_clean()
         assert_same_selection(got, ref)
