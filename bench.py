@@ -819,7 +819,7 @@ def run_e2e(args, inp, lws, dev, stream, decoded=None, fine=None):
                 x = dev_in[a][l]
                 q = x[1][t]
                 if use_fine:
-                    lws[l].fine_select(x[-1][t], inp.layers[l].w, fine[l][0])
+                    lws[l].fine_select(x[-1][t], inp.layers[l].w, fine[l][0], keys_unchanged=t > 0)
                 if causal:
                     lws[l].attend_append(q, douts[a][l][t], x[2][t], x[3][t], kv_unchanged=t > 0)
                 else:
