@@ -540,12 +540,15 @@ int lsa_topk_tokens(const float* scores, const int32_t* n_tokens, int k, int B, 
  *              (zero it once when it is allocated): the bin counts; every
  *              call leaves it zero again.  Calls that may overlap on the GPU
  *              need workspaces of their own.
- *   flags      0 or LSA_TOKENS_UNCHANGED: the kernel that ran just before this
- *              call on `stream` wrote none of token_keys, chunk_table, kept
- *              and n_kept (true for every decode step of a window after the
- *              first).  The scorer then looks up and loads its key rows while
- *              that kernel is still finishing; it reads q_idx and writes its
- *              outputs only after it.  Without the flag it waits first.
+ *   flags      0 or LSA_TOKENS_UNCHANGED: nothing on `stream` has written
+ *              token_keys, chunk_table, kept, n_kept or w since the previous
+ *              lsa_select_tokens call on it (true for every decode step of a
+ *              window after the first).  The kernels of this call start while
+ *              the preceding kernel is still finishing; with the flag the
+ *              scorer looks up and loads its key rows, and the selection works
+ *              out its counts and offsets, before waiting for it.  q_idx is
+ *              read and every output written only after it.  Without the flag
+ *              both wait first.
  * Device errors as lsa_token_score and lsa_topk_tokens.
  */
 #define LSA_TOKENS_UNCHANGED 1u

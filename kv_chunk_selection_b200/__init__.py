@@ -429,10 +429,11 @@ def lsa_select_tokens(q_idx, w, token_keys, chunk_table, kept, n_kept, max_chunk
     """lsa_token_score then lsa_topk_tokens in one call (same outputs), the
     selection driven by the scorer's score-bin counts.
 
-    ``keys_unchanged=True`` tells the library that the kernel just before this
-    call on the stream wrote none of token_keys, chunk_table, kept and n_kept
-    (every decode step of a window after the first), so the scorer may load its
-    key rows while that kernel finishes."""
+    ``keys_unchanged=True`` tells the library that nothing on the stream has
+    written token_keys, chunk_table, kept, n_kept or w since the previous call
+    of this function on it (every decode step of a window after the first), so
+    the scorer may load its key rows, and the selection work out its counts,
+    while the preceding kernel finishes."""
     _need(q_idx, "q_idx", torch.bfloat16)
     _need(w, "w", torch.float32)
     _need(token_keys, "token_keys", torch.bfloat16)

@@ -92,14 +92,12 @@ struct Partition {
 
 // Sequence offsets counted in 64-token units: an array of chunk offsets
 // (shift 0: cu_kept), or of token offsets that are multiples of 64 (shift 6:
-// cu_sel of the token-level fine stage, read without a packed copy).
-// `l2` reads them through L2 only (a kernel that reads them before its grid
-// dependency wait, while another kernel may still be running on its SM).
+// cu_sel of the token-level fine stage, read without a packed copy).  An
+// earlier kernel on the stream may have written them (ld_dep).
 struct Offsets {
   const int32_t* p;
   int shift;
-  bool l2 = false;
-  __device__ __forceinline__ int raw(int i) const { return l2 ? __ldcg(p + i) : __ldg(p + i); }
+  __device__ __forceinline__ int raw(int i) const { return ld_dep(p + i); }
   __device__ __forceinline__ int operator()(int i) const { return raw(i) >> shift; }
 };
 
@@ -281,6 +279,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     cur.start(cu, E, B, u0);
     const int64_t n_units = u1 - u0;
     const uint32_t smem_base_p = smem_u32(smem);
+    int at_b = -1, n_b = 0;
+    int64_t ckb = 0, n_pos = 0;
     for (int64_t i = 0; i < n_units; ++i) {
       const int s = static_cast<int>(i % kStages);
       if (i >= kStages) {
@@ -297,13 +297,17 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
       }
       const int b = cur.b, g = cur.g, j = cur.j;
-      const int64_t ckb = __ldg(sa.ck + b);
-      const int64_t n_pos = (static_cast<int64_t>(__ldg(sa.ck + b + 1)) - ckb) * kChunkTokens;
+      if (b != at_b) {   // the sequence's compact-buffer offset and recalled positions, once per sequence
+        at_b = b;
+        n_b = units_of(cu, E, b);
+        ckb = ld_dep(sa.ck + b);
+        n_pos = (static_cast<int64_t>(ld_dep(sa.ck + b + 1)) - ckb) * kChunkTokens;
+      }
       const uint32_t st = smem_base_p + s * kStageBytes;
       int64_t row_of[2];   // rows lane and lane + 32: compact-buffer row, or -1 (zeros)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int p = __ldg(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + lane + 32 * h);
+        const int p = ld_dep(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + lane + 32 * h);
         const bool okp = p >= 0 && p < n_pos && ckb + p / kChunkTokens < sa.ck_chunks;
         if (!okp) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
         row_of[h] = okp ? (g * sa.ck_chunks + ckb + p / kChunkTokens) * kChunkTokens + p % kChunkTokens : -1;
@@ -320,7 +324,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         cp_async_16_zfill(st + 2 * kBoxBytes + off, sa.v_buf + src, nb);
       }
       cp_async_mbar_arrive_noinc(&full[s]);
-      cur.advance(cu, E, B, units_of(cu, E, cur.b));
+      cur.advance(cu, E, B, n_b);
     }
     cp_async_wait_all();   // every copy this lane issued has landed before the warp leaves
     return;
@@ -337,6 +341,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       const int64_t n_units = u1 - u0;
       int64_t issued = 0;
       bool waited = !kv_unchanged;   // the local chunks are written by the preceding kernel
+      int at_b = -1, cb = 0, n_kept_b = 0;
       for (int64_t i = 0; i < n_units; ++i) {
         const int s = static_cast<int>(i % kStages);
         if (i >= kStages) {
@@ -347,8 +352,11 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             break;
           }
         }
-        const int cb = cu(cur.b);
-        const int n_kept_b = cu(cur.b + 1) - cb;
+        if (cur.b != at_b) {   // the sequence's offsets, once per sequence
+          at_b = cur.b;
+          cb = cu(cur.b);
+          n_kept_b = cu(cur.b + 1) - cb;
+        }
         const bool local = E && cur.j == n_kept_b;
         uint8_t* st = smem + s * kStageBytes;
         if (local && !waited) {
@@ -423,7 +431,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     // the row that receives this step's own token (-1: none).
     int valid_local = 64, new_row = -1;
     if (E) {
-      valid_local = __ldg(local_len + b);
+      valid_local = ld_dep(local_len + b);
       if (valid_local < 0 || valid_local > kChunkTokens) {
         if (tid == 0 && g == 0) set_status(status, LSA_DEV_ERR_BAD_COUNT);
         valid_local = min(max(valid_local, 0), kChunkTokens);
@@ -449,8 +457,8 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           q + (static_cast<int64_t>(b) * kNumQHeads + g * kGroup + gl) * kHeadDim);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        bq[t][0] = __ldg(qrow + 8 * t + c4);
-        bq[t][1] = __ldg(qrow + 8 * t + 4 + c4);
+        bq[t][0] = ld_dep(qrow + 8 * t + c4);
+        bq[t][1] = ld_dep(qrow + 8 * t + 4 + c4);
       }
     }
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -479,7 +487,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             // ldmatrix offsets read it) and into the local chunk in memory.
             const int kv = lane >> 4, x = lane & 15;
             const int64_t pg = static_cast<int64_t>(b) * kNumKVHeads + g;
-            const uint4 val = __ldg((kv ? app.v_new : app.k_new) + pg * 16 + x);
+            const uint4 val = ld_dep((kv ? app.v_new : app.k_new) + pg * 16 + x);
             const uint32_t off = (2 * kv + (x >> 3)) * kBoxBytes + new_row * 128 + (((x & 7) ^ (new_row & 7)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + off), "r"(val.x), "r"(val.y),
                          "r"(val.z), "r"(val.w)
@@ -650,8 +658,8 @@ attn_merge_kernel(const int32_t* __restrict__ cu_raw, int shift, int E, int B, i
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // The offsets were final before the attention grid started (it waits for
   // their writer before it lets this grid launch, or they did not change); they
-  // are read through L2 before the wait.
-  const Offsets cu{cu_raw, shift, true};
+  // are read before the wait.
+  const Offsets cu{cu_raw, shift};
   const bool bad = offsets_bad(cu, B, cap, shift != 0, max_sel);
   if (tid == 0) {
     int nt = 0, items = 0;

@@ -40,10 +40,43 @@ constexpr int kScoreBins = 4096;
 // see a quarter of the atomic adds each; the selection sums the copies.
 constexpr int kScoreBinReplicas = 4;
 
+// Loads of data that an earlier kernel on the stream may write: in a kernel
+// launched as a programmatic dependent, everything read after griddep_wait
+// (scores, counts, selections, offsets, and the caller's own inputs, which its
+// kernels may produce).  Such a grid starts while its predecessors still run,
+// so that data is not read-only for the grid's lifetime, which the
+// non-coherent path (ld.global.nc: __ldg, or a const __restrict__ pointer)
+// assumes: an nc load may be scheduled ahead of griddep_wait and return what
+// was there before.  These are plain global loads (ld.global), which the wait
+// makes see the predecessors' writes, kept after it by the volatile asm and
+// its clobber.  (ld.global.cg, which skips L1, measured 1.5x slower here: the
+// warps of a CTA re-read the same query rows, head weights and offsets.)
+__device__ __forceinline__ float ld_dep(const float* p) {
+  float v;
+  asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_dep(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_dep(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_dep(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float score_bin_scale(const float* w) {
   float wsum = 0.f;   // head order, as every kernel that needs it
 #pragma unroll
-  for (int h = 0; h < kIndexHeads; ++h) wsum += __ldg(w + h);
+  for (int h = 0; h < kIndexHeads; ++h) wsum += ld_dep(w + h);
   return (wsum > 0.f && wsum < 3.0e38f) ? static_cast<float>(kScoreBins) / wsum : 0.f;
 }
 

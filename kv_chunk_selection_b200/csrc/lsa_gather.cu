@@ -144,7 +144,7 @@ append_token_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v
   for (int i = threadIdx.x; i < 2 * kVecPerToken; i += blockDim.x) {
     const int kv = i / kVecPerToken, r = i % kVecPerToken;
     const int g = r / kVecPerRow, e = r % kVecPerRow;
-    const uint4 v = __ldg((kv ? v_new : k_new) + static_cast<int64_t>(b) * kVecPerToken + r);
+    const uint4 v = ld_dep((kv ? v_new : k_new) + static_cast<int64_t>(b) * kVecPerToken + r);
     (kv ? v_local : k_local)[((static_cast<int64_t>(b) * kNumKVHeads + g) * kChunkTokens + pos) * kVecPerRow + e] = v;
   }
   __syncthreads();
@@ -174,7 +174,7 @@ gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ 
   const int b = blockIdx.y;
   const int u = blockIdx.x / kNumKVHeads, g = blockIdx.x % kNumKVHeads;
   const int tid = threadIdx.x;
-  const int s0 = __ldg(cu_sel + b), s1 = __ldg(cu_sel + b + 1);
+  const int s0 = ld_dep(cu_sel + b), s1 = ld_dep(cu_sel + b + 1);
   const int n = s1 - s0;
   const bool lead = blockIdx.x == 0 && tid == 0;
   if (s0 < 0 || n < 0 || n > max_sel || (n % kChunkTokens) != 0 || (s0 % kChunkTokens) != 0) {
@@ -186,7 +186,7 @@ gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ 
     if (b == 0) cu_units[0] = s0 / kChunkTokens;
   }
   if (u * kChunkTokens >= n) return;
-  const int64_t c0 = __ldg(cu_kept + b), c1 = __ldg(cu_kept + b + 1);
+  const int64_t c0 = ld_dep(cu_kept + b), c1 = ld_dep(cu_kept + b + 1);
   const int64_t ou = s0 / kChunkTokens + u;
   if (c0 < 0 || c1 < c0 || c1 > buf_chunks || ou >= out_chunks) {
     if (tid == 0) set_status(status, ou >= out_chunks ? LSA_DEV_ERR_CAPACITY : LSA_DEV_ERR_BAD_COUNT);
@@ -201,12 +201,12 @@ gather_tokens_kernel(const uint4* __restrict__ k_buf, const uint4* __restrict__ 
     const int idx = tid + e * kTokThreads;
     const int kv = idx / (kChunkTokens * kRowVecs), rem = idx % (kChunkTokens * kRowVecs);
     const int r = rem / kRowVecs, x = rem % kRowVecs;
-    const int p = __ldg(my_sel + r);
+    const int p = ld_dep(my_sel + r);
     ok[e] = p >= 0 && p < n_pos;
     v[e] = make_uint4(0, 0, 0, 0);
     if (ok[e]) {
       const int64_t src = (g * buf_chunks + c0 + p / kChunkTokens) * kChunkTokens + p % kChunkTokens;
-      v[e] = __ldg((kv ? v_buf : k_buf) + src * kRowVecs + x);
+      v[e] = ld_dep((kv ? v_buf : k_buf) + src * kRowVecs + x);
     }
   }
 #pragma unroll

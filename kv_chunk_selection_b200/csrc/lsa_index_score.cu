@@ -91,20 +91,20 @@ struct TokenRows {
                 : nullptr;
   }
   __device__ int count(int b) const {
-    const int n = __ldg(n_kept + b);
+    const int n = ld_dep(n_kept + b);
     return (n < 0 || n > max_kept) ? -1 : n * kChunkTokens;
   }
   __device__ int64_t stride() const { return static_cast<int64_t>(max_kept) * kChunkTokens; }
   __device__ void on_count(int b, int n) const { n_tokens[b] = n < 0 ? 0 : n; }
   __device__ bool key_row(int b, int p, int64_t* row, unsigned* err) const {
     const int j = p / kChunkTokens, i = p % kChunkTokens;
-    const int c = __ldg(kept + static_cast<int64_t>(b) * max_kept + j);
+    const int c = ld_dep(kept + static_cast<int64_t>(b) * max_kept + j);
     if (c < 0 || c >= max_chunks) {
       *err = LSA_DEV_ERR_BAD_CHUNK;
       return false;
     }
     const int64_t slot =
-        table ? __ldg(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
+        table ? ld_dep(table + static_cast<int64_t>(b) * max_chunks + c) : static_cast<int64_t>(b) * max_chunks + c;
     if (slot < 0 || slot >= n_slots) {
       *err = LSA_DEV_ERR_BAD_SLOT;
       return false;
@@ -139,7 +139,12 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
   }
   if (blockIdx.x == 0 && threadIdx.x == 0 && !keys_unchanged) rows.on_count(b, n);
   const int base = blockIdx.x * kTile;
-  if (base >= n) return;
+  if (base >= n) {
+    // Every CTA waits before it ends, so this grid never completes before the
+    // preceding one (the next kernel's wait covers both).
+    if (keys_unchanged) griddep_wait();
+    return;
+  }
   if (smem_u32(smem) & 1023u) {   // the swizzle atoms assume 1024-byte alignment
     if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
     return;
@@ -192,7 +197,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     for (int it = 0; it < 16; ++it) {
       const int r = it * (kThreads / 16) + (tid >> 4);
       const int64_t krow = row_at[r];
-      v[it] = krow >= 0 ? __ldg(reinterpret_cast<const uint4*>(keys + krow * kIndexDim) + piece)
+      v[it] = krow >= 0 ? ld_dep(reinterpret_cast<const uint4*>(keys + krow * kIndexDim) + piece)
                         : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
@@ -211,7 +216,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
 #pragma unroll
     for (int i = tid; i < kIndexHeads * 16; i += kThreads) {
       const int h = i >> 4, j = i & 15;
-      *reinterpret_cast<uint4*>(sb + sw128_offset(h, j, kIndexHeads)) = __ldg(qb + i);
+      *reinterpret_cast<uint4*>(sb + sw128_offset(h, j, kIndexHeads)) = ld_dep(qb + i);
     }
   }
   fence_proxy_async_smem();   // generic-proxy smem writes -> visible to the tensor core
@@ -245,7 +250,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16), logit);
     float s = 0.f;
 #pragma unroll
-    for (int h = 0; h < kIndexHeads; ++h) s += __ldg(w + h) * (1.f / (1.f + fast_exp2(logit[h] * neg_scale_log2)));
+    for (int h = 0; h < kIndexHeads; ++h) s += ld_dep(w + h) * (1.f / (1.f + fast_exp2(logit[h] * neg_scale_log2)));
     if (row_ok[tid]) {
       scores[static_cast<int64_t>(b) * rows.stride() + base + tid] = s;
       if (ghist) {

@@ -93,7 +93,7 @@ constexpr int kMaxPerThread = 16;   // candidates kept in registers per thread (
 // Key of candidate i: the descending key of its score.
 struct ScoreKey {
   const float* sc;
-  __device__ __forceinline__ uint32_t operator()(int i) const { return desc_key(__ldg(sc + i)); }
+  __device__ __forceinline__ uint32_t operator()(int i) const { return desc_key(ld_dep(sc + i)); }
 };
 
 // Selects the kc smallest keys among candidates 0..cand-1 (kc < cand) and
@@ -261,13 +261,13 @@ topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_chun
   int part = 0;
   unsigned dummy = 0;
   for (int bb = tid; bb <= b; bb += kThreads)
-    part += kept_count(__ldg(n_chunks + bb), k_per_seq ? __ldg(k_per_seq + bb) : k_all, n_local, max_chunks,
+    part += kept_count(ld_dep(n_chunks + bb), k_per_seq ? ld_dep(k_per_seq + bb) : k_all, n_local, max_chunks,
                        max_kept, &dummy);
   int tot = 0;
   block_exclusive_scan(part, warp_sums, &tot);
   unsigned err = 0;
-  const int n = __ldg(n_chunks + b);
-  const int nk = kept_count(n, k_per_seq ? __ldg(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
+  const int n = ld_dep(n_chunks + b);
+  const int nk = kept_count(n, k_per_seq ? ld_dep(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
   if (tid == 0) {
     cu_kept[b + 1] = tot;
     if (b == 0) cu_kept[0] = 0;
@@ -330,7 +330,7 @@ __device__ void cluster_select_and_write(const float* __restrict__ sc, int cand,
   const int n_own = hi - lo;
   uint32_t kr[kPer];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) kr[e] = (e < n_own) ? desc_key(__ldg(sc + lo + e)) : 0u;
+  for (int e = 0; e < kPer; ++e) kr[e] = (e < n_own) ? desc_key(ld_dep(sc + lo + e)) : 0u;
 
   // ---- smallest and largest key of the whole cluster ------------------------
   uint32_t kmin = 0xffffffffu, kmax = 0u;
@@ -485,13 +485,13 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
   int part = 0;
   unsigned dummy = 0;
   for (int bb = tid; bb <= b; bb += kThreads)
-    part += kept_count(__ldg(n_chunks + bb), k_per_seq ? __ldg(k_per_seq + bb) : k_all, n_local, max_chunks,
+    part += kept_count(ld_dep(n_chunks + bb), k_per_seq ? ld_dep(k_per_seq + bb) : k_all, n_local, max_chunks,
                        max_kept, &dummy);
   int tot = 0;
   block_exclusive_scan(part, warp_sums, &tot);
   unsigned err = 0;
-  const int n = __ldg(n_chunks + b);
-  const int nk = kept_count(n, k_per_seq ? __ldg(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
+  const int n = ld_dep(n_chunks + b);
+  const int nk = kept_count(n, k_per_seq ? ld_dep(k_per_seq + b) : k_all, n_local, max_chunks, max_kept, &err);
   if (rank == 0 && tid == 0) {
     cu_kept[b + 1] = tot;
     if (b == 0) cu_kept[0] = 0;
@@ -524,9 +524,12 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
 // so that fewer of its atomic adds meet on one address; the bin that holds
 // the k-th best score is then known before any score is read again.  A
 // cluster of 8 CTAs per sequence, each owning an eighth of the positions:
-//   1. right after the grid dependency wait every thread issues its loads at
-//      once: up to kPer scores of its CTA's slice (in registers), four bins of
-//      the counts, the token counts and the head weights;
+//   1. what the scorer does not write (the bin scale from the head weights,
+//      the token counts from the kept counts as the scorer computes them, the
+//      output offsets), before the grid dependency wait when the caller
+//      promises those inputs settled; after the wait every thread issues its
+//      loads at once: up to kPer scores of its CTA's slice (in registers) and
+//      four bins of the counts;
 //   2. every CTA sums the count copies and finds that boundary bin b* (one
 //      block scan; all reach the same answer from the same counts);
 //   3. each CTA classifies its slice: a token in a bin above b* is selected
@@ -535,8 +538,10 @@ topk_cluster_kernel(const float* __restrict__ scores, const int32_t* __restrict_
 //      there are few);
 //   4. each CTA pushes its count of selected tokens and its candidates into
 //      every CTA's shared memory, and one cluster barrier publishes them; then
-//      every CTA ranks all candidates by (key, position) the same way, takes
-//      the r best (r = k - tokens above b*), and knows its own output offset;
+//      every CTA ranks all candidates by (key, position) the same way (one warp
+//      per candidate, its lanes comparing it against 32 others per ballot),
+//      takes the r best (r = k - tokens above b*), and knows its own output
+//      offset;
 //   5. each CTA writes its slice's positions in ascending order.
 // Every token above b* outscores every token in or below it, so this is the
 // exact top-k.  When the counts cannot be trusted (they do not add up to the
@@ -552,10 +557,10 @@ static_assert(kScoreBinReplicas * kScoreBins / 4 == kClusterCtas * 512, "each CT
 
 template <int kPer>
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads, 1)
-select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_tokens,
+select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict__ n_kept, int max_kept,
                      const float* __restrict__ w, int k, int max_tokens, int max_sel, int32_t* __restrict__ hist,
                      int32_t* __restrict__ sel, int32_t* __restrict__ n_sel, int32_t* __restrict__ cu_sel,
-                     unsigned* status) {
+                     unsigned* status, int kept_stable) {
   __shared__ uint32_t bits[kSelSliceWords];
   __shared__ uint32_t all_key[kClusterCtas * kSelMaxCand];   // [rank r][i]: CTA r's candidates, pushed by r
   __shared__ int all_pos[kClusterCtas * kSelMaxCand];
@@ -563,15 +568,39 @@ select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict
   __shared__ int warp_sums[32];
   __shared__ int hist_s[256];
   __shared__ int sel2[2];
-  __shared__ int s_bstar, s_above, s_ncand;
-  griddep_wait();   // the scorer has finished: scores, n_tokens and the bin counts are final
+  __shared__ int s_bstar, s_above, s_ncand, s_earlier;
   const int b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
   const float* sc = scores + static_cast<int64_t>(b) * max_tokens;
   int4* hrow = reinterpret_cast<int4*>(hist + static_cast<int64_t>(b) * kScoreBinReplicas * kScoreBins);
 
-  // ---- 1. every load at once ------------------------------------------------------
+  // ---- 1. what the scorer does not write; then every load at once ------------------
+  // The bin scale, the token counts as the scorer writes them (64 n_kept[b];
+  // 0 when n_kept is out of range) and the offsets, as lsa_topk_tokens
+  // computes them from those: min(k, n) positions per sequence (identical in
+  // every CTA of the cluster).  With kept_stable (the caller's promise that no
+  // kernel still running writes w or the kept counts) they are worked out
+  // before the grid dependency wait, while the scorer runs.
+  float scale = 0.f;
+  int tot = 0, n = 0, nk = 0;
+  unsigned err = 0;
+  auto counts = [&]() {
+    scale = score_bin_scale(w);
+    auto tokens_of = [&](int bb) {
+      const int m = ld_dep(n_kept + bb);
+      return (m < 0 || m > max_kept) ? 0 : m * kChunkTokens;
+    };
+    int part = 0;
+    unsigned dummy = 0;
+    for (int bb = tid; bb <= b; bb += kThreads) part += kept_count(tokens_of(bb), k, 0, max_tokens, max_sel, &dummy);
+    block_exclusive_scan(part, warp_sums, &tot);
+    n = tokens_of(b);
+    nk = kept_count(n, k, 0, max_tokens, max_sel, &err);
+  };
+  if (kept_stable) counts();
+  griddep_wait();   // the scorer has finished: scores and the bin counts are final, the outputs free
+  if (!kept_stable) counts();
   // This CTA's slice of positions, in whole bitmap words, sized from the row
   // length (so the loads need not wait for the token count): thread t holds
   // positions lo + j * 1024 + t, j < kPer.
@@ -583,7 +612,7 @@ select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int p = lo + j * kThreads + tid;
-    v[j] = (sliced && p < hi_row) ? __ldg(sc + p) : 0.f;
+    v[j] = (sliced && p < hi_row) ? ld_dep(sc + p) : 0.f;
   }
   int c4[4] = {0, 0, 0, 0};   // bins 4 tid .. 4 tid + 3, summed over the copies
 #pragma unroll
@@ -591,22 +620,10 @@ select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict
     const int4 x = hrow[rep * (kScoreBins / 4) + tid];
     c4[0] += x.x; c4[1] += x.y; c4[2] += x.z; c4[3] += x.w;
   }
-  const float scale = score_bin_scale(w);
   auto clear_counts = [&]() {   // this CTA's eighth of the counts, zero for the next call
     if (tid < 512) hrow[rank * 512 + tid] = make_int4(0, 0, 0, 0);
   };
-
-  // Offsets and counts, as lsa_topk_tokens: min(k, n) positions per sequence
-  // (identical in every CTA of the cluster, written by rank 0).
-  int part = 0;
-  unsigned dummy = 0;
-  for (int bb = tid; bb <= b; bb += kThreads) part += kept_count(__ldg(n_tokens + bb), k, 0, max_tokens, max_sel, &dummy);
-  int tot = 0;
-  block_exclusive_scan(part, warp_sums, &tot);
-  unsigned err = 0;
-  const int n = __ldg(n_tokens + b);
-  const int nk = kept_count(n, k, 0, max_tokens, max_sel, &err);
-  if (rank == 0 && tid == 0) {
+  if (rank == 0 && tid == 0) {   // (rank 0 writes the offsets)
     cu_sel[b + 1] = tot;
     if (b == 0) cu_sel[0] = 0;
     n_sel[b] = nk;
@@ -624,7 +641,7 @@ select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict
   const int own = c4[0] + c4[1] + c4[2] + c4[3];
   int total = 0;
   const int below = block_exclusive_scan(own, warp_sums, &total);   // tokens in bins under 4 tid
-  if (tid == 0) { s_bstar = -1; s_above = 0; s_ncand = 0; }
+  if (tid == 0) { s_bstar = -1; s_above = 0; s_ncand = 0; s_earlier = 0; }
   __syncthreads();
   if (total == n && sliced && scale > 0.f) {                         // cluster-uniform
     int above = total - below - own;                                 // tokens in bins over 4 tid + 3
@@ -701,25 +718,43 @@ select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict
     const int r_take = nk - above_all;
     fast = fast && r_take >= 0 && r_take <= mt;                      // cluster-uniform
     if (fast) {
-      // Candidate t = (CTA r, index i) of the slotted lists, ranked against all.
-      bool taken = false, earlier = false;
-      if (tid < kClusterCtas * kSelMaxCand) {
-        const int r = tid / kSelMaxCand, i = tid - r * kSelMaxCand;
-        if (i < x_cand[r]) {
-          const uint32_t ki = all_key[tid];
-          const int pi = all_pos[tid];
-          int rnk = 0;
-          for (int rr = 0; rr < kClusterCtas; ++rr)
-            for (int jj = 0; jj < x_cand[rr]; ++jj) {
-              const uint32_t kj = all_key[rr * kSelMaxCand + jj];
-              rnk += (kj < ki) || (kj == ki && all_pos[rr * kSelMaxCand + jj] < pi);
-            }
-          taken = rnk < r_take;
-          earlier = taken && r < static_cast<int>(rank);
-          if (taken && r == static_cast<int>(rank)) atomicOr(&bits[(pi - lo) >> 5], 1u << ((pi - lo) & 31));
+      // Candidate f of the flat list (the CTAs' lists in rank order) is slot
+      // (r, f - start[r]) of the slotted arrays.  Warp w ranks candidates
+      // w, w + 32, ...: its lanes compare the candidate with 32 others per
+      // ballot, and the count of candidates before it decides.
+      int start[kClusterCtas + 1];
+      start[0] = 0;
+#pragma unroll
+      for (int r = 0; r < kClusterCtas; ++r) start[r + 1] = start[r] + x_cand[r];
+      auto slot_of = [&](int f) {   // the last list that starts at or before f (start is non-decreasing)
+        int r = 0, base = 0;
+#pragma unroll
+        for (int q = 1; q < kClusterCtas; ++q)
+          if (f >= start[q]) { r = q; base = start[q]; }
+        return r * kSelMaxCand + (f - base);
+      };
+      for (int f = warp; f < mt; f += kThreads / 32) {
+        const int si = slot_of(f);
+        const uint32_t ki = all_key[si];
+        const int pi = all_pos[si];
+        int before = 0;
+        for (int j0 = 0; j0 < mt; j0 += 32) {
+          bool bj = false;
+          if (j0 + lane < mt) {
+            const int sj = slot_of(j0 + lane);
+            const uint32_t kj = all_key[sj];
+            bj = (kj < ki) || (kj == ki && all_pos[sj] < pi);
+          }
+          before += __popc(__ballot_sync(0xffffffffu, bj));
+        }
+        if (lane == 0 && before < r_take) {
+          const int r = si / kSelMaxCand;
+          if (r < static_cast<int>(rank)) atomicAdd(&s_earlier, 1);
+          if (r == static_cast<int>(rank)) atomicOr(&bits[(pi - lo) >> 5], 1u << ((pi - lo) & 31));
         }
       }
-      off += __syncthreads_count(earlier);   // also publishes the bits
+      __syncthreads();   // the bits and the count of earlier ranks' taken candidates
+      off += s_earlier;
       // ---- 5. this slice's positions, ascending ---------------------------------------
       griddep_launch_dependents();
       const int words = hi > lo ? (hi - lo + 31) >> 5 : 0;
@@ -843,8 +878,8 @@ extern "C" int lsa_select_tokens(const void* q_idx, const float* w, const void* 
   auto kernel = max_tokens <= topk::kClusterThreads * 4   ? topk::select_tokens_kernel<4>
                 : max_tokens <= topk::kClusterThreads * 8 ? topk::select_tokens_kernel<8>
                                                           : topk::select_tokens_kernel<16>;
-  launch_pdl(true, kernel, dim3(topk::kClusterCtas, B), dim3(topk::kThreads), 0, s, scores, n_tokens, w, k,
-             max_tokens, max_sel, hist, sel, n_sel, cu_sel, lsa_device_status_ptr());
+  launch_pdl(true, kernel, dim3(topk::kClusterCtas, B), dim3(topk::kThreads), 0, s, scores, n_kept, max_kept, w, k,
+             max_tokens, max_sel, hist, sel, n_sel, cu_sel, lsa_device_status_ptr(), keys_unchanged);
   return launch_status();
 }
 

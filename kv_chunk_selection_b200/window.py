@@ -176,9 +176,9 @@ class LayerWindow:
     def fine_select(self, q_tok, w, token_keys, buf: int = 0, stream=None, keys_unchanged: bool = False):
         """Token-level stage of one step: scores of the recalled tokens from the step's
         indexer query q_tok [B, 16, 128] and the fine_k best (packed into dense
-        units when the window is causal).  ``keys_unchanged``: the previous kernel
-        on the stream wrote neither the token keys nor this window's kept lists
-        (true for every step but the first)."""
+        units when the window is causal).  ``keys_unchanged``: nothing on the
+        stream has written the token keys, the head weights or this window's kept
+        lists since the previous step's call (true for every step but the first)."""
         if self.fused_select:
             lsa_select_tokens(q_tok, w, token_keys, self.chunk_table, self.kept[buf], self.n_kept[buf],
                               self.max_chunks, self.fine_k, self.tok_scores, self.n_tokens, self.sel, self.n_sel,

@@ -360,6 +360,45 @@ def test_fine_stage_short_and_empty_sequences():
     assert_attention_close(out[1:2], chunk_ref[1:2])
 
 
+@pytest.mark.parametrize("keys_unchanged", [False, True])
+def test_fine_steps_pipelined_select_own_scores(keys_unchanged):
+    """Fine steps back to back on one stream, no host synchronisation between
+    them (each kernel a programmatic dependent of the one before, as in a
+    window): three windows of 64 steps, each step's selection copied aside on
+    the stream, then every selection checked bit for bit against the oracle's
+    top-k of that step's own fp32 scores.  A selection kernel that read its
+    scores before the scorer had finished them would differ here."""
+    inp = workloads.make_inputs("tiny", DEV)
+    L = inp.layers[0]
+    tok_keys, q_tok = workloads.fine_inputs(inp, 0, DEV)
+    kn, vn = workloads.decoded_tokens(inp, 0, DEV)
+    k = 256
+    for _ in range(3):
+        lw = LayerWindow(inp.n_chunks, inp.k_per_seq, inp.chunk_table, inp.max_chunks, DEV, fine_k=k, causal=True)
+        outs = torch.empty((64, 1, 64, 128), device=DEV)
+        sel_at = torch.empty((64,) + tuple(lw.sel.shape), dtype=lw.sel.dtype, device=DEV)
+        nsel_at = torch.empty((64,) + tuple(lw.n_sel.shape), dtype=lw.n_sel.dtype, device=DEV)
+        sc_at = torch.empty((64,) + tuple(lw.tok_scores.shape), dtype=lw.tok_scores.dtype, device=DEV)
+        lw.select(L.q_idx[0], L.w, L.chunk_keys)
+        lw.gather(L.k_pool, L.v_pool)
+        lw.reset_local()
+        for t in range(64):
+            lw.append(kn[0, t], vn[0, t])
+            lw.fine_select(q_tok[0, t], L.w, tok_keys, keys_unchanged=keys_unchanged and t > 0)
+            lw.attend(L.q[0, t], outs[t])
+            sel_at[t].copy_(lw.sel)
+            nsel_at[t].copy_(lw.n_sel)
+            sc_at[t].copy_(lw.tok_scores)
+        torch.cuda.synchronize()
+        status_clean()
+        n = int(lw.n_tokens[0])
+        for t in range(64):
+            own = f64(sc_at[t])[0, :n]
+            want = list(oracle.topk_tokens([own], k)[0])
+            got = sel_at[t, 0, : int(nsel_at[t, 0])].cpu().tolist()
+            assert got == want, f"step {t}: selection differs from the top-k of its own scores"
+
+
 def test_window_tiny_fine_and_causal():
     """A whole tiny window with the fine stage (k = 256 of 576 recalled tokens) and
     the causal local chunk, all 64 steps, against the oracle step by step."""
