@@ -909,6 +909,17 @@ def run_attn_only(args):
     qs = workloads.randn_bf16((workloads.TAU, B, 64, 128), 3, dev)
     out = torch.empty((B, 64, 128), device=dev)
     ws = lsa.new_attn_workspace(B, dev)
+    if args.settle_gib > 0:
+        # A process that has not yet written much device memory runs this kernel
+        # about 8% faster than one that has (measured: 32.2 us against 34.5 us
+        # per 500K launch after writing 5 GiB elsewhere, with the copy bandwidth,
+        # clocks and temperatures unchanged); the pipeline always runs in the
+        # second state, so the timing does too.
+        scratch = torch.empty((args.settle_gib << 30,), dtype=torch.uint8, device=dev)
+        scratch.fill_(1)
+        torch.cuda.synchronize()
+        del scratch
+        torch.cuda.empty_cache()   # returned to the driver: a profiler's replays need not save it
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         lsa.lsa_sparse_decode_attn(qs[0], kbuf, vbuf, cu, out, ws)     # first call sets kernel attributes
@@ -940,7 +951,7 @@ def run_attn_only(args):
     return {"mode": "attn-only", "workload": args.workload, "kept_chunks": total, "launches_per_replay": args.steps,
             "replays": args.repeats, "median_us": med * 1e6, "min_us": times[0] * 1e6, "bytes_per_launch": nbytes,
             "median_gbs": nbytes / med / 1e9, "frac_of_measured": nbytes / med / 1e9 / peak,
-            "peak_source": kind, "device_status": bits, "source_digest": source_digest()}
+            "peak_source": kind, "device_status": bits, "source_digest": source_digest(), "settle_gib": args.settle_gib}
 
 
 def run_fine_only(args):
@@ -1173,6 +1184,8 @@ def main():
     ap.add_argument("--causal", action="store_true",
                     help="append each step's token to a local chunk and attend it (decoded window)")
     ap.add_argument("--repeats", type=int, default=5, help="graph replays timed in --attn-only mode")
+    ap.add_argument("--settle-gib", type=int, default=5,
+                    help="GiB of device memory written before the --attn-only timing (0: a fresh process)")
     ap.add_argument("--attn-only", action="store_true",
                     help="time attention launches alone on a random compact buffer (profiling case)")
     ap.add_argument("--fine-only", action="store_true",
