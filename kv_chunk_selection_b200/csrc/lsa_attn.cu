@@ -274,15 +274,34 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     // 256-byte rows instead of 32 scattered pieces.  The pieces land at their
     // swizzled places in the stage; each lane arrives on the stage's full
     // barrier when its copies have landed.  A position outside the sequence's
-    // recalled tokens is written as zeros.
+    // recalled tokens is written as zeros.  The positions of the next unit
+    // are loaded while this one waits for its stage and issues its copies, so
+    // their L2 round trip is off the producer's path.
     UnitCursor cur;
     cur.start(cu, E, B, u0);
     const int64_t n_units = u1 - u0;
     const uint32_t smem_base_p = smem_u32(smem);
     int at_b = -1, n_b = 0;
     int64_t ckb = 0, n_pos = 0;
+    auto load_pos = [&](const UnitCursor& c, int* p) {   // positions lane and lane + 32 of unit c
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        p[h] = ld_dep(sa.sel + static_cast<int64_t>(c.b) * sa.max_sel + c.j * kChunkTokens + lane + 32 * h);
+    };
+    int p_cur[2] = {0, 0}, p_nxt[2] = {0, 0};
+    if (n_units > 0) load_pos(cur, p_cur);
     for (int64_t i = 0; i < n_units; ++i) {
       const int s = static_cast<int>(i % kStages);
+      const int b = cur.b, g = cur.g;
+      if (b != at_b) {   // the sequence's compact-buffer offset and recalled positions, once per sequence
+        at_b = b;
+        n_b = units_of(cu, E, b);
+        ckb = ld_dep(sa.ck + b);
+        n_pos = (static_cast<int64_t>(ld_dep(sa.ck + b + 1)) - ckb) * kChunkTokens;
+      }
+      UnitCursor nxt = cur;
+      nxt.advance(cu, E, B, n_b);
+      if (i + 1 < n_units) load_pos(nxt, p_nxt);
       if (i >= kStages) {
         const unsigned par = static_cast<unsigned>(((i / kStages) - 1) & 1);
         int okw = 1;
@@ -296,18 +315,11 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
           break;
         }
       }
-      const int b = cur.b, g = cur.g, j = cur.j;
-      if (b != at_b) {   // the sequence's compact-buffer offset and recalled positions, once per sequence
-        at_b = b;
-        n_b = units_of(cu, E, b);
-        ckb = ld_dep(sa.ck + b);
-        n_pos = (static_cast<int64_t>(ld_dep(sa.ck + b + 1)) - ckb) * kChunkTokens;
-      }
       const uint32_t st = smem_base_p + s * kStageBytes;
       int64_t row_of[2];   // rows lane and lane + 32: compact-buffer row, or -1 (zeros)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int p = ld_dep(sa.sel + static_cast<int64_t>(b) * sa.max_sel + j * kChunkTokens + lane + 32 * h);
+        const int p = p_cur[h];
         const bool okp = p >= 0 && p < n_pos && ckb + p / kChunkTokens < sa.ck_chunks;
         if (!okp) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
         row_of[h] = okp ? (g * sa.ck_chunks + ckb + p / kChunkTokens) * kChunkTokens + p % kChunkTokens : -1;
@@ -324,7 +336,9 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         cp_async_16_zfill(st + 2 * kBoxBytes + off, sa.v_buf + src, nb);
       }
       cp_async_mbar_arrive_noinc(&full[s]);
-      cur.advance(cu, E, B, n_b);
+      cur = nxt;
+      p_cur[0] = p_nxt[0];
+      p_cur[1] = p_nxt[1];
     }
     cp_async_wait_all();   // every copy this lane issued has landed before the warp leaves
     return;
