@@ -186,6 +186,7 @@ inline int grid_for(int sms) { return sms * kCtasPerSm < kMaxCtas ? sms * kCtasP
 // partials; large launches keep one CTA per SM.
 constexpr int64_t kMinUnitsPerCta = 4;
 constexpr int64_t kMinIndexedUnitsPerCta = 2;   // the in-place fine stage: more CTAs issue its row copies
+constexpr int kPosAhead = 2;                     // units whose positions the in-place producer loads ahead (4: no gain)
 inline int grid_for_units(int sms, int64_t max_units, int64_t per_cta = kMinUnitsPerCta) {
   const int64_t want = (max_units + per_cta - 1) / per_cta;
   const int full = grid_for(sms);
@@ -274,9 +275,10 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     // 256-byte rows instead of 32 scattered pieces.  The pieces land at their
     // swizzled places in the stage; each lane arrives on the stage's full
     // barrier when its copies have landed.  A position outside the sequence's
-    // recalled tokens is written as zeros.  The positions of the next unit
-    // are loaded while this one waits for its stage and issues its copies, so
-    // their L2 round trip is off the producer's path.
+    // recalled tokens is written as zeros.  The positions of a unit are
+    // loaded kPosAhead units ahead, while the units before it wait for their
+    // stages and issue their copies, so their L2 round trips are off the
+    // producer's path.
     UnitCursor cur;
     cur.start(cu, E, B, u0);
     const int64_t n_units = u1 - u0;
@@ -288,8 +290,20 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       for (int h = 0; h < 2; ++h)
         p[h] = ld_dep(sa.sel + static_cast<int64_t>(c.b) * sa.max_sel + c.j * kChunkTokens + lane + 32 * h);
     };
-    int p_cur[2] = {0, 0}, p_nxt[2] = {0, 0};
-    if (n_units > 0) load_pos(cur, p_cur);
+    // The look-ahead cursor `la` is the unit whose positions load next; la_nb
+    // is the unit count of its sequence.
+    UnitCursor la = cur;
+    int la_nb = n_units > 0 ? units_of(cu, E, la.b) : 0;
+    auto la_next = [&](int* p) {
+      load_pos(la, p);
+      const int prev = la.b;
+      la.advance(cu, E, B, la_nb);
+      if (la.b != prev && la.b < B) la_nb = units_of(cu, E, la.b);
+    };
+    int pq[kPosAhead + 1][2] = {};   // positions of units i .. i + kPosAhead
+#pragma unroll
+    for (int q = 0; q < kPosAhead; ++q)
+      if (q < n_units) la_next(pq[q]);
     for (int64_t i = 0; i < n_units; ++i) {
       const int s = static_cast<int>(i % kStages);
       const int b = cur.b, g = cur.g;
@@ -299,9 +313,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         ckb = ld_dep(sa.ck + b);
         n_pos = (static_cast<int64_t>(ld_dep(sa.ck + b + 1)) - ckb) * kChunkTokens;
       }
-      UnitCursor nxt = cur;
-      nxt.advance(cu, E, B, n_b);
-      if (i + 1 < n_units) load_pos(nxt, p_nxt);
+      if (i + kPosAhead < n_units) la_next(pq[kPosAhead]);
       if (i >= kStages) {
         const unsigned par = static_cast<unsigned>(((i / kStages) - 1) & 1);
         int okw = 1;
@@ -319,7 +331,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
       int64_t row_of[2];   // rows lane and lane + 32: compact-buffer row, or -1 (zeros)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int p = p_cur[h];
+        const int p = pq[0][h];
         const bool okp = p >= 0 && p < n_pos && ckb + p / kChunkTokens < sa.ck_chunks;
         if (!okp) set_status(status, LSA_DEV_ERR_BAD_CHUNK);
         row_of[h] = okp ? (g * sa.ck_chunks + ckb + p / kChunkTokens) * kChunkTokens + p % kChunkTokens : -1;
@@ -336,9 +348,12 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         cp_async_16_zfill(st + 2 * kBoxBytes + off, sa.v_buf + src, nb);
       }
       cp_async_mbar_arrive_noinc(&full[s]);
-      cur = nxt;
-      p_cur[0] = p_nxt[0];
-      p_cur[1] = p_nxt[1];
+      cur.advance(cu, E, B, n_b);
+#pragma unroll
+      for (int q = 0; q < kPosAhead; ++q) {
+        pq[q][0] = pq[q + 1][0];
+        pq[q][1] = pq[q + 1][1];
+      }
     }
     cp_async_wait_all();   // every copy this lane issued has landed before the warp leaves
     return;
