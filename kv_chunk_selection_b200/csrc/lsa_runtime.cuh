@@ -33,8 +33,12 @@ EncodeTiledFn tensor_map_encoder();
 // launched once every CTA of the previous kernel on the stream has signalled
 // griddepcontrol.launch_dependents, so its launch latency overlaps that
 // kernel's run.  Every kernel launched this way executes griddepcontrol.wait
-// before its first global-memory access, which orders it after the previous
-// kernel's completion and memory flush.
+// before its first global-memory access (except the reads that a caller's
+// flag declares settled: LSA_ATTN_KV_UNCHANGED, LSA_TOKENS_UNCHANGED), which
+// orders it after the previous kernel's completion and memory flush; its
+// loads after the wait are plain (ld_dep), never non-coherent; and every CTA
+// that ends early waits first, so the grid never completes before the one it
+// depends on.
 //
 // With pdl == false it is an ordinary stream-ordered launch (the griddepcontrol
 // instructions are then no-ops).  The kernels of the per-step chain use PDL;
