@@ -206,6 +206,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   // The 128-byte TMA swizzle pattern repeats every 1024 bytes and the fragment
   // addressing below assumes each box starts on such a boundary.
   if (smem_u32(smem_raw) & 1023u) {
+    griddep_wait();   // every CTA waits before it ends
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
     return;
   }
@@ -229,6 +230,7 @@ sparse_decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
   // (Indexed: token offsets, multiples of 64, at most max_sel per sequence;
   // buf_chunks is then the unit capacity B * max_sel / 64.)
   if (offsets_bad(cu, B, buf_chunks, indexed, sa.max_sel)) {
+    if (kv_unchanged) griddep_wait();   // every CTA waits before it ends
     if (blockIdx.x == 0 && tid == 0) set_status(status, LSA_DEV_ERR_CAPACITY);
     return;
   }

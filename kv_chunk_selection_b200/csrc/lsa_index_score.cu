@@ -146,6 +146,7 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
     return;
   }
   if (smem_u32(smem) & 1023u) {   // the swizzle atoms assume 1024-byte alignment
+    if (keys_unchanged) griddep_wait();   // every CTA waits before it ends
     if (threadIdx.x == 0) set_status(status, LSA_DEV_ERR_INTERNAL);
     return;
   }
