@@ -73,11 +73,16 @@ __device__ __forceinline__ uint4 ld_dep(const uint4* p) {
   return v;
 }
 
+// Bins per unit of score, from sum_h w[h] summed in head order from 0 (as
+// every kernel that needs it sums it).
+__device__ __forceinline__ float score_bin_scale_of_sum(float wsum) {
+  return (wsum > 0.f && wsum < 3.0e38f) ? static_cast<float>(kScoreBins) / wsum : 0.f;
+}
 __device__ __forceinline__ float score_bin_scale(const float* w) {
-  float wsum = 0.f;   // head order, as every kernel that needs it
+  float wsum = 0.f;
 #pragma unroll
   for (int h = 0; h < kIndexHeads; ++h) wsum += ld_dep(w + h);
-  return (wsum > 0.f && wsum < 3.0e38f) ? static_cast<float>(kScoreBins) / wsum : 0.f;
+  return score_bin_scale_of_sum(wsum);
 }
 
 __device__ __forceinline__ int score_bin(float s, float scale) {

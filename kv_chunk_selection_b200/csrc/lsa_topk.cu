@@ -578,25 +578,39 @@ select_tokens_kernel(const float* __restrict__ scores, const int32_t* __restrict
   // ---- 1. what the scorer does not write; then every load at once ------------------
   // The bin scale, the token counts as the scorer writes them (64 n_kept[b];
   // 0 when n_kept is out of range) and the offsets, as lsa_topk_tokens
-  // computes them from those: min(k, n) positions per sequence (identical in
-  // every CTA of the cluster).  With kept_stable (the caller's promise that no
+  // computes them from those: min(k, n) positions per sequence (rank 0's
+  // warp 0 sums them over sequences 0 .. b).  With kept_stable (the caller's promise that no
   // kernel still running writes w or the kept counts) they are worked out
   // before the grid dependency wait, while the scorer runs.
   float scale = 0.f;
   int tot = 0, n = 0, nk = 0;
   unsigned err = 0;
   auto counts = [&]() {
-    scale = score_bin_scale(w);
-    auto tokens_of = [&](int bb) {
-      const int m = ld_dep(n_kept + bb);
-      return (m < 0 || m > max_kept) ? 0 : m * kChunkTokens;
-    };
-    int part = 0;
-    unsigned dummy = 0;
-    for (int bb = tid; bb <= b; bb += kThreads) part += kept_count(tokens_of(bb), k, 0, max_tokens, max_sel, &dummy);
-    block_exclusive_scan(part, warp_sums, &tot);
-    n = tokens_of(b);
+    // Every load first, so that they take one round trip: this sequence's
+    // kept count, the head weights, and (for the lanes of rank 0's warp 0,
+    // which alone needs the offsets) the kept counts of sequences 0 .. b.
+    const bool lead = rank == 0 && warp == 0;
+    const int m_own = ld_dep(n_kept + b);
+    float wv[kIndexHeads];
+#pragma unroll
+    for (int h = 0; h < kIndexHeads; ++h) wv[h] = ld_dep(w + h);
+    const int m_lane = (lead && lane <= b) ? ld_dep(n_kept + lane) : 0;
+    float wsum = 0.f;
+#pragma unroll
+    for (int h = 0; h < kIndexHeads; ++h) wsum += wv[h];
+    scale = score_bin_scale_of_sum(wsum);
+    auto tokens_of = [&](int m) { return (m < 0 || m > max_kept) ? 0 : m * kChunkTokens; };
+    n = tokens_of(m_own);
     nk = kept_count(n, k, 0, max_tokens, max_sel, &err);
+    if (lead) {   // warp-uniform
+      unsigned dummy = 0;
+      int part = lane <= b ? kept_count(tokens_of(m_lane), k, 0, max_tokens, max_sel, &dummy) : 0;
+      for (int bb = lane + 32; bb <= b; bb += 32)
+        part += kept_count(tokens_of(ld_dep(n_kept + bb)), k, 0, max_tokens, max_sel, &dummy);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      tot = part;
+    }
   };
   if (kept_stable) counts();
   griddep_wait();   // the scorer has finished: scores and the bin counts are final, the outputs free
