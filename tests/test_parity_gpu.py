@@ -441,6 +441,28 @@ def test_fused_append_step_matches_two_launch_path_and_oracle():
     assert_attention_close(out_f, ref)
 
 
+def test_rejected_offsets_under_kv_unchanged_report_capacity_and_the_stream_goes_on():
+    """Offsets that the attention rejects (a total beyond the compact buffer)
+    make every CTA leave before any K/V read; with LSA_ATTN_KV_UNCHANGED each
+    CTA first waits for the preceding kernel, so the grid still completes after
+    it.  CAPACITY is reported, and the next, correct call on the stream matches
+    the oracle."""
+    q, kb, vb, cu = ragged_buffers([3, 1], seed=97)
+    ws = lsa.new_attn_workspace(2)
+    out = torch.full((2, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out, ws)
+    bad = cu.clone()
+    bad[-1] = kb.shape[1] + 1          # one chunk more than the buffer holds
+    lsa.lsa_sparse_decode_attn(q, kb, vb, bad, out, ws, kv_unchanged=True)
+    assert lsa.read_device_status() & 8          # CAPACITY
+    out2 = torch.full((2, 64, 128), float("nan"), device=DEV)
+    lsa.lsa_sparse_decode_attn(q, kb, vb, cu, out2, ws, kv_unchanged=True)
+    torch.cuda.synchronize()
+    status_clean()
+    ref = oracle.sparse_decode_attn(f64(q), f64(cm(kb)), f64(cm(vb)), i64(cu))
+    assert_attention_close(out2, ref)
+
+
 def test_fused_append_full_local_chunk_reports_capacity():
     n_kept = [2]
     q, kb, vb, cu = ragged_buffers(n_kept, seed=93)
