@@ -140,9 +140,15 @@ index_score_kernel(const __nv_bfloat16* __restrict__ q_idx, const float* __restr
   if (blockIdx.x == 0 && threadIdx.x == 0 && !keys_unchanged) rows.on_count(b, n);
   const int base = blockIdx.x * kTile;
   if (base >= n) {
-    // Every CTA waits before it ends, so this grid never completes before the
-    // preceding one (the next kernel's wait covers both).
-    if (keys_unchanged) griddep_wait();
+    // No rows here (a sequence shorter than the longest).  The sequence's
+    // first CTA still waits and writes its count, so this grid never
+    // completes before the preceding one (the next kernel's wait covers
+    // both); the other empty CTAs leave at once and free their SM slots for
+    // CTAs with rows to load.
+    if (keys_unchanged && blockIdx.x == 0) {
+      griddep_wait();
+      if (threadIdx.x == 0) rows.on_count(b, n);
+    }
     return;
   }
   if (smem_u32(smem) & 1023u) {   // the swizzle atoms assume 1024-byte alignment
