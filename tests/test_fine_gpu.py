@@ -324,6 +324,33 @@ def test_fine_step_attention_matches_oracle(name, kw, k):
     assert_attention_close(out, ref, heads=heads)
 
 
+def test_select_tokens_flagged_writes_every_count_including_empty_sequences():
+    """With LSA_TOKENS_UNCHANGED the scorer's CTAs that find no rows leave at
+    once, but each sequence's first CTA still waits and writes its token count:
+    a flagged call into fresh outputs (counts set to -1) equals the unflagged
+    call bit for bit, the sequence with nothing recalled included."""
+    B = 3
+    n_chunks = torch.tensor([0, 3, 40], dtype=torch.int32, device=DEV)
+    k_per_seq = torch.tensor([0, 2, 9], dtype=torch.int32, device=DEV)
+    max_chunks = 40
+    g = torch.Generator(device=DEV).manual_seed(18)
+    n_slots = B * max_chunks
+    keys = torch.randn((n_slots, 128), generator=g, device=DEV).to(torch.bfloat16)
+    tok_keys = torch.randn((n_slots, 64, 128), generator=g, device=DEV).to(torch.bfloat16)
+    w = torch.rand(16, generator=g, device=DEV)
+    q_idx = torch.randn((B, 16, 128), generator=g, device=DEV).to(torch.bfloat16)
+    q_tok = torch.randn((B, 16, 128), generator=g, device=DEV).to(torch.bfloat16)
+    lw = LayerWindow(n_chunks, k_per_seq, None, max_chunks, DEV, fine_k=256)
+    lw.select(q_idx, w, keys)
+    ws = lsa.new_select_tokens_workspace(lw.B)
+    ref = fused_selection(lw, q_tok, w, tok_keys, 256, ws)
+    got = fused_selection(lw, q_tok, w, tok_keys, 256, ws, keys_unchanged=True)
+    torch.cuda.synchronize()
+    status_clean()
+    assert i64(got[1]).tolist() == [0, 192, 640]
+    assert_same_selection(got, ref)
+
+
 def test_fine_stage_short_and_empty_sequences():
     """A sequence with fewer recalled tokens than k keeps them all (the step then
     equals chunk attention); a sequence with nothing recalled gets zeros."""
